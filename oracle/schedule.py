@@ -59,8 +59,15 @@ def set_utilization(ws: Sequence[Sequence[int]]) -> Fraction:
 
     [EB] §5.2 (CumUtil: "U(.) denotes GPU utilization"); read as Eq. (3)
     applied to the one step that runs S: sum_d W_d / (D * max_d W_d).
+    A set that carries no work at all leaves every device idle and is given
+    U = 0 (a reading: Eq. (3) is 0/0 there; in an episode every micro-batch
+    carries T k > 0 token-expert pairs, so this only concerns stand-alone
+    calls on arbitrary loads).
     """
-    return utilization([combined(ws)])
+    W = combined(ws)
+    if max(W) == 0:
+        return Fraction(0)
+    return utilization([W])
 
 
 def _pad_to_m(chosen: List[int], pending: Sequence[int], m: int) -> List[int]:

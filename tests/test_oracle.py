@@ -381,3 +381,13 @@ def test_moe_layer_slot_gates_brute_force():
     # gates differ between slots, so swapping them changes the result
     out_sw = omoe.moe_layer(h, idx, gate[:, ::-1], 0, lambda l, e: W[e], E, 0, "f32")
     assert not np.array_equal(out, out_sw)
+
+
+def test_zero_work_sets_rank_lowest():
+    """Reading for loads with no work: U = 0, so such a set never beats one
+    that carries work, and adding it never raises U (CumUtil skips it)."""
+    w = {0: [0, 0], 1: [3, 1], 2: [0, 0]}
+    assert osch.set_utilization([w[0]]) == 0
+    assert osch.cumutil([0, 1, 2], w, 1) == [0, 1]
+    # every set holding micro-batch 1 has U = 4/6; the largest one wins
+    assert osch.maxutil([0, 1, 2], w, 1) == [0, 1, 2]

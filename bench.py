@@ -1,0 +1,439 @@
+"""Benchmark of the cross-layer MoE step (EasyBalance) on B200.
+
+A bench "step" is one whole episode of Algorithm 1 on the Qwen3-30B-A3B-shaped
+workload (48 MoE layers, 128 experts, top-8, hidden 2048, expert FFN 768,
+D = 8 virtual ranks, M = 8 micro-batches x 1024 tokens): from reset until every
+micro-batch has passed all 48 layers, each scheduler step running routing,
+loads, the RunSet choice, permutation, the two grouped expert GEMMs and the
+combine.  Throughput counts token-layer passes: M * T * L per episode.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 (launched with torchrun) runs one independent replica per GPU: the path
+has no exchange step on one GPU ("replicas only"); value = all ranks' tokens /
+the slowest rank's time.  --impl reference times the CPU oracle (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "cross-layer MoE step tokens/s at Qwen3-30B shape (1 B200); under-util 1−u"
+UNIT = "tokens/s"
+POLICY_NAMES = {0: "cumutil", 1: "maxutil", 2: "lockstep", 3: "diffpeak"}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="qwen3_bf16")
+    p.add_argument("--policy", default="maxutil", choices=list(POLICY_NAMES.values()))
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def dist_setup(args):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: int):
+        self.gpu = gpu
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu)], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in out.strip().splitlines():
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d.get("hbm_gbs", 6650.0), "measured"
+    return 6650.0, "fallback"
+
+
+def ncu_traffic(name: str):
+    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
+    summary says it matches the current build (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d.get(name)
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ our arm
+
+def run_ours(args, world, rank, local):
+    import numpy as np
+    import torch
+
+    import cross_layer_expert_b200 as eb
+    import synth
+    from cross_layer_expert_b200 import build
+
+    if rank == 0 or not os.path.exists(build.LIB):
+        build.build()
+    barrier(world)
+    eb.load()
+    wl = synth.get(args.workload)
+    policy = {v: k for k, v in POLICY_NAMES.items()}[args.policy]
+    dev = torch.device("cuda", torch.cuda.current_device())
+    logits_np = synth.logits(wl)
+    logits = torch.from_numpy(logits_np).to(dev)
+    h0 = synth.hidden_torch(wl).to(dev)
+    wgu, wdn = synth.weights_torch(wl, device=dev)
+    torch.cuda.synchronize()
+
+    def cfg_for(pol, compute=1):
+        return eb.make_config(L=wl.L, E=wl.E, k=wl.k, H=wl.H, F=wl.F, D=wl.D, M=wl.M, T=wl.T,
+                              n_shared=wl.n_shared, dtype=eb.DTYPE_BF16, policy=pol,
+                              m=wl.m_default, compute=compute)
+
+    # exact under-utilisation of every policy (routing + scheduling only)
+    under = {}
+    for pol, name in POLICY_NAMES.items():
+        c = eb.Context(cfg_for(pol, compute=0))
+        c.eb_episode(logits, None, None, None)
+        num, den, den_sep = c.eb_utilization()
+        under[name] = round(1 - num / den, 6)
+        under["separate"] = round(1 - num / den_sep, 6)
+        c.close()
+
+    ctx = eb.Context(cfg_for(policy))
+    hidden = torch.empty_like(h0)
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        hidden.copy_(h0)
+        ctx.eb_episode(logits, hidden, wgu, wdn)
+    assert ctx.eb_sync_status() == eb.EB_OK
+    rows, _ = ctx.eb_trace()
+    n_steps = rows.shape[0]
+    # algorithmic bytes of one episode, per kernel (bf16 = 2 bytes)
+    b = 2
+    R = rows[:, 4].astype(np.int64)
+    P_touch = rows[:, 5].astype(np.int64)
+    alg = {
+        "gemm_gateup": int((P_touch * 2 * wl.F * wl.H * b + R * (wl.H + wl.F) * b).sum()),
+        "gemm_down": int((P_touch * wl.H * wl.F * b + R * (wl.F + wl.H) * b).sum()),
+        "permute": int(sum(bin(int(m)).count("1") for m in rows[:, 0]) * wl.T * wl.H * b
+                       + (R * (wl.H * b + 4)).sum()),
+        "combine": int((R * (wl.H * b + 8)).sum()
+                       + 2 * sum(bin(int(m)).count("1") for m in rows[:, 0]) * wl.T * wl.H * b),
+    }
+    flops_gemm = int((R * 6 * wl.H * wl.F).sum())
+
+    clocks = ClockSampler(local)
+    launches0 = ctx.eb_launch_count()
+    ctx.eb_profile(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for _ in range(args.steps):
+        hidden.copy_(h0)
+        ctx.eb_episode(logits, hidden, wgu, wdn)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = t_start.elapsed_time(t_stop)
+    prof = ctx.eb_profile_read()
+    ctx.eb_profile(False)
+    launches = ctx.eb_launch_count() - launches0
+    assert ctx.eb_sync_status() == eb.EB_OK
+    ms_max = max_over_ranks(ms_total, world)
+    tokens = wl.M * wl.T * wl.L * args.steps * world
+    value = tokens / (ms_max / 1e3)
+
+    # roofline of the dominant kernel
+    kern = max(("gemm_gateup", "gemm_down", "permute", "combine"), key=lambda k: prof[k][0])
+    kms, kl = prof[kern]
+    peak, peak_src = measured_peaks()
+    achieved = alg[kern] * args.steps / (kms / 1e3) / 1e9
+    roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kern),
+            "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
+            else "fallback 6650 GB/s",
+            "alg_bytes_per_launch": int(alg[kern] * args.steps / max(1, kl)),
+            "avg_launch_ms": round(kms / max(1, kl), 5)}
+    gemm_ms = prof["gemm_gateup"][0] + prof["gemm_down"][0]
+    kernels = {k: {"ms_per_episode": round(v[0] / args.steps, 4), "launches": v[1]}
+               for k, v in prof.items()}
+    for k in ("gemm_gateup", "gemm_down", "permute", "combine"):
+        kernels[k]["GBps"] = round(alg[k] * args.steps / (prof[k][0] / 1e3) / 1e9, 1)
+    kernels["gemm_tflops"] = round(flops_gemm * args.steps / (gemm_ms / 1e3) / 1e12, 2)
+
+    # end to end: host buffers, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        lg_host = torch.from_numpy(logits_np).pin_memory()
+        h_host = h0.cpu().pin_memory()
+        out_host = torch.empty_like(h_host).pin_memory()
+        lg_dev = torch.empty_like(logits)
+        barrier(world)
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        k_e2e = max(1, args.steps // 2)
+        for _ in range(k_e2e):
+            lg_dev.copy_(lg_host, non_blocking=True)
+            hidden.copy_(h_host, non_blocking=True)
+            ctx.eb_episode(lg_dev, hidden, wgu, wdn)
+            out_host.copy_(hidden, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        ms_e2e = max_over_ranks(e0.elapsed_time(e1), world)
+        e2e = {"value": round(wl.M * wl.T * wl.L * k_e2e * world / (ms_e2e / 1e3), 1),
+               "unit": UNIT,
+               "h2d_bytes_per_step": int(lg_host.numel() * 4 + h_host.numel() * h_host.element_size()),
+               "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
+               "steps": k_e2e}
+    ctx.close()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, policy, logits_np, h0, wgu, wdn)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded Dirichlet task-profile routing skew; N(0,0.02) weights)",
+            "config": {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
+                                   f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",
+                       "policy": args.policy, "m": wl.m_default, "step": "one Algorithm-1 episode",
+                       "tokens_per_step": wl.M * wl.T * wl.L, "scheduler_steps": n_steps,
+                       "l2": "inputs larger than L2 (58 GB of expert weights streamed per episode)",
+                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+            "e2e": e2e, "gpu_launches": int(launches), "roofline": roof,
+            "cpu_baseline": cpu, "clocks": clk, "under_util": under, "kernels": kernels,
+        }
+        print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ oracle
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def episode_loads(wl, logits_np):
+    """Loads of every (micro-batch, layer) through the oracle (not timed)."""
+    import numpy as np
+    import oracle
+    return np.stack([np.stack([oracle.loads(oracle.histogram(oracle.route(logits_np[j, l], wl.k)[0],
+                                                             wl.E), wl.D) for l in range(wl.L)])
+                     for j in range(wl.M)])
+
+
+def oracle_sample(wl, policy, logits_np, h0_np, fetch_expert, n_tokens: int, route_tokens: int,
+                  full_loads, ffn_layers: int):
+    """Times the oracle on a bounded sample; returns (seconds per token-layer, detail).
+
+    The expert weights the sampled tokens need are fetched before the clock
+    starts (fetch_expert(l, e) -> float32 arrays); the oracle's own float64
+    conversion and arithmetic are timed.
+    """
+    import numpy as np
+    import oracle
+    from oracle import moe as omoe
+
+    t0 = time.perf_counter()
+    for l in range(wl.L):
+        idx, _ = oracle.route(logits_np[0, l, :route_tokens], wl.k)
+        oracle.loads(oracle.histogram(idx, wl.E), wl.D)
+    t_route = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.run_episode(full_loads, policy, wl.m_default)
+    t_sched = time.perf_counter() - t0
+    toks = [(j % wl.M, (j * 131) % wl.T) for j in range(n_tokens)]
+    need = set()
+    for l in range(ffn_layers):
+        rows = np.stack([logits_np[j, l, t] for j, t in toks])
+        need |= {(l, int(e)) for e in oracle.route(rows, wl.k)[0].reshape(-1)}
+        need |= {(l, wl.E + s) for s in range(wl.n_shared)}
+    weights = {key: fetch_expert(*key) for key in sorted(need)}
+    t0 = time.perf_counter()
+    omoe.forward_tokens(np.stack([h0_np[j, t] for j, t in toks]), lambda j, l: logits_np[j, l],
+                        toks, ffn_layers, wl.E, wl.k, wl.n_shared, wl.dtype,
+                        lambda l, e: weights[(l, e)])
+    t_ffn = time.perf_counter() - t0
+    per_tl = (t_route / (route_tokens * wl.L) + t_sched / (wl.M * wl.T * wl.L)
+              + t_ffn / (n_tokens * ffn_layers))
+    detail = (f"oracle on a bounded sample: routing+loads of {route_tokens} tokens x {wl.L} layers "
+              f"({t_route:.2f}s), the full-episode schedule ({t_sched:.2f}s), expert FFN + combine "
+              f"of {n_tokens} token(s) through {ffn_layers} layers ({t_ffn:.2f}s); time per "
+              f"token-layer = sum of the three per-unit costs")
+    return per_tl, detail
+
+
+def make_fetch(wgu, wdn, F):
+    def fetch(l, e):
+        gu = wgu[l, e].float().cpu().numpy()
+        return gu[:F], gu[F:], wdn[l, e].float().cpu().numpy()
+    return fetch
+
+
+def cpu_baseline(wl, policy, logits_np, h0, wgu, wdn, n_tokens=4, ffn_layers=8):
+    import numpy as np
+    h0_np = h0.float().cpu().numpy().astype(np.float64)
+    per_tl, detail = oracle_sample(wl, policy, logits_np, h0_np, make_fetch(wgu, wdn, wl.F),
+                                   n_tokens, 256, episode_loads(wl, logits_np), ffn_layers)
+    return {"value": round(1.0 / per_tl, 2), "unit": UNIT, "cores": _blas_threads(),
+            "kind": "oracle", "sample": detail + " (expert weights copied from the device)"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the CPU oracle as it stands, on the host cores."""
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import synth
+    wl = synth.get(args.workload)
+    policy = {v: k for k, v in POLICY_NAMES.items()}[args.policy]
+    logits_np = synth.logits(wl)
+    h0_np = synth.hidden(wl).astype(np.float64)
+    if wl.dtype == "bf16":
+        h0_np = torch.from_numpy(synth.hidden(wl)).to(torch.bfloat16).double().numpy()
+    def fetch(l, e):  # one expert's weights drawn on the host
+        g = torch.Generator().manual_seed((wl.seed * 7919 + l * 1009 + e) & 0x7FFFFFFF)
+        gu = (torch.randn((2 * wl.F, wl.H), generator=g) * 0.02).to(torch.bfloat16).float().numpy()
+        dn = (torch.randn((wl.H, wl.F), generator=g) * 0.02).to(torch.bfloat16).float().numpy()
+        return gu[:wl.F], gu[wl.F:], dn
+
+    times, detail = [], ""
+    full_loads = episode_loads(wl, logits_np)
+    for i in range(args.warmup + args.steps):
+        per_tl, detail = oracle_sample(wl, policy, logits_np, h0_np, fetch, 1, 64, full_loads, 4)
+        if i >= args.warmup:
+            times.append(per_tl)
+    per_tl = statistics.median(times)
+    value = 1.0 / per_tl
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(per_tl * wl.M * wl.T * wl.L * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": wl.name, "policy": args.policy,
+                                            "m": wl.m_default},
+            "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _blas_threads(),
+                             "kind": "oracle", "sample": detail + " (host-drawn weights)"},
+            "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,450 @@
+// The C ABI of include/eb.h: argument checks, the context and its device
+// state, the workspace layout and the step / episode drivers.
+//
+// [EB] = "EasyBalance: Cross-Layer Load Balancing in Distributed MoE
+// Inference"; Algorithm 1 in its §4.2 is the loop eb_episode runs.
+#include <cuda_runtime.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <vector>
+
+#include "eb_internal.cuh"
+#include "gemm_tc.cuh"
+
+using namespace eb;
+
+struct eb_ctx {
+  eb_config cfg;
+  Dims d;
+  CtxDev dev;
+  void* dev_alloc = nullptr;
+  int device = 0;
+  int num_sms = 148;
+  bool use_tc = false;
+  cudaStream_t last_stream = nullptr;
+  uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
+  cudaEvent_t events[8] = {};
+  // cached TMA maps (rebuilt when a pointer changes)
+  TcMaps maps;
+  const void* map_keys[4] = {nullptr, nullptr, nullptr, nullptr};
+  // kernel launches enqueued since create, and optional per-kernel event timing
+  long long launches = 0;
+  bool prof = false;
+  struct Mark {
+    int kernel;
+    cudaEvent_t a, b;
+  };
+  std::vector<Mark> marks;
+  std::vector<cudaEvent_t> pool;
+};
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kLookahead = 4;  // steps enqueued ahead of the host's completion check
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool use_tc_for(const eb_config& c) {
+  if (c.dtype != EB_DTYPE_BF16) return false;
+  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC;
+}
+
+Dims make_dims(const eb_config& c) {
+  Dims d;
+  d.L = c.L; d.E = c.E; d.k = c.k; d.H = c.H; d.F = c.F; d.D = c.D; d.M = c.M; d.T = c.T;
+  d.n_shared = c.n_shared; d.Etot = c.E + c.n_shared; d.renorm = c.renorm; d.dtype = c.dtype;
+  d.policy = c.policy; d.m = c.m; d.residual = c.residual; d.compute = c.compute;
+  d.NC = (c.T + kChunk - 1) / kChunk;
+  d.kk = c.k + c.n_shared;
+  d.max_steps = c.M * c.L;
+  return d;
+}
+
+size_t elem_size(int dtype) { return dtype == EB_DTYPE_BF16 ? 2 : 4; }
+
+// Offsets of the workspace buffers; returns the total size.
+size_t layout(const eb_config& c, char* base, Work* w) {
+  const Dims d = make_dims(c);
+  const size_t M = c.M, T = c.T;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return base ? (void*)(base + o) : nullptr;
+  };
+  Work x{};
+  x.idx = (int32_t*)take(sizeof(int32_t) * M * T * c.k);
+  x.gate = (float*)take(sizeof(float) * M * T * c.k);
+  x.chunk_hist = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
+  const size_t nseg = M * (size_t)d.Etot;
+  if (c.compute) {
+    x.base = (int32_t*)take(sizeof(int32_t) * M * d.NC * d.Etot);
+    x.pos = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
+    x.seg_rows = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
+    x.seg_wid = (int32_t*)take(sizeof(int32_t) * nseg);
+    x.seg_items1 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
+    x.seg_items2 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
+    x.Rcap = (long long)(M * T * d.kk);
+    const size_t es = elem_size(c.dtype);
+    x.A = take(es * (size_t)x.Rcap * c.H);
+    x.act = take(es * (size_t)x.Rcap * c.F);
+    x.y = take(es * (size_t)x.Rcap * c.H);
+  }
+  if (w) *w = x;
+  return off;
+}
+
+eb_status cuda_status(cudaError_t e) { return e == cudaSuccess ? EB_OK : EB_ERR_CUDA; }
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+cudaEvent_t take_event(eb_ctx* x) {
+  if (!x->pool.empty()) {
+    cudaEvent_t e = x->pool.back();
+    x->pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launches one stage, counting it and (when profiling) bracketing it with
+// events on its stream.
+template <typename F>
+cudaError_t timed(eb_ctx* x, int kernel, int n_launch, cudaStream_t s, F&& launch) {
+  if (!x->prof) {
+    x->launches += n_launch;
+    return launch();
+  }
+  eb_ctx::Mark mk{kernel, take_event(x), take_event(x)};
+  cudaEventRecord(mk.a, s);
+  const cudaError_t e = launch();
+  cudaEventRecord(mk.b, s);
+  x->marks.push_back(mk);
+  x->launches += n_launch;
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* eb_status_string(eb_status s) {
+  switch (s) {
+    case EB_OK: return "ok";
+    case EB_ERR_INVALID_ARG: return "invalid argument";
+    case EB_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case EB_ERR_NONFINITE: return "non-finite router logit";
+    case EB_ERR_CUDA: return "CUDA runtime error";
+    case EB_ERR_TIMEOUT: return "bounded device wait expired";
+    case EB_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+eb_status eb_config_check(const eb_config* c) {
+  if (!c) return EB_ERR_INVALID_ARG;
+  if (c->L < 1 || c->E < 1 || c->k < 1 || c->D < 1 || c->M < 1 || c->T < 1 || c->m < 1)
+    return EB_ERR_INVALID_ARG;
+  if (c->k > c->E || c->m > c->M || c->n_shared < 0) return EB_ERR_INVALID_ARG;
+  if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
+  if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
+  if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_SIMT) return EB_ERR_INVALID_ARG;
+  if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
+      c->k + c->n_shared > EB_MAX_K)
+    return EB_ERR_UNSUPPORTED;
+  if ((long long)c->M * c->L * c->T * c->E > (1ll << 40)) return EB_ERR_UNSUPPORTED;
+  if (c->policy == EB_SCHED_MAXUTIL && maxutil_candidates(c->M, c->m) > kMaxUtilCandidateCap)
+    return EB_ERR_UNSUPPORTED;
+  if (c->compute) {
+    if (c->H < 1 || c->F < 1) return EB_ERR_INVALID_ARG;
+    const int vec = c->dtype == EB_DTYPE_BF16 ? 8 : 4;  // 16-byte rows
+    if (c->H % vec != 0) return EB_ERR_UNSUPPORTED;
+    if ((long long)c->M * c->T * (c->k + c->n_shared) > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
+    if (c->dtype == EB_DTYPE_F32 && c->gemm == EB_GEMM_TC) return EB_ERR_UNSUPPORTED;
+    if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
+      if (c->gemm == EB_GEMM_TC) return EB_ERR_UNSUPPORTED;
+    }
+  }
+  return EB_OK;
+}
+
+eb_status eb_workspace_size(const eb_config* c, size_t* bytes) {
+  const eb_status s = eb_config_check(c);
+  if (s != EB_OK) return s;
+  if (!bytes) return EB_ERR_INVALID_ARG;
+  *bytes = layout(*c, nullptr, nullptr);
+  return EB_OK;
+}
+
+eb_status eb_create(const eb_config* c, eb_ctx** out) {
+  const eb_status s = eb_config_check(c);
+  if (s != EB_OK) return s;
+  if (!out) return EB_ERR_INVALID_ARG;
+  eb_ctx* x = new eb_ctx();
+  x->cfg = *c;
+  x->d = make_dims(*c);
+  // the tensor-core engine needs 128-row feature tiles; otherwise SIMT
+  x->use_tc = use_tc_for(*c) && c->H % 128 == 0 && c->F % 128 == 0;
+  cudaError_t e = cudaGetDevice(&x->device);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&x->num_sms, cudaDevAttrMultiProcessorCount, x->device);
+  const size_t n_state = align_up(sizeof(State));
+  const size_t n_hist = align_up(sizeof(int32_t) * c->M * c->E);
+  const size_t n_w = align_up(sizeof(int32_t) * c->M * c->D);
+  const size_t n_trace = align_up(sizeof(long long) * kTraceCols * x->d.max_steps);
+  const size_t n_tl = align_up(sizeof(int32_t) * c->M * (size_t)x->d.max_steps);
+  char* p = nullptr;
+  if (e == cudaSuccess) e = cudaMalloc(&p, n_state + n_hist + n_w + n_trace + n_tl);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, n_state + n_hist + n_w + n_trace + n_tl);
+  if (e == cudaSuccess) {
+    x->dev_alloc = p;
+    x->dev.st = (State*)p;
+    x->dev.hist = (int32_t*)(p + n_state);
+    x->dev.w = (int32_t*)(p + n_state + n_hist);
+    x->dev.trace = (long long*)(p + n_state + n_hist + n_w);
+    x->dev.trace_layers = (int32_t*)(p + n_state + n_hist + n_w + n_trace);
+    e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
+  }
+  for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
+    e = cudaEventCreateWithFlags(&x->events[i], cudaEventDisableTiming);
+  if (e == cudaSuccess && x->use_tc) e = gemm_tc_prepare();
+  if (e == cudaSuccess) e = launch_reset(x->d, x->dev, nullptr);
+  if (e == cudaSuccess) e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) {
+    eb_destroy(x);
+    return EB_ERR_CUDA;
+  }
+  *out = x;
+  return EB_OK;
+}
+
+eb_status eb_destroy(eb_ctx* x) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (x->last_stream) cudaStreamSynchronize(x->last_stream);
+  for (int i = 0; i < kLookahead; ++i)
+    if (x->events[i]) cudaEventDestroy(x->events[i]);
+  for (auto& mk : x->marks) {
+    cudaEventDestroy(mk.a);
+    cudaEventDestroy(mk.b);
+  }
+  for (auto e : x->pool) cudaEventDestroy(e);
+  if (x->host_pending) cudaFreeHost(x->host_pending);
+  if (x->dev_alloc) cudaFree(x->dev_alloc);
+  delete x;
+  return EB_OK;
+}
+
+eb_status eb_reset(eb_ctx* x, void* stream) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  x->last_stream = s;
+  x->launches += 1;
+  return cuda_status(launch_reset(x->d, x->dev, s));
+}
+
+static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
+                              const void* wdn, void* workspace, size_t ws_bytes,
+                              cudaStream_t s) {
+  const eb_config& c = x->cfg;
+  if (!logits || !workspace) return EB_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & (kAlign - 1)) != 0) return EB_ERR_INVALID_ARG;
+  if (c.compute && (!hidden || !wgu || !wdn)) return EB_ERR_INVALID_ARG;
+  if (c.compute && (!aligned16(hidden) || !aligned16(wgu) || !aligned16(wdn)))
+    return EB_ERR_INVALID_ARG;
+  Work w;
+  const size_t need = layout(c, (char*)workspace, &w);
+  if (ws_bytes < need) return EB_ERR_WORKSPACE;
+  x->last_stream = s;
+  const bool tc = c.compute && x->use_tc;
+  if (tc && (x->map_keys[0] != wgu || x->map_keys[1] != wdn || x->map_keys[2] != workspace)) {
+    if (make_tc_maps(x->d, w, wgu, wdn, &x->maps) != cudaSuccess) return EB_ERR_UNSUPPORTED;
+    x->map_keys[0] = wgu;
+    x->map_keys[1] = wdn;
+    x->map_keys[2] = workspace;
+  }
+  cudaError_t e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, logits, s); });
+  if (e == cudaSuccess)
+    e = timed(x, 1, 1, s, [&] {
+      return launch_schedule_step(x->d, x->dev, w, tc ? kTcRows : kSimtRows,
+                                  tc ? kTcFeat : kSimtFeat, s);
+    });
+  if (c.compute) {
+    if (e == cudaSuccess)
+      e = timed(x, 2, 1, s, [&] { return launch_permute(x->d, x->dev, w, hidden, s); });
+    if (e == cudaSuccess) {
+      if (tc) {
+        e = timed(x, 3, 1, s, [&] { return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 1); });
+        if (e == cudaSuccess)
+          e = timed(x, 4, 1, s, [&] { return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 2); });
+      } else {
+        e = timed(x, 3, 1, s, [&] { return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, 1); });
+        if (e == cudaSuccess)
+          e = timed(x, 4, 1, s, [&] { return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, 2); });
+      }
+    }
+    if (e == cudaSuccess)
+      e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });
+  }
+  return cuda_status(e);
+}
+
+eb_status eb_moe_step(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
+                      const void* wdn, void* workspace, size_t ws_bytes, void* stream,
+                      uint32_t* runset_host) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  const eb_status st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s);
+  if (st != EB_OK) return st;
+  if (runset_host) {
+    cudaError_t e = cudaMemcpyAsync(runset_host, &x->dev.st->runset, sizeof(uint32_t),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return cuda_status(e);
+  }
+  return EB_OK;
+}
+
+eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
+                     const void* wdn, void* workspace, size_t ws_bytes, void* stream,
+                     int* n_steps) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  eb_status st = eb_reset(x, stream);
+  if (st != EB_OK) return st;
+  const int max_steps = x->d.max_steps;
+  for (int i = 0; i < max_steps; ++i) {
+    st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s);
+    if (st != EB_OK) return st;
+    const int slot = i % kLookahead;
+    cudaError_t e = cudaMemcpyAsync(&x->host_pending[slot], &x->dev.st->pending, sizeof(uint32_t),
+                                    cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaEventRecord(x->events[slot], s);
+    if (e != cudaSuccess) return EB_ERR_CUDA;
+    // check the step enqueued kLookahead - 1 steps ago; the GPU keeps working
+    const int chk = i - (kLookahead - 1);
+    if (chk >= 0) {
+      const int cs = chk % kLookahead;
+      if (cudaEventSynchronize(x->events[cs]) != cudaSuccess) return EB_ERR_CUDA;
+      if (x->host_pending[cs] == 0) break;
+    }
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) return EB_ERR_CUDA;
+  int steps = 0;
+  if (cudaMemcpy(&steps, &x->dev.st->n_steps, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EB_ERR_CUDA;
+  if (n_steps) *n_steps = steps;
+  return EB_OK;
+}
+
+eb_status eb_utilization(eb_ctx* x, int64_t* num, int64_t* den, int64_t* den_sep) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (x->last_stream && cudaStreamSynchronize(x->last_stream) != cudaSuccess) return EB_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return EB_ERR_CUDA;
+  State h;
+  if (cudaMemcpy(&h, x->dev.st, sizeof(State), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EB_ERR_CUDA;
+  if (num) *num = h.num;
+  if (den) *den = h.den;
+  if (den_sep) *den_sep = h.den_sep;
+  return EB_OK;
+}
+
+eb_status eb_trace(eb_ctx* x, int64_t* rows, int32_t* layers, int max_steps, int* n_steps) {
+  if (!x || max_steps < 0 || (max_steps > 0 && !rows)) return EB_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return EB_ERR_CUDA;
+  State h;
+  if (cudaMemcpy(&h, x->dev.st, sizeof(State), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EB_ERR_CUDA;
+  const int n = h.n_steps < x->d.max_steps ? h.n_steps : x->d.max_steps;
+  const int cp = n < max_steps ? n : max_steps;
+  if (cp > 0) {
+    if (cudaMemcpy(rows, x->dev.trace, sizeof(long long) * kTraceCols * cp, cudaMemcpyDeviceToHost) !=
+        cudaSuccess)
+      return EB_ERR_CUDA;
+    if (layers && cudaMemcpy(layers, x->dev.trace_layers, sizeof(int32_t) * x->d.M * cp,
+                             cudaMemcpyDeviceToHost) != cudaSuccess)
+      return EB_ERR_CUDA;
+  }
+  if (n_steps) *n_steps = h.n_steps;
+  return EB_OK;
+}
+
+eb_status eb_profile(eb_ctx* x, int enable) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (x->last_stream && cudaStreamSynchronize(x->last_stream) != cudaSuccess) return EB_ERR_CUDA;
+  for (auto& mk : x->marks) {
+    x->pool.push_back(mk.a);
+    x->pool.push_back(mk.b);
+  }
+  x->marks.clear();
+  x->prof = enable != 0;
+  return EB_OK;
+}
+
+eb_status eb_profile_read(eb_ctx* x, double* ms, int64_t* launches) {
+  if (!x || !ms || !launches) return EB_ERR_INVALID_ARG;
+  for (int i = 0; i < EB_PROF_KERNELS; ++i) {
+    ms[i] = 0.0;
+    launches[i] = 0;
+  }
+  for (auto& mk : x->marks) {
+    if (cudaEventSynchronize(mk.b) != cudaSuccess) return EB_ERR_CUDA;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, mk.a, mk.b) != cudaSuccess) return EB_ERR_CUDA;
+    ms[mk.kernel] += t;
+    launches[mk.kernel] += 1;
+    x->pool.push_back(mk.a);
+    x->pool.push_back(mk.b);
+  }
+  x->marks.clear();
+  return EB_OK;
+}
+
+eb_status eb_launch_count(eb_ctx* x, int64_t* n) {
+  if (!x || !n) return EB_ERR_INVALID_ARG;
+  *n = x->launches;
+  return EB_OK;
+}
+
+eb_status eb_sync_status(eb_ctx* x) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return EB_ERR_CUDA;
+  int status = 0;
+  if (cudaMemcpy(&status, &x->dev.st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EB_ERR_CUDA;
+  return status;
+}
+
+eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t* idx, float* gate,
+                   int32_t* hist, int32_t* status_dev, void* stream) {
+  if (n < 0 || E < 1 || k < 1 || k > E) return EB_ERR_INVALID_ARG;
+  if (E > EB_MAX_ETOT || k > EB_MAX_K) return EB_ERR_UNSUPPORTED;
+  if (!hist || (n > 0 && (!logits || !idx || !gate))) return EB_ERR_INVALID_ARG;
+  return cuda_status(launch_route_rows(logits, n, E, k, renorm, idx, gate, hist, status_dev,
+                                       (cudaStream_t)stream));
+}
+
+eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream) {
+  if (M < 0 || E < 1 || D < 1 || E % D != 0) return EB_ERR_INVALID_ARG;
+  if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
+  return cuda_status(launch_loads(hist, M, E, D, w, (cudaStream_t)stream));
+}
+
+eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int m, int policy,
+                      uint32_t* runset_mask, int64_t* step_stats, void* stream) {
+  if (M < 1 || D < 1 || m < 1 || m > M || !w || !runset_mask) return EB_ERR_INVALID_ARG;
+  if (policy < EB_SCHED_CUMUTIL || policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
+  if (M > EB_MAX_M || D > EB_MAX_D) return EB_ERR_UNSUPPORTED;
+  if (M < 32 && (pending_mask >> M) != 0) return EB_ERR_INVALID_ARG;
+  if (policy == EB_SCHED_MAXUTIL && maxutil_candidates(__builtin_popcount(pending_mask), m) >
+                                        kMaxUtilCandidateCap)
+    return EB_ERR_UNSUPPORTED;
+  return cuda_status(launch_schedule_once(w, pending_mask, M, D, m, policy, runset_mask,
+                                          (long long*)step_stats, (cudaStream_t)stream));
+}
+
+}  // extern "C"

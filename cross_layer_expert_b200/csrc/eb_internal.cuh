@@ -1,0 +1,109 @@
+// Internal declarations shared by the CUDA sources of the cross-layer MoE
+// step library.  Citations: [EB] = "EasyBalance: Cross-Layer Load Balancing in
+// Distributed MoE Inference" (Wu, Gao, Li, Wu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/eb.h"
+
+namespace eb {
+
+// Tokens handled by one routing / permute / combine CTA.  The per-chunk
+// expert counts written by routing give every (micro-batch, chunk, expert) a
+// fixed base row, so the permutation is deterministic.
+constexpr int kChunk = 64;
+
+// Sizes of GEMM work items: RN token rows per item and FM output features per
+// item (the tcgen05 tile is 128 x 128; the SIMT tile 64 x 64).
+constexpr int kTcRows = 128;
+constexpr int kTcFeat = 128;
+constexpr int kSimtRows = 64;
+constexpr int kSimtFeat = 64;
+
+// Columns of a trace row: RunSet mask, sum_d W_d, max_d W_d, sum_j max_d w_j,
+// permuted rows R, non-empty (layer, expert) segments.
+constexpr int kTraceCols = 6;
+
+// Exact per-step and per-episode accounting lives in this device struct.
+struct State {
+  int32_t layer[EB_MAX_M];       // l_j: next layer of micro-batch j
+  int32_t step_layer[EB_MAX_M];  // layer micro-batch j runs at in this step, -1 if not run
+  int32_t run_list[EB_MAX_M];    // RunSet members, ascending
+  int32_t group_of[EB_MAX_M];    // segment group (one per distinct layer) of each micro-batch
+  int32_t group_layer[EB_MAX_M]; // layer of each group, ascending
+  uint32_t pending;              // S: micro-batches with l_j < L
+  uint32_t need_route;           // micro-batches whose logits at l_j must be routed
+  uint32_t runset;               // RunSet of the current step
+  int32_t n_run;
+  int32_t n_groups;
+  int32_t n_steps;   // steps with a non-empty RunSet since reset
+  int32_t status;    // first device-side error (EB_OK if none)
+  int32_t nseg;      // segments of this step: n_groups * (E + n_shared)
+  int32_t items1;    // work items of the gate/up GEMM
+  int32_t items2;    // work items of the down GEMM
+  int32_t rows;      // permuted rows of this step
+  int32_t pad0;
+  long long num, den, den_sep;  // utilisation accumulators (Eq. (3))
+};
+
+// Plain-old-data copy of the configuration used by kernels.
+struct Dims {
+  int L, E, k, H, F, D, M, T, n_shared, Etot, renorm, dtype, policy, m, residual, compute;
+  int NC;     // routing chunks per micro-batch: ceil(T / kChunk)
+  int kk;     // slots per token including shared experts: k + n_shared
+  int max_steps;
+};
+
+// Pointers into the caller's workspace.
+struct Work {
+  int32_t* idx;        // [M][T][k]
+  float* gate;         // [M][T][k]
+  int32_t* chunk_hist; // [M][NC][E]
+  int32_t* base;       // [M][NC][Etot]: first row of (j, chunk, expert)
+  int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
+  int32_t* seg_rows;   // [M*Etot + 1]
+  int32_t* seg_wid;    // [M*Etot]: layer * Etot + expert
+  int32_t* seg_items1; // [M*Etot + 1]
+  int32_t* seg_items2; // [M*Etot + 1]
+  void* A;             // [Rcap][H] permuted tokens
+  void* act;           // [Rcap][F] SwiGLU activations
+  void* y;             // [Rcap][H] expert outputs
+  long long Rcap;
+};
+
+// Device state owned by a context.
+struct CtxDev {
+  State* st;
+  int32_t* hist;        // [M][E]: counts of micro-batch j at layer l_j
+  int32_t* w;           // [M][D]
+  long long* trace;     // [max_steps][kTraceCols]
+  int32_t* trace_layers;  // [max_steps][M]
+};
+
+// ---- launchers (all asynchronous on `s`) ----
+cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
+                              cudaStream_t s);
+cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
+                              float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
+cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn, int fm,
+                                 cudaStream_t s);
+cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
+                                 int policy, uint32_t* runset, long long* stats, cudaStream_t s);
+cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s);
+cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
+cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
+                           cudaStream_t s);
+cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
+                           cudaStream_t s);
+// GEMM `which` (1: gate/up + SwiGLU, 2: down) on the CUDA cores.
+cudaError_t launch_gemm_simt(const Dims& d, const CtxDev& c, const Work& w, const void* w_gateup,
+                             const void* w_down, cudaStream_t s, int which);
+
+// MaxUtil enumerates complements of size <= |S| - m; this caps the candidate
+// count a single step may need (sum_{c <= M-m} C(M, c)).
+constexpr unsigned long long kMaxUtilCandidateCap = 1ull << 25;
+unsigned long long maxutil_candidates(int n, int m);
+
+}  // namespace eb

@@ -1,0 +1,480 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a):
+// one persistent launch per GEMM over every (layer, expert) segment of the
+// step, so experts of different layers share a launch.
+//
+// Expert FFN of [EB] Eq. (1), read as SwiGLU:
+//   GEMM 1:  act = bf16( silu(A W_gate^T) * (A W_up^T) )   (fp32 accumulation)
+//   GEMM 2:  y   = bf16( act W_down^T )
+//
+// Layout ("swap AB"): the 128 weight rows of an output-feature block are the
+// MMA's M side and the segment's token rows its N side (N = the chunk's row
+// count rounded up to 16, at most 128), so a segment of a few dozen rows costs
+// a narrow MMA instead of a half-empty 128-row tile.  D[f, r] accumulates in
+// TMEM; lane f of the accumulator belongs to epilogue thread f.
+//
+// Work item = (segment, 128-feature block, 128-row chunk), chunks innermost,
+// so CTAs that run side by side read the same weight tile (L2 reuse).  Roles
+// per CTA (192 threads): warp 0 issues TMA loads into a ring of shared-memory
+// stages, warp 1 allocates TMEM and one thread issues the MMAs, warps 2-5 drain
+// the accumulator (double buffered, so the drain overlaps the next item).
+// Operands are K-major with the 128-byte swizzle in both TMA and the MMA
+// descriptors.  Every mbarrier wait is bounded: on expiry the CTA records
+// EB_ERR_TIMEOUT in the step's status word, waits (bounded) for its own copies
+// and MMAs in flight, frees its TMEM and returns.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "eb_internal.cuh"
+#include "gemm_tc.cuh"
+
+namespace eb {
+namespace {
+
+constexpr int kBM = 128;        // weight rows (features) per MMA tile
+constexpr int kBN = kTcRows;    // token rows per item (max MMA N)
+constexpr int kBK = 64;         // K elements per stage: 128 bytes of bf16 = one swizzle row
+constexpr int kTileBytes = kBM * kBK * 2;  // 16 KiB
+constexpr int kXBytes = kBN * kBK * 2;     // 16 KiB
+constexpr int kThreads = 192;
+constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase of parity `parity` to complete.  Returns false
+// (and raises the CTA's abort flag) if it does not within the limit, or if
+// another role of the CTA has aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          int* status) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        atomicCAS(status, EB_OK, EB_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// K-major operand, 128-byte swizzle: rows of 128 B, 8-row atoms 1024 B apart.
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);  // start address (16 B units)
+  d |= (uint64_t)1 << 16;                     // leading byte offset (unused when swizzled)
+  d |= (uint64_t)(1024 >> 4) << 32;           // stride byte offset: next 8-row atom
+  d |= (uint64_t)1 << 46;                     // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                     // SWIZZLE_128B
+  return d;
+}
+
+// kind::f16 instruction descriptor: D fp32, A and B bf16, both K-major.
+__device__ __forceinline__ uint32_t idesc_bf16(int M, int N) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+         ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit accumulator -> 32 registers per thread.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+      "%28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ int find_segment(const int32_t* items, int nseg, int item) {
+  int lo = 0, hi = nseg;  // items[lo] <= item < items[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (items[mid] <= item) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+struct Item {
+  int r0;     // first token row of the chunk
+  int n;      // token rows in the chunk (1..128)
+  int f0;     // first output feature of the block
+  int wrow;   // first weight row (gate rows for GEMM 1)
+};
+
+template <bool GATEUP>
+__device__ __forceinline__ Item decode(const Dims& d, const int32_t* seg_rows,
+                                       const int32_t* seg_wid, const int32_t* seg_items,
+                                       int nseg, int item) {
+  const int s = find_segment(seg_items, nseg, item);
+  const int local = item - seg_items[s];
+  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
+  const int nch = (cnt + kBN - 1) / kBN;
+  const int chunk = local % nch, mb = local / nch;
+  Item it;
+  it.r0 = rb + chunk * kBN;
+  it.n = min(kBN, cnt - chunk * kBN);
+  it.f0 = mb * kBM;
+  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
+  return it;
+}
+
+template <bool GATEUP>
+struct Cfg {
+  static constexpr int kStages = GATEUP ? 4 : 6;
+  static constexpr int kStageBytes = (GATEUP ? 2 : 1) * kTileBytes + kXBytes;
+  static constexpr int kAccCols = (GATEUP ? 2 : 1) * kBN;  // TMEM columns per accumulator
+  static constexpr int kTmemCols = 2 * kAccCols;            // double buffered: 512 / 256
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* barriers */ + 1024 /* align */;
+};
+
+// GATEUP: map_w = w_gateup [L*Etot*2F, H], map_x = A [Rcap, H], out = act [Rcap, F]
+// DOWN:   map_w = w_down   [L*Etot*H, F],  map_x = act [Rcap, F], out = y [Rcap, H]
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+              Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
+              const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
+              __nv_bfloat16* __restrict__ out) {
+  using C = Cfg<GATEUP>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;                      // [kStages]
+  uint64_t* empty = bars + C::kStages;        // [kStages]
+  uint64_t* tfull = bars + 2 * C::kStages;    // [2]
+  uint64_t* tempty = tfull + 2;               // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nseg = st->nseg;
+  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
+  if (total == 0) return;  // uniform across the CTA: nothing to do this step
+  const int K = GATEUP ? d.H : d.F;
+  const int nk = K / kBK;
+  const int NOUT = GATEUP ? d.F : d.H;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 128);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;  // per stage: armed at least once / parity of last arm
+      bool ok = true;
+      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const Item it = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = stage_base + stage * C::kStageBytes;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, C::kStageBytes);
+          tma_load_2d(smem_u32(sb), &map_w, kb * kBK, it.wrow, fb);
+          if (GATEUP) tma_load_2d(smem_u32(sb + kTileBytes), &map_w, kb * kBK, it.wrow + d.F, fb);
+          tma_load_2d(smem_u32(sb + (GATEUP ? 2 : 1) * kTileBytes), &map_x, kb * kBK, it.r0, fb);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {  // let our own copies land before the CTA's shared memory goes away
+        for (int s = 0; s < C::kStages; ++s)
+          if ((armed >> s) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s]), (armed_par >> s) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint32_t last_bar = 0, last_par = 0;
+      bool ok = true, issued = false;
+      for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
+        const Item it = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+        const int N = ((it.n + 15) / 16) * 16;
+        const uint32_t idesc = idesc_bf16(kBM, N);
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_gate = tmem + acc * C::kAccCols;
+        const uint32_t d_up = d_gate + kBN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(stage_base + stage * C::kStageBytes);
+          const uint32_t sx = sb + (GATEUP ? 2 : 1) * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks) {
+            const uint32_t koff = ks * 32;  // 16 bf16 = 32 bytes along K
+            const uint32_t acc_flag = (kb | ks) != 0;
+            mma_bf16(d_gate, sdesc(sb + koff), sdesc(sx + koff), idesc, acc_flag);
+            if (GATEUP) mma_bf16(d_up, sdesc(sb + kTileBytes + koff), sdesc(sx + koff), idesc, acc_flag);
+          }
+          mma_commit(smem_u32(&empty[stage]));
+          last_bar = smem_u32(&empty[stage]);
+          last_par = phase;
+          issued = true;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tfull[acc]));
+        last_bar = smem_u32(&tfull[acc]);
+        last_par = acc_phase;
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued) {  // MMAs still reading shared memory / writing TMEM
+        const unsigned long long t0 = global_ns();
+        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;            // TMEM lane quarter this warp may read
+    const int frow = q * 32 + lane;    // feature row of this thread within the tile
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+      const Item it = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      __nv_bfloat16* orow = out + (size_t)it.r0 * NOUT + it.f0 + frow;
+      for (int cb = 0; cb < it.n; cb += 32) {
+        float g[32];
+        tmem_ld32(tbase + cb, g);
+        if (GATEUP) {
+          float u[32];
+          tmem_ld32(tbase + kBN + cb, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (cb + i < it.n) {
+              const float a = g[i] / (1.f + expf(-g[i])) * u[i];
+              orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(a);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (cb + i < it.n) orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(g[i]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty[acc]));
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::kTmemCols));
+  }
+}
+
+}  // namespace
+
+int gemm_tc_smem_bytes(bool gateup) {
+  return gateup ? Cfg<true>::kSmemBytes : Cfg<false>::kSmemBytes;
+}
+
+cudaError_t gemm_tc_prepare() {
+  cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       Cfg<true>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  return cudaFuncSetAttribute(k_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              Cfg<false>::kSmemBytes);
+}
+
+cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                           int grid, cudaStream_t s, int which) {
+  if (which == 1)
+    k_gemm_tc<true><<<grid, kThreads, Cfg<true>::kSmemBytes, s>>>(
+        maps.w_gateup, maps.A, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1,
+        static_cast<__nv_bfloat16*>(w.act));
+  else
+    k_gemm_tc<false><<<grid, kThreads, Cfg<false>::kSmemBytes, s>>>(
+        maps.w_down, maps.act, d, c.st, w.seg_rows, w.seg_wid, w.seg_items2,
+        static_cast<__nv_bfloat16*>(w.y));
+  return cudaGetLastError();
+}
+
+}  // namespace eb
+
+namespace eb {
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x 128 rows.
+cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, int cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
+                         TcMaps* maps) {
+  const unsigned long long experts = (unsigned long long)d.L * d.Etot;
+  cudaError_t e = encode(&maps->w_gateup, w_gateup, experts * 2 * d.F, d.H);
+  if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F);
+  if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H);
+  if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F);
+  return e;
+}
+
+}  // namespace eb

@@ -1,0 +1,31 @@
+// Host-side interface of the tcgen05 grouped expert GEMMs.
+#pragma once
+
+#include <cuda.h>
+
+#include "eb_internal.cuh"
+
+namespace eb {
+
+// TMA descriptors of the four bf16 operands (128-byte swizzle, 64-element K
+// boxes of 128 rows).
+struct TcMaps {
+  CUtensorMap w_gateup;  // [L*Etot*2F rows, H cols]
+  CUtensorMap w_down;    // [L*Etot*H rows, F cols]
+  CUtensorMap A;         // [Rcap rows, H cols]
+  CUtensorMap act;       // [Rcap rows, F cols]
+};
+
+// Encodes the maps for these buffers; returns cudaErrorInvalidValue if the
+// driver rejects a map (alignment, strides).
+cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
+                         TcMaps* maps);
+// Opts the kernels into their dynamic shared memory (once per device).
+cudaError_t gemm_tc_prepare();
+int gemm_tc_smem_bytes(bool gateup);
+// GEMM `which` (1: gate/up + SwiGLU, 2: down) of a step; grid = persistent
+// CTAs (one per SM).
+cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                           int grid, cudaStream_t s, int which);
+
+}  // namespace eb

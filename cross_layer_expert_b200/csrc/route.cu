@@ -1,0 +1,195 @@
+// Routing: softmax top-k with renormalised gates and per-expert token counts.
+//
+// [EB] §2.1: W_l, I_l = topk(G(h'_l)) -- each token picks its top-k experts and
+// weighs them.  The counts T_e per expert are what a rank's load is built
+// from ([SysLB] §1: L_r = sum_{e in E_r} T_e).
+//
+// One warp routes one token: the E logits are read coalesced (lane i holds
+// experts i, i+32, ...), the k winners come out of k rounds of a warp-wide
+// argmax under the order (logit descending, expert index ascending), and the
+// gates exp(l_s - l_max) / sum_{s'} exp(l_s' - l_max) are formed from the
+// winners alone when renormalised (the full softmax denominator cancels).
+// Counts go to shared-memory atomics (integers, so the result is exact and
+// order-free) and are written once per (micro-batch, chunk): no global
+// atomics and no zeroing pass in the step path.
+#include <math.h>
+
+#include "eb_internal.cuh"
+
+namespace eb {
+namespace {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+__device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
+  return v1 > v2 || (v1 == v2 && e1 < e2);
+}
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(kFull, x, off);
+  return x;
+}
+
+// Routes one token row with the calling warp.  Lane s < k returns slot s.
+template <int VPL>
+__device__ __forceinline__ void route_row(const float* __restrict__ row, int E, int k, int renorm,
+                                          int lane, int& out_e, float& out_g, bool& nonfinite) {
+  float v[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = i * 32 + lane;
+    float x = -INFINITY;
+    if (e < E) {
+      x = __ldg(row + e);
+      if (!isfinite(x)) {
+        nonfinite = true;
+        x = -INFINITY;  // selection stays among real experts; the call reports the error
+      }
+    }
+    v[i] = x;
+  }
+  unsigned taken = 0;
+  float top_v = -INFINITY, vmax = -INFINITY;
+  int top_e = 0;
+  for (int s = 0; s < k; ++s) {
+    float bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, be)) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+      const float ov = __shfl_xor_sync(kFull, bv, off);
+      const int oe = __shfl_xor_sync(kFull, be, off);
+      if (better(ov, oe, bv, be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    if (lane == s) {
+      top_v = bv;
+      top_e = be;
+    }
+    if (s == 0) vmax = bv;
+  }
+  const float ex = (lane < k) ? expf(top_v - vmax) : 0.f;
+  float denom;
+  if (renorm) {
+    denom = warp_sum(ex);
+  } else {
+    float part = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (i * 32 + lane < E) part += expf(v[i] - vmax);
+    denom = warp_sum(part);
+  }
+  out_e = top_e;
+  out_g = ex / denom;
+}
+
+template <int VPL>
+__device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
+                            int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
+                            int* hist_s, bool& nonfinite) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int t = t0 + warp; t < t1; t += nwarps) {
+    int e;
+    float g;
+    route_row<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, g, nonfinite);
+    if (lane < k) {
+      idx[(size_t)t * k + lane] = e;
+      gate[(size_t)t * k + lane] = g;
+      atomicAdd(&hist_s[e], 1);
+    }
+  }
+}
+
+// Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
+// is in need_route; its counts land in chunk_hist[j][c][:].
+template <int VPL>
+__global__ void __launch_bounds__(256) k_route_step(Dims d, State* __restrict__ st,
+                                                     const float* __restrict__ logits,
+                                                     int32_t* __restrict__ idx,
+                                                     float* __restrict__ gate,
+                                                     int32_t* __restrict__ chunk_hist) {
+  const int c = blockIdx.x, j = blockIdx.y;
+  if (!((st->need_route >> j) & 1u)) return;
+  const int l = st->layer[j];
+  __shared__ int hist_s[EB_MAX_ETOT];
+  __shared__ int bad;
+  for (int e = threadIdx.x; e < d.E; e += blockDim.x) hist_s[e] = 0;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const float* blk = logits + ((size_t)j * d.L + l) * (size_t)d.T * d.E;
+  const int t0 = c * kChunk, t1 = min(d.T, t0 + kChunk);
+  bool nonfinite = false;
+  route_chunk<VPL>(blk, t0, t1, d.E, d.k, d.renorm, idx + (size_t)j * d.T * d.k,
+                   gate + (size_t)j * d.T * d.k, hist_s, nonfinite);
+  if (nonfinite) bad = 1;
+  __syncthreads();
+  int32_t* out = chunk_hist + ((size_t)j * d.NC + c) * d.E;
+  for (int e = threadIdx.x; e < d.E; e += blockDim.x) out[e] = hist_s[e];
+  if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
+}
+
+// Stand-alone path: rows [c*kChunk, ...) of an [n, E] block; counts summed
+// into hist[E] with one global atomic per (CTA, expert) with a non-zero count.
+template <int VPL>
+__global__ void __launch_bounds__(256) k_route_rows(const float* __restrict__ logits, int n, int E,
+                                                     int k, int renorm, int32_t* __restrict__ idx,
+                                                     float* __restrict__ gate,
+                                                     int32_t* __restrict__ hist,
+                                                     int32_t* __restrict__ status) {
+  __shared__ int hist_s[EB_MAX_ETOT];
+  __shared__ int bad;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist_s[e] = 0;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * kChunk, t1 = min(n, t0 + kChunk);
+  bool nonfinite = false;
+  route_chunk<VPL>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
+  if (nonfinite) bad = 1;
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist_s[e]) atomicAdd(&hist[e], hist_s[e]);
+  if (threadIdx.x == 0 && bad && status) atomicExch(status, EB_ERR_NONFINITE);
+}
+
+int vpl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
+
+}  // namespace
+
+cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
+                              cudaStream_t s) {
+  dim3 grid(d.NC, d.M);
+  switch (vpl_for(d.E)) {
+    case 1: k_route_step<1><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 2: k_route_step<2><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 4: k_route_step<4><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    default: k_route_step<8><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
+                              float* gate, int32_t* hist, int32_t* status, cudaStream_t s) {
+  cudaError_t err = cudaMemsetAsync(hist, 0, sizeof(int32_t) * (size_t)E, s);
+  if (err != cudaSuccess || n == 0) return err;
+  dim3 grid((n + kChunk - 1) / kChunk);
+  switch (vpl_for(E)) {
+    case 1: k_route_rows<1><<<grid, 256, 0, s>>>(logits, n, E, k, renorm, idx, gate, hist, status); break;
+    case 2: k_route_rows<2><<<grid, 256, 0, s>>>(logits, n, E, k, renorm, idx, gate, hist, status); break;
+    case 4: k_route_rows<4><<<grid, 256, 0, s>>>(logits, n, E, k, renorm, idx, gate, hist, status); break;
+    default: k_route_rows<8><<<grid, 256, 0, s>>>(logits, n, E, k, renorm, idx, gate, hist, status); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace eb

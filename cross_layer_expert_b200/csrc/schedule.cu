@@ -1,0 +1,571 @@
+// Loads, the RunSet scheduler, exact utilisation accounting and the segment
+// plan of one step -- one CTA, everything in shared memory.
+//
+// [EB] §2.3 Eq. (2) w_hat = max_d w_d, Eq. (3) u = sum sum w / (sum w_hat D);
+// [EB] §4.2 Algorithm 1 and the minimum RunSet size m; [EB] §5.2 CumUtil
+// (add j+1 iff U(S u {w_{j+1}}) > U(S)), MaxUtil (best U over the candidate
+// subsets) and DiffPeak (add j+1 iff its peak device is new).
+//
+// U(S) = sum_d W_d / (D max_d W_d) is compared exactly:
+//   U(A) > U(B)  <=>  sum_A * max_B > sum_B * max_A   (int64; D cancels),
+// a set without work counts as U = 0.  MaxUtil ties go to the larger set,
+// then to the smaller bitmask.  CumUtil and DiffPeak pad a short RunSet to m
+// with the lowest skipped indices.
+//
+// MaxUtil enumerates the complements C of the pending set P with
+// |C| <= |P| - m (so every candidate S = P \ C has |S| >= m): the threads
+// split the candidate ranks, unrank a first complement in colexicographic
+// order and walk on with Gosper's next-combination step.
+#include "eb_internal.cuh"
+
+namespace eb {
+namespace {
+
+constexpr int kThreads = 1024;
+
+struct Cand {
+  long long sum, mx;
+  int size;
+  uint32_t mask;
+};
+
+__device__ __forceinline__ bool cand_better(const Cand& a, const Cand& b) {
+  if (a.mx == 0 || b.mx == 0) {
+    if (a.mx != b.mx) return a.mx != 0;  // a set with work beats one without
+  } else {
+    const long long l = a.sum * b.mx, r = b.sum * a.mx;
+    if (l != r) return l > r;
+  }
+  if (a.size != b.size) return a.size > b.size;
+  return a.mask < b.mask;
+}
+
+// Shared-memory workspace of the scheduler.
+struct SchedSmem {
+  int w[EB_MAX_M][EB_MAX_D];  // loads of pending micro-batches, by position in P
+  long long wsum[EB_MAX_M];
+  long long tot[EB_MAX_D];
+  long long totsum;
+  int P[EB_MAX_M];            // pending micro-batch ids, ascending
+  int n;
+  uint32_t binom[33][33];
+  Cand red[kThreads / 32];
+  uint32_t result;
+};
+
+__device__ __forceinline__ uint64_t gosper_next(uint64_t v) {
+  const uint64_t t = v | (v - 1);
+  return (t + 1) | (((~t & (t + 1)) - 1) >> __ffsll((long long)v));
+}
+
+// The r-th c-subset of {0..n-1} in colexicographic order.
+__device__ uint32_t unrank_colex(uint32_t r, int c, const uint32_t (*B)[33]) {
+  uint32_t mask = 0;
+  for (int i = c; i >= 1; --i) {
+    int x = i - 1;
+    while (B[x + 1][i] <= r) ++x;
+    r -= B[x][i];
+    mask |= 1u << x;
+  }
+  return mask;
+}
+
+__device__ Cand eval_complement(const SchedSmem& sm, int D, uint32_t cm) {
+  long long mx = 0;
+  long long sum = sm.totsum;
+  for (uint32_t b = cm; b; b &= b - 1) sum -= sm.wsum[__ffs(b) - 1];
+  for (int dd = 0; dd < D; ++dd) {
+    long long Wd = sm.tot[dd];
+    for (uint32_t b = cm; b; b &= b - 1) Wd -= sm.w[__ffs(b) - 1][dd];
+    mx = Wd > mx ? Wd : mx;
+  }
+  uint32_t mask = 0;
+  for (int i = 0; i < sm.n; ++i)
+    if (!((cm >> i) & 1u)) mask |= 1u << sm.P[i];
+  return Cand{sum, mx, sm.n - __popc(cm), mask};
+}
+
+__device__ Cand shfl_cand(const Cand& c, int off) {
+  Cand o;
+  o.sum = __shfl_xor_sync(0xffffffffu, c.sum, off);
+  o.mx = __shfl_xor_sync(0xffffffffu, c.mx, off);
+  o.size = __shfl_xor_sync(0xffffffffu, c.size, off);
+  o.mask = __shfl_xor_sync(0xffffffffu, c.mask, off);
+  return o;
+}
+
+// All threads of the block: MaxUtil over complements of size <= n - m.
+__device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
+  const int n = sm.n, cmax = n - m;
+  unsigned long long N = 0;
+  for (int c = 0; c <= cmax; ++c) N += sm.binom[n][c];
+  const unsigned long long per = (N + blockDim.x - 1) / blockDim.x;
+  unsigned long long r = per * threadIdx.x;
+  const unsigned long long r_end = r + per < N ? r + per : N;
+  Cand best{0, 0, -1, 0xffffffffu};
+  bool have = false;
+  if (r < r_end) {
+    int c = 0;
+    unsigned long long q = r;
+    while (q >= sm.binom[n][c]) {
+      q -= sm.binom[n][c];
+      ++c;
+    }
+    uint64_t cm = c == 0 ? 0 : unrank_colex((uint32_t)q, c, sm.binom);
+    for (; r < r_end; ++r) {
+      const Cand cd = eval_complement(sm, D, (uint32_t)cm);
+      if (!have || cand_better(cd, best)) {
+        best = cd;
+        have = true;
+      }
+      if (++q == sm.binom[n][c]) {
+        ++c;
+        q = 0;
+        cm = (c >= 64) ? 0 : ((1ull << c) - 1);
+      } else {
+        cm = gosper_next(cm);
+      }
+    }
+  }
+  // block reduction; threads without candidates carry size = -1 (never wins)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int off = 16; off; off >>= 1) {
+    const Cand o = shfl_cand(best, off);
+    if (o.size >= 0 && (best.size < 0 || cand_better(o, best))) best = o;
+  }
+  if (lane == 0) sm.red[warp] = best;
+  __syncthreads();
+  if (warp == 0) {
+    best = lane < (int)(blockDim.x >> 5) ? sm.red[lane] : Cand{0, 0, -1, 0xffffffffu};
+    for (int off = 16; off; off >>= 1) {
+      const Cand o = shfl_cand(best, off);
+      if (o.size >= 0 && (best.size < 0 || cand_better(o, best))) best = o;
+    }
+    if (lane == 0) sm.result = best.mask;
+  }
+  __syncthreads();
+  return sm.result;
+}
+
+// Thread 0 only: CumUtil (policy 0) or DiffPeak (policy 3), padded to m.
+__device__ uint32_t scan_policy(const SchedSmem& sm, int D, int m, int policy) {
+  const int n = sm.n;
+  long long W[EB_MAX_D];
+  for (int dd = 0; dd < D; ++dd) W[dd] = sm.w[0][dd];
+  long long sum = sm.wsum[0], mx = 0;
+  for (int dd = 0; dd < D; ++dd) mx = W[dd] > mx ? W[dd] : mx;
+  uint32_t chosen = 1u;  // positions in P
+  unsigned long long peaks = 0;
+  auto peak_of = [&](int i) {
+    int best = 0;
+    for (int dd = 1; dd < D; ++dd)
+      if (sm.w[i][dd] > sm.w[i][best]) best = dd;
+    return best;
+  };
+  if (policy == EB_SCHED_DIFFPEAK) peaks = 1ull << peak_of(0);
+  for (int i = 1; i < n; ++i) {
+    if (policy == EB_SCHED_DIFFPEAK) {
+      const int p = peak_of(i);
+      if (!((peaks >> p) & 1ull)) {
+        peaks |= 1ull << p;
+        chosen |= 1u << i;
+      }
+      continue;
+    }
+    long long nmx = 0;
+    for (int dd = 0; dd < D; ++dd) {
+      const long long v = W[dd] + sm.w[i][dd];
+      nmx = v > nmx ? v : nmx;
+    }
+    const long long nsum = sum + sm.wsum[i];
+    // U(S u {i}) > U(S) <=> nsum * mx > sum * nmx; a set without work has U = 0
+    bool gain;
+    if (nmx == 0 || mx == 0) gain = (nmx != 0 && mx == 0);
+    else gain = nsum * mx > sum * nmx;
+    if (gain) {
+      chosen |= 1u << i;
+      for (int dd = 0; dd < D; ++dd) W[dd] += sm.w[i][dd];
+      sum = nsum;
+      mx = nmx;
+    }
+  }
+  for (int i = 0; i < n && __popc(chosen) < m; ++i) chosen |= 1u << i;
+  uint32_t mask = 0;
+  for (int i = 0; i < n; ++i)
+    if ((chosen >> i) & 1u) mask |= 1u << sm.P[i];
+  return mask;
+}
+
+// All threads: loads w[j][:] of the pending set must be in sm.w (by position);
+// returns the RunSet mask (over micro-batch ids).
+__device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending) {
+  if (threadIdx.x == 0) {
+    // binomial table for the MaxUtil enumeration
+    for (int a = 0; a <= 32; ++a)
+      for (int b = 0; b <= 32; ++b)
+        sm.binom[a][b] = (b == 0) ? 1u : (a == 0 ? 0u : 0u);
+    for (int a = 1; a <= 32; ++a)
+      for (int b = 1; b <= 32; ++b) sm.binom[a][b] = sm.binom[a - 1][b - 1] + sm.binom[a - 1][b];
+    long long ts = 0;
+    for (int dd = 0; dd < D; ++dd) {
+      long long t = 0;
+      for (int i = 0; i < sm.n; ++i) t += sm.w[i][dd];
+      sm.tot[dd] = t;
+      ts += t;
+    }
+    sm.totsum = ts;
+    for (int i = 0; i < sm.n; ++i) {
+      long long s = 0;
+      for (int dd = 0; dd < D; ++dd) s += sm.w[i][dd];
+      sm.wsum[i] = s;
+    }
+  }
+  __syncthreads();
+  if (policy == EB_SCHED_LOCKSTEP || sm.n <= m) return pending;
+  if (policy == EB_SCHED_MAXUTIL) return maxutil_block(sm, D, m);
+  if (threadIdx.x == 0) sm.result = scan_policy(sm, D, m, policy);
+  __syncthreads();
+  return sm.result;
+}
+
+// ---------------------------------------------------------------- block scan
+// Exclusive scan of v[0..n) in place (all threads); returns the total.
+__device__ int block_exclusive_scan(int* v, int n, int* tmp /* [kThreads] */) {
+  const int per = (n + blockDim.x - 1) / blockDim.x;
+  const int b = threadIdx.x * per, e = min(n, b + per);
+  int local = 0;
+  for (int i = b; i < e; ++i) local += v[i];
+  tmp[threadIdx.x] = local;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < (int)blockDim.x; ++i) {
+      const int t = tmp[i];
+      tmp[i] = run;
+      run += t;
+    }
+    tmp[blockDim.x] = run;
+  }
+  __syncthreads();
+  int run = tmp[threadIdx.x];
+  for (int i = b; i < e; ++i) {
+    const int t = v[i];
+    v[i] = run;
+    run += t;
+  }
+  const int total = tmp[blockDim.x];
+  __syncthreads();
+  return total;
+}
+
+struct PlanSmem {
+  int tmp[kThreads + 1];
+};
+
+__global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn,
+                                                             int fm) {
+  __shared__ SchedSmem sm;
+  __shared__ PlanSmem pl;
+  State* st = c.st;
+  const int tid = threadIdx.x;
+  const uint32_t need = st->need_route;
+  // 1. fold fresh chunk counts into hist[j][:] and loads w[j][:]
+  for (int i = tid; i < d.M * d.E; i += blockDim.x) {
+    const int j = i / d.E, e = i % d.E;
+    if ((need >> j) & 1u) {
+      int s = 0;
+      for (int ch = 0; ch < d.NC; ++ch) s += wk.chunk_hist[((size_t)j * d.NC + ch) * d.E + e];
+      c.hist[i] = s;
+    }
+  }
+  __syncthreads();
+  const int per = d.E / d.D;
+  for (int i = tid; i < d.M * d.D; i += blockDim.x) {
+    const int j = i / d.D, dd = i % d.D;
+    if ((need >> j) & 1u) {
+      int s = 0;
+      for (int e = dd * per; e < (dd + 1) * per; ++e) s += c.hist[j * d.E + e];
+      c.w[i] = s;
+    }
+  }
+  // 2. pending set
+  const uint32_t pending = st->pending;
+  if (tid == 0) {
+    int n = 0;
+    for (int j = 0; j < d.M; ++j)
+      if ((pending >> j) & 1u) sm.P[n++] = j;
+    sm.n = n;
+  }
+  __syncthreads();
+  if (sm.n == 0) {  // episode finished: this step does nothing
+    if (tid == 0) {
+      st->runset = 0;
+      st->n_run = 0;
+      st->need_route = 0;
+      st->nseg = 0;
+      st->items1 = 0;
+      st->items2 = 0;
+      st->rows = 0;
+      for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
+    }
+    return;
+  }
+  for (int i = tid; i < sm.n * d.D; i += blockDim.x) {
+    const int p = i / d.D, dd = i % d.D;
+    sm.w[p][dd] = c.w[sm.P[p] * d.D + dd];
+  }
+  __syncthreads();
+  // 3. RunSet
+  const uint32_t run = choose_runset(sm, d.D, d.m, d.policy, pending);
+  // 4. accounting, trace and Algorithm 1 bookkeeping (thread 0)
+  if (tid == 0) {
+    long long sumW = 0, maxW = 0, summax = 0;
+    for (int dd = 0; dd < d.D; ++dd) {
+      long long Wd = 0;
+      for (int p = 0; p < sm.n; ++p)
+        if ((run >> sm.P[p]) & 1u) Wd += sm.w[p][dd];
+      sumW += Wd;
+      maxW = Wd > maxW ? Wd : maxW;
+    }
+    for (int p = 0; p < sm.n; ++p)
+      if ((run >> sm.P[p]) & 1u) {
+        long long mx = 0;
+        for (int dd = 0; dd < d.D; ++dd) mx = sm.w[p][dd] > mx ? sm.w[p][dd] : mx;
+        summax += mx;
+      }
+    st->num += sumW;
+    st->den += (long long)d.D * maxW;
+    st->den_sep += (long long)d.D * summax;
+    const int step = st->n_steps;
+    if (step < d.max_steps) {
+      c.trace[step * kTraceCols + 0] = run;
+      c.trace[step * kTraceCols + 1] = sumW;
+      c.trace[step * kTraceCols + 2] = maxW;
+      c.trace[step * kTraceCols + 3] = summax;
+      c.trace[step * kTraceCols + 4] = 0;
+      c.trace[step * kTraceCols + 5] = 0;
+      for (int j = 0; j < d.M; ++j)
+        c.trace_layers[step * d.M + j] = ((run >> j) & 1u) ? st->layer[j] : -1;
+    }
+    st->n_steps = step + 1;
+    int nr = 0;
+    uint32_t still = 0;
+    for (int j = 0; j < d.M; ++j) {
+      if ((run >> j) & 1u) {
+        st->step_layer[j] = st->layer[j];
+        st->run_list[nr++] = j;
+        st->layer[j] += 1;
+      } else {
+        st->step_layer[j] = -1;
+      }
+      if (st->layer[j] < d.L) still |= 1u << j;
+    }
+    st->n_run = nr;
+    st->runset = run;
+    st->pending = still;
+    st->need_route = run & still;
+    // segment groups: distinct layers of the RunSet, ascending
+    int G = 0;
+    for (int a = 0; a < nr; ++a) {
+      const int l = st->step_layer[st->run_list[a]];
+      bool seen = false;
+      for (int g = 0; g < G; ++g) seen |= (st->group_layer[g] == l);
+      if (!seen) {
+        int g = G++;
+        while (g > 0 && st->group_layer[g - 1] > l) {
+          st->group_layer[g] = st->group_layer[g - 1];
+          --g;
+        }
+        st->group_layer[g] = l;
+      }
+    }
+    for (int a = 0; a < nr; ++a) {
+      const int j = st->run_list[a];
+      for (int g = 0; g < G; ++g)
+        if (st->group_layer[g] == st->step_layer[j]) st->group_of[j] = g;
+    }
+    st->n_groups = G;
+    st->nseg = G * d.Etot;
+  }
+  if (!d.compute) return;
+  __syncthreads();
+  // 5. segment plan: rows of (group, expert) are counted into seg_rows and
+  //    scanned in place; GEMM work items per segment likewise.
+  const int G = st->n_groups, nr = st->n_run, Et = d.Etot, nseg = G * Et;
+  const int mb1 = d.F / fm, mb2 = d.H / fm;
+  __shared__ int s_nonempty;
+  if (tid == 0) s_nonempty = 0;
+  __syncthreads();
+  int my_nonempty = 0;
+  for (int i = tid; i < nseg; i += blockDim.x) {
+    const int g = i / Et, e = i % Et;
+    int cnt = 0;
+    for (int a = 0; a < nr; ++a) {
+      const int j = st->run_list[a];
+      if (st->group_of[j] != g) continue;
+      cnt += (e < d.E) ? c.hist[j * d.E + e] : d.T;
+    }
+    const int nch = (cnt + rn - 1) / rn;
+    my_nonempty += cnt > 0;
+    wk.seg_rows[i] = cnt;
+    wk.seg_items1[i] = nch * mb1;
+    wk.seg_items2[i] = nch * mb2;
+    wk.seg_wid[i] = st->group_layer[g] * Et + e;
+  }
+  if (my_nonempty) atomicAdd(&s_nonempty, my_nonempty);
+  __syncthreads();
+  const int rows = block_exclusive_scan(wk.seg_rows, nseg, pl.tmp);
+  const int it1 = block_exclusive_scan(wk.seg_items1, nseg, pl.tmp);
+  const int it2 = block_exclusive_scan(wk.seg_items2, nseg, pl.tmp);
+  if (tid == 0) {
+    wk.seg_rows[nseg] = rows;
+    wk.seg_items1[nseg] = it1;
+    wk.seg_items2[nseg] = it2;
+    st->rows = rows;
+    st->items1 = it1;
+    st->items2 = it2;
+    const int step = st->n_steps - 1;  // the row written above
+    if (step < d.max_steps) {
+      c.trace[step * kTraceCols + 4] = rows;
+      c.trace[step * kTraceCols + 5] = s_nonempty;
+    }
+  }
+  __syncthreads();
+  // bases: first row of (j, chunk, expert)
+  for (int i = tid; i < nr * Et; i += blockDim.x) {
+    const int a = i / Et, e = i % Et;
+    const int j = st->run_list[a], g = st->group_of[j];
+    int run_row = wk.seg_rows[g * Et + e];
+    for (int b = 0; b < a; ++b) {
+      const int jb = st->run_list[b];
+      if (st->group_of[jb] == g) run_row += (e < d.E) ? c.hist[jb * d.E + e] : d.T;
+    }
+    for (int ch = 0; ch < d.NC; ++ch) {
+      wk.base[((size_t)j * d.NC + ch) * Et + e] = run_row;
+      run_row += (e < d.E) ? wk.chunk_hist[((size_t)j * d.NC + ch) * d.E + e]
+                           : min(kChunk, d.T - ch * kChunk);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __restrict__ w,
+                                                             uint32_t pending, int M, int D,
+                                                             int m, int policy,
+                                                             uint32_t* __restrict__ runset_out,
+                                                             long long* __restrict__ stats) {
+  __shared__ SchedSmem sm;
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    int n = 0;
+    for (int j = 0; j < M; ++j)
+      if ((pending >> j) & 1u) sm.P[n++] = j;
+    sm.n = n;
+  }
+  __syncthreads();
+  if (sm.n == 0) {
+    if (tid == 0) {
+      *runset_out = 0;
+      if (stats) stats[0] = stats[1] = stats[2] = 0;
+    }
+    return;
+  }
+  for (int i = tid; i < sm.n * D; i += blockDim.x) {
+    const int p = i / D, dd = i % D;
+    sm.w[p][dd] = w[sm.P[p] * D + dd];
+  }
+  __syncthreads();
+  const uint32_t run = choose_runset(sm, D, m, policy, pending);
+  if (tid == 0) {
+    *runset_out = run;
+    if (stats) {
+      long long sumW = 0, maxW = 0, summax = 0;
+      for (int dd = 0; dd < D; ++dd) {
+        long long Wd = 0;
+        for (int p = 0; p < sm.n; ++p)
+          if ((run >> sm.P[p]) & 1u) Wd += sm.w[p][dd];
+        sumW += Wd;
+        maxW = Wd > maxW ? Wd : maxW;
+      }
+      for (int p = 0; p < sm.n; ++p)
+        if ((run >> sm.P[p]) & 1u) {
+          long long mx = 0;
+          for (int dd = 0; dd < D; ++dd) mx = sm.w[p][dd] > mx ? sm.w[p][dd] : mx;
+          summax += mx;
+        }
+      stats[0] = sumW;
+      stats[1] = maxW;
+      stats[2] = summax;
+    }
+  }
+}
+
+__global__ void k_loads(const int32_t* __restrict__ hist, int M, int E, int D,
+                        int32_t* __restrict__ w) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * D) return;
+  const int j = i / D, dd = i % D, per = E / D;
+  int s = 0;
+  for (int e = dd * per; e < (dd + 1) * per; ++e) s += hist[j * E + e];
+  w[i] = s;
+}
+
+__global__ void k_reset(Dims d, State* st) {
+  if (threadIdx.x != 0) return;
+  const uint32_t all = d.M >= 32 ? 0xffffffffu : ((1u << d.M) - 1u);
+  for (int j = 0; j < EB_MAX_M; ++j) {
+    st->layer[j] = 0;
+    st->step_layer[j] = -1;
+    st->run_list[j] = 0;
+    st->group_of[j] = 0;
+    st->group_layer[j] = 0;
+  }
+  st->pending = d.L > 0 ? all : 0u;
+  st->need_route = st->pending;
+  st->runset = 0;
+  st->n_run = 0;
+  st->n_groups = 0;
+  st->n_steps = 0;
+  st->status = EB_OK;
+  st->nseg = 0;
+  st->items1 = st->items2 = 0;
+  st->rows = 0;
+  st->num = st->den = st->den_sep = 0;
+}
+
+}  // namespace
+
+unsigned long long maxutil_candidates(int n, int m) {
+  if (n <= m) return 1;
+  unsigned long long total = 0, b = 1;  // b = C(n, c)
+  for (int c = 0; c <= n - m; ++c) {
+    total += b;
+    b = b * (unsigned long long)(n - c) / (unsigned long long)(c + 1);
+  }
+  return total;
+}
+
+cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn, int fm,
+                                 cudaStream_t s) {
+  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn, fm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
+                                 int policy, uint32_t* runset, long long* stats, cudaStream_t s) {
+  k_schedule_once<<<1, kThreads, 0, s>>>(w, pending, M, D, m, policy, runset, stats);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s) {
+  const int n = M * D;
+  if (n == 0) return cudaSuccess;
+  k_loads<<<(n + 255) / 256, 256, 0, s>>>(hist, M, E, D, w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s) {
+  k_reset<<<1, 32, 0, s>>>(d, c.st);
+  return cudaGetLastError();
+}
+
+}  // namespace eb

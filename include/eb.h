@@ -1,0 +1,219 @@
+/*
+ * eb.h -- C ABI of the B200 cross-layer MoE step (EasyBalance).
+ *
+ * The library runs one EasyBalance step on one GPU for M micro-batches that
+ * each sit at their own MoE layer, with D expert-parallel ranks simulated on
+ * the device.  Cited sources:
+ *   [EB]      "EasyBalance: Cross-Layer Load Balancing in Distributed MoE
+ *             Inference" (Wu, Gao, Li, Wu).
+ *   [EB-read] deep-read page "EasyBalance：分布式 MoE 推理的跨层负载均衡".
+ *   [SysLB]   page "系统侧负载均衡：EPLB、LPLB、UltraEP 与 MoonEP".
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers unless a parameter says "host".
+ *     They are owned by the caller; the library never frees them.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously on it unless stated.
+ *   - Argument errors are detected on the host before anything is enqueued
+ *     and returned as a negative eb_status; nothing runs in that case.
+ *   - Errors the device detects (a non-finite router logit, an expired
+ *     bounded wait) are recorded in the context's status word and returned by
+ *     eb_sync_status().
+ *   - There is no CPU fallback: a shape the kernels do not support returns
+ *     EB_ERR_UNSUPPORTED.
+ *   - A context is not thread-safe; its calls must be ordered on one stream.
+ *   - All integer outputs (indices, histograms, loads, RunSets, utilisation
+ *     numerators and denominators) are exact.
+ */
+#ifndef EB_H
+#define EB_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int eb_status;
+#define EB_OK 0
+#define EB_ERR_INVALID_ARG (-1) /* null pointer, size out of range, m > M ... */
+#define EB_ERR_UNSUPPORTED (-2) /* valid but outside the kernels' limits     */
+#define EB_ERR_NONFINITE (-3)   /* a NaN or Inf router logit was seen        */
+#define EB_ERR_CUDA (-4)        /* a CUDA runtime call failed                */
+#define EB_ERR_TIMEOUT (-5)     /* a bounded device-side wait expired        */
+#define EB_ERR_WORKSPACE (-6)   /* workspace smaller than eb_workspace_size  */
+
+/* RunSet policies, [EB] §4.2 and §5.2. */
+#define EB_SCHED_CUMUTIL 0  /* O(n) scan: add j iff U(S+{j}) > U(S)          */
+#define EB_SCHED_MAXUTIL 1  /* argmax U(S) over all S with |S| >= m          */
+#define EB_SCHED_LOCKSTEP 2 /* every pending micro-batch: layer-by-layer     */
+#define EB_SCHED_DIFFPEAK 3 /* add j iff its peak device is not yet taken    */
+
+/* storage type of hidden states, expert weights and intermediates */
+#define EB_DTYPE_F32 0
+#define EB_DTYPE_BF16 1
+
+/* expert GEMM engine: AUTO = tensor cores (tcgen05) for bf16, SIMT for f32 */
+#define EB_GEMM_AUTO 0
+#define EB_GEMM_TC 1
+#define EB_GEMM_SIMT 2
+
+/* Limits of this build. */
+#define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */
+#define EB_MAX_D 64   /* virtual ranks                                   */
+#define EB_MAX_ETOT 256 /* routed + shared experts per layer            */
+#define EB_MAX_K 32   /* experts per token                               */
+
+typedef struct eb_config {
+  int L;        /* MoE layers (l_max)                                    */
+  int E;        /* routed experts per layer                              */
+  int k;        /* experts per token, 1 <= k <= min(E, EB_MAX_K)         */
+  int H;        /* hidden size                                           */
+  int F;        /* expert FFN width (SwiGLU inner size)                  */
+  int D;        /* virtual EP ranks; E % D == 0; rank d holds experts
+                   [d E/D, (d+1) E/D)  ([EB] §5 Models: even mapping)     */
+  int M;        /* micro-batches, 1..EB_MAX_M                            */
+  int T;        /* tokens per micro-batch, >= 1                          */
+  int n_shared; /* always-on shared experts per layer (gate 1.0, not
+                   counted in the workloads w)                           */
+  int renorm;   /* 1: gates renormalised over the top-k                  */
+  int dtype;    /* EB_DTYPE_*                                            */
+  int policy;   /* EB_SCHED_*                                            */
+  int m;        /* minimum RunSet size, 1..M ([EB] §4.2)                 */
+  int residual; /* 1: h_{l+1} = h_l + MoE_l(h_l); 0: h_{l+1} = MoE_l(h_l) */
+  int compute;  /* 1: full step; 0: routing + scheduling only            */
+  int gemm;     /* EB_GEMM_*                                             */
+} eb_config;
+
+typedef struct eb_ctx eb_ctx;
+
+/* Human-readable name of a status code (static string). */
+const char* eb_status_string(eb_status s);
+
+/* Checks a configuration without touching the GPU. */
+eb_status eb_config_check(const eb_config* cfg);
+
+/* Bytes of device workspace eb_moe_step needs for `cfg` (host only).  The
+ * caller allocates it (256-byte aligned) and keeps it, unchanged, for a whole
+ * episode: it carries the routed indices and gates of deferred micro-batches
+ * from one step to the next. */
+eb_status eb_workspace_size(const eb_config* cfg, size_t* bytes);
+
+/* Creates a context on the current CUDA device.  The context owns a small
+ * device state (per-micro-batch layers l_j, the pending set S, histograms,
+ * loads, the exact utilisation accumulators and the per-step trace). */
+eb_status eb_create(const eb_config* cfg, eb_ctx** out);
+eb_status eb_destroy(eb_ctx* ctx);
+
+/* Algorithm 1 initialisation ([EB] §4.2): l_j = 0 for all j, S_0 = all
+ * micro-batches, RunSet_0 = all (every micro-batch routes at step 1), and
+ * zeroed accumulators and trace.  Enqueued on `stream`. */
+eb_status eb_reset(eb_ctx* ctx, void* stream);
+
+/*
+ * One EasyBalance step, [EB] §4.2 Algorithm 1 loop body, entirely on device:
+ *   1. route the micro-batches of the previous RunSet at their layer l_j:
+ *      softmax top-k of the fp32 logits, renormalised gates ([EB] §2.1);
+ *      per-expert counts T_e folded into w_j over the contiguous map
+ *      ([SysLB] §1; [EB] §2.3);
+ *   2. RunSet = Schedule(S, m) with cfg.policy; exact int64 utilisation
+ *      accumulators ([EB] Eq. (2), (3)); trace row;
+ *   3. permute the RunSet's tokens into segments keyed (layer, expert)
+ *      -- micro-batches at the same layer share a segment --, one grouped
+ *      SwiGLU expert GEMM over all segments (experts of different layers in
+ *      one launch), and the gated combine in slot order ([EB] Eq. (1)),
+ *      written back into `hidden`;
+ *   4. l_j += 1 for the RunSet; finished micro-batches leave S.
+ * Once S is empty a step does nothing.
+ *
+ * logits    [M, L, T, E] float32: the router logits of micro-batch j at
+ *           layer l; only the blocks (j, l_j) of routed micro-batches are read.
+ * hidden    [M, T, H] cfg.dtype, updated in place for RunSet micro-batches.
+ * w_gateup  [L, E + n_shared, 2F, H] cfg.dtype, row-major; rows 0..F-1 of an
+ *           expert are its gate projection, rows F..2F-1 its up projection.
+ *           Must be 16-byte aligned.
+ * w_down    [L, E + n_shared, H, F] cfg.dtype.  Must be 16-byte aligned.
+ * workspace at least eb_workspace_size() bytes, 256-byte aligned.
+ * runset_host  optional host pointer: if non-NULL the call waits for the step
+ *           and stores its RunSet bitmask (bit j = micro-batch j; 0 = nothing
+ *           ran because S was empty).
+ * With cfg.compute == 0 only steps 1, 2 and 4 run (hidden and weights may be
+ * NULL).
+ */
+eb_status eb_moe_step(eb_ctx* ctx, const float* logits, void* hidden, const void* w_gateup,
+                      const void* w_down, void* workspace, size_t workspace_bytes, void* stream,
+                      uint32_t* runset_host);
+
+/* A whole episode: eb_reset, then eb_moe_step until S is empty.  Steps are
+ * enqueued a few ahead of the host's completion check, so the GPU never waits
+ * for the host; steps enqueued after S became empty do nothing.  Returns the
+ * number of steps that ran in *n_steps (host).  Waits for completion. */
+eb_status eb_episode(eb_ctx* ctx, const float* logits, void* hidden, const void* w_gateup,
+                     const void* w_down, void* workspace, size_t workspace_bytes, void* stream,
+                     int* n_steps);
+
+/* Exact utilisation totals of the steps run since eb_reset (waits for the
+ * context's work):
+ *   num     = sum over steps of sum_d W_d            (work done)
+ *   den     = D * sum over steps of max_d W_d         ([EB] Eq. (3) denominator)
+ *   den_sep = D * sum over executed (j, l) of max_d w_{j,l}
+ *             (each micro-batch run on its own: the "maximum workload" of
+ *             [EB] Fig. 6).
+ * u = num / den; the no-combination baseline is num / den_sep. */
+eb_status eb_utilization(eb_ctx* ctx, int64_t* num, int64_t* den, int64_t* den_sep);
+
+/* Per-step trace since eb_reset (waits).  Host arrays: rows [max_steps][6]
+ * int64 = (RunSet mask, sum_d W_d, max_d W_d, sum_{j in RunSet} max_d w_j,
+ * permuted token rows R of the step, non-empty (layer, expert) segments);
+ * layers [max_steps][M] int32 = layer at which micro-batch j ran in that step,
+ * or -1.  *n_steps receives the number of steps recorded (may exceed
+ * max_steps; only max_steps rows are written).  layers may be NULL. */
+eb_status eb_trace(eb_ctx* ctx, int64_t* rows, int32_t* layers, int max_steps, int* n_steps);
+
+/* Measurement support.  eb_profile(ctx, 1) brackets every kernel the context
+ * enqueues with CUDA events on the launching stream (eb_profile(ctx, 0) stops;
+ * both drop earlier marks).  eb_profile_read waits for them and returns, per
+ * kernel, the summed milliseconds and the number of launches since, then
+ * clears the marks.  Kernel order: route, schedule+plan, permute, GEMM 1
+ * (gate/up + SwiGLU), GEMM 2 (down), combine.  eb_launch_count returns the
+ * kernels the context has enqueued since eb_create. */
+#define EB_PROF_KERNELS 6
+eb_status eb_profile(eb_ctx* ctx, int enable);
+eb_status eb_profile_read(eb_ctx* ctx, double* ms, int64_t* launches);
+eb_status eb_launch_count(eb_ctx* ctx, int64_t* n);
+
+/* Waits for the context's work and returns the device-side status. */
+eb_status eb_sync_status(eb_ctx* ctx);
+
+/* ---------------------------------------------------------------------------
+ * Stand-alone stages (stateless; device pointers; async on `stream`).
+ * ------------------------------------------------------------------------ */
+
+/* Router top-k over n independent token rows, [EB] §2.1 topk(G(h')):
+ * logits [n, E] float32 -> idx [n, k] int32 (descending logit; equal logits
+ * to the lower expert index), gate [n, k] float32 (softmax probabilities of
+ * the selected experts, renormalised to sum 1 if renorm), hist [E] int32
+ * (tokens per expert, T_e of [SysLB] §1; overwritten).  status_dev is an
+ * optional device int32: if non-NULL it is set to EB_ERR_NONFINITE when a
+ * NaN or Inf logit is seen (and left unchanged otherwise). */
+eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t* idx, float* gate,
+                   int32_t* hist, int32_t* status_dev, void* stream);
+
+/* Virtual-rank loads under the contiguous map: w[j][d] = sum of hist[j][e]
+ * over e in [d E/D, (d+1) E/D).  hist [M, E] int32 -> w [M, D] int32. */
+eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream);
+
+/* RunSet = Schedule(S, m) for one step ([EB] §4.2, §5.2).
+ * w [M, D] int32 loads; pending_mask: bit j set = j in S.
+ * runset_mask (device uint32) receives the RunSet bitmask; step_stats
+ * (device int64[3], may be NULL) receives (sum_d W_d, max_d W_d,
+ * sum_{j in RunSet} max_d w_j).  If |S| <= m the RunSet is S. */
+eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int m, int policy,
+                      uint32_t* runset_mask, int64_t* step_stats, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EB_H */

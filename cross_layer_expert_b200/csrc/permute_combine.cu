@@ -34,6 +34,10 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // CTA (c, j): chunk c of RunSet micro-batch j.  Row of (t, s) = base of
 // (j, c, expert) + number of earlier (t', s') of this chunk with the same
 // expert, so rows follow (micro-batch, token, slot) order inside a segment.
+// Each chunk's ranks are computed by kPermSplit CTAs (cheap, identical); each
+// copies a quarter of the chunk's tokens, so the HBM-bound copy has 4x the CTAs.
+constexpr int kPermSplit = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* __restrict__ st,
                                                           const int32_t* __restrict__ idx,
@@ -41,7 +45,7 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
                                                           int32_t* __restrict__ pos,
                                                           const T* __restrict__ hidden,
                                                           T* __restrict__ A) {
-  const int c = blockIdx.x, j = blockIdx.y;
+  const int c = blockIdx.x / kPermSplit, part = blockIdx.x % kPermSplit, j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
   __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
   __shared__ int running[EB_MAX_ETOT];
@@ -76,7 +80,7 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
       const int t = p / k, s = p % k;
       const int row = bj[e] + cnt[warp][e] + rank;
       dest[t * kk + s] = row;
-      pos[((size_t)j * d.T + t0 + t) * kk + s] = row;
+      if (part == 0) pos[((size_t)j * d.T + t0 + t) * kk + s] = row;
     }
     __syncthreads();
   }
@@ -84,11 +88,13 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
     const int t = i / d.n_shared, s = i % d.n_shared;
     const int row = bj[E + s] + t;
     dest[t * kk + k + s] = row;
-    pos[((size_t)j * d.T + t0 + t) * kk + k + s] = row;
+    if (part == 0) pos[((size_t)j * d.T + t0 + t) * kk + k + s] = row;
   }
   __syncthreads();
   const int nvec = d.H * (int)sizeof(T) / 16;
-  for (int t = warp; t < nt; t += kPermThreads / 32) {
+  const int per = (nt + kPermSplit - 1) / kPermSplit;
+  const int ta = part * per, tb = min(nt, ta + per);
+  for (int t = ta + warp; t < tb; t += kPermThreads / 32) {
     const uint4* src = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + t) * d.H);
     for (int v = lane; v < nvec; v += 32) {
       const uint4 val = __ldg(src + v);
@@ -110,6 +116,10 @@ struct Vec<float> {
   __device__ static void load_plain(const float* p, int v, float* out) {
     const float4 x = reinterpret_cast<const float4*>(p)[v];
     out[0] = x.x; out[1] = x.y; out[2] = x.z; out[3] = x.w;
+  }
+  __device__ static void unpack(const uint4& x, float* out) {
+    out[0] = __uint_as_float(x.x); out[1] = __uint_as_float(x.y);
+    out[2] = __uint_as_float(x.z); out[3] = __uint_as_float(x.w);
   }
   __device__ static void store(float* p, int v, const float* in) {
     reinterpret_cast<float4*>(p)[v] = make_float4(in[0], in[1], in[2], in[3]);
@@ -138,6 +148,15 @@ struct Vec<__nv_bfloat16> {
       out[2 * i + 1] = f.y;
     }
   }
+  __device__ static void unpack(const uint4& x, float* out) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&x);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      out[2 * i] = f.x;
+      out[2 * i + 1] = f.y;
+    }
+  }
   __device__ static void store(__nv_bfloat16* p, int v, const float* in) {
     uint4 x;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&x);
@@ -147,37 +166,48 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
+constexpr int kCombineTokens = 8;  // one warp per token
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_combine(Dims d, const State* __restrict__ st,
                                                   const float* __restrict__ gate,
                                                   const int32_t* __restrict__ pos,
                                                   const T* __restrict__ y, T* hidden) {
-  const int c = blockIdx.x, j = blockIdx.y;
+  const int j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
-  __shared__ int s_row[8][kMaxSlots];
-  __shared__ float s_gate[8][kMaxSlots];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  const int t0 = c * kChunk, nt = min(kChunk, d.T - t0);
+  __shared__ int s_row[kCombineTokens][kMaxSlots];
+  __shared__ float s_gate[kCombineTokens][kMaxSlots];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * kCombineTokens + warp;
+  if (t >= d.T) return;
   const int k = d.k, kk = d.kk;
   constexpr int VE = Vec<T>::n;
   const int nvec = d.H / VE;
-  for (int tl = warp; tl < nt; tl += nwarps) {
-    const size_t tok = (size_t)j * d.T + t0 + tl;
-    if (lane < kk) s_row[warp][lane] = pos[tok * kk + lane];
-    if (lane < k) s_gate[warp][lane] = gate[tok * k + lane];
-    __syncwarp();
-    T* out = hidden + tok * d.H;
-    for (int v = lane; v < nvec; v += 32) {
-      float acc[VE];
-      if (d.residual) {
-        Vec<T>::load_plain(out, v, acc);
-      } else {
+  const size_t tok = (size_t)j * d.T + t;
+  if (lane < kk) s_row[warp][lane] = pos[tok * kk + lane];
+  if (lane < k) s_gate[warp][lane] = gate[tok * k + lane];
+  __syncwarp();
+  T* out = hidden + tok * d.H;
+  for (int v = lane; v < nvec; v += 32) {
+    float acc[VE];
+    if (d.residual) {
+      Vec<T>::load_plain(out, v, acc);
+    } else {
 #pragma unroll
-        for (int i = 0; i < VE; ++i) acc[i] = 0.f;
-      }
-      for (int s = 0; s < kk; ++s) {
+      for (int i = 0; i < VE; ++i) acc[i] = 0.f;
+    }
+    for (int s0 = 0; s0 < kk; s0 += 8) {
+      uint4 raw[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (s0 + u < kk)
+          raw[u] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)s_row[warp][s0 + u] * d.H) + v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int s = s0 + u;
+        if (s >= kk) break;
         float yv[VE];
-        Vec<T>::load(y + (size_t)s_row[warp][s] * d.H, v, yv);
+        Vec<T>::unpack(raw[u], yv);
         if (s < k) {
           const float g = s_gate[warp][s];
 #pragma unroll
@@ -187,9 +217,8 @@ __global__ void __launch_bounds__(256) k_combine(Dims d, const State* __restrict
           for (int i = 0; i < VE; ++i) acc[i] += yv[i];
         }
       }
-      Vec<T>::store(out, v, acc);
     }
-    __syncwarp();
+    Vec<T>::store(out, v, acc);
   }
 }
 
@@ -197,7 +226,7 @@ __global__ void __launch_bounds__(256) k_combine(Dims d, const State* __restrict
 
 cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                            cudaStream_t s) {
-  dim3 grid(d.NC, d.M);
+  dim3 grid(d.NC * kPermSplit, d.M);
   if (d.dtype == EB_DTYPE_BF16)
     k_permute<__nv_bfloat16><<<grid, kPermThreads, 0, s>>>(
         d, c.st, w.idx, w.base, w.pos, static_cast<const __nv_bfloat16*>(hidden),
@@ -211,7 +240,7 @@ cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const 
 
 cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
                            cudaStream_t s) {
-  dim3 grid(d.NC, d.M);
+  dim3 grid((d.T + kCombineTokens - 1) / kCombineTokens, d.M);
   if (d.dtype == EB_DTYPE_BF16)
     k_combine<__nv_bfloat16><<<grid, 256, 0, s>>>(d, c.st, w.gate, w.pos,
                                                   static_cast<const __nv_bfloat16*>(w.y),

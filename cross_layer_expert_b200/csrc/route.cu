@@ -6,7 +6,9 @@
 //
 // One warp routes one token: the E logits are read coalesced (lane i holds
 // experts i, i+32, ...), the k winners come out of k rounds of a warp-wide
-// argmax under the order (logit descending, expert index ascending), and the
+// argmax under the order (logit descending, expert index ascending) -- a
+// hardware max-reduction over order-preserving integer keys, then a
+// min-reduction over the expert ids holding the maximum --, and the
 // gates exp(l_s - l_max) / sum_{s'} exp(l_s' - l_max) are formed from the
 // winners alone when renormalised (the full softmax denominator cancels).
 // Counts go to shared-memory atomics (integers, so the result is exact and
@@ -21,21 +23,27 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 
-__device__ __forceinline__ bool better(float v1, int e1, float v2, int e2) {
-  return v1 > v2 || (v1 == v2 && e1 < e2);
-}
-
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll
   for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(kFull, x, off);
   return x;
 }
 
+// Order-preserving map of a finite float to uint32 (-0 is folded into +0
+// first, so equal floats map to equal keys).
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
 // Routes one token row with the calling warp.  Lane s < k returns slot s.
+// Each of the k rounds takes the warp maximum of the lanes' best keys, then
+// the smallest expert index among the lanes holding it.
 template <int VPL>
 __device__ __forceinline__ void route_row(const float* __restrict__ row, int E, int k, int renorm,
                                           int lane, int& out_e, float& out_g, bool& nonfinite) {
   float v[VPL];
+  uint32_t key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = i * 32 + lane;
@@ -48,36 +56,37 @@ __device__ __forceinline__ void route_row(const float* __restrict__ row, int E, 
       }
     }
     v[i] = x;
+    key[i] = e < E ? order_key(x) : 0u;  // real experts (even -inf) rank above padding
+    if (e < E && key[i] == 0u) key[i] = 1u;
   }
-  unsigned taken = 0;
   float top_v = -INFINITY, vmax = -INFINITY;
   int top_e = 0;
   for (int s = 0; s < k; ++s) {
-    float bv = -INFINITY;
+    uint32_t bk = 0;
     int be = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = i * 32 + lane;
-      if (e < E && !((taken >> i) & 1u) && better(v[i], e, bv, be)) {
-        bv = v[i];
-        be = e;
+      // ascending i visits ascending expert ids of this lane: strict > keeps the lowest
+      if (key[i] > bk) {
+        bk = key[i];
+        be = i * 32 + lane;
       }
     }
+    const uint32_t wk = __reduce_max_sync(kFull, bk);
+    const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
+    float wv = 0.f;
 #pragma unroll
-    for (int off = 16; off; off >>= 1) {
-      const float ov = __shfl_xor_sync(kFull, bv, off);
-      const int oe = __shfl_xor_sync(kFull, be, off);
-      if (better(ov, oe, bv, be)) {
-        bv = ov;
-        be = oe;
+    for (int i = 0; i < VPL; ++i)
+      if (i * 32 + lane == we) {
+        wv = v[i];
+        key[i] = 0u;  // taken
       }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+    wv = __shfl_sync(kFull, wv, we & 31);
     if (lane == s) {
-      top_v = bv;
-      top_e = be;
+      top_v = wv;
+      top_e = we;
     }
-    if (s == 0) vmax = bv;
+    if (s == 0) vmax = wv;
   }
   const float ex = (lane < k) ? expf(top_v - vmax) : 0.f;
   float denom;
@@ -114,7 +123,7 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
 // is in need_route; its counts land in chunk_hist[j][c][:].
 template <int VPL>
-__global__ void __launch_bounds__(256) k_route_step(Dims d, State* __restrict__ st,
+__global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__ st,
                                                      const float* __restrict__ logits,
                                                      int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
@@ -170,10 +179,10 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               cudaStream_t s) {
   dim3 grid(d.NC, d.M);
   switch (vpl_for(d.E)) {
-    case 1: k_route_step<1><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    case 2: k_route_step<2><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    case 4: k_route_step<4><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    default: k_route_step<8><<<grid, 256, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
   }
   return cudaGetLastError();
 }

@@ -199,67 +199,84 @@ __device__ uint32_t scan_policy(const SchedSmem& sm, int D, int m, int policy) {
 // All threads: loads w[j][:] of the pending set must be in sm.w (by position);
 // returns the RunSet mask (over micro-batch ids).
 __device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending) {
-  if (threadIdx.x == 0) {
-    // binomial table for the MaxUtil enumeration
-    for (int a = 0; a <= 32; ++a)
-      for (int b = 0; b <= 32; ++b)
-        sm.binom[a][b] = (b == 0) ? 1u : (a == 0 ? 0u : 0u);
-    for (int a = 1; a <= 32; ++a)
-      for (int b = 1; b <= 32; ++b) sm.binom[a][b] = sm.binom[a - 1][b - 1] + sm.binom[a - 1][b];
+  const int tid = threadIdx.x;
+  if (policy == EB_SCHED_MAXUTIL) {
+    // binomial table for the MaxUtil enumeration: C(a, b) by the exact
+    // multiplicative recurrence C(a, i) = C(a, i-1) (a - i + 1) / i
+    for (int i = tid; i < 33 * 33; i += blockDim.x) {
+      const int a = i / 33, b = i % 33;
+      unsigned long long c = b <= a ? 1ull : 0ull;
+      for (int q = 1; q <= b && b <= a; ++q) c = c * (unsigned long long)(a - q + 1) / q;
+      sm.binom[a][b] = (uint32_t)c;
+    }
+  }
+  for (int dd = tid; dd < D; dd += blockDim.x) {
+    long long t = 0;
+    for (int i = 0; i < sm.n; ++i) t += sm.w[i][dd];
+    sm.tot[dd] = t;
+  }
+  for (int i = tid; i < sm.n; i += blockDim.x) {
+    long long t = 0;
+    for (int dd = 0; dd < D; ++dd) t += sm.w[i][dd];
+    sm.wsum[i] = t;
+  }
+  __syncthreads();
+  if (tid == 0) {
     long long ts = 0;
-    for (int dd = 0; dd < D; ++dd) {
-      long long t = 0;
-      for (int i = 0; i < sm.n; ++i) t += sm.w[i][dd];
-      sm.tot[dd] = t;
-      ts += t;
-    }
+    for (int i = 0; i < sm.n; ++i) ts += sm.wsum[i];
     sm.totsum = ts;
-    for (int i = 0; i < sm.n; ++i) {
-      long long s = 0;
-      for (int dd = 0; dd < D; ++dd) s += sm.w[i][dd];
-      sm.wsum[i] = s;
-    }
   }
   __syncthreads();
   if (policy == EB_SCHED_LOCKSTEP || sm.n <= m) return pending;
   if (policy == EB_SCHED_MAXUTIL) return maxutil_block(sm, D, m);
-  if (threadIdx.x == 0) sm.result = scan_policy(sm, D, m, policy);
+  if (tid == 0) sm.result = scan_policy(sm, D, m, policy);
   __syncthreads();
   return sm.result;
 }
 
 // ---------------------------------------------------------------- block scan
 // Exclusive scan of v[0..n) in place (all threads); returns the total.
-__device__ int block_exclusive_scan(int* v, int n, int* tmp /* [kThreads] */) {
+// Each thread owns a contiguous run; run totals are scanned with warp
+// shuffles, then across the warps.
+__device__ int block_exclusive_scan(int* v, int n, int* tmp /* >= 33 ints */) {
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int b = threadIdx.x * per, e = min(n, b + per);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int local = 0;
   for (int i = b; i < e; ++i) local += v[i];
-  tmp[threadIdx.x] = local;
+  int incl = local;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  if (lane == 31) tmp[warp] = incl;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int i = 0; i < (int)blockDim.x; ++i) {
-      const int t = tmp[i];
-      tmp[i] = run;
-      run += t;
+  if (warp == 0) {
+    int x = lane < nw ? tmp[lane] : 0;
+    int xi = x;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, xi, off);
+      if (lane >= off) xi += y;
     }
-    tmp[blockDim.x] = run;
+    if (lane < nw) tmp[lane] = xi - x;  // exclusive warp offsets
+    if (lane == 31) tmp[32] = xi;       // block total
   }
   __syncthreads();
-  int run = tmp[threadIdx.x];
+  int run = tmp[warp] + incl - local;
   for (int i = b; i < e; ++i) {
     const int t = v[i];
     v[i] = run;
     run += t;
   }
-  const int total = tmp[blockDim.x];
+  const int total = tmp[32];
   __syncthreads();
   return total;
 }
 
 struct PlanSmem {
-  int tmp[kThreads + 1];
+  int tmp[33];
 };
 
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn,

@@ -37,15 +37,20 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every source into one shared library (objects in parallel)."""
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, out: str = LIB, defines=()) -> str:
+    """Compile every source into one shared library (objects in parallel).
+
+    `out` and `defines` (e.g. ["EB_L2_PREFETCH=8"]) build tuning variants
+    beside the default library."""
+    if not force and out == LIB and not _stale():
         return LIB
-    os.makedirs(LIB_DIR, exist_ok=True)
-    obj_dir = os.path.join(LIB_DIR, "obj")
+    lib_dir = os.path.dirname(os.path.abspath(out))
+    os.makedirs(lib_dir, exist_ok=True)
+    tag = os.path.splitext(os.path.basename(out))[0]
+    obj_dir = os.path.join(lib_dir, "obj" if out == LIB else "obj_" + tag)
     os.makedirs(obj_dir, exist_ok=True)
     flags = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC",
-                    "-I", os.path.join(ROOT, "include")]
+                    "-I", os.path.join(ROOT, "include")] + [f"-D{x}" for x in defines]
     procs = []
     objs = []
     for src in SOURCES:
@@ -57,18 +62,18 @@ def build(force: bool = False, verbose: bool = False) -> str:
         procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)))
     errors = []
     for src, p in procs:
-        out, _ = p.communicate()
+        log, _ = p.communicate()
         if p.returncode != 0:
-            errors.append(f"{src}:\n{out.decode(errors='replace')}")
+            errors.append(f"{src}:\n{log.decode(errors='replace')}")
     if errors:
         raise RuntimeError("nvcc failed:\n" + "\n".join(errors))
-    tmp = LIB + ".tmp"
+    tmp = out + ".tmp"
     cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs
     r = subprocess.run(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT)
     if r.returncode != 0:
         raise RuntimeError("link failed:\n" + r.stdout.decode(errors="replace"))
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, out)
+    return out
 
 
 if __name__ == "__main__":

@@ -16,8 +16,12 @@ namespace eb {
 constexpr int kChunk = 64;
 
 // Sizes of GEMM work items: RN token rows per item and FM output features per
-// item (the tcgen05 tile is 128 x 128; the SIMT tile 64 x 64).
-constexpr int kTcRows = 128;
+// item (the tcgen05 tile is 128 features x kTcRows tokens; the SIMT tile
+// 64 x 64).
+#ifndef EB_TC_ROWS
+#define EB_TC_ROWS 128
+#endif
+constexpr int kTcRows = EB_TC_ROWS;
 constexpr int kTcFeat = 128;
 constexpr int kSimtRows = 64;
 constexpr int kSimtFeat = 64;

@@ -34,9 +34,20 @@ constexpr int kBM = 128;        // weight rows (features) per MMA tile
 constexpr int kBN = kTcRows;    // token rows per item (max MMA N)
 constexpr int kBK = 64;         // K elements per stage: 128 bytes of bf16 = one swizzle row
 constexpr int kTileBytes = kBM * kBK * 2;  // 16 KiB
-constexpr int kXBytes = kBN * kBK * 2;     // 16 KiB
-constexpr int kThreads = 192;
+constexpr int kXBytes = kBN * kBK * 2;     // 16 or 32 KiB
+#ifndef EB_EPI_WARPS
+#define EB_EPI_WARPS 4
+#endif
+constexpr int kEpiWarps = EB_EPI_WARPS;    // 4 or 8: warps draining TMEM
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
+
+// Weight tiles are prefetched into L2 this many k-blocks ahead of the
+// shared-memory ring (0: off), so the ring's loads mostly hit L2.
+#ifndef EB_L2_PREFETCH
+#define EB_L2_PREFETCH 0
+#endif
+constexpr int kPrefetch = EB_L2_PREFETCH;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -100,6 +111,13 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y)
+               : "memory");
 }
 
 // K-major operand, 128-byte swizzle: rows of 128 B, 8-row atoms 1024 B apart.
@@ -196,10 +214,11 @@ __device__ __forceinline__ Item decode(const Dims& d, const int32_t* seg_rows,
 
 template <bool GATEUP>
 struct Cfg {
-  static constexpr int kStages = GATEUP ? 4 : 6;
   static constexpr int kStageBytes = (GATEUP ? 2 : 1) * kTileBytes + kXBytes;
+  static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kAccCols = (GATEUP ? 2 : 1) * kBN;  // TMEM columns per accumulator
-  static constexpr int kTmemCols = 2 * kAccCols;            // double buffered: 512 / 256
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;  // double buffer if it fits
+  static constexpr int kTmemCols = kAccBufs * kAccCols;     // 256 or 512
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /* barriers */ + 1024 /* align */;
 };
 
@@ -239,7 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 128);
+      mbar_init(smem_u32(&tempty[i]), 32 * kEpiWarps);
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -264,7 +283,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const Item it = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+        Item nx = it;
+        const bool has_next = kPrefetch > 0 && item + (int)gridDim.x < total;
+        if (has_next) nx = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item + gridDim.x);
+        if (kPrefetch > 0 && item == (int)blockIdx.x) {
+          for (int p = 0; p < kPrefetch && p < nk; ++p) {
+            tma_prefetch_2d(&map_w, p * kBK, it.wrow);
+            if (GATEUP) tma_prefetch_2d(&map_w, p * kBK, it.wrow + d.F);
+          }
+        }
         for (int kb = 0; kb < nk; ++kb) {
+          if (kPrefetch > 0) {
+            const int pk = kb + kPrefetch;
+            if (pk < nk) {
+              tma_prefetch_2d(&map_w, pk * kBK, it.wrow);
+              if (GATEUP) tma_prefetch_2d(&map_w, pk * kBK, it.wrow + d.F);
+            } else if (has_next && pk - nk < nk) {
+              tma_prefetch_2d(&map_w, (pk - nk) * kBK, nx.wrow);
+              if (GATEUP) tma_prefetch_2d(&map_w, (pk - nk) * kBK, nx.wrow + d.F);
+            }
+          }
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
             ok = false;
             break;
@@ -341,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_commit(smem_u32(&tfull[acc]));
         last_bar = smem_u32(&tfull[acc]);
         last_par = acc_phase;
-        if (++acc == 2) {
+        if (++acc == C::kAccBufs) {
           acc = 0;
           acc_phase ^= 1;
         }
@@ -356,6 +394,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;            // TMEM lane quarter this warp may read
     const int frow = q * 32 + lane;    // feature row of this thread within the tile
+    const int cgrp = (warp - 2) >> 2;  // with 8 warps, two warps split a quarter's columns
+    constexpr int kColStep = 32 * (kEpiWarps / 4);
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int item = blockIdx.x; item < total; item += gridDim.x) {
@@ -364,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
       __nv_bfloat16* orow = out + (size_t)it.r0 * NOUT + it.f0 + frow;
-      for (int cb = 0; cb < it.n; cb += 32) {
+      for (int cb = cgrp * 32; cb < it.n; cb += kColStep) {
         float g[32];
         tmem_ld32(tbase + cb, g);
         if (GATEUP) {
@@ -385,7 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&tempty[acc]));
-      if (++acc == 2) {
+      if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1;
       }
@@ -450,13 +490,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x 128 rows.
-cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, int cols) {
+// Row-major bf16 matrix [rows, cols] read in boxes of 64 columns x box_rows rows.
+cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, int cols,
+                   int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return cudaErrorNotSupported;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -470,10 +511,10 @@ cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, 
 cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
                          TcMaps* maps) {
   const unsigned long long experts = (unsigned long long)d.L * d.Etot;
-  cudaError_t e = encode(&maps->w_gateup, w_gateup, experts * 2 * d.F, d.H);
-  if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F);
-  if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H);
-  if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F);
+  cudaError_t e = encode(&maps->w_gateup, w_gateup, experts * 2 * d.F, d.H, kBM);
+  if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F, kBM);
+  if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H, kBN);
+  if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kBN);
   return e;
 }
 

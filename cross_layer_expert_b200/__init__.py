@@ -25,6 +25,7 @@ EB_ERR_NONFINITE = -3
 EB_ERR_CUDA = -4
 EB_ERR_TIMEOUT = -5
 EB_ERR_WORKSPACE = -6
+EB_ERR_TOO_LARGE = -7
 
 CUMUTIL, MAXUTIL, LOCKSTEP, DIFFPEAK = 0, 1, 2, 3
 DTYPE_F32, DTYPE_BF16 = 0, 1
@@ -33,7 +34,7 @@ GEMM_AUTO, GEMM_TC, GEMM_SIMT = 0, 1, 2
 EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_create", "eb_destroy",
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
-            "eb_profile_read", "eb_launch_count"]
+            "eb_profile_read", "eb_launch_count", "eb_route_loads_static"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine")
 
@@ -82,6 +83,7 @@ def load() -> ctypes.CDLL:
         "eb_profile": (I, [P, I]),
         "eb_profile_read": (I, [P, P, P]),
         "eb_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "eb_route_loads_static": (I, [P, I, I, I, I, I, I, P, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -150,6 +152,17 @@ def eb_schedule(w, pending_mask: int, m: int, policy: int, runset, stats=None, s
     M, D = w.shape
     _check(load().eb_schedule(_ptr(w), pending_mask, M, D, m, policy, _ptr(runset), _ptr(stats),
                               _stream(stream)), "eb_schedule")
+
+
+def eb_route_loads_static(logits, k: int, renorm: bool, D: int, idx, gate, w, status=None,
+                          stream=None) -> None:
+    """No-allocation routing + loads: logits [n_mb, T, E] f32 -> idx [n_mb, T, k] i32,
+    gate [n_mb, T, k] f32, w [n_mb, D] i32.  For callers that cannot allocate
+    device memory; the library's fixed 4 MiB device array holds the counts."""
+    n_mb, T, E = logits.shape
+    _check(load().eb_route_loads_static(_ptr(logits), n_mb, T, E, k, int(renorm), D, _ptr(idx),
+                                        _ptr(gate), _ptr(w), _ptr(status), _stream(stream)),
+           "eb_route_loads_static")
 
 
 class Context:

@@ -141,6 +141,7 @@ const char* eb_status_string(eb_status s) {
     case EB_ERR_CUDA: return "CUDA runtime error";
     case EB_ERR_TIMEOUT: return "bounded device wait expired";
     case EB_ERR_WORKSPACE: return "workspace too small";
+    case EB_ERR_TOO_LARGE: return "exceeds the fixed scratch capacity of a no-allocation call";
     default: return "unknown status";
   }
 }

@@ -202,3 +202,115 @@ cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int reno
 }
 
 }  // namespace eb
+
+// ---------------------------------------------------------------------------
+// Routing + loads for callers that cannot allocate device memory.
+//
+// The step path keeps its per-(micro-batch, chunk, expert) counts in the
+// caller's workspace.  Some callers cannot provide one: a serving process
+// whose device memory is fixed once at start-up (a pre-reserved pool, or an
+// allocator that refuses new cudaMalloc after warm-up), or a caller that must
+// not call cudaMalloc / cudaFree because they can synchronise the device and
+// stall work on other streams.  eb_route_loads_static serves them: the counts
+// live in the file-scope array below, which every GPU that loads this library
+// holds (4 MiB) until the process exits.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace eb {
+namespace {
+
+constexpr long long kStaticCountInts = 1ll << 20;  // 4 MiB of int32 counts
+static __device__ __align__(256) int32_t g_static_counts[kStaticCountInts];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+int32_t* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_counts on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up with
+// cudaGetSymbolAddress once per device (with that device current) and cached.
+cudaError_t static_counts_ptr(int32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_static_mu);
+  if (!g_static_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_counts);
+    if (e != cudaSuccess) return e;
+    g_static_ptr[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_static_ptr[dev];
+  return cudaSuccess;
+}
+
+// CTA (c, j): chunk c of micro-batch j of logits [n_mb, T, E]; writes every
+// count of its (j, c) row, so nothing in the scratch needs to start at zero.
+template <int VPL>
+__global__ void __launch_bounds__(1024) k_route_counts_static(const float* __restrict__ logits,
+                                                              int T, int E, int k, int renorm, int NC,
+                                                              int32_t* __restrict__ idx,
+                                                              float* __restrict__ gate,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ status) {
+  const int c = blockIdx.x, j = blockIdx.y;
+  __shared__ int hist_s[EB_MAX_ETOT];
+  __shared__ int bad;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist_s[e] = 0;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+  const int t0 = c * kChunk, t1 = min(T, t0 + kChunk);
+  bool nonfinite = false;
+  route_chunk<VPL>(logits + (size_t)j * T * E, t0, t1, E, k, renorm, idx + (size_t)j * T * k,
+                   gate + (size_t)j * T * k, hist_s, nonfinite);
+  if (nonfinite) bad = 1;
+  __syncthreads();
+  int32_t* out = counts + ((size_t)j * NC + c) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) out[e] = hist_s[e];
+  if (threadIdx.x == 0 && bad && status) atomicExch(status, EB_ERR_NONFINITE);
+}
+
+// w[j][d] = sum over chunks and over the contiguous expert block of rank d.
+__global__ void k_fold_static(const int32_t* __restrict__ counts, int n_mb, int NC, int E, int D,
+                              int32_t* __restrict__ w) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_mb * D) return;
+  const int j = i / D, dd = i % D, per = E / D;
+  int s = 0;
+  for (int ch = 0; ch < NC; ++ch) {
+    const int32_t* row = counts + ((size_t)j * NC + ch) * E;
+    for (int e = dd * per; e < (dd + 1) * per; ++e) s += row[e];
+  }
+  w[i] = s;
+}
+
+}  // namespace
+}  // namespace eb
+
+extern "C" eb_status eb_route_loads_static(const float* logits, int n_mb, int T, int E, int k,
+                                           int renorm, int D, int32_t* idx, float* gate,
+                                           int32_t* w, int32_t* status_dev, void* stream) {
+  using namespace eb;
+  if (n_mb < 1 || T < 1 || E < 1 || k < 1 || k > E || D < 1 || E % D != 0)
+    return EB_ERR_INVALID_ARG;
+  if (!logits || !idx || !gate || !w) return EB_ERR_INVALID_ARG;
+  if (E > EB_MAX_ETOT || k > EB_MAX_K || n_mb > 65535) return EB_ERR_UNSUPPORTED;
+  const int NC = (T + kChunk - 1) / kChunk;
+  if ((long long)n_mb * NC * E > kStaticCountInts) return EB_ERR_TOO_LARGE;
+  int32_t* counts = nullptr;
+  if (static_counts_ptr(&counts) != cudaSuccess) return EB_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  dim3 grid(NC, n_mb);
+  switch (vpl_for(E)) {
+    case 1: k_route_counts_static<1><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    case 2: k_route_counts_static<2><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    case 4: k_route_counts_static<4><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    default: k_route_counts_static<8><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
+  const int n = n_mb * D;
+  k_fold_static<<<(n + 255) / 256, 256, 0, s>>>(counts, n_mb, NC, E, D, w);
+  return cudaGetLastError() == cudaSuccess ? EB_OK : EB_ERR_CUDA;
+}

@@ -43,6 +43,7 @@ typedef int eb_status;
 #define EB_ERR_CUDA (-4)        /* a CUDA runtime call failed                */
 #define EB_ERR_TIMEOUT (-5)     /* a bounded device-side wait expired        */
 #define EB_ERR_WORKSPACE (-6)   /* workspace smaller than eb_workspace_size  */
+#define EB_ERR_TOO_LARGE (-7)   /* beyond the fixed capacity of a no-allocation call */
 
 /* RunSet policies, [EB] §4.2 and §5.2. */
 #define EB_SCHED_CUMUTIL 0  /* O(n) scan: add j iff U(S+{j}) > U(S)          */
@@ -211,6 +212,34 @@ eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* s
  * sum_{j in RunSet} max_d w_j).  If |S| <= m the RunSet is S. */
 eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int m, int policy,
                       uint32_t* runset_mask, int64_t* step_stats, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * No-allocation routing + loads.  The paper has no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- a serving
+ * process whose memory is fixed at start-up (a pre-reserved pool, or an
+ * allocator that refuses cudaMalloc after warm-up), or a caller that must
+ * not call cudaMalloc / cudaFree because they can synchronise the device.
+ *
+ * Routes n_mb independent micro-batches (as eb_route does for each) and folds
+ * their expert counts into virtual-rank loads (as eb_loads does):
+ *   logits [n_mb, T, E] float32 -> idx [n_mb, T, k] int32,
+ *   gate [n_mb, T, k] float32, w [n_mb, D] int32 (contiguous map).
+ * status_dev: optional device int32, set to EB_ERR_NONFINITE on a NaN/Inf.
+ * The caller passes inputs and outputs; the intermediate per-(micro-batch,
+ * 64-token chunk, expert) counts live in a file-scope device array of
+ * 2^20 int32 (4 MiB) that every GPU loading the library holds until exit.
+ * n_mb * ceil(T / 64) * E above 2^20 returns EB_ERR_TOO_LARGE before any
+ * launch.  The call allocates nothing (no cudaMalloc, cudaFree or allocating
+ * library routine).  Its first call on a device looks the array's device
+ * address up (cudaGetSymbolAddress) and caches it: make that first call
+ * before any stream capture.  Every call shares the one array: calls that
+ * overlap on the GPU (other streams, other threads) race on it, so order
+ * them on one stream.  Each call writes every count it reads, so stale
+ * contents from an earlier call never leak into a result.
+ * ------------------------------------------------------------------------ */
+eb_status eb_route_loads_static(const float* logits, int n_mb, int T, int E, int k, int renorm,
+                                int D, int32_t* idx, float* gate, int32_t* w, int32_t* status_dev,
+                                void* stream);
 
 #ifdef __cplusplus
 }

@@ -41,6 +41,9 @@ def parse():
     p.add_argument("--policy", default="maxutil", choices=list(POLICY_NAMES.values()))
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-under-util", action="store_true")
+    p.add_argument("--layers", type=int, default=0,
+                   help="override the workload's MoE layer count (small profiling cases)")
     return p.parse_args()
 
 
@@ -160,6 +163,8 @@ def run_ours(args, world, rank, local):
     barrier(world)
     eb.load()
     wl = synth.get(args.workload)
+    if args.layers:
+        wl = wl.replace(L=args.layers)
     policy = {v: k for k, v in POLICY_NAMES.items()}[args.policy]
     dev = torch.device("cuda", torch.cuda.current_device())
     logits_np = synth.logits(wl)
@@ -175,7 +180,7 @@ def run_ours(args, world, rank, local):
 
     # exact under-utilisation of every policy (routing + scheduling only)
     under = {}
-    for pol, name in POLICY_NAMES.items():
+    for pol, name in ([] if args.no_under_util else POLICY_NAMES.items()):
         c = eb.Context(cfg_for(pol, compute=0))
         c.eb_episode(logits, None, None, None)
         num, den, den_sep = c.eb_utilization()
@@ -289,6 +294,7 @@ def run_ours(args, world, rank, local):
             "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded Dirichlet task-profile routing skew; N(0,0.02) weights)",
+            "workload_layers": wl.L,
             "config": {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
                                    f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",
                        "policy": args.policy, "m": wl.m_default, "step": "one Algorithm-1 episode",

@@ -34,7 +34,8 @@ GEMM_AUTO, GEMM_TC, GEMM_SIMT = 0, 1, 2
 EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_create", "eb_destroy",
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
-            "eb_profile_read", "eb_launch_count", "eb_route_loads_static"]
+            "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
+            "eb_selftest_timeout"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine")
 
@@ -84,6 +85,7 @@ def load() -> ctypes.CDLL:
         "eb_profile_read": (I, [P, P, P]),
         "eb_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
         "eb_route_loads_static": (I, [P, I, I, I, I, I, I, P, P, P, P, P]),
+        "eb_selftest_timeout": (I, [ctypes.c_int64, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -163,6 +165,13 @@ def eb_route_loads_static(logits, k: int, renorm: bool, D: int, idx, gate, w, st
     _check(load().eb_route_loads_static(_ptr(logits), n_mb, T, E, k, int(renorm), D, _ptr(idx),
                                         _ptr(gate), _ptr(w), _ptr(status), _stream(stream)),
            "eb_route_loads_static")
+
+
+def eb_selftest_timeout(limit_ns: int, status, stream=None) -> None:
+    """Runs the GEMMs' bounded device wait on a barrier nothing arrives on;
+    `status` (1-element int32 device tensor) receives EB_ERR_TIMEOUT."""
+    _check(load().eb_selftest_timeout(int(limit_ns), _ptr(status), _stream(stream)),
+           "eb_selftest_timeout")
 
 
 class Context:

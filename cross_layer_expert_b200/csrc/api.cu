@@ -270,8 +270,8 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   cudaError_t e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, logits, s); });
   if (e == cudaSuccess)
     e = timed(x, 1, 1, s, [&] {
-      return launch_schedule_step(x->d, x->dev, w, tc ? kTcRows : kSimtRows,
-                                  tc ? kTcFeat : kSimtFeat, s);
+      return launch_schedule_step(x->d, x->dev, w, tc ? kTcRows1 : kSimtRows,
+                                  tc ? kTcRows2 : kSimtRows, tc ? kTcFeat : kSimtFeat, s);
     });
   if (c.compute) {
     if (e == cudaSuccess)
@@ -418,6 +418,12 @@ eb_status eb_sync_status(eb_ctx* x) {
   if (cudaMemcpy(&status, &x->dev.st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return EB_ERR_CUDA;
   return status;
+}
+
+eb_status eb_selftest_timeout(int64_t limit_ns, int32_t* status_dev, void* stream) {
+  if (!status_dev || limit_ns < 1000 || limit_ns > 2000000000ll) return EB_ERR_INVALID_ARG;
+  return cuda_status(launch_selftest_wait((unsigned long long)limit_ns, status_dev,
+                                          (cudaStream_t)stream));
 }
 
 eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t* idx, float* gate,

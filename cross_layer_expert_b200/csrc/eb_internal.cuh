@@ -15,13 +15,17 @@ namespace eb {
 // fixed base row, so the permutation is deterministic.
 constexpr int kChunk = 64;
 
-// Sizes of GEMM work items: RN token rows per item and FM output features per
-// item (the tcgen05 tile is 128 features x kTcRows tokens; the SIMT tile
-// 64 x 64).
-#ifndef EB_TC_ROWS
-#define EB_TC_ROWS 128
+// Sizes of GEMM work items: token rows per item and output features per item.
+// The tcgen05 tiles are 128 features x kTcRows1 tokens (gate/up GEMM) and
+// 128 features x kTcRows2 tokens (down GEMM); the SIMT tile is 64 x 64.
+#ifndef EB_TC_ROWS1
+#define EB_TC_ROWS1 128
 #endif
-constexpr int kTcRows = EB_TC_ROWS;
+#ifndef EB_TC_ROWS2
+#define EB_TC_ROWS2 256
+#endif
+constexpr int kTcRows1 = EB_TC_ROWS1;
+constexpr int kTcRows2 = EB_TC_ROWS2;
 constexpr int kTcFeat = 128;
 constexpr int kSimtRows = 64;
 constexpr int kSimtFeat = 64;
@@ -91,8 +95,9 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               cudaStream_t s);
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
                               float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
-cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn, int fm,
-                                 cudaStream_t s);
+// rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm: features per item.
+cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
+                                 int fm, cudaStream_t s);
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
                                  int policy, uint32_t* runset, long long* stats, cudaStream_t s);
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s);

@@ -31,12 +31,10 @@ namespace eb {
 namespace {
 
 constexpr int kBM = 128;        // weight rows (features) per MMA tile
-constexpr int kBN = kTcRows;    // token rows per item (max MMA N)
 constexpr int kBK = 64;         // K elements per stage: 128 bytes of bf16 = one swizzle row
 constexpr int kTileBytes = kBM * kBK * 2;  // 16 KiB
-constexpr int kXBytes = kBN * kBK * 2;     // 16 or 32 KiB
 #ifndef EB_EPI_WARPS
-#define EB_EPI_WARPS 4
+#define EB_EPI_WARPS 8
 #endif
 constexpr int kEpiWarps = EB_EPI_WARPS;    // 4 or 8: warps draining TMEM
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -79,14 +77,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 // (and raises the CTA's abort flag) if it does not within the limit, or if
 // another role of the CTA has aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (*abort_flag) return false;
-      if (global_ns() - t0 > kWaitLimitNs) {
+      if (global_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         atomicCAS(status, EB_OK, EB_ERR_TIMEOUT);
         return false;
@@ -196,9 +195,13 @@ struct Item {
 };
 
 template <bool GATEUP>
+struct Cfg;
+
+template <bool GATEUP>
 __device__ __forceinline__ Item decode(const Dims& d, const int32_t* seg_rows,
                                        const int32_t* seg_wid, const int32_t* seg_items,
                                        int nseg, int item) {
+  constexpr int kBN = Cfg<GATEUP>::kBN;
   const int s = find_segment(seg_items, nseg, item);
   const int local = item - seg_items[s];
   const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
@@ -214,6 +217,8 @@ __device__ __forceinline__ Item decode(const Dims& d, const int32_t* seg_rows,
 
 template <bool GATEUP>
 struct Cfg {
+  static constexpr int kBN = GATEUP ? kTcRows1 : kTcRows2;  // token rows per item (max MMA N)
+  static constexpr int kXBytes = kBN * kBK * 2;              // 16 or 32 KiB
   static constexpr int kStageBytes = (GATEUP ? 2 : 1) * kTileBytes + kXBytes;
   static constexpr int kStages = (196608 / kStageBytes) < 8 ? (196608 / kStageBytes) : 8;
   static constexpr int kAccCols = (GATEUP ? 2 : 1) * kBN;  // TMEM columns per accumulator
@@ -231,6 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
               __nv_bfloat16* __restrict__ out) {
   using C = Cfg<GATEUP>;
+  constexpr int kBN = C::kBN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -440,7 +446,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Failure-detection self-test: waits, with the GEMM's bounded wait, on an
+// mbarrier nothing ever arrives on; the wait expires after limit_ns and
+// leaves EB_ERR_TIMEOUT in *status.  Nothing faults and the context stays
+// usable.
+__global__ void k_selftest_wait(unsigned long long limit_ns, int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns))
+    atomicExch(status, EB_OK);  // not reached: nothing arrives on the barrier
+}
+
 }  // namespace
+
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s) {
+  k_selftest_wait<<<1, 32, 0, s>>>(limit_ns, status);
+  return cudaGetLastError();
+}
 
 int gemm_tc_smem_bytes(bool gateup) {
   return gateup ? Cfg<true>::kSmemBytes : Cfg<false>::kSmemBytes;
@@ -513,8 +541,8 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   const unsigned long long experts = (unsigned long long)d.L * d.Etot;
   cudaError_t e = encode(&maps->w_gateup, w_gateup, experts * 2 * d.F, d.H, kBM);
   if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F, kBM);
-  if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H, kBN);
-  if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kBN);
+  if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H, kTcRows1);
+  if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kTcRows2);
   return e;
 }
 

@@ -23,6 +23,8 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
 // Opts the kernels into their dynamic shared memory (once per device).
 cudaError_t gemm_tc_prepare();
 int gemm_tc_smem_bytes(bool gateup);
+// Runs the GEMM's bounded mbarrier wait on a barrier nothing arrives on.
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) of a step; grid = persistent
 // CTAs (one per SM).
 cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,

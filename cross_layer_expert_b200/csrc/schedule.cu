@@ -279,12 +279,24 @@ struct PlanSmem {
   int tmp[33];
 };
 
-__global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn,
-                                                             int fm) {
+__global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
+                                                             int rn2, int fm) {
   __shared__ SchedSmem sm;
   __shared__ PlanSmem pl;
-  State* st = c.st;
+  // the step state lives in shared memory for the whole kernel (thread 0's
+  // bookkeeping would otherwise be a chain of dependent global loads)
+  __shared__ State ss;
+  State* st = &ss;
   const int tid = threadIdx.x;
+  constexpr int kStateWords = sizeof(State) / sizeof(int);
+  for (int i = tid; i < kStateWords; i += blockDim.x)
+    reinterpret_cast<int*>(&ss)[i] = reinterpret_cast<const int*>(c.st)[i];
+  __syncthreads();
+  auto write_back = [&]() {
+    __syncthreads();
+    for (int i = tid; i < kStateWords; i += blockDim.x)
+      reinterpret_cast<int*>(c.st)[i] = reinterpret_cast<const int*>(&ss)[i];
+  };
   const uint32_t need = st->need_route;
   // 1. fold fresh chunk counts into hist[j][:] and loads w[j][:]
   for (int i = tid; i < d.M * d.E; i += blockDim.x) {
@@ -325,6 +337,7 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
       st->rows = 0;
       for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
     }
+    write_back();
     return;
   }
   for (int i = tid; i < sm.n * d.D; i += blockDim.x) {
@@ -404,7 +417,10 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     st->n_groups = G;
     st->nseg = G * d.Etot;
   }
-  if (!d.compute) return;
+  if (!d.compute) {
+    write_back();
+    return;
+  }
   __syncthreads();
   // 5. segment plan: rows of (group, expert) are counted into seg_rows and
   //    scanned in place; GEMM work items per segment likewise.
@@ -422,11 +438,10 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
       if (st->group_of[j] != g) continue;
       cnt += (e < d.E) ? c.hist[j * d.E + e] : d.T;
     }
-    const int nch = (cnt + rn - 1) / rn;
     my_nonempty += cnt > 0;
     wk.seg_rows[i] = cnt;
-    wk.seg_items1[i] = nch * mb1;
-    wk.seg_items2[i] = nch * mb2;
+    wk.seg_items1[i] = (cnt + rn1 - 1) / rn1 * mb1;
+    wk.seg_items2[i] = (cnt + rn2 - 1) / rn2 * mb2;
     wk.seg_wid[i] = st->group_layer[g] * Et + e;
   }
   if (my_nonempty) atomicAdd(&s_nonempty, my_nonempty);
@@ -463,6 +478,7 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
                            : min(kChunk, d.T - ch * kChunk);
     }
   }
+  write_back();
 }
 
 __global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __restrict__ w,
@@ -561,9 +577,9 @@ unsigned long long maxutil_candidates(int n, int m) {
   return total;
 }
 
-cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn, int fm,
-                                 cudaStream_t s) {
-  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn, fm);
+cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
+                                 int fm, cudaStream_t s) {
+  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn1, rn2, fm);
   return cudaGetLastError();
 }
 

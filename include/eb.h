@@ -184,6 +184,14 @@ eb_status eb_profile(eb_ctx* ctx, int enable);
 eb_status eb_profile_read(eb_ctx* ctx, double* ms, int64_t* launches);
 eb_status eb_launch_count(eb_ctx* ctx, int64_t* n);
 
+/* Failure-detection self-test (the pages describe no failure handling).  Every
+ * device-side wait of the tensor-core GEMMs is bounded; when one expires the
+ * kernel records EB_ERR_TIMEOUT, finishes its own copies, frees its TMEM and
+ * returns instead of hanging.  This call runs that same bounded wait on a
+ * barrier nothing ever arrives on, with a limit of limit_ns nanoseconds
+ * (1e3..2e9), and leaves EB_ERR_TIMEOUT in the device int32 *status_dev. */
+eb_status eb_selftest_timeout(int64_t limit_ns, int32_t* status_dev, void* stream);
+
 /* Waits for the context's work and returns the device-side status. */
 eb_status eb_sync_status(eb_ctx* ctx);
 

@@ -163,7 +163,7 @@ def schedule(policy: int, pending: Sequence[int], w: dict, m: int) -> List[int]:
     return SCHEDULERS[policy](pending, w, m)
 
 
-def run_episode(loads_all: np.ndarray, policy: int, m: int):
+def run_episode(loads_all: np.ndarray, policy: int, m: int, maxutil_impl=None):
     """Algorithm 1 of [EB] §4.2 over pre-routed workloads.
 
     loads_all[j, l] is the D-vector w of micro-batch j at MoE layer l (the
@@ -172,6 +172,9 @@ def run_episode(loads_all: np.ndarray, policy: int, m: int):
     Start: l_j = 0 and S_0 = all micro-batches.  Each step picks
     RunSet_i = Schedule(S_{i-1}, m), runs it, advances l_j for j in the RunSet
     and drops the micro-batches that reached l_max.  Stops when S is empty.
+
+    maxutil_impl optionally replaces the Python MaxUtil enumeration by another
+    implementation of the same definition (oracle.native.maxutil, plain C).
 
     Returns a dict with the per-step list of (runset, layers, sumW, maxW,
     summax) and the episode totals num = sum sumW, den = D sum maxW (the
@@ -187,7 +190,10 @@ def run_episode(loads_all: np.ndarray, policy: int, m: int):
     while S:
         pending = sorted(S)
         w = {j: [int(x) for x in loads_all[j, layer[j]]] for j in pending}
-        run = schedule(policy, pending, w, m)
+        if policy == MAXUTIL and maxutil_impl is not None:
+            run = maxutil_impl(pending, w, m)
+        else:
+            run = schedule(policy, pending, w, m)
         if not run:
             raise RuntimeError("empty RunSet")
         W = combined([w[j] for j in run])

@@ -41,10 +41,15 @@ class Inputs:
         else:
             self.w_gateup = self.w_down = None
         self._cache = {}
+        self._cache_layer = None
 
     def expert(self, l: int, e: int):
-        """(w_gate [F,H], w_up [F,H], w_down [H,F]) float64 on the host."""
+        """(w_gate [F,H], w_up [F,H], w_down [H,F]) float64 on the host (only
+        the current layer's experts are kept)."""
         key = (l, e)
+        if l != self._cache_layer:
+            self._cache = {}
+            self._cache_layer = l
         if key not in self._cache:
             gu = self.w_gateup[l, e].float().cpu().numpy().astype(np.float64)
             dn = self.w_down[l, e].float().cpu().numpy().astype(np.float64)
@@ -70,10 +75,18 @@ def run_episode(inp: Inputs, policy: int, m: int = 0, gemm: int = 0):
     return hidden, rows, layers, util, steps
 
 
+def oracle_loads(inp: Inputs):
+    if getattr(inp, "_loads", None) is None:
+        wl = inp.wl
+        inp._loads = oracle.route_all(inp.logits_np, wl.k, wl.D)[3]
+    return inp._loads
+
+
 def oracle_episode(inp: Inputs, policy: int, m: int = 0):
+    from oracle import native
     wl = inp.wl
-    _, _, _, ld = oracle.route_all(inp.logits_np, wl.k, wl.D)
-    return oracle.run_episode(ld, policy, m or wl.m_default)
+    return oracle.run_episode(oracle_loads(inp), policy, m or wl.m_default,
+                              maxutil_impl=native.maxutil if wl.M > 12 else None)
 
 
 def check_schedule(rows, layers, util, steps, ref, M: int):

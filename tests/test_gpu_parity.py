@@ -124,15 +124,22 @@ def test_schedule_random_matches_oracle(torch, policy):
 
 
 def test_maxutil_m32_sampled(torch):
-    """MaxUtil at M = 32, m = 24 (about 15M complements per call) against the
-    oracle's enumeration of all admissible subsets."""
+    """MaxUtil at M = 32, m = 24 (about 15M admissible subsets per call)
+    against the oracle's exhaustive enumeration (plain C)."""
+    from oracle import native
     rng = np.random.default_rng(7)
-    for trial in range(2):
-        w = rng.integers(0, 200, size=(32, 8))
+    for trial, D in enumerate((8, 16)):
+        w = rng.integers(0, 200, size=(32, D))
         mask, _ = _gpu_schedule(torch, w, 0xFFFFFFFF, 24, osch.MAXUTIL)
         pend = list(range(32))
-        ref = osch.maxutil(pend, {j: [int(x) for x in w[j]] for j in pend}, 24)
+        ref = native.maxutil(pend, {j: [int(x) for x in w[j]] for j in pend}, 24)
         assert mask == sum(1 << j for j in ref)
+    # a pending set with holes: 28 of 32
+    pend = [j for j in range(32) if j % 8 != 3]
+    w = rng.integers(0, 50, size=(32, 8))
+    mask, _ = _gpu_schedule(torch, w, sum(1 << j for j in pend), 22, osch.MAXUTIL)
+    ref = native.maxutil(pend, {j: [int(x) for x in w[j]] for j in pend}, 22)
+    assert mask == sum(1 << j for j in ref)
 
 
 # ------------------------------------------------------------------ episodes

@@ -391,3 +391,25 @@ def test_zero_work_sets_rank_lowest():
     assert osch.cumutil([0, 1, 2], w, 1) == [0, 1]
     # every set holding micro-batch 1 has U = 4/6; the largest one wins
     assert osch.maxutil([0, 1, 2], w, 1) == [0, 1, 2]
+
+
+def test_native_maxutil_matches_python():
+    """The plain-C exhaustive MaxUtil agrees with the Python one."""
+    from oracle import native
+    rng = np.random.default_rng(16)
+    for trial in range(300):
+        M = int(rng.integers(1, 11))
+        D = int(rng.integers(1, 9))
+        pending = sorted(rng.choice(M, size=int(rng.integers(1, M + 1)), replace=False).tolist())
+        hi = int(rng.choice([2, 5, 50]))
+        w = {j: [int(x) for x in rng.integers(0, hi, size=D)] for j in pending}
+        m = int(rng.integers(1, M + 1))
+        assert native.maxutil(pending, w, m) == osch.maxutil(pending, w, m), (pending, w, m)
+    # golden hand cases
+    for ln in _read_golden("cumutil_maxutil_hand.txt"):
+        head, ws, want = [x.strip() for x in ln.split("|")]
+        pol, m = head.split()
+        if pol != "maxutil":
+            continue
+        w = {j: [int(x) for x in v.split()] for j, v in enumerate(ws.split(";"))}
+        assert native.maxutil(sorted(w), w, int(m)) == [int(x) for x in want.split()]

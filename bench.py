@@ -398,10 +398,12 @@ def run_reference(args, world, rank):
     h0_np = synth.hidden(wl).astype(np.float64)
     if wl.dtype == "bf16":
         h0_np = torch.from_numpy(synth.hidden(wl)).to(torch.bfloat16).double().numpy()
+    sg, sd = ((3.0 * wl.H) ** -0.5, (3.0 * wl.F) ** -0.5) if wl.w_init == "fan_in" else (wl.w_std,) * 2
+
     def fetch(l, e):  # one expert's weights drawn on the host
         g = torch.Generator().manual_seed((wl.seed * 7919 + l * 1009 + e) & 0x7FFFFFFF)
-        gu = (torch.randn((2 * wl.F, wl.H), generator=g) * 0.02).to(torch.bfloat16).float().numpy()
-        dn = (torch.randn((wl.H, wl.F), generator=g) * 0.02).to(torch.bfloat16).float().numpy()
+        gu = (torch.randn((2 * wl.F, wl.H), generator=g) * sg).to(torch.bfloat16).float().numpy()
+        dn = (torch.randn((wl.H, wl.F), generator=g) * sd).to(torch.bfloat16).float().numpy()
         return gu[:wl.F], gu[wl.F:], dn
 
     times, detail = [], ""

@@ -14,7 +14,7 @@ experts, top-6, hidden 2048, expert FFN 1408).  The paper measures on
 LongBench's 13 tasks with trained weights; neither is available here, so
 seeded Dirichlet / Zipf "task profiles" stand in for the tasks' routing skew
 (the paper's Fig. 7 shows the skew is task- and layer-dependent) and weights
-are N(0, 0.02).
+are random (below).
 
 Logit recipes (noise is always N(0,1) per (micro-batch, layer, token, expert)):
 
@@ -31,6 +31,12 @@ Logit recipes (noise is always N(0,1) per (micro-batch, layer, token, expert)):
                      seeded permutation rolled by floor(l / 4) * (E / D)
                      positions: the hot set moves by one virtual rank every
                      4 layers.
+
+Weights: ``w_init="normal"`` draws N(0, w_std^2) (the stated N(0, 0.02) of
+the tiny and Moonlight-shaped stacks); ``w_init="fan_in"`` draws
+N(0, 1 / (3 fan_in)) per matrix -- the variance of a linear layer's default
+initialisation -- for stacks whose description says only "random-init
+weights" (Qwen3-shaped ones).
 """
 from __future__ import annotations
 
@@ -65,6 +71,8 @@ class Workload:
     zipf_s: float = 1.2
     n_profiles: int = 13
     compute: bool = True  # False: routing and scheduling only (no expert FFN)
+    w_init: str = "normal"  # "normal": N(0, w_std^2); "fan_in": N(0, 1/(3 fan_in))
+    w_std: float = 0.02
     seed: int = BASE_SEED
 
     @property
@@ -89,13 +97,13 @@ WORKLOADS = {
                                alpha=0.3),
     # Qwen3-30B-A3B shape: the throughput workload
     "qwen3_bf16": Workload("qwen3_bf16", L=48, E=128, k=8, H=2048, F=768, D=8, M=8,
-                           T=1024, profile="task_profiles", alpha=0.2),
+                           T=1024, profile="task_profiles", alpha=0.2, w_init="fan_in"),
     # routing + scheduling only sweep at the Qwen3-30B shape (D and M vary)
     "sweep": Workload("sweep", L=48, E=128, k=8, H=2048, F=768, D=8, M=8, T=256,
                       profile="sweep_profiles", compute=False),
     # long-context prefill at the Qwen3-30B shape
     "longctx_bf16": Workload("longctx_bf16", L=48, E=128, k=8, H=2048, F=768, D=8,
-                             M=8, T=8192, profile="zipf_rotating", zipf_s=1.5),
+                             M=8, T=8192, profile="zipf_rotating", zipf_s=1.5, w_init="fan_in"),
     # small cases the oracle finishes in seconds; several GEMM tiles and a
     # ragged token tail (T not a multiple of 64 or 128)
     "small_bf16": Workload("small_bf16", L=6, E=16, k=4, H=256, F=384, D=4, M=4,
@@ -175,8 +183,8 @@ def logits(w: Workload, episode: int = 0, mbs: Optional[range] = None,
     return out
 
 
-def hidden(w: Workload, episode: int = 0) -> np.ndarray:
-    """Initial hidden states h_0 [M, T, H] float32 drawn from N(0, 1).
+def hidden(w: Workload, episode: int = 0, scale: float = 1.0) -> np.ndarray:
+    """Initial hidden states h_0 [M, T, H] float32 drawn from N(0, scale^2).
 
     For bf16 workloads the caller converts to bfloat16 (the stored input).
     """
@@ -184,18 +192,21 @@ def hidden(w: Workload, episode: int = 0) -> np.ndarray:
     for j in range(w.M):
         out[j] = _rng(w.seed, _TAG_HIDDEN, episode, j).standard_normal((w.T, w.H),
                                                                       dtype=np.float32)
+    if scale != 1.0:
+        out *= np.float32(scale)
     return out
 
 
-def hidden_torch(w: Workload, episode: int = 0):
+def hidden_torch(w: Workload, episode: int = 0, scale: float = 1.0):
     """h_0 as a torch CPU tensor in the workload's storage type."""
     import torch
-    t = torch.from_numpy(hidden(w, episode))
+    t = torch.from_numpy(hidden(w, episode, scale))
     return t.to(torch.bfloat16) if w.dtype == "bf16" else t
 
 
-def weights_torch(w: Workload, device="cpu", std: float = 0.02):
-    """Expert weights N(0, std^2) as torch tensors on `device`.
+def weights_torch(w: Workload, device="cpu"):
+    """Expert weights as torch tensors on `device` (see the module docstring
+    for the two initialisations).
 
     Returns (w_gateup [L, E_tot, 2F, H], w_down [L, E_tot, H, F]).  Along the
     2F axis the first F rows are the gate projection and the next F the up
@@ -206,13 +217,17 @@ def weights_torch(w: Workload, device="cpu", std: float = 0.02):
     import torch
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Et = w.E_tot
+    if w.w_init == "fan_in":
+        std_gu, std_dn = (3.0 * w.H) ** -0.5, (3.0 * w.F) ** -0.5
+    else:
+        std_gu = std_dn = w.w_std
     gu = torch.empty((w.L, Et, 2 * w.F, w.H), dtype=dt, device=device)
     dn = torch.empty((w.L, Et, w.H, w.F), dtype=dt, device=device)
     for l in range(w.L):
         g = torch.Generator(device=device)
         g.manual_seed((w.seed * 1000003 + _TAG_WEIGHTS * 7919 + l) & 0x7FFFFFFFFFFF)
         gu[l] = (torch.randn((Et, 2 * w.F, w.H), generator=g, device=device,
-                             dtype=torch.float32) * std).to(dt)
+                             dtype=torch.float32) * std_gu).to(dt)
         dn[l] = (torch.randn((Et, w.H, w.F), generator=g, device=device,
-                             dtype=torch.float32) * std).to(dt)
+                             dtype=torch.float32) * std_dn).to(dt)
     return gu, dn

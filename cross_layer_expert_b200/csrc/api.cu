@@ -22,6 +22,7 @@ struct eb_ctx {
   int device = 0;
   int num_sms = 148;
   bool use_tc = false;
+  bool pair1 = false, pair2 = false;  // GEMM 1 / GEMM 2 on the two-SM engine
   cudaStream_t last_stream = nullptr;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
@@ -48,7 +49,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool use_tc_for(const eb_config& c) {
   if (c.dtype != EB_DTYPE_BF16) return false;
-  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC;
+  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC || c.gemm == EB_GEMM_TC2;
 }
 
 Dims make_dims(const eb_config& c) {
@@ -80,7 +81,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   x.chunk_hist = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
   const size_t nseg = M * (size_t)d.Etot;
   if (c.compute) {
-    x.base = (int32_t*)take(sizeof(int32_t) * M * d.NC * d.Etot);
+    x.prior = (int32_t*)take(sizeof(int32_t) * M * d.Etot);
     x.pos = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
     x.seg_rows = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.seg_wid = (int32_t*)take(sizeof(int32_t) * nseg);
@@ -154,7 +155,7 @@ eb_status eb_config_check(const eb_config* c) {
   if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
   if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
   if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
-  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_SIMT) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TC2) return EB_ERR_INVALID_ARG;
   if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
@@ -166,10 +167,12 @@ eb_status eb_config_check(const eb_config* c) {
     const int vec = c->dtype == EB_DTYPE_BF16 ? 8 : 4;  // 16-byte rows
     if (c->H % vec != 0) return EB_ERR_UNSUPPORTED;
     if ((long long)c->M * c->T * (c->k + c->n_shared) > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
-    if (c->dtype == EB_DTYPE_F32 && c->gemm == EB_GEMM_TC) return EB_ERR_UNSUPPORTED;
+    if (c->dtype == EB_DTYPE_F32 && (c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2))
+      return EB_ERR_UNSUPPORTED;
     if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
-      if (c->gemm == EB_GEMM_TC) return EB_ERR_UNSUPPORTED;
+      if (c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2) return EB_ERR_UNSUPPORTED;
     }
+    if (c->gemm == EB_GEMM_TC2 && (c->H % 256 != 0 || c->F % 256 != 0)) return EB_ERR_UNSUPPORTED;
   }
   return EB_OK;
 }
@@ -193,6 +196,10 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   x->use_tc = use_tc_for(*c) && c->H % 128 == 0 && c->F % 128 == 0;
   cudaError_t e = cudaGetDevice(&x->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&x->num_sms, cudaDevAttrMultiProcessorCount, x->device);
+  // the two-SM engine covers 256 output features per item
+  const bool pairs_ok = x->use_tc && c->gemm != EB_GEMM_TC && x->num_sms >= 2;
+  x->pair1 = pairs_ok && c->F % kTc2Feat == 0;
+  x->pair2 = pairs_ok && c->H % kTc2Feat == 0;
   const size_t n_state = align_up(sizeof(State));
   const size_t n_hist = align_up(sizeof(int32_t) * c->M * c->E);
   const size_t n_w = align_up(sizeof(int32_t) * c->M * c->D);
@@ -267,20 +274,28 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     x->map_keys[1] = wdn;
     x->map_keys[2] = workspace;
   }
+  const bool p1 = tc && x->pair1, p2 = tc && x->pair2;
+  const int rn1 = !tc ? kSimtRows : p1 ? kTc2Rows1 : kTcRows1;
+  const int rn2 = !tc ? kSimtRows : p2 ? kTc2Rows2 : kTcRows2;
+  const int fm1 = !tc ? kSimtFeat : p1 ? kTc2Feat : kTcFeat;
+  const int fm2 = !tc ? kSimtFeat : p2 ? kTc2Feat : kTcFeat;
   cudaError_t e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, logits, s); });
   if (e == cudaSuccess)
-    e = timed(x, 1, 1, s, [&] {
-      return launch_schedule_step(x->d, x->dev, w, tc ? kTcRows1 : kSimtRows,
-                                  tc ? kTcRows2 : kSimtRows, tc ? kTcFeat : kSimtFeat, s);
-    });
+    e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
   if (c.compute) {
     if (e == cudaSuccess)
       e = timed(x, 2, 1, s, [&] { return launch_permute(x->d, x->dev, w, hidden, s); });
     if (e == cudaSuccess) {
       if (tc) {
-        e = timed(x, 3, 1, s, [&] { return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 1); });
+        e = timed(x, 3, 1, s, [&] {
+          return p1 ? launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, 1)
+                    : launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 1);
+        });
         if (e == cudaSuccess)
-          e = timed(x, 4, 1, s, [&] { return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 2); });
+          e = timed(x, 4, 1, s, [&] {
+            return p2 ? launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, 2)
+                      : launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 2);
+          });
       } else {
         e = timed(x, 3, 1, s, [&] { return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, 1); });
         if (e == cudaSuccess)

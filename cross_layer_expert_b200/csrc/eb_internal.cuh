@@ -26,6 +26,10 @@ constexpr int kChunk = 64;
 #endif
 constexpr int kTcRows1 = EB_TC_ROWS1;
 constexpr int kTcRows2 = EB_TC_ROWS2;
+// Two-SM tiles: 256 features x kTc2Rows tokens per CTA pair.
+constexpr int kTc2Rows1 = 128;
+constexpr int kTc2Rows2 = 256;
+constexpr int kTc2Feat = 256;
 constexpr int kTcFeat = 128;
 constexpr int kSimtRows = 64;
 constexpr int kSimtFeat = 64;
@@ -68,8 +72,8 @@ struct Dims {
 struct Work {
   int32_t* idx;        // [M][T][k]
   float* gate;         // [M][T][k]
-  int32_t* chunk_hist; // [M][NC][E]
-  int32_t* base;       // [M][NC][Etot]: first row of (j, chunk, expert)
+  int32_t* chunk_hist; // [M][NC][E]: counts of each 64-token chunk
+  int32_t* prior;      // [M][Etot]: rows of (j's segment, expert) taken by earlier RunSet members
   int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
   int32_t* seg_rows;   // [M*Etot + 1]
   int32_t* seg_wid;    // [M*Etot]: layer * Etot + expert
@@ -84,8 +88,8 @@ struct Work {
 // Device state owned by a context.
 struct CtxDev {
   State* st;
-  int32_t* hist;        // [M][E]: counts of micro-batch j at layer l_j
-  int32_t* w;           // [M][D]
+  int32_t* hist;        // [M][E]: counts of micro-batch j at layer l_j (accumulated by routing)
+  int32_t* w;           // [M][D]: loads of micro-batch j at layer l_j (accumulated by routing)
   long long* trace;     // [max_steps][kTraceCols]
   int32_t* trace_layers;  // [max_steps][M]
 };
@@ -95,9 +99,10 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               cudaStream_t s);
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
                               float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
-// rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm: features per item.
+// rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm1 / fm2:
+// output features per item.
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
-                                 int fm, cudaStream_t s);
+                                 int fm1, int fm2, cudaStream_t s);
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
                                  int policy, uint32_t* runset, long long* stats, cudaStream_t s);
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s);

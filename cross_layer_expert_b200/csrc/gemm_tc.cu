@@ -463,6 +463,323 @@ __global__ void k_selftest_wait(unsigned long long limit_ns, int* status) {
     atomicExch(status, EB_OK);  // not reached: nothing arrives on the barrier
 }
 
+
+// ---------------------------------------------------------------------------
+// Two-SM variant (tcgen05 cta_group::2).  A cluster of two CTAs on an SM pair
+// computes one 256-feature x N-token tile: CTA r holds weight rows
+// [f0 + 128 r, f0 + 128 r + 128) and token rows [r0 + r N/2, r0 + (r+1) N/2)
+// of the operands, the leader CTA (rank 0) issues the M = 256 MMAs, and each
+// CTA's TMEM receives its 128 feature rows x all N tokens.  Each SM therefore
+// fetches only half of the token tile: per output, 1.2x (gate/up) to 1.5x
+// (down) fewer bytes cross L2 -> SM than the one-SM kernel.
+//
+// Barriers: the leader arms its full barrier with both CTAs' bytes and both
+// CTAs' TMA loads complete on it; the leader's commits arrive on the empty
+// and accumulator-full barriers of both CTAs (multicast commit); each CTA's
+// drain warps arrive on the leader's accumulator-empty barrier.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t num_clusters() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+  return r;
+}
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+  return out;
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose completion is counted on the
+// leader CTA's barrier (bar = that barrier's shared::cluster address).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
+                                              uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
+}
+// Arrives on the barrier at this shared-memory offset in both CTAs of the pair
+// once the leader's earlier MMAs have completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  const uint16_t mask = 0x3;
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+template <bool GATEUP>
+struct Cfg2 {
+  static constexpr int kBN = GATEUP ? kTc2Rows1 : kTc2Rows2;  // token rows per pair item
+  static constexpr int kBNc = kBN / 2;                         // token rows per CTA
+  static constexpr int kXBytes = kBNc * kBK * 2;
+  static constexpr int kStageBytes = (GATEUP ? 2 : 1) * kTileBytes + kXBytes;  // per CTA
+  static constexpr int kStages = (204800 / kStageBytes) < 8 ? (204800 / kStageBytes) : 8;
+  static constexpr int kAccCols = (GATEUP ? 2 : 1) * kBN;
+  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
+  static constexpr int kTmemCols = kAccBufs * kAccCols;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 1024;
+};
+
+// One pair item: (segment, 256-feature block, chunk of kBN tokens).
+template <bool GATEUP>
+__device__ __forceinline__ Item decode2(const Dims& d, const int32_t* seg_rows,
+                                        const int32_t* seg_wid, const int32_t* seg_items, int nseg,
+                                        int item) {
+  constexpr int kBN = Cfg2<GATEUP>::kBN;
+  const int s = find_segment(seg_items, nseg, item);
+  const int local = item - seg_items[s];
+  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
+  const int nch = (cnt + kBN - 1) / kBN;
+  const int chunk = local % nch, mb = local / nch;
+  Item it;
+  it.r0 = rb + chunk * kBN;
+  it.n = min(kBN, cnt - chunk * kBN);
+  it.f0 = mb * 256;
+  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
+  return it;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tc2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
+               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
+               __nv_bfloat16* __restrict__ out) {
+  using C = Cfg2<GATEUP>;
+  constexpr int kBN = C::kBN;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;                    // [kStages], used in the leader
+  uint64_t* empty = bars + C::kStages;      // [kStages]
+  uint64_t* tfull = bars + 2 * C::kStages;  // [2]
+  uint64_t* tempty = tfull + 2;             // [2], used in the leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = (int)cluster_id(), npairs = (int)num_clusters();
+  const int nseg = st->nseg;
+  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
+  if (total == 0) return;  // both CTAs of a pair read the same value
+  const int K = GATEUP ? d.H : d.F;
+  const int nk = K / kBK;
+  const int NOUT = GATEUP ? d.F : d.H;
+  constexpr uint32_t kTxBytes = 2u * (uint32_t)C::kStageBytes;  // both CTAs' loads
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 2 * kEpiWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int item = pair; item < total && ok; item += npairs) {
+        const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+        const int N = ((it.n + 15) / 16) * 16;
+        const int wrow = it.wrow + (int)rank * 128;
+        const int xrow = it.r0 + (int)rank * (N / 2);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = stage_base + stage * C::kStageBytes;
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          const uint32_t fb = map_to_rank(fb_local, 0);
+          if (leader) {
+            mbar_expect_tx(fb_local, kTxBytes);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          tma_load_2d_pair(smem_u32(sb), &map_w, kb * kBK, wrow, fb);
+          if (GATEUP) tma_load_2d_pair(smem_u32(sb + kTileBytes), &map_w, kb * kBK, wrow + d.F, fb);
+          tma_load_2d_pair(smem_u32(sb + (GATEUP ? 2 : 1) * kTileBytes), &map_x, kb * kBK, xrow, fb);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {  // the leader's barriers count both CTAs' copies
+        for (int s2 = 0; s2 < C::kStages; ++s2)
+          if ((armed >> s2) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint32_t last_bar = 0, last_par = 0;
+      bool ok = true, issued = false;
+      for (int item = pair; item < total && ok; item += npairs) {
+        const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+        const int N = ((it.n + 15) / 16) * 16;
+        const uint32_t idesc = idesc_bf16(256, N);
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_gate = tmem + acc * C::kAccCols;
+        const uint32_t d_up = d_gate + kBN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(stage_base + stage * C::kStageBytes);
+          const uint32_t sx = sb + (GATEUP ? 2 : 1) * kTileBytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks) {
+            const uint32_t koff = ks * 32;
+            const uint32_t acc_flag = (kb | ks) != 0;
+            mma_bf16_pair(d_gate, sdesc(sb + koff), sdesc(sx + koff), idesc, acc_flag);
+            if (GATEUP)
+              mma_bf16_pair(d_up, sdesc(sb + kTileBytes + koff), sdesc(sx + koff), idesc, acc_flag);
+          }
+          mma_commit_pair(smem_u32(&empty[stage]));
+          last_bar = smem_u32(&empty[stage]);
+          last_par = phase;
+          issued = true;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(smem_u32(&tfull[acc]));
+        last_bar = smem_u32(&tfull[acc]);
+        last_par = acc_phase;
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued) {
+        const unsigned long long t0 = global_ns();
+        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ drain (both CTAs)
+    const int q = warp & 3;
+    const int frow = q * 32 + lane;
+    const int cgrp = (warp - 2) >> 2;
+    constexpr int kColStep = 32 * (kEpiWarps / 4);
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int item = pair; item < total; item += npairs) {
+      const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      __nv_bfloat16* orow = out + (size_t)it.r0 * NOUT + it.f0 + (int)rank * 128 + frow;
+      for (int cb = cgrp * 32; cb < it.n; cb += kColStep) {
+        float g[32];
+        tmem_ld32(tbase + cb, g);
+        if (GATEUP) {
+          float u[32];
+          tmem_ld32(tbase + kBN + cb, u);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (cb + i < it.n) {
+              const float a = g[i] / (1.f + expf(-g[i])) * u[i];
+              orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(a);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (cb + i < it.n) orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(g[i]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair's MMAs or signals may touch it
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::kTmemCols));
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s) {
@@ -477,9 +794,39 @@ int gemm_tc_smem_bytes(bool gateup) {
 cudaError_t gemm_tc_prepare() {
   cudaError_t e = cudaFuncSetAttribute(k_gemm_tc<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        Cfg<true>::kSmemBytes);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(k_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              Cfg<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg2<true>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tc2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             Cfg2<false>::kSmemBytes);
+  return e;
+}
+
+cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                            int grid, cudaStream_t s, int which) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3((unsigned)(grid & ~1));
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (which == 1) {
+    cfg.dynamicSmemBytes = Cfg2<true>::kSmemBytes;
+    return cudaLaunchKernelEx(&cfg, k_gemm_tc2<true>, maps.w_gateup, maps.A2, d, c.st, w.seg_rows,
+                              w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
+  }
+  cfg.dynamicSmemBytes = Cfg2<false>::kSmemBytes;
+  return cudaLaunchKernelEx(&cfg, k_gemm_tc2<false>, maps.w_down, maps.act2, d, c.st, w.seg_rows,
+                            w.seg_wid, w.seg_items2, static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -543,6 +890,8 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F, kBM);
   if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H, kTcRows1);
   if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kTcRows2);
+  if (e == cudaSuccess) e = encode(&maps->A2, w.A, (unsigned long long)w.Rcap, d.H, kTc2Rows1 / 2);
+  if (e == cudaSuccess) e = encode(&maps->act2, w.act, (unsigned long long)w.Rcap, d.F, kTc2Rows2 / 2);
   return e;
 }
 

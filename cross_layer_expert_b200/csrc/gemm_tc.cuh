@@ -14,6 +14,8 @@ struct TcMaps {
   CUtensorMap w_down;    // [L*Etot*H rows, F cols]
   CUtensorMap A;         // [Rcap rows, H cols]
   CUtensorMap act;       // [Rcap rows, F cols]
+  CUtensorMap A2;        // same buffers, boxes of half a pair's token tile
+  CUtensorMap act2;
 };
 
 // Encodes the maps for these buffers; returns cudaErrorInvalidValue if the
@@ -23,6 +25,10 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
 // Opts the kernels into their dynamic shared memory (once per device).
 cudaError_t gemm_tc_prepare();
 int gemm_tc_smem_bytes(bool gateup);
+// Two-SM (cta_group::2) version of launch_gemm_tc: clusters of two CTAs, one
+// per SM pair; each item covers 256 output features.
+cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                            int grid, cudaStream_t s, int which);
 // Runs the GEMM's bounded mbarrier wait on a barrier nothing arrives on.
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) of a step; grid = persistent

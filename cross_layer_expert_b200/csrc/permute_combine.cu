@@ -41,7 +41,9 @@ constexpr int kPermSplit = 4;
 template <typename T>
 __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* __restrict__ st,
                                                           const int32_t* __restrict__ idx,
-                                                          const int32_t* __restrict__ base,
+                                                          const int32_t* __restrict__ chunk_hist,
+                                                          const int32_t* __restrict__ seg_rows,
+                                                          const int32_t* __restrict__ prior,
                                                           int32_t* __restrict__ pos,
                                                           const T* __restrict__ hidden,
                                                           T* __restrict__ A) {
@@ -50,10 +52,29 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
   __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
   __shared__ int running[EB_MAX_ETOT];
   __shared__ int dest[kChunk * kMaxSlots];
+  __shared__ int bj[EB_MAX_ETOT];  // first row of (j, this chunk, expert)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = c * kChunk, nt = min(kChunk, d.T - t0);
-  const int k = d.k, kk = d.kk, E = d.E;
-  const int32_t* bj = base + ((size_t)j * d.NC + c) * d.Etot;
+  const int k = d.k, kk = d.kk, E = d.E, Et = d.Etot;
+  const int g = st->group_of[j];
+  for (int e = tid; e < Et; e += kPermThreads) {
+    int b = seg_rows[g * Et + e] + prior[j * Et + e];
+    if (e < E) {
+      const int32_t* ch = chunk_hist + (size_t)j * d.NC * E + e;
+      int cc = 0;
+      for (; cc + 8 <= c; cc += 8) {  // eight independent loads in flight
+        int part[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) part[u] = __ldg(ch + (size_t)(cc + u) * E);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) b += part[u];
+      }
+      for (; cc < c; ++cc) b += __ldg(ch + (size_t)cc * E);
+    } else {
+      b += c * kChunk;
+    }
+    bj[e] = b;
+  }
   for (int e = tid; e < E; e += kPermThreads) running[e] = 0;
   const int npairs = nt * k;
   const int32_t* idx_c = idx + ((size_t)j * d.T + t0) * k;
@@ -188,37 +209,53 @@ __global__ void __launch_bounds__(256) k_combine(Dims d, const State* __restrict
   if (lane < k) s_gate[warp][lane] = gate[tok * k + lane];
   __syncwarp();
   T* out = hidden + tok * d.H;
-  for (int v = lane; v < nvec; v += 32) {
-    float acc[VE];
+  // two 16-byte vectors per lane per pass: 2 * kk loads in flight
+  for (int v0 = lane; v0 < nvec; v0 += 64) {
+    const int v1 = v0 + 32;
+    const bool has1 = v1 < nvec;
+    float acc0[VE], acc1[VE];
     if (d.residual) {
-      Vec<T>::load_plain(out, v, acc);
+      Vec<T>::load_plain(out, v0, acc0);
+      if (has1) Vec<T>::load_plain(out, v1, acc1);
     } else {
 #pragma unroll
-      for (int i = 0; i < VE; ++i) acc[i] = 0.f;
+      for (int i = 0; i < VE; ++i) acc0[i] = acc1[i] = 0.f;
     }
     for (int s0 = 0; s0 < kk; s0 += 8) {
-      uint4 raw[8];
+      uint4 r0[8], r1[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (s0 + u < kk)
-          raw[u] = __ldg(reinterpret_cast<const uint4*>(y + (size_t)s_row[warp][s0 + u] * d.H) + v);
+      for (int u = 0; u < 8; ++u) {
+        if (s0 + u < kk) {
+          const uint4* yrow = reinterpret_cast<const uint4*>(y + (size_t)s_row[warp][s0 + u] * d.H);
+          r0[u] = __ldg(yrow + v0);
+          if (has1) r1[u] = __ldg(yrow + v1);
+        }
+      }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int s = s0 + u;
         if (s >= kk) break;
-        float yv[VE];
-        Vec<T>::unpack(raw[u], yv);
+        float y0[VE], y1[VE];
+        Vec<T>::unpack(r0[u], y0);
+        if (has1) Vec<T>::unpack(r1[u], y1);
         if (s < k) {
           const float g = s_gate[warp][s];
 #pragma unroll
-          for (int i = 0; i < VE; ++i) acc[i] = fmaf(g, yv[i], acc[i]);
+          for (int i = 0; i < VE; ++i) {
+            acc0[i] = fmaf(g, y0[i], acc0[i]);
+            if (has1) acc1[i] = fmaf(g, y1[i], acc1[i]);
+          }
         } else {
 #pragma unroll
-          for (int i = 0; i < VE; ++i) acc[i] += yv[i];
+          for (int i = 0; i < VE; ++i) {
+            acc0[i] += y0[i];
+            if (has1) acc1[i] += y1[i];
+          }
         }
       }
     }
-    Vec<T>::store(out, v, acc);
+    Vec<T>::store(out, v0, acc0);
+    if (has1) Vec<T>::store(out, v1, acc1);
   }
 }
 
@@ -229,11 +266,11 @@ cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const 
   dim3 grid(d.NC * kPermSplit, d.M);
   if (d.dtype == EB_DTYPE_BF16)
     k_permute<__nv_bfloat16><<<grid, kPermThreads, 0, s>>>(
-        d, c.st, w.idx, w.base, w.pos, static_cast<const __nv_bfloat16*>(hidden),
-        static_cast<__nv_bfloat16*>(w.A));
+        d, c.st, w.idx, w.chunk_hist, w.seg_rows, w.prior, w.pos,
+        static_cast<const __nv_bfloat16*>(hidden), static_cast<__nv_bfloat16*>(w.A));
   else
-    k_permute<float><<<grid, kPermThreads, 0, s>>>(d, c.st, w.idx, w.base, w.pos,
-                                                   static_cast<const float*>(hidden),
+    k_permute<float><<<grid, kPermThreads, 0, s>>>(d, c.st, w.idx, w.chunk_hist, w.seg_rows,
+                                                   w.prior, w.pos, static_cast<const float*>(hidden),
                                                    static_cast<float*>(w.A));
   return cudaGetLastError();
 }

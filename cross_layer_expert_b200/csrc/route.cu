@@ -121,13 +121,17 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
 }
 
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
-// is in need_route; its counts land in chunk_hist[j][c][:].
+// is in need_route; its counts land in chunk_hist[j][c][:] and are added
+// (integer atomics: exact, order-free) to the micro-batch's histogram
+// hist[j][:] and rank loads w[j][:], which the previous step zeroed.
 template <int VPL>
 __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__ st,
                                                      const float* __restrict__ logits,
                                                      int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
-                                                     int32_t* __restrict__ chunk_hist) {
+                                                     int32_t* __restrict__ chunk_hist,
+                                                     int32_t* __restrict__ hist,
+                                                     int32_t* __restrict__ wload) {
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->need_route >> j) & 1u)) return;
   const int l = st->layer[j];
@@ -144,7 +148,16 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
   if (nonfinite) bad = 1;
   __syncthreads();
   int32_t* out = chunk_hist + ((size_t)j * d.NC + c) * d.E;
-  for (int e = threadIdx.x; e < d.E; e += blockDim.x) out[e] = hist_s[e];
+  for (int e = threadIdx.x; e < d.E; e += blockDim.x) {
+    out[e] = hist_s[e];
+    if (hist_s[e]) atomicAdd(&hist[j * d.E + e], hist_s[e]);
+  }
+  const int per = d.E / d.D;
+  for (int r = threadIdx.x; r < d.D; r += blockDim.x) {
+    int sum = 0;
+    for (int e = r * per; e < (r + 1) * per; ++e) sum += hist_s[e];
+    if (sum) atomicAdd(&wload[j * d.D + r], sum);
+  }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
 }
 
@@ -179,10 +192,10 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               cudaStream_t s) {
   dim3 grid(d.NC, d.M);
   switch (vpl_for(d.E)) {
-    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
-    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist); break;
+    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
+    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
+    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
+    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
   }
   return cudaGetLastError();
 }

@@ -23,6 +23,19 @@ namespace {
 
 constexpr int kThreads = 1024;
 
+// Binomial coefficients C(a, b), 0 <= a, b <= 32, built at compile time
+// (Pascal's rule) and placed in constant memory.
+struct BinomTable {
+  uint32_t v[33][33];
+  constexpr BinomTable() : v() {
+    for (int a = 0; a <= 32; ++a) {
+      v[a][0] = 1;
+      for (int b = 1; b <= 32; ++b) v[a][b] = a == 0 ? 0u : v[a - 1][b - 1] + v[a - 1][b];
+    }
+  }
+};
+__constant__ BinomTable kBinom = BinomTable();
+
 struct Cand {
   long long sum, mx;
   int size;
@@ -48,7 +61,6 @@ struct SchedSmem {
   long long totsum;
   int P[EB_MAX_M];            // pending micro-batch ids, ascending
   int n;
-  uint32_t binom[33][33];
   Cand red[kThreads / 32];
   uint32_t result;
 };
@@ -98,7 +110,8 @@ __device__ Cand shfl_cand(const Cand& c, int off) {
 __device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
   const int n = sm.n, cmax = n - m;
   unsigned long long N = 0;
-  for (int c = 0; c <= cmax; ++c) N += sm.binom[n][c];
+  const uint32_t (*B)[33] = kBinom.v;
+  for (int c = 0; c <= cmax; ++c) N += B[n][c];
   const unsigned long long per = (N + blockDim.x - 1) / blockDim.x;
   unsigned long long r = per * threadIdx.x;
   const unsigned long long r_end = r + per < N ? r + per : N;
@@ -107,18 +120,18 @@ __device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
   if (r < r_end) {
     int c = 0;
     unsigned long long q = r;
-    while (q >= sm.binom[n][c]) {
-      q -= sm.binom[n][c];
+    while (q >= B[n][c]) {
+      q -= B[n][c];
       ++c;
     }
-    uint64_t cm = c == 0 ? 0 : unrank_colex((uint32_t)q, c, sm.binom);
+    uint64_t cm = c == 0 ? 0 : unrank_colex((uint32_t)q, c, B);
     for (; r < r_end; ++r) {
       const Cand cd = eval_complement(sm, D, (uint32_t)cm);
       if (!have || cand_better(cd, best)) {
         best = cd;
         have = true;
       }
-      if (++q == sm.binom[n][c]) {
+      if (++q == B[n][c]) {
         ++c;
         q = 0;
         cm = (c >= 64) ? 0 : ((1ull << c) - 1);
@@ -200,16 +213,6 @@ __device__ uint32_t scan_policy(const SchedSmem& sm, int D, int m, int policy) {
 // returns the RunSet mask (over micro-batch ids).
 __device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending) {
   const int tid = threadIdx.x;
-  if (policy == EB_SCHED_MAXUTIL) {
-    // binomial table for the MaxUtil enumeration: C(a, b) by the exact
-    // multiplicative recurrence C(a, i) = C(a, i-1) (a - i + 1) / i
-    for (int i = tid; i < 33 * 33; i += blockDim.x) {
-      const int a = i / 33, b = i % 33;
-      unsigned long long c = b <= a ? 1ull : 0ull;
-      for (int q = 1; q <= b && b <= a; ++q) c = c * (unsigned long long)(a - q + 1) / q;
-      sm.binom[a][b] = (uint32_t)c;
-    }
-  }
   for (int dd = tid; dd < D; dd += blockDim.x) {
     long long t = 0;
     for (int i = 0; i < sm.n; ++i) t += sm.w[i][dd];
@@ -280,7 +283,7 @@ struct PlanSmem {
 };
 
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
-                                                             int rn2, int fm) {
+                                                             int rn2, int fm1, int fm2) {
   __shared__ SchedSmem sm;
   __shared__ PlanSmem pl;
   // the step state lives in shared memory for the whole kernel (thread 0's
@@ -297,26 +300,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     for (int i = tid; i < kStateWords; i += blockDim.x)
       reinterpret_cast<int*>(c.st)[i] = reinterpret_cast<const int*>(&ss)[i];
   };
-  const uint32_t need = st->need_route;
-  // 1. fold fresh chunk counts into hist[j][:] and loads w[j][:]
-  for (int i = tid; i < d.M * d.E; i += blockDim.x) {
-    const int j = i / d.E, e = i % d.E;
-    if ((need >> j) & 1u) {
-      int s = 0;
-      for (int ch = 0; ch < d.NC; ++ch) s += wk.chunk_hist[((size_t)j * d.NC + ch) * d.E + e];
-      c.hist[i] = s;
-    }
-  }
-  __syncthreads();
-  const int per = d.E / d.D;
-  for (int i = tid; i < d.M * d.D; i += blockDim.x) {
-    const int j = i / d.D, dd = i % d.D;
-    if ((need >> j) & 1u) {
-      int s = 0;
-      for (int e = dd * per; e < (dd + 1) * per; ++e) s += c.hist[j * d.E + e];
-      c.w[i] = s;
-    }
-  }
+  // 1. hist[j][:] and w[j][:] of the micro-batches routed for this step were
+  //    accumulated by the routing kernel
   // 2. pending set
   const uint32_t pending = st->pending;
   if (tid == 0) {
@@ -418,6 +403,12 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     st->nseg = G * d.Etot;
   }
   if (!d.compute) {
+    __syncthreads();
+    const uint32_t next = st->need_route;
+    for (int i = tid; i < d.M * d.E; i += blockDim.x)
+      if ((next >> (i / d.E)) & 1u) c.hist[i] = 0;
+    for (int i = tid; i < d.M * d.D; i += blockDim.x)
+      if ((next >> (i / d.D)) & 1u) c.w[i] = 0;
     write_back();
     return;
   }
@@ -425,7 +416,7 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   // 5. segment plan: rows of (group, expert) are counted into seg_rows and
   //    scanned in place; GEMM work items per segment likewise.
   const int G = st->n_groups, nr = st->n_run, Et = d.Etot, nseg = G * Et;
-  const int mb1 = d.F / fm, mb2 = d.H / fm;
+  const int mb1 = d.F / fm1, mb2 = d.H / fm2;
   __shared__ int s_nonempty;
   if (tid == 0) s_nonempty = 0;
   __syncthreads();
@@ -463,21 +454,25 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     }
   }
   __syncthreads();
-  // bases: first row of (j, chunk, expert)
+  // rows of (j's segment, expert) taken by earlier micro-batches of its group;
+  // the permute kernel adds the earlier chunks of j itself
   for (int i = tid; i < nr * Et; i += blockDim.x) {
     const int a = i / Et, e = i % Et;
     const int j = st->run_list[a], g = st->group_of[j];
-    int run_row = wk.seg_rows[g * Et + e];
+    int prior = 0;
     for (int b = 0; b < a; ++b) {
       const int jb = st->run_list[b];
-      if (st->group_of[jb] == g) run_row += (e < d.E) ? c.hist[jb * d.E + e] : d.T;
+      if (st->group_of[jb] == g) prior += (e < d.E) ? c.hist[jb * d.E + e] : d.T;
     }
-    for (int ch = 0; ch < d.NC; ++ch) {
-      wk.base[((size_t)j * d.NC + ch) * Et + e] = run_row;
-      run_row += (e < d.E) ? wk.chunk_hist[((size_t)j * d.NC + ch) * d.E + e]
-                           : min(kChunk, d.T - ch * kChunk);
-    }
+    wk.prior[j * Et + e] = prior;
   }
+  __syncthreads();
+  // the micro-batches routed at the next step start from zero counts
+  const uint32_t next = st->need_route;
+  for (int i = tid; i < d.M * d.E; i += blockDim.x)
+    if ((next >> (i / d.E)) & 1u) c.hist[i] = 0;
+  for (int i = tid; i < d.M * d.D; i += blockDim.x)
+    if ((next >> (i / d.D)) & 1u) c.w[i] = 0;
   write_back();
 }
 
@@ -542,7 +537,10 @@ __global__ void k_loads(const int32_t* __restrict__ hist, int M, int E, int D,
   w[i] = s;
 }
 
-__global__ void k_reset(Dims d, State* st) {
+__global__ void k_reset(Dims d, CtxDev c) {
+  State* st = c.st;
+  for (int i = threadIdx.x; i < d.M * d.E; i += blockDim.x) c.hist[i] = 0;
+  for (int i = threadIdx.x; i < d.M * d.D; i += blockDim.x) c.w[i] = 0;
   if (threadIdx.x != 0) return;
   const uint32_t all = d.M >= 32 ? 0xffffffffu : ((1u << d.M) - 1u);
   for (int j = 0; j < EB_MAX_M; ++j) {
@@ -578,8 +576,8 @@ unsigned long long maxutil_candidates(int n, int m) {
 }
 
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
-                                 int fm, cudaStream_t s) {
-  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn1, rn2, fm);
+                                 int fm1, int fm2, cudaStream_t s) {
+  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn1, rn2, fm1, fm2);
   return cudaGetLastError();
 }
 
@@ -597,7 +595,7 @@ cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, c
 }
 
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s) {
-  k_reset<<<1, 32, 0, s>>>(d, c.st);
+  k_reset<<<1, 1024, 0, s>>>(d, c);
   return cudaGetLastError();
 }
 

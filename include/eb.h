@@ -55,10 +55,15 @@ typedef int eb_status;
 #define EB_DTYPE_F32 0
 #define EB_DTYPE_BF16 1
 
-/* expert GEMM engine: AUTO = tensor cores (tcgen05) for bf16, SIMT for f32 */
+/* expert GEMM engine.  AUTO: tensor cores (tcgen05) for bf16 -- the two-SM
+ * engine (cta_group::2, 256 features per CTA pair) for each GEMM whose output
+ * width is a multiple of 256, else the one-SM engine -- and SIMT for f32.
+ * TC: one-SM tensor-core engine only.  SIMT: CUDA cores.  TC2: two-SM engine
+ * (H and F multiples of 256). */
 #define EB_GEMM_AUTO 0
 #define EB_GEMM_TC 1
 #define EB_GEMM_SIMT 2
+#define EB_GEMM_TC2 3
 
 /* Limits of this build. */
 #define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */

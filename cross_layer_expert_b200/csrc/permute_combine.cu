@@ -115,12 +115,40 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
   const int nvec = d.H * (int)sizeof(T) / 16;
   const int per = (nt + kPermSplit - 1) / kPermSplit;
   const int ta = part * per, tb = min(nt, ta + per);
-  for (int t = ta + warp; t < tb; t += kPermThreads / 32) {
-    const uint4* src = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + t) * d.H);
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 val = __ldg(src + v);
-      for (int s = 0; s < kk; ++s)
-        reinterpret_cast<uint4*>(A + (size_t)dest[t * kk + s] * d.H)[v] = val;
+  // each warp copies two tokens at a time: both rows' 16-byte vectors are
+  // loaded into registers (8 per lane per token) before any store is issued
+  constexpr int kU = 8;
+  for (int t = ta + warp; t < tb; t += 2 * (kPermThreads / 32)) {
+    const int t2 = t + kPermThreads / 32;
+    const bool two = t2 < tb;
+    const uint4* src0 = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + t) * d.H);
+    const uint4* src1 = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + (two ? t2 : t)) * d.H);
+    for (int base = 0; base < nvec; base += 32 * kU) {
+      uint4 v0[kU], v1[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int v = base + u * 32 + lane;
+        if (v < nvec) {
+          v0[u] = __ldg(src0 + v);
+          if (two) v1[u] = __ldg(src1 + v);
+        }
+      }
+      for (int s = 0; s < kk; ++s) {
+        uint4* dst0 = reinterpret_cast<uint4*>(A + (size_t)dest[t * kk + s] * d.H);
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int v = base + u * 32 + lane;
+          if (v < nvec) dst0[v] = v0[u];
+        }
+        if (two) {
+          uint4* dst1 = reinterpret_cast<uint4*>(A + (size_t)dest[t2 * kk + s] * d.H);
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int v = base + u * 32 + lane;
+            if (v < nvec) dst1[v] = v1[u];
+          }
+        }
+      }
     }
   }
 }

@@ -293,7 +293,8 @@ def run_ours(args, world, rank, local):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic (seeded Dirichlet task-profile routing skew; N(0,0.02) weights)",
+            "data": ("synthetic (seeded routing skew: " + wl.profile + "; random-init weights "
+                     + ("N(0, 1/(3 fan_in))" if wl.w_init == "fan_in" else f"N(0, {wl.w_std}^2)") + ")"),
             "workload_layers": wl.L,
             "config": {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
                                    f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",

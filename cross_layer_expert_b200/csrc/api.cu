@@ -22,7 +22,7 @@ struct eb_ctx {
   int device = 0;
   int num_sms = 148;
   bool use_tc = false;
-  bool pair1 = false, pair2 = false;  // GEMM 1 / GEMM 2 on the two-SM engine
+  int eng1 = EB_GEMM_SIMT, eng2 = EB_GEMM_SIMT;  // engine of GEMM 1 / GEMM 2
   cudaStream_t last_stream = nullptr;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
@@ -49,7 +49,56 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool use_tc_for(const eb_config& c) {
   if (c.dtype != EB_DTYPE_BF16) return false;
-  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC || c.gemm == EB_GEMM_TC2;
+  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC || c.gemm == EB_GEMM_TC2 ||
+         c.gemm == EB_GEMM_TM || c.gemm == EB_GEMM_TM2;
+}
+
+// Engine of each GEMM.  AUTO takes the one-SM token-major engine for every
+// GEMM whose tile shape fits (GEMM 1: F a multiple of 128; GEMM 2: H a
+// multiple of 256) and the one-SM weight-major engine otherwise; an explicit
+// choice that does not fit one GEMM runs that GEMM on the weight-major engine.
+void choose_engines(const eb_config& c, bool use_tc, int num_sms, int* g1, int* g2) {
+  *g1 = *g2 = EB_GEMM_SIMT;
+  if (!use_tc) return;
+  const bool pair_ok = num_sms >= 2;
+  const int want = c.gemm == EB_GEMM_AUTO ? EB_GEMM_TM : c.gemm;
+  auto fits = [&](int eng, int which) {
+    const int nout = which == 1 ? c.F : c.H;
+    switch (eng) {
+      case EB_GEMM_TC: return true;
+      case EB_GEMM_TC2: return pair_ok && nout % kTc2Feat == 0;
+      case EB_GEMM_TM: return nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
+      case EB_GEMM_TM2: return pair_ok && nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
+      default: return false;
+    }
+  };
+  *g1 = fits(want, 1) ? want : EB_GEMM_TC;
+  *g2 = fits(want, 2) ? want : EB_GEMM_TC;
+}
+
+// Token rows and output features of one work item of `eng` for GEMM `which`.
+void engine_tiles(int eng, int which, int* rows, int* feats) {
+  switch (eng) {
+    case EB_GEMM_TC:
+      *rows = which == 1 ? kTcRows1 : kTcRows2;
+      *feats = kTcFeat;
+      return;
+    case EB_GEMM_TC2:
+      *rows = which == 1 ? kTc2Rows1 : kTc2Rows2;
+      *feats = kTc2Feat;
+      return;
+    case EB_GEMM_TM:
+      *rows = kTmRows;
+      *feats = which == 1 ? kTmFeat1 : kTmFeat2;
+      return;
+    case EB_GEMM_TM2:
+      *rows = 2 * kTmRows;
+      *feats = which == 1 ? kTmFeat1 : kTmFeat2;
+      return;
+    default:
+      *rows = kSimtRows;
+      *feats = kSimtFeat;
+  }
 }
 
 Dims make_dims(const eb_config& c) {
@@ -87,6 +136,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
     x.seg_wid = (int32_t*)take(sizeof(int32_t) * nseg);
     x.seg_items1 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.seg_items2 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
+    x.gemm_next = (int32_t*)take(sizeof(int32_t) * 2);
     x.Rcap = (long long)(M * T * d.kk);
     const size_t es = elem_size(c.dtype);
     x.A = take(es * (size_t)x.Rcap * c.H);
@@ -155,7 +205,7 @@ eb_status eb_config_check(const eb_config* c) {
   if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
   if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
   if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
-  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TC2) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TM2) return EB_ERR_INVALID_ARG;
   if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
@@ -167,10 +217,11 @@ eb_status eb_config_check(const eb_config* c) {
     const int vec = c->dtype == EB_DTYPE_BF16 ? 8 : 4;  // 16-byte rows
     if (c->H % vec != 0) return EB_ERR_UNSUPPORTED;
     if ((long long)c->M * c->T * (c->k + c->n_shared) > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
-    if (c->dtype == EB_DTYPE_F32 && (c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2))
-      return EB_ERR_UNSUPPORTED;
+    const bool forced_tc = c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2 ||
+                           c->gemm == EB_GEMM_TM || c->gemm == EB_GEMM_TM2;
+    if (c->dtype == EB_DTYPE_F32 && forced_tc) return EB_ERR_UNSUPPORTED;
     if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
-      if (c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2) return EB_ERR_UNSUPPORTED;
+      if (forced_tc) return EB_ERR_UNSUPPORTED;
     }
     if (c->gemm == EB_GEMM_TC2 && (c->H % 256 != 0 || c->F % 256 != 0)) return EB_ERR_UNSUPPORTED;
   }
@@ -197,9 +248,7 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   cudaError_t e = cudaGetDevice(&x->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&x->num_sms, cudaDevAttrMultiProcessorCount, x->device);
   // the two-SM engine covers 256 output features per item
-  const bool pairs_ok = x->use_tc && c->gemm != EB_GEMM_TC && x->num_sms >= 2;
-  x->pair1 = pairs_ok && c->F % kTc2Feat == 0;
-  x->pair2 = pairs_ok && c->H % kTc2Feat == 0;
+  if (e == cudaSuccess) choose_engines(*c, x->use_tc, x->num_sms, &x->eng1, &x->eng2);
   const size_t n_state = align_up(sizeof(State));
   const size_t n_hist = align_up(sizeof(int32_t) * c->M * c->E);
   const size_t n_w = align_up(sizeof(int32_t) * c->M * c->D);
@@ -254,6 +303,17 @@ eb_status eb_reset(eb_ctx* x, void* stream) {
   return cuda_status(launch_reset(x->d, x->dev, s));
 }
 
+static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* wgu,
+                                 const void* wdn, cudaStream_t s, int which) {
+  switch (eng) {
+    case EB_GEMM_TC: return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, which);
+    case EB_GEMM_TC2: return launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
+    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which);
+    case EB_GEMM_TM2: return launch_gemm_tm2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
+    default: return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, which);
+  }
+}
+
 static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
                               const void* wdn, void* workspace, size_t ws_bytes,
                               cudaStream_t s) {
@@ -274,11 +334,10 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     x->map_keys[1] = wdn;
     x->map_keys[2] = workspace;
   }
-  const bool p1 = tc && x->pair1, p2 = tc && x->pair2;
-  const int rn1 = !tc ? kSimtRows : p1 ? kTc2Rows1 : kTcRows1;
-  const int rn2 = !tc ? kSimtRows : p2 ? kTc2Rows2 : kTcRows2;
-  const int fm1 = !tc ? kSimtFeat : p1 ? kTc2Feat : kTcFeat;
-  const int fm2 = !tc ? kSimtFeat : p2 ? kTc2Feat : kTcFeat;
+  const int g1 = c.compute ? x->eng1 : EB_GEMM_SIMT, g2 = c.compute ? x->eng2 : EB_GEMM_SIMT;
+  int rn1, fm1, rn2, fm2;
+  engine_tiles(g1, 1, &rn1, &fm1);
+  engine_tiles(g2, 2, &rn2, &fm2);
   cudaError_t e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, logits, s); });
   if (e == cudaSuccess)
     e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
@@ -286,21 +345,9 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     if (e == cudaSuccess)
       e = timed(x, 2, 1, s, [&] { return launch_permute(x->d, x->dev, w, hidden, s); });
     if (e == cudaSuccess) {
-      if (tc) {
-        e = timed(x, 3, 1, s, [&] {
-          return p1 ? launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, 1)
-                    : launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 1);
-        });
-        if (e == cudaSuccess)
-          e = timed(x, 4, 1, s, [&] {
-            return p2 ? launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, 2)
-                      : launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, 2);
-          });
-      } else {
-        e = timed(x, 3, 1, s, [&] { return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, 1); });
-        if (e == cudaSuccess)
-          e = timed(x, 4, 1, s, [&] { return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, 2); });
-      }
+      e = timed(x, 3, 1, s, [&] { return launch_engine(x, g1, w, wgu, wdn, s, 1); });
+      if (e == cudaSuccess)
+        e = timed(x, 4, 1, s, [&] { return launch_engine(x, g2, w, wgu, wdn, s, 2); });
     }
     if (e == cudaSuccess)
       e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });

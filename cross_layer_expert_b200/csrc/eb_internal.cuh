@@ -31,6 +31,10 @@ constexpr int kTc2Rows1 = 128;
 constexpr int kTc2Rows2 = 256;
 constexpr int kTc2Feat = 256;
 constexpr int kTcFeat = 128;
+// Token-major tiles: 128 tokens x (128 gate/up features | 256 down features).
+constexpr int kTmRows = 128;
+constexpr int kTmFeat1 = 128;
+constexpr int kTmFeat2 = 256;
 constexpr int kSimtRows = 64;
 constexpr int kSimtFeat = 64;
 
@@ -79,6 +83,7 @@ struct Work {
   int32_t* seg_wid;    // [M*Etot]: layer * Etot + expert
   int32_t* seg_items1; // [M*Etot + 1]
   int32_t* seg_items2; // [M*Etot + 1]
+  int32_t* gemm_next;  // [2]: next dynamically claimed item of GEMM 1 / GEMM 2 (zeroed by the plan)
   void* A;             // [Rcap][H] permuted tokens
   void* act;           // [Rcap][F] SwiGLU activations
   void* y;             // [Rcap][H] expert outputs

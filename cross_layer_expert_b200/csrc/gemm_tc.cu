@@ -22,6 +22,8 @@
 // EB_ERR_TIMEOUT in the step's status word, waits (bounded) for its own copies
 // and MMAs in flight, frees its TMEM and returns.
 #include <cuda.h>
+
+#include <atomic>
 #include <cuda_bf16.h>
 
 #include "eb_internal.cuh"
@@ -780,6 +782,632 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Token-major variant.  Tokens are the MMA's M side (128 per accumulator) and
+// 256 weight rows its N side (GEMM 1: the gate and up rows of one 128-feature
+// block; GEMM 2: 256 output features), so every MMA is 128 x 256 x 16 -- large
+// enough to run at the tensor pipe's rate with operands read fresh from
+// shared memory -- and a token's accumulator row holds its 256 outputs, so
+// the drain writes contiguous 16-byte chunks.
+//
+// One work item is one 128-token chunk of a segment against one weight tile.
+// Only the chunk's own token rows are loaded (32-row boxes); the rest of the
+// 128-row operand is stale shared memory whose products land in accumulator
+// rows that are never stored.  Items are claimed dynamically from a
+// step-wide counter, so CTAs finish together whatever the segment sizes.
+// ---------------------------------------------------------------------------
+
+// Segment plan (row offsets, expert ids, item offsets) of up to kSegCache
+// segments is copied into shared memory at kernel start, so the per-item
+// decode (a binary search over item offsets) runs on shared memory instead
+// of dependent global loads; larger plans are read from global memory.
+constexpr int kSegCache = 1536;
+constexpr int kSegCacheBytes = ((3 * 4 * (kSegCache + 1)) + 127) / 128 * 128;
+
+struct SegView {
+  const int32_t* rows;
+  const int32_t* wid;
+  const int32_t* items;
+};
+
+__device__ __forceinline__ SegView cache_segments(uint8_t* buf, int nseg, const int32_t* seg_rows,
+                                                  const int32_t* seg_wid,
+                                                  const int32_t* seg_items) {
+  if (nseg > kSegCache) return {seg_rows, seg_wid, seg_items};
+  int32_t* r = reinterpret_cast<int32_t*>(buf);
+  int32_t* w = r + kSegCache + 1;
+  int32_t* it = w + kSegCache + 1;
+  for (int i = threadIdx.x; i <= nseg; i += blockDim.x) {
+    r[i] = seg_rows[i];
+    it[i] = seg_items[i];
+    if (i < nseg) w[i] = seg_wid[i];
+  }
+  return {r, w, it};
+}
+
+constexpr int kTmBox = 32;                    // token rows per TMA box
+constexpr int kTmBoxBytes = kTmBox * kBK * 2;  // 4 KiB
+
+template <bool GATEUP>
+struct CfgTM {
+  static constexpr int kRows = kTmRows;  // token rows per item (MMA M)
+  static constexpr int kN = 256;         // weight rows per item (MMA N)
+  static constexpr int kFeat = GATEUP ? kTmFeat1 : kTmFeat2;  // output features per item
+  static constexpr int kABytes = kRows * kBK * 2;   // 16 KiB token tile
+  static constexpr int kBBytes = kN * kBK * 2;      // 32 KiB weight tile
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = 196608 / kStageBytes;  // 4
+  static constexpr int kAccCols = kN;
+  static constexpr int kAccBufs = 2;
+  static constexpr int kTmemCols = kAccBufs * kAccCols;  // 512
+  static constexpr int kQueue = 8;  // claimed items queued for the MMA issuer and the drain
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kSegCacheBytes + 1024;
+  static_assert(kRows == 128 && kFeat * (GATEUP ? 2 : 1) == kN, "token-major tile shape");
+  static_assert((2 * kStages + 4 + 2 * kQueue) * 8 + 8 + 4 * kQueue <= 1024, "barrier region");
+};
+
+template <bool GATEUP>
+__device__ __forceinline__ Item decode_tm(const Dims& d, const int32_t* seg_rows,
+                                          const int32_t* seg_wid, const int32_t* seg_items,
+                                          int nseg, int item) {
+  using C = CfgTM<GATEUP>;
+  const int s = find_segment(seg_items, nseg, item);
+  const int local = item - seg_items[s];
+  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
+  const int nch = (cnt + C::kRows - 1) / C::kRows;
+  const int chunk = local % nch, mb = local / nch;
+  Item it;
+  it.r0 = rb + chunk * C::kRows;
+  it.n = min(C::kRows, cnt - chunk * C::kRows);
+  it.f0 = mb * C::kFeat;
+  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
+  return it;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// map_x: token rows [Rcap, K] in boxes of 32 rows; map_w: weights in boxes of
+// 128 rows.  GATEUP: out = act [Rcap, F]; else out = y [Rcap, H].  next_item:
+// the step's claim counter (zero before the launch).
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+              Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
+              const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
+              int32_t* __restrict__ next_item, __nv_bfloat16* __restrict__ out) {
+  using C = CfgTM<GATEUP>;
+  constexpr int Q = C::kQueue;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;                      // [kStages] k-block landed
+  uint64_t* empty = bars + C::kStages;        // [kStages] k-block consumed by the MMAs
+  uint64_t* tfull = bars + 2 * C::kStages;    // [2] accumulator complete
+  uint64_t* tempty = tfull + 2;               // [2] accumulator drained
+  uint64_t* iready = tempty + 2;              // [Q] item queue entry written
+  uint64_t* ifree = iready + Q;               // [Q] entry read by the MMA issuer and the drain
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ifree + Q);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* iq = const_cast<int*>(abort_flag) + 1;  // [Q] claimed items, -1 ends the sequence
+  uint8_t* seg_buf = reinterpret_cast<uint8_t*>(bars) + 1024;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nseg = st->nseg;
+  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
+  if (total == 0) return;
+  const int K = GATEUP ? d.H : d.F;
+  const int nk = K / kBK;
+  const int NOUT = GATEUP ? d.F : d.H;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), kEpiWarps);
+    }
+    for (int i = 0; i < Q; ++i) {
+      mbar_init(smem_u32(&iready[i]), 1);
+      mbar_init(smem_u32(&ifree[i]), kEpiWarps + 1);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const SegView sv = cache_segments(seg_buf, nseg, seg_rows, seg_wid, seg_items);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    // A CTA's first item is blockIdx.x; each further one is gridDim.x plus
+    // the next value of the claim counter, claimed when the current item
+    // starts and decoded once its last k-block is issued (both off the
+    // k-block path).  Claimed items go to the MMA issuer and the drain
+    // through a queue in shared memory.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      int item = (int)blockIdx.x < total ? (int)blockIdx.x : -1;
+      Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item < 0 ? 0 : item);
+      for (int u = 0; ok; ++u) {
+        const int qs = u % Q;
+        if (u >= Q && !mbar_wait(smem_u32(&ifree[qs]), (uint32_t)(((u / Q) - 1) & 1), abort_flag,
+                                 &st->status)) {
+          ok = false;
+          break;
+        }
+        iq[qs] = item;
+        mbar_arrive(smem_u32(&iready[qs]));  // releases iq[qs]
+        if (item < 0) break;
+        const int claim = atomicAdd(next_item, 1);  // used after the k-loop
+        const int nbox = (it.n + kTmBox - 1) / kTmBox;
+        const uint32_t tx = (uint32_t)(nbox * kTmBoxBytes + C::kBBytes);
+        // weight rows of the 256-row N tile: GATEUP gate rows then up rows of
+        // the feature block; else 256 consecutive output rows
+        const int w0 = it.wrow, w1 = GATEUP ? it.wrow + d.F : it.wrow + 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = stage_base + stage * C::kStageBytes;
+          const uint32_t fb = smem_u32(&full[stage]);
+          mbar_expect_tx(fb, tx);
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d(smem_u32(sb + b * kTmBoxBytes), &map_x, kb * kBK, it.r0 + b * kTmBox, fb);
+          tma_load_2d(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
+          tma_load_2d(smem_u32(sb + C::kABytes + C::kBBytes / 2), &map_w, kb * kBK, w1, fb);
+          armed |= 1u << stage;
+          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        const int nxt = (int)gridDim.x + claim;
+        item = nxt < total ? nxt : -1;
+        if (item >= 0) it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+      }
+      if (!ok) {  // let every issued copy land before the CTA exits
+        for (int s2 = 0; s2 < C::kStages; ++s2)
+          if ((armed >> s2) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint32_t last_bar = 0, last_par = 0;
+      bool ok = true, issued = false;
+      const uint32_t idesc = idesc_bf16(C::kRows, C::kN);
+      for (int u = 0; ok; ++u) {
+        const int qs = u % Q;
+        if (!mbar_wait(smem_u32(&iready[qs]), (uint32_t)((u / Q) & 1), abort_flag, &st->status)) {
+          ok = false;
+          break;
+        }
+        const int item = iq[qs];
+        mbar_arrive(smem_u32(&ifree[qs]));
+        if (item < 0) break;
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem + acc * C::kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks) {
+            const uint32_t koff = ks * 32;
+            mma_bf16(dcol, sdesc(sa + koff), sdesc(sb + koff), idesc, (kb | ks) != 0);
+          }
+          mma_commit(smem_u32(&empty[stage]));
+          last_bar = smem_u32(&empty[stage]);
+          last_par = phase;
+          issued = true;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tfull[acc]));
+        last_bar = smem_u32(&tfull[acc]);
+        last_par = acc_phase;
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued) {
+        const unsigned long long t0 = global_ns();
+        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ drain
+    // warp w reads TMEM lanes (tokens) 32 (w % 4) .. +31; with 8 warps two
+    // warps share a lane quarter and split its 32-column blocks.
+    const int q = warp & 3;
+    const int cgrp = (warp - 2) >> 2;
+    constexpr int kGroups = kEpiWarps / 4;
+    constexpr int kBlocks = C::kFeat / 32;  // 32-feature blocks of an item's output
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int u = 0;; ++u) {
+      const int qs = u % Q;
+      if (!mbar_wait(smem_u32(&iready[qs]), (uint32_t)((u / Q) & 1), abort_flag, &st->status)) break;
+      const int item = iq[qs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ifree[qs]));
+      if (item < 0) break;
+      const Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
+      tc_fence_after();
+      const int row = q * 32 + lane;  // token row within the item
+      const bool live = row < it.n;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      __nv_bfloat16* orow = out + (size_t)(it.r0 + row) * NOUT + it.f0;
+      // a lane quarter past the chunk's last token has nothing to drain
+      const int b_end = q * 32 < it.n ? kBlocks : 0;
+      for (int b = cgrp; b < b_end; b += kGroups) {
+        float g[32];
+        tmem_ld32(tbase + b * 32, g);
+        uint32_t packed[16];
+        if (GATEUP) {
+          float uu[32];
+          tmem_ld32(tbase + 128 + b * 32, uu);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = g[2 * i] / (1.f + expf(-g[2 * i])) * uu[2 * i];
+            const float a1 = g[2 * i + 1] / (1.f + expf(-g[2 * i + 1])) * uu[2 * i + 1];
+            packed[i] = pack_bf16x2(a0, a1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+        }
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + b * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::kTmemCols));
+  }
+}
+
+
+// ---------------------------------------------------------------------------
+// Two-SM token-major variant (cta_group::2).  A CTA pair computes 256 tokens
+// x 256 weight rows: CTA r holds token rows [r0 + 128 r, r0 + 128 r + 128) as
+// its half of the MMA's A operand and weight rows 128 r .. 128 r + 127 of the
+// tile as its half of B (GEMM 1: r = 0 the gate rows, r = 1 the up rows of a
+// 128-feature block; GEMM 2: the lower / upper 128 of 256 features).  Every
+// MMA is 256 x 256 x 16 over the pair, so a weight tile read into the pair
+// serves twice the tokens of the one-SM engine; CTA r's accumulator holds
+// its 128 tokens' 256 outputs, so SwiGLU and the stores stay local.
+// ---------------------------------------------------------------------------
+
+template <bool GATEUP>
+struct CfgTM2 {
+  static constexpr int kRows = 2 * kTmRows;          // token rows per pair item
+  static constexpr int kFeat = GATEUP ? kTmFeat1 : kTmFeat2;
+  static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KiB: this CTA's tokens
+  static constexpr int kBBytes = 128 * kBK * 2;      // 16 KiB: this CTA's weight rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = 204800 / kStageBytes;  // 6
+  static constexpr int kAccCols = 256;
+  static constexpr int kAccBufs = 2;
+  static constexpr int kTmemCols = kAccBufs * kAccCols;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kSegCacheBytes + 1024;
+};
+
+template <bool GATEUP>
+__device__ __forceinline__ Item decode_tm2(const Dims& d, const int32_t* seg_rows,
+                                           const int32_t* seg_wid, const int32_t* seg_items,
+                                           int nseg, int item) {
+  using C = CfgTM2<GATEUP>;
+  const int s = find_segment(seg_items, nseg, item);
+  const int local = item - seg_items[s];
+  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
+  const int nch = (cnt + C::kRows - 1) / C::kRows;
+  const int chunk = local % nch, mb = local / nch;
+  Item it;
+  it.r0 = rb + chunk * C::kRows;
+  it.n = min(C::kRows, cnt - chunk * C::kRows);
+  it.f0 = mb * C::kFeat;
+  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
+  return it;
+}
+
+template <bool GATEUP>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_gemm_tm2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
+               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
+               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
+               __nv_bfloat16* __restrict__ out) {
+  using C = CfgTM2<GATEUP>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
+  uint64_t* full = bars;                    // [kStages], used in the leader
+  uint64_t* empty = bars + C::kStages;      // [kStages]
+  uint64_t* tfull = bars + 2 * C::kStages;  // [2]
+  uint64_t* tempty = tfull + 2;             // [2], used in the leader
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint8_t* seg_buf = reinterpret_cast<uint8_t*>(bars) + 1024;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int pair = (int)cluster_id(), npairs = (int)num_clusters();
+  const int nseg = st->nseg;
+  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
+  if (total == 0) return;  // both CTAs of a pair read the same value
+  const int K = GATEUP ? d.H : d.F;
+  const int nk = K / kBK;
+  const int NOUT = GATEUP ? d.F : d.H;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < C::kStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&tfull[i]), 1);
+      mbar_init(smem_u32(&tempty[i]), 2 * kEpiWarps);
+    }
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  const SegView sv = cache_segments(seg_buf, nseg, seg_rows, seg_wid, seg_items);
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::kTmemCols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+  }
+  tc_fence_before();
+  cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (both CTAs)
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int item = pair; item < total && ok; item += npairs) {
+        const Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+        // token rows of each CTA and the 32-row boxes that cover them
+        const int n0 = min(it.n, kTmRows), n1 = it.n - n0;
+        const int nb0 = (n0 + kTmBox - 1) / kTmBox, nb1 = (n1 + kTmBox - 1) / kTmBox;
+        const int nbox = rank == 0 ? nb0 : nb1;
+        const int xrow = it.r0 + (int)rank * kTmRows;
+        const int wrow = GATEUP ? it.wrow + (int)rank * d.F : it.wrow + (int)rank * 128;
+        const uint32_t tx = (uint32_t)((nb0 + nb1) * kTmBoxBytes + 2 * C::kBBytes);
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = stage_base + stage * C::kStageBytes;
+          const uint32_t fb_local = smem_u32(&full[stage]);
+          const uint32_t fb = map_to_rank(fb_local, 0);
+          if (leader) {
+            mbar_expect_tx(fb_local, tx);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          for (int b = 0; b < nbox; ++b)
+            tma_load_2d_pair(smem_u32(sb + b * kTmBoxBytes), &map_x, kb * kBK, xrow + b * kTmBox, fb);
+          tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, wrow, fb);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok && leader) {  // the leader's barriers count both CTAs' copies
+        for (int s2 = 0; s2 < C::kStages; ++s2)
+          if ((armed >> s2) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      uint32_t last_bar = 0, last_par = 0;
+      bool ok = true, issued = false;
+      const uint32_t idesc = idesc_bf16(256, 256);
+      for (int item = pair; item < total && ok; item += npairs) {
+        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dcol = tmem + acc * C::kAccCols;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
+          const uint32_t sb = sa + C::kABytes;
+#pragma unroll
+          for (int ks = 0; ks < kBK / 16; ++ks) {
+            const uint32_t koff = ks * 32;
+            mma_bf16_pair(dcol, sdesc(sa + koff), sdesc(sb + koff), idesc, (kb | ks) != 0);
+          }
+          mma_commit_pair(smem_u32(&empty[stage]));
+          last_bar = smem_u32(&empty[stage]);
+          last_par = phase;
+          issued = true;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        mma_commit_pair(smem_u32(&tfull[acc]));
+        last_bar = smem_u32(&tfull[acc]);
+        last_par = acc_phase;
+        if (++acc == C::kAccBufs) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok && issued) {
+        const unsigned long long t0 = global_ns();
+        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ drain (both CTAs)
+    const int q = warp & 3;
+    const int cgrp = (warp - 2) >> 2;
+    constexpr int kGroups = kEpiWarps / 4;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int item = pair; item < total; item += npairs) {
+      const Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
+      tc_fence_after();
+      const int nmine = min(max(it.n - (int)rank * kTmRows, 0), kTmRows);  // this CTA's tokens
+      const int row = q * 32 + lane;
+      const bool live = row < nmine;
+      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
+      __nv_bfloat16* orow = out + (size_t)(it.r0 + (int)rank * kTmRows + row) * NOUT + it.f0;
+      constexpr int kBlocks = C::kFeat / 32;
+      const int b_end = q * 32 < nmine ? kBlocks : 0;
+      for (int b = cgrp; b < b_end; b += kGroups) {
+        float g[32];
+        tmem_ld32(tbase + b * 32, g);
+        uint32_t packed[16];
+        if (GATEUP) {
+          float u[32];
+          tmem_ld32(tbase + 128 + b * 32, u);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = g[2 * i] / (1.f + expf(-g[2 * i])) * u[2 * i];
+            const float a1 = g[2 * i + 1] / (1.f + expf(-g[2 * i + 1])) * u[2 * i + 1];
+            packed[i] = pack_bf16x2(a0, a1);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
+        }
+        if (live) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + b * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
+      if (++acc == C::kAccBufs) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();  // neither CTA leaves while the pair's MMAs or signals may touch it
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"((uint32_t)C::kTmemCols));
+  }
+}
+
+// CTA pairs of `kernel` that fit on the device at once (one CTA per SM; an
+// SM pair must sit in one GPC, so an odd SM count per GPC leaves SMs out).
+// Queried once per device and kernel.
+template <typename Kernel>
+int resident_pairs(Kernel kernel, cudaLaunchConfig_t cfg, int fallback) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fallback;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  cfg.gridDim = dim3(2 * (unsigned)fallback);
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+    (void)cudaGetLastError();
+    n = fallback;
+  }
+  n = n < fallback ? n : fallback;
+  cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
 }  // namespace
 
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s) {
@@ -803,7 +1431,56 @@ cudaError_t gemm_tc_prepare() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_gemm_tc2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg2<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM<true>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM2<true>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM2<false>::kSmemBytes);
   return e;
+}
+
+cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                            int grid, cudaStream_t s, int which) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (which == 1) {
+    cfg.dynamicSmemBytes = CfgTM2<true>::kSmemBytes;
+    cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<true>, cfg, grid / 2));
+    return cudaLaunchKernelEx(&cfg, k_gemm_tm2<true>, maps.w_gateup, maps.A32, d, c.st, w.seg_rows,
+                              w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
+  }
+  cfg.dynamicSmemBytes = CfgTM2<false>::kSmemBytes;
+  cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<false>, cfg, grid / 2));
+  return cudaLaunchKernelEx(&cfg, k_gemm_tm2<false>, maps.w_down, maps.act32, d, c.st, w.seg_rows,
+                            w.seg_wid, w.seg_items2, static_cast<__nv_bfloat16*>(w.y));
+}
+
+cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                           int grid, cudaStream_t s, int which) {
+  if (which == 1)
+    k_gemm_tm<true><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
+        maps.w_gateup, maps.A32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1, w.gemm_next,
+        static_cast<__nv_bfloat16*>(w.act));
+  else
+    k_gemm_tm<false><<<grid, kThreads, CfgTM<false>::kSmemBytes, s>>>(
+        maps.w_down, maps.act32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items2, w.gemm_next + 1,
+        static_cast<__nv_bfloat16*>(w.y));
+  return cudaGetLastError();
 }
 
 cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -814,17 +1491,18 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3((unsigned)(grid & ~1));
   cfg.blockDim = dim3(kThreads);
   cfg.stream = s;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (which == 1) {
     cfg.dynamicSmemBytes = Cfg2<true>::kSmemBytes;
+    cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<true>, cfg, grid / 2));
     return cudaLaunchKernelEx(&cfg, k_gemm_tc2<true>, maps.w_gateup, maps.A2, d, c.st, w.seg_rows,
                               w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
   }
   cfg.dynamicSmemBytes = Cfg2<false>::kSmemBytes;
+  cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<false>, cfg, grid / 2));
   return cudaLaunchKernelEx(&cfg, k_gemm_tc2<false>, maps.w_down, maps.act2, d, c.st, w.seg_rows,
                             w.seg_wid, w.seg_items2, static_cast<__nv_bfloat16*>(w.y));
 }
@@ -892,6 +1570,8 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kTcRows2);
   if (e == cudaSuccess) e = encode(&maps->A2, w.A, (unsigned long long)w.Rcap, d.H, kTc2Rows1 / 2);
   if (e == cudaSuccess) e = encode(&maps->act2, w.act, (unsigned long long)w.Rcap, d.F, kTc2Rows2 / 2);
+  if (e == cudaSuccess) e = encode(&maps->A32, w.A, (unsigned long long)w.Rcap, d.H, kTmBox);
+  if (e == cudaSuccess) e = encode(&maps->act32, w.act, (unsigned long long)w.Rcap, d.F, kTmBox);
   return e;
 }
 

@@ -16,6 +16,8 @@ struct TcMaps {
   CUtensorMap act;       // [Rcap rows, F cols]
   CUtensorMap A2;        // same buffers, boxes of half a pair's token tile
   CUtensorMap act2;
+  CUtensorMap A32;       // same buffers, boxes of 32 rows (token-major engines)
+  CUtensorMap act32;
 };
 
 // Encodes the maps for these buffers; returns cudaErrorInvalidValue if the
@@ -28,6 +30,14 @@ int gemm_tc_smem_bytes(bool gateup);
 // Two-SM (cta_group::2) version of launch_gemm_tc: clusters of two CTAs, one
 // per SM pair; each item covers 256 output features.
 cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                            int grid, cudaStream_t s, int which);
+// Token-major engine: 128 token rows x 256 weight rows per MMA (GEMM 1: 128
+// features of gate and up; GEMM 2: 256 features).
+cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
+                           int grid, cudaStream_t s, int which);
+// Two-SM token-major engine: a CTA pair computes 256 tokens x 256 weight
+// rows per MMA (cta_group::2); each CTA holds 128 tokens and half the weights.
+cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                             int grid, cudaStream_t s, int which);
 // Runs the GEMM's bounded mbarrier wait on a barrier nothing arrives on.
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s);

@@ -447,6 +447,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     st->rows = rows;
     st->items1 = it1;
     st->items2 = it2;
+    wk.gemm_next[0] = 0;
+    wk.gemm_next[1] = 0;
     const int step = st->n_steps - 1;  // the row written above
     if (step < d.max_steps) {
       c.trace[step * kTraceCols + 4] = rows;

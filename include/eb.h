@@ -55,15 +55,27 @@ typedef int eb_status;
 #define EB_DTYPE_F32 0
 #define EB_DTYPE_BF16 1
 
-/* expert GEMM engine.  AUTO: tensor cores (tcgen05) for bf16 -- the two-SM
- * engine (cta_group::2, 256 features per CTA pair) for each GEMM whose output
- * width is a multiple of 256, else the one-SM engine -- and SIMT for f32.
- * TC: one-SM tensor-core engine only.  SIMT: CUDA cores.  TC2: two-SM engine
- * (H and F multiples of 256). */
+/* expert GEMM engine (all tensor-core engines use tcgen05 with TMA-fed
+ * operands and TMEM accumulators, and need bf16 with H and F multiples of 128).
+ *   AUTO  bf16: TM for each GEMM it fits, else TC; f32: SIMT.
+ *   TC    one SM per tile; weight rows are the MMA's M side (128 features),
+ *         tokens its N side.
+ *   SIMT  CUDA cores (any shape, f32 or bf16).
+ *   TC2   as TC over an SM pair (cta_group::2, 256 features); F and H
+ *         multiples of 256.
+ *   TM    token-major, one SM: 128 tokens x 256 weight rows per MMA (gate/up:
+ *         128 features of each; down: 256 features); work items are claimed
+ *         dynamically, so CTAs finish together whatever the segment sizes.
+ *   TM2   token-major over an SM pair (cta_group::2): 256 tokens x 256 weight
+ *         rows per MMA, each SM holding 128 tokens and half the weight rows.
+ * TM and TM2 need F a multiple of 128 (gate/up) and H a multiple of 256
+ * (down); a GEMM they do not fit runs on TC. */
 #define EB_GEMM_AUTO 0
 #define EB_GEMM_TC 1
 #define EB_GEMM_SIMT 2
 #define EB_GEMM_TC2 3
+#define EB_GEMM_TM 4
+#define EB_GEMM_TM2 5
 
 /* Limits of this build. */
 #define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */

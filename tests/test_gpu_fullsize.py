@@ -149,12 +149,14 @@ def test_full_shape_chain(torch_mod, name):
         _free()
 
 
+@pytest.mark.parametrize("gemm", [0, 1, 3, 5])
 @pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16", "qwen3_bf16",
                                   "moonlight_bf16", "longctx_bf16"])
-def test_single_step_expert_outputs(torch_mod, name):
+def test_single_step_expert_outputs(torch_mod, name, gemm):
     """The MoE output alone (residual off), one step from h_0 scaled so that
     the expert outputs are O(1): a strong check of the grouped GEMMs, SwiGLU
-    and the gated combine against the oracle at full per-layer sizes."""
+    and the gated combine against the oracle at full per-layer sizes, for
+    every tensor-core engine (gemm 0 is the default, one-SM token-major)."""
     import cross_layer_expert_b200 as eb
     from _common import lib_config
     from oracle import moe as omoe
@@ -169,7 +171,9 @@ def test_single_step_expert_outputs(torch_mod, name):
                  "moonlight_bf16": 1.0, "longctx_bf16": 3.0}[name]
         h0 = synth.hidden_torch(wl, scale=scale).cuda()
         h0_np = h0.float().cpu().numpy().astype(np.float64)
-        cfg = lib_config(wl, osch.MAXUTIL)
+        if gemm == 3 and (wl.H % 256 or wl.F % 256):
+            pytest.skip("the two-SM weight-major engine needs H and F multiples of 256")
+        cfg = lib_config(wl, osch.MAXUTIL, gemm=gemm)
         cfg.residual = 0
         ctx = eb.Context(cfg)
         hidden = h0.clone()

@@ -134,16 +134,25 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
-def ncu_traffic(name: str):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
-    summary says it matches the current build (else None)."""
+def ncu_traffic(name: str, alg_bytes_per_launch: float):
+    """Per-launch DRAM bytes (read + write) of a kernel, from the committed
+    ncu summary profiles/traffic.json: the measured DRAM bytes per algorithmic
+    byte of captured launches, times this run's algorithmic bytes per launch.
+    None when there is no summary for the kernel or its source file changed
+    since the counters were taken (the summary records the file's SHA-256)."""
+    import hashlib
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
-            d = json.load(f)
-        return d.get(name)
+            e = json.load(f).get(name)
+        if not e:
+            return None
+        with open(os.path.join(ROOT, e["source"]), "rb") as f:
+            if hashlib.sha256(f.read()).hexdigest() != e["source_sha256"]:
+                return None
+        return int(e["dram_bytes_per_alg_byte"] * alg_bytes_per_launch)
     except Exception:
         return None
 
@@ -241,11 +250,12 @@ def run_ours(args, world, rank, local):
     kms, kl = prof[kern]
     peak, peak_src = measured_peaks()
     achieved = alg[kern] * args.steps / (kms / 1e3) / 1e9
+    alg_launch = alg[kern] * args.steps / max(1, kl)
     roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kern),
+            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kern, alg_launch),
             "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
             else "fallback 6650 GB/s",
-            "alg_bytes_per_launch": int(alg[kern] * args.steps / max(1, kl)),
+            "alg_bytes_per_launch": int(alg_launch),
             "avg_launch_ms": round(kms / max(1, kl), 5)}
     gemm_ms = prof["gemm_gateup"][0] + prof["gemm_down"][0]
     kernels = {k: {"ms_per_episode": round(v[0] / args.steps, 4), "launches": v[1]}

@@ -1128,24 +1128,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 
 // ---------------------------------------------------------------------------
-// Two-SM token-major variant (cta_group::2).  A CTA pair computes 256 tokens
-// x 256 weight rows: CTA r holds token rows [r0 + 128 r, r0 + 128 r + 128) as
-// its half of the MMA's A operand and weight rows 128 r .. 128 r + 127 of the
-// tile as its half of B (GEMM 1: r = 0 the gate rows, r = 1 the up rows of a
-// 128-feature block; GEMM 2: the lower / upper 128 of 256 features).  Every
-// MMA is 256 x 256 x 16 over the pair, so a weight tile read into the pair
-// serves twice the tokens of the one-SM engine; CTA r's accumulator holds
-// its 128 tokens' 256 outputs, so SwiGLU and the stores stay local.
+// Two-SM token-major variant (cta_group::2).  A CTA pair computes one chunk
+// of up to 256 tokens against 256 weight rows.  The weight tile is split
+// between the pair's shared memories (B operand halves), so each SM loads
+// half of it; the chunk's tokens are split too (A operand halves):
+//  - more than 128 tokens: an M = 256 MMA, 128 tokens per CTA;
+//  - up to 128 tokens: an M = 128 MMA, 64 tokens per CTA.
+// Both shapes run at the tensor pipe's full rate, so a small segment costs a
+// pair no more SM time than the one-SM engine and half the shared-memory
+// bytes per SM.
+//
+// B half of CTA r: GEMM 1: gate rows f0 + 64 r .. + 63 then the matching up
+// rows (two 64-row boxes); GEMM 2: output rows f0 + 128 r .. + 127.  With this
+// order every accumulator lane holds the gate and up values of the same
+// features side by side (SwiGLU stays in one thread), for both MMA shapes:
+//  - M = 256: lane l is token 128 r + l; columns [128 G, 128 G + 64) are the
+//    gate and [128 G + 64, 128 G + 128) the up values of features
+//    f0 + 64 G .. (GEMM 1, G = 0, 1); columns 0..255 are features f0..f0+255
+//    (GEMM 2).
+//  - M = 128: lane l < 64 is token 64 r + l with columns 0..127 = the pair's
+//    N columns 0..127; lane 64 + l is the same token with N columns 128..255.
 // ---------------------------------------------------------------------------
 
 template <bool GATEUP>
 struct CfgTM2 {
-  static constexpr int kRows = 2 * kTmRows;          // token rows per pair item
+  static constexpr int kRows = 2 * kTmRows;          // token rows per pair item (at most)
   static constexpr int kFeat = GATEUP ? kTmFeat1 : kTmFeat2;
-  static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KiB: this CTA's tokens
+  static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KiB: this CTA's tokens (at most)
   static constexpr int kBBytes = 128 * kBK * 2;      // 16 KiB: this CTA's weight rows
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 204800 / kStageBytes;  // 6
+  static constexpr int kStages = 196608 / kStageBytes;  // 6
   static constexpr int kAccCols = 256;
   static constexpr int kAccBufs = 2;
   static constexpr int kTmemCols = kAccBufs * kAccCols;
@@ -1170,6 +1182,15 @@ __device__ __forceinline__ Item decode_tm2(const Dims& d, const int32_t* seg_row
   return it;
 }
 
+// Tokens of a pair item held by CTA `rank`, and where they start in the item.
+__device__ __forceinline__ void pair_split(int n, uint32_t rank, int* first, int* count) {
+  const int per = n > kTmRows ? kTmRows : kTmRows / 2;  // tokens per CTA: M / 2
+  *first = (int)rank * per;
+  *count = min(max(n - *first, 0), per);
+}
+
+// map_w: GATEUP w_gateup in boxes of 64 rows, else w_down in boxes of 128
+// rows; map_x: token rows in boxes of 32 rows.
 template <bool GATEUP>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tm2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
@@ -1232,15 +1253,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
       bool ok = true;
+      Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, pair < total ? pair : 0);
       for (int item = pair; item < total && ok; item += npairs) {
-        const Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
-        // token rows of each CTA and the 32-row boxes that cover them
-        const int n0 = min(it.n, kTmRows), n1 = it.n - n0;
-        const int nb0 = (n0 + kTmBox - 1) / kTmBox, nb1 = (n1 + kTmBox - 1) / kTmBox;
-        const int nbox = rank == 0 ? nb0 : nb1;
-        const int xrow = it.r0 + (int)rank * kTmRows;
-        const int wrow = GATEUP ? it.wrow + (int)rank * d.F : it.wrow + (int)rank * 128;
-        const uint32_t tx = (uint32_t)((nb0 + nb1) * kTmBoxBytes + 2 * C::kBBytes);
+        int first0, cnt0, first1, cnt1, first, cnt;
+        pair_split(it.n, 0, &first0, &cnt0);
+        pair_split(it.n, 1, &first1, &cnt1);
+        pair_split(it.n, rank, &first, &cnt);
+        const int nbox = (cnt + kTmBox - 1) / kTmBox;
+        const uint32_t tx = (uint32_t)(((cnt0 + kTmBox - 1) / kTmBox + (cnt1 + kTmBox - 1) / kTmBox) *
+                                           kTmBoxBytes +
+                                       2 * C::kBBytes);
+        const int xrow = it.r0 + first;
+        // this CTA's B half (see the layout note above)
+        const int w0 = GATEUP ? it.wrow + 64 * (int)rank : it.wrow + 128 * (int)rank;
+        const int w1 = it.wrow + d.F + 64 * (int)rank;  // GATEUP only: the up rows
+        const int next = item + npairs;
+        Item nx = it;
         for (int kb = 0; kb < nk; ++kb) {
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
             ok = false;
@@ -1256,12 +1284,20 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           for (int b = 0; b < nbox; ++b)
             tma_load_2d_pair(smem_u32(sb + b * kTmBoxBytes), &map_x, kb * kBK, xrow + b * kTmBox, fb);
-          tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, wrow, fb);
+          if (GATEUP) {
+            tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
+            tma_load_2d_pair(smem_u32(sb + C::kABytes + C::kBBytes / 2), &map_w, kb * kBK, w1, fb);
+          } else {
+            tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
+          }
           if (++stage == C::kStages) {
             stage = 0;
             phase ^= 1;
           }
+          // decode the next item while this item's copies are in flight
+          if (kb == 0 && next < total) nx = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, next);
         }
+        it = nx;
       }
       if (!ok && leader) {  // the leader's barriers count both CTAs' copies
         for (int s2 = 0; s2 < C::kStages; ++s2)
@@ -1282,8 +1318,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t acc_phase = 0;
       uint32_t last_bar = 0, last_par = 0;
       bool ok = true, issued = false;
-      const uint32_t idesc = idesc_bf16(256, 256);
+      Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, pair < total ? pair : 0);
       for (int item = pair; item < total && ok; item += npairs) {
+        const uint32_t idesc = idesc_bf16(it.n > kTmRows ? 256 : 128, 256);
+        const int next = item + npairs;
+        Item nx = it;
         if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
           ok = false;
           break;
@@ -1311,6 +1350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             stage = 0;
             phase ^= 1;
           }
+          if (kb == 0 && next < total) nx = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, next);
         }
         if (!ok) break;
         mma_commit_pair(smem_u32(&tfull[acc]));
@@ -1320,6 +1360,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc = 0;
           acc_phase ^= 1;
         }
+        it = nx;
       }
       if (!ok && issued) {
         const unsigned long long t0 = global_ns();
@@ -1329,6 +1370,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ drain (both CTAs)
+    // warp w reads TMEM lanes 32 (w % 4) .. +31; the two warps sharing a lane
+    // quarter split its 32-feature blocks.
     const int q = warp & 3;
     const int cgrp = (warp - 2) >> 2;
     constexpr int kGroups = kEpiWarps / 4;
@@ -1338,20 +1381,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
       if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
       tc_fence_after();
-      const int nmine = min(max(it.n - (int)rank * kTmRows, 0), kTmRows);  // this CTA's tokens
-      const int row = q * 32 + lane;
-      const bool live = row < nmine;
+      int first, cnt;
+      pair_split(it.n, rank, &first, &cnt);
+      const bool wide = it.n > kTmRows;  // M = 256
+      // token of this lane within the CTA's share, the features it holds and
+      // the 32-feature blocks that cover them
+      const int tok = wide ? q * 32 + lane : (q & 1) * 32 + lane;
+      const bool live = tok < cnt;
+      const int fbase = wide ? 0 : (q >> 1) * (C::kFeat / 2);
+      const int nblk = (wide ? C::kFeat : C::kFeat / 2) / 32;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      __nv_bfloat16* orow = out + (size_t)(it.r0 + (int)rank * kTmRows + row) * NOUT + it.f0;
-      constexpr int kBlocks = C::kFeat / 32;
-      const int b_end = q * 32 < nmine ? kBlocks : 0;
+      __nv_bfloat16* orow = out + (size_t)(it.r0 + first + tok) * NOUT + it.f0 + fbase;
+      // a lane quarter whose tokens are all past the share has nothing to drain
+      const int b_end = ((wide ? q * 32 : (q & 1) * 32) < cnt) ? nblk : 0;
       for (int b = cgrp; b < b_end; b += kGroups) {
         float g[32];
-        tmem_ld32(tbase + b * 32, g);
         uint32_t packed[16];
         if (GATEUP) {
+          // features 64 G + 32 h of this lane's range: gate at column 128 G + 32 h,
+          // up 64 columns further
+          const int G = b >> 1, h = b & 1;
           float u[32];
-          tmem_ld32(tbase + 128 + b * 32, u);
+          tmem_ld32(tbase + 128 * G + 32 * h, g);
+          tmem_ld32(tbase + 128 * G + 64 + 32 * h, u);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float a0 = g[2 * i] / (1.f + expf(-g[2 * i])) * u[2 * i];
@@ -1359,6 +1411,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             packed[i] = pack_bf16x2(a0, a1);
           }
         } else {
+          tmem_ld32(tbase + 32 * b, g);
 #pragma unroll
           for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
         }
@@ -1461,7 +1514,7 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
   if (which == 1) {
     cfg.dynamicSmemBytes = CfgTM2<true>::kSmemBytes;
     cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<true>, cfg, grid / 2));
-    return cudaLaunchKernelEx(&cfg, k_gemm_tm2<true>, maps.w_gateup, maps.A32, d, c.st, w.seg_rows,
+    return cudaLaunchKernelEx(&cfg, k_gemm_tm2<true>, maps.w_gateup64, maps.A32, d, c.st, w.seg_rows,
                               w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
   }
   cfg.dynamicSmemBytes = CfgTM2<false>::kSmemBytes;
@@ -1570,6 +1623,7 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kTcRows2);
   if (e == cudaSuccess) e = encode(&maps->A2, w.A, (unsigned long long)w.Rcap, d.H, kTc2Rows1 / 2);
   if (e == cudaSuccess) e = encode(&maps->act2, w.act, (unsigned long long)w.Rcap, d.F, kTc2Rows2 / 2);
+  if (e == cudaSuccess) e = encode(&maps->w_gateup64, w_gateup, experts * 2 * d.F, d.H, 64);
   if (e == cudaSuccess) e = encode(&maps->A32, w.A, (unsigned long long)w.Rcap, d.H, kTmBox);
   if (e == cudaSuccess) e = encode(&maps->act32, w.act, (unsigned long long)w.Rcap, d.F, kTmBox);
   return e;

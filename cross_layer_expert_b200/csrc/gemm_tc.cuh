@@ -16,6 +16,7 @@ struct TcMaps {
   CUtensorMap act;       // [Rcap rows, F cols]
   CUtensorMap A2;        // same buffers, boxes of half a pair's token tile
   CUtensorMap act2;
+  CUtensorMap w_gateup64;  // w_gateup in boxes of 64 rows (two-SM token-major engine)
   CUtensorMap A32;       // same buffers, boxes of 32 rows (token-major engines)
   CUtensorMap act32;
 };
@@ -35,8 +36,9 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
 // features of gate and up; GEMM 2: 256 features).
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                            int grid, cudaStream_t s, int which);
-// Two-SM token-major engine: a CTA pair computes 256 tokens x 256 weight
-// rows per MMA (cta_group::2); each CTA holds 128 tokens and half the weights.
+// Two-SM token-major engine (cta_group::2): a CTA pair computes a chunk of up
+// to 256 tokens against 256 weight rows; each CTA holds half the tokens and
+// half the weight rows (M = 256 MMAs above 128 tokens, M = 128 below).
 cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                             int grid, cudaStream_t s, int which);
 // Runs the GEMM's bounded mbarrier wait on a barrier nothing arrives on.

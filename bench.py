@@ -70,13 +70,21 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest of every rank's x (all ranks call it, in the same order)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def job_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput: the units every rank processed over the slowest
+    rank's time (replicas do equal work, so weak scaling)."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 class ClockSampler:
@@ -242,8 +250,7 @@ def run_ours(args, world, rank, local):
     launches = ctx.eb_launch_count() - launches0
     assert ctx.eb_sync_status() == eb.EB_OK
     ms_max = max_over_ranks(ms_total, world)
-    tokens = wl.M * wl.T * wl.L * args.steps * world
-    value = tokens / (ms_max / 1e3)
+    value = job_throughput(wl.M * wl.T * wl.L * args.steps, ms_max, world)
 
     # roofline of the dominant kernel
     kern = max(("gemm_gateup", "gemm_down", "permute", "combine"), key=lambda k: prof[k][0])
@@ -286,7 +293,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
         barrier(world)
         ms_e2e = max_over_ranks(e0.elapsed_time(e1), world)
-        e2e = {"value": round(wl.M * wl.T * wl.L * k_e2e * world / (ms_e2e / 1e3), 1),
+        e2e = {"value": round(job_throughput(wl.M * wl.T * wl.L * k_e2e, ms_e2e, world), 1),
                "unit": UNIT,
                "h2d_bytes_per_step": int(lg_host.numel() * 4 + h_host.numel() * h_host.element_size()),
                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),

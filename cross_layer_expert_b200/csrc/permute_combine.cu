@@ -11,9 +11,14 @@
 // [EB-read] §2.1: scheduling may change neither the expert set, the gates nor
 // the aggregation order -- the slot order here is fixed.
 //
-// Both kernels are HBM-bound copies: one warp per token row, 16-byte vector
-// loads and stores, each row read once and written (permute) k + n_shared
-// times or k + n_shared rows read and one written (combine).
+// The permutation is two launches: k_positions computes every (token, slot)
+// row of the RunSet (a light pass over the routing indices), then
+// k_permute_copy moves the rows.  The copy and the combine are HBM-bound and
+// persistent: a grid of resident CTAs sized to the SM count strides over the
+// RunSet's tokens, one warp per token row with 16-byte vector loads and
+// stores, so the work spreads evenly over the SMs whatever the RunSet size
+// (no partial last wave).  Each row is read once and written k + n_shared
+// times (permute), or k + n_shared rows are read and one written (combine).
 #include <cuda_bf16.h>
 
 #include "eb_internal.cuh"
@@ -34,24 +39,16 @@ __device__ __forceinline__ unsigned lanemask_lt() {
 // CTA (c, j): chunk c of RunSet micro-batch j.  Row of (t, s) = base of
 // (j, c, expert) + number of earlier (t', s') of this chunk with the same
 // expert, so rows follow (micro-batch, token, slot) order inside a segment.
-// Each chunk's ranks are computed by kPermSplit CTAs (cheap, identical); each
-// copies a quarter of the chunk's tokens, so the HBM-bound copy has 4x the CTAs.
-constexpr int kPermSplit = 4;
-
-template <typename T>
-__global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* __restrict__ st,
-                                                          const int32_t* __restrict__ idx,
-                                                          const int32_t* __restrict__ chunk_hist,
-                                                          const int32_t* __restrict__ seg_rows,
-                                                          const int32_t* __restrict__ prior,
-                                                          int32_t* __restrict__ pos,
-                                                          const T* __restrict__ hidden,
-                                                          T* __restrict__ A) {
-  const int c = blockIdx.x / kPermSplit, part = blockIdx.x % kPermSplit, j = blockIdx.y;
+__global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State* __restrict__ st,
+                                                            const int32_t* __restrict__ idx,
+                                                            const int32_t* __restrict__ chunk_hist,
+                                                            const int32_t* __restrict__ seg_rows,
+                                                            const int32_t* __restrict__ prior,
+                                                            int32_t* __restrict__ pos) {
+  const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
   __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
   __shared__ int running[EB_MAX_ETOT];
-  __shared__ int dest[kChunk * kMaxSlots];
   __shared__ int bj[EB_MAX_ETOT];  // first row of (j, this chunk, expert)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = c * kChunk, nt = min(kChunk, d.T - t0);
@@ -78,6 +75,7 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
   for (int e = tid; e < E; e += kPermThreads) running[e] = 0;
   const int npairs = nt * k;
   const int32_t* idx_c = idx + ((size_t)j * d.T + t0) * k;
+  int32_t* pos_c = pos + ((size_t)j * d.T + t0) * kk;
   for (int r0 = 0; r0 < npairs; r0 += kPermThreads) {
     for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) cnt[i / E][i % E] = 0;
     __syncthreads();
@@ -97,55 +95,68 @@ __global__ void __launch_bounds__(kPermThreads) k_permute(Dims d, const State* _
       running[ee] = run;
     }
     __syncthreads();
-    if (e >= 0) {
-      const int t = p / k, s = p % k;
-      const int row = bj[e] + cnt[warp][e] + rank;
-      dest[t * kk + s] = row;
-      if (part == 0) pos[((size_t)j * d.T + t0 + t) * kk + s] = row;
-    }
+    if (e >= 0) pos_c[(p / k) * kk + p % k] = bj[e] + cnt[warp][e] + rank;
     __syncthreads();
   }
   for (int i = tid; i < nt * d.n_shared; i += kPermThreads) {
     const int t = i / d.n_shared, s = i % d.n_shared;
-    const int row = bj[E + s] + t;
-    dest[t * kk + k + s] = row;
-    if (part == 0) pos[((size_t)j * d.T + t0 + t) * kk + k + s] = row;
+    pos_c[t * kk + k + s] = bj[E + s] + t;
   }
-  __syncthreads();
+}
+
+// Token u of the RunSet (members in ascending order, T tokens each).
+__device__ __forceinline__ size_t runset_token(const State* st, int T, int u) {
+  return (size_t)st->run_list[u / T] * T + (u % T);
+}
+
+// Persistent copy: warp w moves tokens w, w + W, ... (W = warps in the grid),
+// two at a time: both rows' 16-byte vectors are loaded into registers (8 per
+// lane per token) before the k + n_shared stores of each.
+template <typename T>
+__global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const State* __restrict__ st,
+                                                               const int32_t* __restrict__ pos,
+                                                               const T* __restrict__ hidden,
+                                                               T* __restrict__ A) {
+  const int lane = threadIdx.x & 31;
+  const int W = (int)(gridDim.x * (kPermThreads / 32));
+  const int wid = (int)(blockIdx.x * (kPermThreads / 32) + (threadIdx.x >> 5));
+  const int units = st->n_run * d.T;
+  const int kk = d.kk;
   const int nvec = d.H * (int)sizeof(T) / 16;
-  const int per = (nt + kPermSplit - 1) / kPermSplit;
-  const int ta = part * per, tb = min(nt, ta + per);
-  // each warp copies two tokens at a time: both rows' 16-byte vectors are
-  // loaded into registers (8 per lane per token) before any store is issued
   constexpr int kU = 8;
-  for (int t = ta + warp; t < tb; t += 2 * (kPermThreads / 32)) {
-    const int t2 = t + kPermThreads / 32;
-    const bool two = t2 < tb;
-    const uint4* src0 = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + t) * d.H);
-    const uint4* src1 = reinterpret_cast<const uint4*>(hidden + ((size_t)j * d.T + t0 + (two ? t2 : t)) * d.H);
+  for (int u = wid; u < units; u += 2 * W) {
+    const int u2 = u + W;
+    const bool two = u2 < units;
+    const size_t tok0 = runset_token(st, d.T, u), tok1 = runset_token(st, d.T, two ? u2 : u);
+    // slot rows of both tokens, one per lane
+    const int row0 = lane < kk ? __ldg(pos + tok0 * kk + lane) : 0;
+    const int row1 = lane < kk ? __ldg(pos + tok1 * kk + lane) : 0;
+    const uint4* src0 = reinterpret_cast<const uint4*>(hidden + tok0 * d.H);
+    const uint4* src1 = reinterpret_cast<const uint4*>(hidden + tok1 * d.H);
     for (int base = 0; base < nvec; base += 32 * kU) {
       uint4 v0[kU], v1[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int v = base + u * 32 + lane;
+      for (int q = 0; q < kU; ++q) {
+        const int v = base + q * 32 + lane;
         if (v < nvec) {
-          v0[u] = __ldg(src0 + v);
-          if (two) v1[u] = __ldg(src1 + v);
+          v0[q] = __ldg(src0 + v);
+          if (two) v1[q] = __ldg(src1 + v);
         }
       }
       for (int s = 0; s < kk; ++s) {
-        uint4* dst0 = reinterpret_cast<uint4*>(A + (size_t)dest[t * kk + s] * d.H);
+        uint4* dst0 = reinterpret_cast<uint4*>(A + (size_t)__shfl_sync(kFull, row0, s) * d.H);
+        const int r1 = __shfl_sync(kFull, row1, s);
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
-          const int v = base + u * 32 + lane;
-          if (v < nvec) dst0[v] = v0[u];
+        for (int q = 0; q < kU; ++q) {
+          const int v = base + q * 32 + lane;
+          if (v < nvec) dst0[v] = v0[q];
         }
         if (two) {
-          uint4* dst1 = reinterpret_cast<uint4*>(A + (size_t)dest[t2 * kk + s] * d.H);
+          uint4* dst1 = reinterpret_cast<uint4*>(A + (size_t)r1 * d.H);
 #pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int v = base + u * 32 + lane;
-            if (v < nvec) dst1[v] = v1[u];
+          for (int q = 0; q < kU; ++q) {
+            const int v = base + q * 32 + lane;
+            if (v < nvec) dst1[v] = v1[q];
           }
         }
       }
@@ -215,104 +226,133 @@ struct Vec<__nv_bfloat16> {
   }
 };
 
-constexpr int kCombineTokens = 8;  // one warp per token
+constexpr int kCombineThreads = 256;
 
+// Persistent: warp w combines tokens w, w + W, ... of the RunSet.
 template <typename T>
-__global__ void __launch_bounds__(256) k_combine(Dims d, const State* __restrict__ st,
-                                                  const float* __restrict__ gate,
-                                                  const int32_t* __restrict__ pos,
-                                                  const T* __restrict__ y, T* hidden) {
-  const int j = blockIdx.y;
-  if (!((st->runset >> j) & 1u)) return;
-  __shared__ int s_row[kCombineTokens][kMaxSlots];
-  __shared__ float s_gate[kCombineTokens][kMaxSlots];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int t = blockIdx.x * kCombineTokens + warp;
-  if (t >= d.T) return;
+__global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State* __restrict__ st,
+                                                             const float* __restrict__ gate,
+                                                             const int32_t* __restrict__ pos,
+                                                             const T* __restrict__ y, T* hidden) {
+  const int lane = threadIdx.x & 31;
+  const int W = (int)(gridDim.x * (kCombineThreads / 32));
+  const int wid = (int)(blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5));
+  const int units = st->n_run * d.T;
   const int k = d.k, kk = d.kk;
   constexpr int VE = Vec<T>::n;
   const int nvec = d.H / VE;
-  const size_t tok = (size_t)j * d.T + t;
-  if (lane < kk) s_row[warp][lane] = pos[tok * kk + lane];
-  if (lane < k) s_gate[warp][lane] = gate[tok * k + lane];
-  __syncwarp();
-  T* out = hidden + tok * d.H;
-  // two 16-byte vectors per lane per pass: 2 * kk loads in flight
-  for (int v0 = lane; v0 < nvec; v0 += 64) {
-    const int v1 = v0 + 32;
-    const bool has1 = v1 < nvec;
-    float acc0[VE], acc1[VE];
-    if (d.residual) {
-      Vec<T>::load_plain(out, v0, acc0);
-      if (has1) Vec<T>::load_plain(out, v1, acc1);
-    } else {
+  for (int u = wid; u < units; u += W) {
+    const size_t tok = runset_token(st, d.T, u);
+    // slot rows and gates, one per lane
+    const int my_row = lane < kk ? __ldg(pos + tok * kk + lane) : 0;
+    const float my_gate = lane < k ? __ldg(gate + tok * k + lane) : 0.f;
+    T* out = hidden + tok * d.H;
+    // two 16-byte vectors per lane per pass: 2 * kk loads in flight
+    for (int v0 = lane; v0 < nvec; v0 += 64) {
+      const int v1 = v0 + 32;
+      const bool has1 = v1 < nvec;
+      float acc0[VE], acc1[VE];
+      if (d.residual) {
+        Vec<T>::load_plain(out, v0, acc0);
+        if (has1) Vec<T>::load_plain(out, v1, acc1);
+      } else {
 #pragma unroll
-      for (int i = 0; i < VE; ++i) acc0[i] = acc1[i] = 0.f;
-    }
-    for (int s0 = 0; s0 < kk; s0 += 8) {
-      uint4 r0[8], r1[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (s0 + u < kk) {
-          const uint4* yrow = reinterpret_cast<const uint4*>(y + (size_t)s_row[warp][s0 + u] * d.H);
-          r0[u] = __ldg(yrow + v0);
-          if (has1) r1[u] = __ldg(yrow + v1);
-        }
+        for (int i = 0; i < VE; ++i) acc0[i] = acc1[i] = 0.f;
       }
+      for (int s0 = 0; s0 < kk; s0 += 8) {
+        uint4 r0[8], r1[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s0 + u;
-        if (s >= kk) break;
-        float y0[VE], y1[VE];
-        Vec<T>::unpack(r0[u], y0);
-        if (has1) Vec<T>::unpack(r1[u], y1);
-        if (s < k) {
-          const float g = s_gate[warp][s];
-#pragma unroll
-          for (int i = 0; i < VE; ++i) {
-            acc0[i] = fmaf(g, y0[i], acc0[i]);
-            if (has1) acc1[i] = fmaf(g, y1[i], acc1[i]);
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < VE; ++i) {
-            acc0[i] += y0[i];
-            if (has1) acc1[i] += y1[i];
+        for (int q = 0; q < 8; ++q) {
+          const int row = __shfl_sync(kFull, my_row, (s0 + q) & 31);
+          if (s0 + q < kk) {
+            const uint4* yrow = reinterpret_cast<const uint4*>(y + (size_t)row * d.H);
+            r0[q] = __ldg(yrow + v0);
+            if (has1) r1[q] = __ldg(yrow + v1);
           }
         }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const int s = s0 + q;
+          const float g = __shfl_sync(kFull, my_gate, s & 31);
+          if (s >= kk) break;
+          float y0[VE], y1[VE];
+          Vec<T>::unpack(r0[q], y0);
+          if (has1) Vec<T>::unpack(r1[q], y1);
+          if (s < k) {
+#pragma unroll
+            for (int i = 0; i < VE; ++i) {
+              acc0[i] = fmaf(g, y0[i], acc0[i]);
+              if (has1) acc1[i] = fmaf(g, y1[i], acc1[i]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < VE; ++i) {
+              acc0[i] += y0[i];
+              if (has1) acc1[i] += y1[i];
+            }
+          }
+        }
       }
+      Vec<T>::store(out, v0, acc0);
+      if (has1) Vec<T>::store(out, v1, acc1);
     }
-    Vec<T>::store(out, v0, acc0);
-    if (has1) Vec<T>::store(out, v1, acc1);
   }
 }
 
 }  // namespace
 
+// Resident CTAs of a persistent kernel: its blocks per SM (by registers and
+// shared memory) times the SM count, queried on the first launch and kept in
+// the caller's `cache`.
+int persistent_grid(const void* kernel, int threads, int& cache) {
+  if (cache == 0) {
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, 0) == cudaSuccess &&
+        sms > 0 && per_sm > 0)
+      cache = sms * per_sm;
+    else
+      cache = 148;
+  }
+  return cache;
+}
+
+int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb_f32 = 0;
+
 cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                            cudaStream_t s) {
-  dim3 grid(d.NC * kPermSplit, d.M);
+  k_positions<<<dim3(d.NC, d.M), kPermThreads, 0, s>>>(d, c.st, w.idx, w.chunk_hist, w.seg_rows,
+                                                      w.prior, w.pos);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
   if (d.dtype == EB_DTYPE_BF16)
-    k_permute<__nv_bfloat16><<<grid, kPermThreads, 0, s>>>(
-        d, c.st, w.idx, w.chunk_hist, w.seg_rows, w.prior, w.pos,
-        static_cast<const __nv_bfloat16*>(hidden), static_cast<__nv_bfloat16*>(w.A));
+    k_permute_copy<__nv_bfloat16>
+        <<<persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads, g_grid_copy_bf16),
+           kPermThreads, 0, s>>>(
+            d, c.st, w.pos, static_cast<const __nv_bfloat16*>(hidden),
+            static_cast<__nv_bfloat16*>(w.A));
   else
-    k_permute<float><<<grid, kPermThreads, 0, s>>>(d, c.st, w.idx, w.chunk_hist, w.seg_rows,
-                                                   w.prior, w.pos, static_cast<const float*>(hidden),
-                                                   static_cast<float*>(w.A));
+    k_permute_copy<float>
+        <<<persistent_grid((const void*)k_permute_copy<float>, kPermThreads, g_grid_copy_f32),
+           kPermThreads, 0, s>>>(d, c.st, w.pos, static_cast<const float*>(hidden),
+                                 static_cast<float*>(w.A));
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
                            cudaStream_t s) {
-  dim3 grid((d.T + kCombineTokens - 1) / kCombineTokens, d.M);
   if (d.dtype == EB_DTYPE_BF16)
-    k_combine<__nv_bfloat16><<<grid, 256, 0, s>>>(d, c.st, w.gate, w.pos,
-                                                  static_cast<const __nv_bfloat16*>(w.y),
-                                                  static_cast<__nv_bfloat16*>(hidden));
+    k_combine<__nv_bfloat16>
+        <<<persistent_grid((const void*)k_combine<__nv_bfloat16>, kCombineThreads, g_grid_comb_bf16),
+           kCombineThreads, 0, s>>>(
+            d, c.st, w.gate, w.pos, static_cast<const __nv_bfloat16*>(w.y),
+            static_cast<__nv_bfloat16*>(hidden));
   else
-    k_combine<float><<<grid, 256, 0, s>>>(d, c.st, w.gate, w.pos, static_cast<const float*>(w.y),
-                                          static_cast<float*>(hidden));
+    k_combine<float>
+        <<<persistent_grid((const void*)k_combine<float>, kCombineThreads, g_grid_comb_f32),
+           kCombineThreads, 0, s>>>(d, c.st, w.gate, w.pos, static_cast<const float*>(w.y),
+                                    static_cast<float*>(hidden));
   return cudaGetLastError();
 }
 

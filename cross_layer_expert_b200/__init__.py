@@ -29,7 +29,7 @@ EB_ERR_TOO_LARGE = -7
 
 CUMUTIL, MAXUTIL, LOCKSTEP, DIFFPEAK = 0, 1, 2, 3
 DTYPE_F32, DTYPE_BF16 = 0, 1
-GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TC2, GEMM_TM, GEMM_TM2 = 0, 1, 2, 3, 4, 5
+GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TC2, GEMM_TM, GEMM_TM2, GEMM_TMG = 0, 1, 2, 3, 4, 5, 6
 
 EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_create", "eb_destroy",
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",

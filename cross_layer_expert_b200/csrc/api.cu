@@ -50,7 +50,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 bool use_tc_for(const eb_config& c) {
   if (c.dtype != EB_DTYPE_BF16) return false;
   return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC || c.gemm == EB_GEMM_TC2 ||
-         c.gemm == EB_GEMM_TM || c.gemm == EB_GEMM_TM2;
+         c.gemm == EB_GEMM_TM || c.gemm == EB_GEMM_TM2 || c.gemm == EB_GEMM_TMG;
 }
 
 // Engine of each GEMM.  AUTO takes the one-SM token-major engine for every
@@ -68,12 +68,15 @@ void choose_engines(const eb_config& c, bool use_tc, int num_sms, int* g1, int* 
       case EB_GEMM_TC: return true;
       case EB_GEMM_TC2: return pair_ok && nout % kTc2Feat == 0;
       case EB_GEMM_TM: return nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
+      case EB_GEMM_TMG: return which == 1 && nout % kTmFeat1 == 0;
       case EB_GEMM_TM2: return pair_ok && nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
       default: return false;
     }
   };
   *g1 = fits(want, 1) ? want : EB_GEMM_TC;
-  *g2 = fits(want, 2) ? want : EB_GEMM_TC;
+  // TMG gathers GEMM 1's input; its GEMM 2 is the token-major one
+  const int want2 = want == EB_GEMM_TMG ? EB_GEMM_TM : want;
+  *g2 = fits(want2, 2) ? want2 : EB_GEMM_TC;
 }
 
 // Token rows and output features of one work item of `eng` for GEMM `which`.
@@ -88,6 +91,7 @@ void engine_tiles(int eng, int which, int* rows, int* feats) {
       *feats = kTc2Feat;
       return;
     case EB_GEMM_TM:
+    case EB_GEMM_TMG:
       *rows = kTmRows;
       *feats = which == 1 ? kTmFeat1 : kTmFeat2;
       return;
@@ -132,6 +136,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   if (c.compute) {
     x.prior = (int32_t*)take(sizeof(int32_t) * M * d.Etot);
     x.pos = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
+    x.rowmap = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
     x.seg_rows = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.seg_wid = (int32_t*)take(sizeof(int32_t) * nseg);
     x.seg_items1 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
@@ -205,7 +210,7 @@ eb_status eb_config_check(const eb_config* c) {
   if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
   if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
   if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
-  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TM2) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TMG) return EB_ERR_INVALID_ARG;
   if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
@@ -218,7 +223,7 @@ eb_status eb_config_check(const eb_config* c) {
     if (c->H % vec != 0) return EB_ERR_UNSUPPORTED;
     if ((long long)c->M * c->T * (c->k + c->n_shared) > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
     const bool forced_tc = c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2 ||
-                           c->gemm == EB_GEMM_TM || c->gemm == EB_GEMM_TM2;
+                           c->gemm == EB_GEMM_TM || c->gemm == EB_GEMM_TM2 || c->gemm == EB_GEMM_TMG;
     if (c->dtype == EB_DTYPE_F32 && forced_tc) return EB_ERR_UNSUPPORTED;
     if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
       if (forced_tc) return EB_ERR_UNSUPPORTED;
@@ -308,7 +313,8 @@ static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* 
   switch (eng) {
     case EB_GEMM_TC: return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     case EB_GEMM_TC2: return launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
-    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which);
+    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, false);
+    case EB_GEMM_TMG: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, true);
     case EB_GEMM_TM2: return launch_gemm_tm2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     default: return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, which);
   }
@@ -334,6 +340,13 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     x->map_keys[1] = wdn;
     x->map_keys[2] = workspace;
   }
+  // GEMM 1 on the gathering engine reads its token rows from `hidden` itself
+  // (no permuted copy)
+  const bool gather = c.compute && x->eng1 == EB_GEMM_TMG;
+  if (gather && x->map_keys[3] != hidden) {
+    if (make_hidden_map(x->d, hidden, &x->maps) != cudaSuccess) return EB_ERR_UNSUPPORTED;
+    x->map_keys[3] = hidden;
+  }
   const int g1 = c.compute ? x->eng1 : EB_GEMM_SIMT, g2 = c.compute ? x->eng2 : EB_GEMM_SIMT;
   int rn1, fm1, rn2, fm2;
   engine_tiles(g1, 1, &rn1, &fm1);
@@ -343,7 +356,7 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
   if (c.compute) {
     if (e == cudaSuccess)
-      e = timed(x, 2, 2, s, [&] { return launch_permute(x->d, x->dev, w, hidden, s); });
+      e = timed(x, 2, gather ? 1 : 2, s, [&] { return launch_permute(x->d, x->dev, w, hidden, !gather, s); });
     if (e == cudaSuccess) {
       e = timed(x, 3, 1, s, [&] { return launch_engine(x, g1, w, wgu, wdn, s, 1); });
       if (e == cudaSuccess)

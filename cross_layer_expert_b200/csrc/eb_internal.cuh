@@ -79,6 +79,7 @@ struct Work {
   int32_t* chunk_hist; // [M][NC][E]: counts of each 64-token chunk
   int32_t* prior;      // [M][Etot]: rows of (j's segment, expert) taken by earlier RunSet members
   int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
+  int32_t* rowmap;     // [Rcap]: token (j * T + t) of each permuted row
   int32_t* seg_rows;   // [M*Etot + 1]
   int32_t* seg_wid;    // [M*Etot]: layer * Etot + expert
   int32_t* seg_items1; // [M*Etot + 1]
@@ -112,8 +113,10 @@ cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int 
                                  int policy, uint32_t* runset, long long* stats, cudaStream_t s);
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s);
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
+// Rows of every (token, slot) of the RunSet (pos, rowmap); with `copy`, also
+// the permuted copy A of the token rows.
 cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
-                           cudaStream_t s);
+                           bool copy, cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
                            cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) on the CUDA cores.

@@ -114,6 +114,17 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Four rows y0..y3 (x .. x + box width) of a tensor whose map has a one-row
+// box, landing as four consecutive shared-memory rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0,
+                                            int y1, int y2, int y3, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -870,15 +881,19 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// map_x: token rows [Rcap, K] in boxes of 32 rows; map_w: weights in boxes of
-// 128 rows.  GATEUP: out = act [Rcap, F]; else out = y [Rcap, H].  next_item:
-// the step's claim counter (zero before the launch).
-template <bool GATEUP>
+// map_x: token rows [Rcap, K] in boxes of 32 rows -- or, GATHER, the caller's
+// hidden states [M*T, H] in one-row boxes, gathered row by row through
+// rowmap (permuted row -> token) so the permuted copy is never written;
+// map_w: weights in boxes of 128 rows.  GATEUP: out = act [Rcap, F]; else
+// out = y [Rcap, H].  next_item: the step's claim counter (zero before the
+// launch).
+template <bool GATEUP, bool GATHER>
 __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-              int32_t* __restrict__ next_item, __nv_bfloat16* __restrict__ out) {
+              int32_t* __restrict__ next_item, const int32_t* __restrict__ rowmap,
+              __nv_bfloat16* __restrict__ out) {
   using C = CfgTM<GATEUP>;
   constexpr int Q = C::kQueue;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -940,7 +955,82 @@ __global__ void __launch_bounds__(kThreads, 1)
     // starts and decoded once its last k-block is issued (both off the
     // k-block path).  Claimed items go to the MMA issuer and the drain
     // through a queue in shared memory.
-    if (lane == 0) {
+    if (GATHER) {
+      // The whole warp runs the loop: lane 0 waits on the barriers, arms
+      // them and loads the weights; lane i gathers token rows 4i .. 4i + 3
+      // of the chunk (rows past the chunk repeat its last row).
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      int item = (int)blockIdx.x < total ? (int)blockIdx.x : -1;
+      Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item < 0 ? 0 : item);
+      for (int u = 0;; ++u) {
+        const int qs = u % Q;
+        int good = 1;
+        if (lane == 0) {
+          if (u >= Q && !mbar_wait(smem_u32(&ifree[qs]), (uint32_t)(((u / Q) - 1) & 1),
+                                   abort_flag, &st->status)) {
+            good = 0;
+          } else {
+            iq[qs] = item;
+            mbar_arrive(smem_u32(&iready[qs]));  // releases iq[qs]
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) {
+          ok = false;
+          break;
+        }
+        if (item < 0) break;
+        int claim = 0;
+        if (lane == 0) claim = atomicAdd(next_item, 1);  // used after the k-loop
+        const int g0 = 4 * lane;
+        const bool active = g0 < it.n;
+        int y[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[i] = active ? __ldg(rowmap + it.r0 + min(g0 + i, it.n - 1)) : 0;
+        const uint32_t tx = (uint32_t)(((it.n + 3) / 4) * 4 * kBK * 2 + C::kBBytes);
+        const int w0 = it.wrow, w1 = GATEUP ? it.wrow + d.F : it.wrow + 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          int good2 = 1;
+          if (lane == 0) good2 = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status);
+          if (!__shfl_sync(0xffffffffu, good2, 0)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sb = stage_base + stage * C::kStageBytes;
+          const uint32_t fb = smem_u32(&full[stage]);
+          if (lane == 0) {
+            mbar_expect_tx(fb, tx);
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          __syncwarp();
+          if (active) tma_gather4(smem_u32(sb + g0 * kBK * 2), &map_x, kb * kBK, y[0], y[1], y[2], y[3], fb);
+          if (lane == 0) {
+            tma_load_2d(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
+            tma_load_2d(smem_u32(sb + C::kABytes + C::kBBytes / 2), &map_w, kb * kBK, w1, fb);
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        const int nxt = (int)gridDim.x + __shfl_sync(0xffffffffu, claim, 0);
+        item = nxt < total ? nxt : -1;
+        if (item >= 0) it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+      }
+      if (!ok && lane == 0) {  // let every issued copy land before the CTA exits
+        for (int s2 = 0; s2 < C::kStages; ++s2)
+          if ((armed >> s2) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    } else if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
@@ -1485,10 +1575,13 @@ cudaError_t gemm_tc_prepare() {
     e = cudaFuncSetAttribute(k_gemm_tc2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg2<false>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemm_tm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<true>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemm_tm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM<true>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<false>::kSmemBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_gemm_tm2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1524,15 +1617,19 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
 }
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                           int grid, cudaStream_t s, int which) {
-  if (which == 1)
-    k_gemm_tm<true><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
+                           int grid, cudaStream_t s, int which, bool gather) {
+  if (which == 1 && gather)
+    k_gemm_tm<true, true><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
+        maps.w_gateup, maps.hidden_rows, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1, w.gemm_next,
+        w.rowmap, static_cast<__nv_bfloat16*>(w.act));
+  else if (which == 1)
+    k_gemm_tm<true, false><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
         maps.w_gateup, maps.A32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1, w.gemm_next,
-        static_cast<__nv_bfloat16*>(w.act));
+        w.rowmap, static_cast<__nv_bfloat16*>(w.act));
   else
-    k_gemm_tm<false><<<grid, kThreads, CfgTM<false>::kSmemBytes, s>>>(
+    k_gemm_tm<false, false><<<grid, kThreads, CfgTM<false>::kSmemBytes, s>>>(
         maps.w_down, maps.act32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items2, w.gemm_next + 1,
-        static_cast<__nv_bfloat16*>(w.y));
+        w.rowmap, static_cast<__nv_bfloat16*>(w.y));
   return cudaGetLastError();
 }
 
@@ -1613,6 +1710,10 @@ cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, 
 }
 
 }  // namespace
+
+cudaError_t make_hidden_map(const Dims& d, const void* hidden, TcMaps* maps) {
+  return encode(&maps->hidden_rows, hidden, (unsigned long long)d.M * d.T, d.H, 1);
+}
 
 cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
                          TcMaps* maps) {

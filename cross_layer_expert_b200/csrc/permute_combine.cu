@@ -12,8 +12,9 @@
 // the aggregation order -- the slot order here is fixed.
 //
 // The permutation is two launches: k_positions computes every (token, slot)
-// row of the RunSet (a light pass over the routing indices), then
-// k_permute_copy moves the rows.  The copy and the combine are HBM-bound and
+// row of the RunSet and its inverse, the token of every row (a light pass
+// over the routing indices); k_permute_copy then moves the rows -- unless
+// GEMM 1 gathers them from the hidden states itself.  The copy and the combine are HBM-bound and
 // persistent: a grid of resident CTAs sized to the SM count strides over the
 // RunSet's tokens, one warp per token row with 16-byte vector loads and
 // stores, so the work spreads evenly over the SMs whatever the RunSet size
@@ -44,7 +45,8 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
                                                             const int32_t* __restrict__ chunk_hist,
                                                             const int32_t* __restrict__ seg_rows,
                                                             const int32_t* __restrict__ prior,
-                                                            int32_t* __restrict__ pos) {
+                                                            int32_t* __restrict__ pos,
+                                                            int32_t* __restrict__ rowmap) {
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
   __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
@@ -95,12 +97,17 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
       running[ee] = run;
     }
     __syncthreads();
-    if (e >= 0) pos_c[(p / k) * kk + p % k] = bj[e] + cnt[warp][e] + rank;
+    if (e >= 0) {
+      const int row = bj[e] + cnt[warp][e] + rank;
+      pos_c[(p / k) * kk + p % k] = row;
+      rowmap[row] = j * d.T + t0 + p / k;
+    }
     __syncthreads();
   }
   for (int i = tid; i < nt * d.n_shared; i += kPermThreads) {
     const int t = i / d.n_shared, s = i % d.n_shared;
     pos_c[t * kk + k + s] = bj[E + s] + t;
+    rowmap[bj[E + s] + t] = j * d.T + t0 + t;
   }
 }
 
@@ -321,11 +328,11 @@ int persistent_grid(const void* kernel, int threads, int& cache) {
 int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb_f32 = 0;
 
 cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
-                           cudaStream_t s) {
+                           bool copy, cudaStream_t s) {
   k_positions<<<dim3(d.NC, d.M), kPermThreads, 0, s>>>(d, c.st, w.idx, w.chunk_hist, w.seg_rows,
-                                                      w.prior, w.pos);
+                                                      w.prior, w.pos, w.rowmap);
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  if (e != cudaSuccess || !copy) return e;
   if (d.dtype == EB_DTYPE_BF16)
     k_permute_copy<__nv_bfloat16>
         <<<persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads, g_grid_copy_bf16),

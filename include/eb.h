@@ -68,6 +68,9 @@ typedef int eb_status;
  *         dynamically, so CTAs finish together whatever the segment sizes.
  *   TM2   token-major over an SM pair (cta_group::2): 256 tokens x 256 weight
  *         rows per MMA, each SM holding 128 tokens and half the weight rows.
+ *   TMG   as TM, but GEMM 1 reads its token rows straight from `hidden` with
+ *         TMA gather4 (four rows per copy) instead of from a permuted copy,
+ *         which is then not written.
  * TM and TM2 need F a multiple of 128 (gate/up) and H a multiple of 256
  * (down); a GEMM they do not fit runs on TC. */
 #define EB_GEMM_AUTO 0
@@ -76,6 +79,7 @@ typedef int eb_status;
 #define EB_GEMM_TC2 3
 #define EB_GEMM_TM 4
 #define EB_GEMM_TM2 5
+#define EB_GEMM_TMG 6
 
 /* Limits of this build. */
 #define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */

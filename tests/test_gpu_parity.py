@@ -164,14 +164,15 @@ def small_expected(small_inputs):
 
 @pytest.mark.parametrize("name", SMALL)
 @pytest.mark.parametrize("policy", [0, 1, 2, 3])
-@pytest.mark.parametrize("gemm", [0, 1, 2, 3, 5])
+@pytest.mark.parametrize("gemm", [0, 1, 2, 3, 5, 6])
 def test_small_episode_matches_oracle(small_inputs, small_expected, name, policy, gemm):
     """gemm 0: default engine (one-SM token-major tensor-core engine for bf16,
     SIMT for fp32); 1: one-SM weight-major; 2: SIMT; 3: two-SM weight-major;
-    5: two-SM token-major (the tensor-core engines take bf16 only)."""
+    5: two-SM token-major; 6: token-major with GEMM 1 gathering its rows
+    from the hidden states (the tensor-core engines take bf16 only)."""
     inp = small_inputs[name]
     wl = inp.wl
-    if wl.dtype == "f32" and gemm in (1, 3, 5):
+    if wl.dtype == "f32" and gemm in (1, 3, 5, 6):
         pytest.skip("the tensor-core engines take bf16 operands")
     if gemm == 3 and (wl.H % 256 or wl.F % 256):
         pytest.skip("the two-SM weight-major engine needs H and F multiples of 256")

@@ -24,11 +24,12 @@ from .schedule import (CUMUTIL, DIFFPEAK, LOCKSTEP, MAXUTIL, run_episode,  # noq
                        set_utilization, utilization)
 
 
-def route_all(logits: np.ndarray, k: int, D: int, renorm: bool = True):
+def route_all(logits: np.ndarray, k: int, D: int, renorm: bool = True, expert_rank=None):
     """Route every (micro-batch, layer) block of logits [M, L, T, E].
 
     Returns idx [M, L, T, k] int32, gate [M, L, T, k] float64, hist [M, L, E]
-    and loads [M, L, D] (int64).
+    and loads [M, L, D] (int64) under the contiguous map, or under
+    expert_rank if given.
     """
     M, L, T, E = logits.shape
     idx = np.empty((M, L, T, k), dtype=np.int32)
@@ -38,4 +39,4 @@ def route_all(logits: np.ndarray, k: int, D: int, renorm: bool = True):
         for l in range(L):
             idx[j, l], gate[j, l] = route(logits[j, l], k, renorm)
             hist[j, l] = histogram(idx[j, l], E)
-    return idx, gate, hist, loads(hist, D)
+    return idx, gate, hist, loads(hist, D, expert_rank)

@@ -59,20 +59,30 @@ def histogram(idx: np.ndarray, E: int) -> np.ndarray:
     return np.bincount(np.asarray(idx).reshape(-1), minlength=E).astype(np.int64)
 
 
-def loads(hist: np.ndarray, D: int) -> np.ndarray:
+def loads(hist: np.ndarray, D: int, expert_rank=None) -> np.ndarray:
     """Virtual-rank workload vector w = (w_1..w_D) of one (micro-batch, layer).
 
     [SysLB] §1: the load of rank r is the sum of T_e over its local experts.
     [EB] §5 Models: experts are evenly distributed over the devices; read as the
     contiguous map, rank d holding experts [d E/D, (d+1) E/D).
     [EB] §2.3 writes this vector as w^(l) = (w_1^(l), ..., w_D^(l)).
+    expert_rank (length E, values in [0, D)) replaces the contiguous map by
+    an arbitrary placement, as a load balancer such as EPLB would choose
+    ([EB] §5.3 treats placement as orthogonal to scheduling); E need not then
+    be a multiple of D.
     """
     hist = np.asarray(hist, dtype=np.int64)
     E = hist.shape[-1]
-    if D < 1 or E % D != 0:
-        raise ValueError("E must be a multiple of D")
-    per = E // D
+    if D < 1:
+        raise ValueError("D must be positive")
+    if expert_rank is None:
+        if E % D != 0:
+            raise ValueError("E must be a multiple of D")
+        expert_rank = [e // (E // D) for e in range(E)]
+    expert_rank = list(expert_rank)
+    if len(expert_rank) != E or any(not (0 <= r < D) for r in expert_rank):
+        raise ValueError("expert_rank must give a rank in [0, D) for each of the E experts")
     w = np.zeros(hist.shape[:-1] + (D,), dtype=np.int64)
-    for d in range(D):
-        w[..., d] = hist[..., d * per:(d + 1) * per].sum(axis=-1)
+    for e, r in enumerate(expert_rank):
+        w[..., r] += hist[..., e]
     return w

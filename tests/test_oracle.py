@@ -273,6 +273,33 @@ def test_histogram_and_loads():
         oracle.loads(h, 5)
 
 
+def test_loads_with_expert_map():
+    """An arbitrary expert -> rank placement: each rank sums exactly the
+    experts mapped to it (brute force per rank), the contiguous map is the
+    default, E need not be a multiple of D, and bad maps are rejected."""
+    rng = np.random.default_rng(10)
+    h = rng.integers(0, 50, size=(3, 12))
+    contiguous = [e // 3 for e in range(12)]
+    assert np.array_equal(oracle.loads(h, 4, contiguous), oracle.loads(h, 4))
+    for D in (1, 3, 5, 7):
+        emap = rng.integers(0, D, size=12).tolist()
+        w = oracle.loads(h, D, emap)
+        for j in range(3):
+            for d in range(D):
+                assert w[j, d] == sum(int(h[j, e]) for e in range(12) if emap[e] == d)
+        assert np.array_equal(w.sum(axis=-1), h.sum(axis=-1))
+    # a rank with no experts carries no load; a permutation of the contiguous
+    # map permutes the loads
+    w = oracle.loads(h, 5, [0] * 6 + [2] * 6)
+    assert (w[:, [1, 3, 4]] == 0).all()
+    perm = [3, 0, 2, 1]
+    w = oracle.loads(h, 4, [perm[e // 3] for e in range(12)])
+    assert np.array_equal(w[:, perm], oracle.loads(h, 4))
+    for bad in ([0] * 11, [0] * 11 + [4], [-1] + [0] * 11):
+        with pytest.raises(ValueError):
+            oracle.loads(h, 4, bad)
+
+
 # ------------------------------------------------------------ expert / combine
 
 def test_round_bf16():

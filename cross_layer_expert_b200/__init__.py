@@ -35,7 +35,7 @@ EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_crea
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
-            "eb_selftest_timeout"]
+            "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine")
 
@@ -80,6 +80,8 @@ def load() -> ctypes.CDLL:
         "eb_sync_status": (I, [P]),
         "eb_route": (I, [P, I, I, I, I, P, P, P, P, P]),
         "eb_loads": (I, [P, I, I, I, P, P]),
+        "eb_loads_mapped": (I, [P, I, I, I, P, P, P, P]),
+        "eb_set_expert_map": (I, [P, P]),
         "eb_schedule": (I, [P, U32, I, I, I, I, P, P, P]),
         "eb_profile": (I, [P, I]),
         "eb_profile_read": (I, [P, P, P]),
@@ -149,6 +151,15 @@ def eb_loads(hist, D: int, w, stream=None) -> None:
     _check(load().eb_loads(_ptr(hist), M, E, D, _ptr(w), _stream(stream)), "eb_loads")
 
 
+def eb_loads_mapped(hist, D: int, expert_rank, w, status=None, stream=None) -> None:
+    """hist [M, E] i32 -> w [M, D] i32 under the placement expert_rank
+    (device [E] i32); status: optional device i32 set on an out-of-range rank."""
+    M, E = hist.shape
+    _check(load().eb_loads_mapped(_ptr(hist), M, E, D, _ptr(expert_rank), _ptr(w),
+                                  _ptr(status) if status is not None else None, _stream(stream)),
+           "eb_loads_mapped")
+
+
 def eb_schedule(w, pending_mask: int, m: int, policy: int, runset, stats=None, stream=None) -> None:
     """w [M, D] i32 -> runset (1-element u32/i32 device tensor), stats [3] i64."""
     M, D = w.shape
@@ -203,6 +214,16 @@ class Context:
 
     def eb_reset(self, stream=None) -> None:
         _check(load().eb_reset(self.handle, _stream(stream)), "eb_reset")
+
+    def eb_set_expert_map(self, expert_rank=None) -> None:
+        """Placement of the E experts on the D ranks (a sequence of ints), or
+        None for the contiguous map."""
+        if expert_rank is None:
+            _check(load().eb_set_expert_map(self.handle, None), "eb_set_expert_map")
+            return
+        arr = (ctypes.c_int32 * len(expert_rank))(*[int(r) for r in expert_rank])
+        _check(load().eb_set_expert_map(self.handle, ctypes.cast(arr, ctypes.c_void_p)),
+               "eb_set_expert_map")
 
     def eb_moe_step(self, logits, hidden, w_gateup, w_down, stream=None, want_runset=False):
         out = ctypes.c_uint32(0)

@@ -259,9 +259,10 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   const size_t n_w = align_up(sizeof(int32_t) * c->M * c->D);
   const size_t n_trace = align_up(sizeof(long long) * kTraceCols * x->d.max_steps);
   const size_t n_tl = align_up(sizeof(int32_t) * c->M * (size_t)x->d.max_steps);
+  const size_t n_map = align_up(sizeof(int32_t) * c->E);
   char* p = nullptr;
-  if (e == cudaSuccess) e = cudaMalloc(&p, n_state + n_hist + n_w + n_trace + n_tl);
-  if (e == cudaSuccess) e = cudaMemset(p, 0, n_state + n_hist + n_w + n_trace + n_tl);
+  if (e == cudaSuccess) e = cudaMalloc(&p, n_state + n_hist + n_w + n_trace + n_tl + n_map);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, n_state + n_hist + n_w + n_trace + n_tl + n_map);
   if (e == cudaSuccess) {
     x->dev_alloc = p;
     x->dev.st = (State*)p;
@@ -269,6 +270,8 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->dev.w = (int32_t*)(p + n_state + n_hist);
     x->dev.trace = (long long*)(p + n_state + n_hist + n_w);
     x->dev.trace_layers = (int32_t*)(p + n_state + n_hist + n_w + n_trace);
+    x->dev.emap = (int32_t*)(p + n_state + n_hist + n_w + n_trace + n_tl);
+    x->dev.use_emap = 0;
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
   for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
@@ -306,6 +309,22 @@ eb_status eb_reset(eb_ctx* x, void* stream) {
   x->last_stream = s;
   x->launches += 1;
   return cuda_status(launch_reset(x->d, x->dev, s));
+}
+
+eb_status eb_set_expert_map(eb_ctx* x, const int32_t* expert_rank) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (!expert_rank) {
+    x->dev.use_emap = 0;
+    return EB_OK;
+  }
+  for (int e = 0; e < x->cfg.E; ++e)
+    if (expert_rank[e] < 0 || expert_rank[e] >= x->cfg.D) return EB_ERR_INVALID_ARG;
+  // synchronous: no step of this context may be in flight
+  const cudaError_t err = cudaMemcpy(x->dev.emap, expert_rank, sizeof(int32_t) * x->cfg.E,
+                                     cudaMemcpyHostToDevice);
+  if (err != cudaSuccess) return EB_ERR_CUDA;
+  x->dev.use_emap = 1;
+  return EB_OK;
 }
 
 static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* wgu,
@@ -513,7 +532,15 @@ eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t
 eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream) {
   if (M < 0 || E < 1 || D < 1 || E % D != 0) return EB_ERR_INVALID_ARG;
   if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
-  return cuda_status(launch_loads(hist, M, E, D, w, (cudaStream_t)stream));
+  return cuda_status(launch_loads(hist, M, E, D, nullptr, w, nullptr, (cudaStream_t)stream));
+}
+
+eb_status eb_loads_mapped(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
+                          int32_t* w, int32_t* status_dev, void* stream) {
+  if (M < 0 || E < 1 || D < 1 || !expert_rank) return EB_ERR_INVALID_ARG;
+  if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_loads(hist, M, E, D, expert_rank, w, status_dev, (cudaStream_t)stream));
 }
 
 eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int m, int policy,

@@ -98,6 +98,8 @@ struct CtxDev {
   int32_t* w;           // [M][D]: loads of micro-batch j at layer l_j (accumulated by routing)
   long long* trace;     // [max_steps][kTraceCols]
   int32_t* trace_layers;  // [max_steps][M]
+  int32_t* emap;        // [E]: rank of each expert (a custom placement)
+  int use_emap;         // 0: contiguous map, experts [d E/D, (d+1) E/D) on rank d
 };
 
 // ---- launchers (all asynchronous on `s`) ----
@@ -111,7 +113,11 @@ cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, 
                                  int fm1, int fm2, cudaStream_t s);
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
                                  int policy, uint32_t* runset, long long* stats, cudaStream_t s);
-cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s);
+// expert_rank: device [E] placement, or nullptr for the contiguous map;
+// status (device, may be nullptr) gets EB_ERR_INVALID_ARG for a rank outside
+// [0, D) (that expert's count is then dropped).
+cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
+                         int32_t* w, int32_t* status, cudaStream_t s);
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
 // Rows of every (token, slot) of the RunSet (pos, rowmap); with `copy`, also
 // the permuted copy A of the token rows.

@@ -123,7 +123,9 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
 // is in need_route; its counts land in chunk_hist[j][c][:] and are added
 // (integer atomics: exact, order-free) to the micro-batch's histogram
-// hist[j][:] and rank loads w[j][:], which the previous step zeroed.
+// hist[j][:] and rank loads w[j][:], which the previous step zeroed.  The
+// loads fold the counts by the context's expert placement: contiguous
+// blocks of E/D experts, or emap[e] if one was set.
 template <int VPL>
 __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__ st,
                                                      const float* __restrict__ logits,
@@ -131,13 +133,16 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
                                                      float* __restrict__ gate,
                                                      int32_t* __restrict__ chunk_hist,
                                                      int32_t* __restrict__ hist,
-                                                     int32_t* __restrict__ wload) {
+                                                     int32_t* __restrict__ wload,
+                                                     const int32_t* __restrict__ emap) {
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->need_route >> j) & 1u)) return;
   const int l = st->layer[j];
   __shared__ int hist_s[EB_MAX_ETOT];
+  __shared__ int w_s[EB_MAX_D];
   __shared__ int bad;
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) hist_s[e] = 0;
+  for (int r = threadIdx.x; r < d.D; r += blockDim.x) w_s[r] = 0;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   const float* blk = logits + ((size_t)j * d.L + l) * (size_t)d.T * d.E;
@@ -152,11 +157,19 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
     out[e] = hist_s[e];
     if (hist_s[e]) atomicAdd(&hist[j * d.E + e], hist_s[e]);
   }
-  const int per = d.E / d.D;
-  for (int r = threadIdx.x; r < d.D; r += blockDim.x) {
-    int sum = 0;
-    for (int e = r * per; e < (r + 1) * per; ++e) sum += hist_s[e];
-    if (sum) atomicAdd(&wload[j * d.D + r], sum);
+  if (emap) {  // custom placement (ranks validated on the host)
+    for (int e = threadIdx.x; e < d.E; e += blockDim.x)
+      if (hist_s[e]) atomicAdd(&w_s[emap[e]], hist_s[e]);
+    __syncthreads();
+    for (int r = threadIdx.x; r < d.D; r += blockDim.x)
+      if (w_s[r]) atomicAdd(&wload[j * d.D + r], w_s[r]);
+  } else {
+    const int per = d.E / d.D;
+    for (int r = threadIdx.x; r < d.D; r += blockDim.x) {
+      int sum = 0;
+      for (int e = r * per; e < (r + 1) * per; ++e) sum += hist_s[e];
+      if (sum) atomicAdd(&wload[j * d.D + r], sum);
+    }
   }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
 }
@@ -191,11 +204,12 @@ int vpl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
                               cudaStream_t s) {
   dim3 grid(d.NC, d.M);
+  const int32_t* emap = c.use_emap ? c.emap : nullptr;
   switch (vpl_for(d.E)) {
-    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
-    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
-    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
-    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w); break;
+    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
   }
   return cudaGetLastError();
 }

@@ -530,12 +530,22 @@ __global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __res
 }
 
 __global__ void k_loads(const int32_t* __restrict__ hist, int M, int E, int D,
-                        int32_t* __restrict__ w) {
+                        const int32_t* __restrict__ expert_rank, int32_t* __restrict__ w,
+                        int32_t* __restrict__ status) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= M * D) return;
-  const int j = i / D, dd = i % D, per = E / D;
+  const int j = i / D, dd = i % D;
   int s = 0;
-  for (int e = dd * per; e < (dd + 1) * per; ++e) s += hist[j * E + e];
+  if (expert_rank) {  // custom placement: the experts whose rank is dd
+    for (int e = 0; e < E; ++e) {
+      const int r = expert_rank[e];
+      if (r == dd) s += hist[j * E + e];
+      else if ((r < 0 || r >= D) && dd == 0 && status) atomicExch(status, EB_ERR_INVALID_ARG);
+    }
+  } else {
+    const int per = E / D;
+    for (int e = dd * per; e < (dd + 1) * per; ++e) s += hist[j * E + e];
+  }
   w[i] = s;
 }
 
@@ -589,10 +599,11 @@ cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int 
   return cudaGetLastError();
 }
 
-cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, int32_t* w, cudaStream_t s) {
+cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
+                         int32_t* w, int32_t* status, cudaStream_t s) {
   const int n = M * D;
   if (n == 0) return cudaSuccess;
-  k_loads<<<(n + 255) / 256, 256, 0, s>>>(hist, M, E, D, w);
+  k_loads<<<(n + 255) / 256, 256, 0, s>>>(hist, M, E, D, expert_rank, w, status);
   return cudaGetLastError();
 }
 

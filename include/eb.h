@@ -133,12 +133,22 @@ eb_status eb_destroy(eb_ctx* ctx);
  * zeroed accumulators and trace.  Enqueued on `stream`. */
 eb_status eb_reset(eb_ctx* ctx, void* stream);
 
+/* Expert placement used to fold expert counts into rank loads.  By default
+ * rank d holds experts [d E/D, (d+1) E/D) ([EB] §5 Models, "evenly
+ * distributed").  expert_rank (HOST array of cfg.E int32, each in
+ * [0, cfg.D)) replaces it by any placement -- e.g. one a load balancer such
+ * as EPLB chose, which [EB] §5.3 treats as orthogonal to scheduling; NULL
+ * restores the contiguous map.  Copied synchronously into the context (call
+ * it with none of the context's steps in flight); takes effect from the next
+ * routing.  EB_ERR_INVALID_ARG for a rank outside [0, D). */
+eb_status eb_set_expert_map(eb_ctx* ctx, const int32_t* expert_rank);
+
 /*
  * One EasyBalance step, [EB] §4.2 Algorithm 1 loop body, entirely on device:
  *   1. route the micro-batches of the previous RunSet at their layer l_j:
  *      softmax top-k of the fp32 logits, renormalised gates ([EB] §2.1);
- *      per-expert counts T_e folded into w_j over the contiguous map
- *      ([SysLB] §1; [EB] §2.3);
+ *      per-expert counts T_e folded into w_j over the contiguous map, or
+ *      the placement set by eb_set_expert_map ([SysLB] §1; [EB] §2.3);
  *   2. RunSet = Schedule(S, m) with cfg.policy; exact int64 utilisation
  *      accumulators ([EB] Eq. (2), (3)); trace row;
  *   3. permute the RunSet's tokens into segments keyed (layer, expert)
@@ -233,6 +243,14 @@ eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t
 /* Virtual-rank loads under the contiguous map: w[j][d] = sum of hist[j][e]
  * over e in [d E/D, (d+1) E/D).  hist [M, E] int32 -> w [M, D] int32. */
 eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream);
+
+/* Virtual-rank loads under an arbitrary placement: w[j][d] = sum of
+ * hist[j][e] over the experts e with expert_rank[e] == d.  expert_rank is a
+ * DEVICE array of E int32; E need not be a multiple of D.  An entry outside
+ * [0, D) drops that expert's counts and sets *status_dev (optional device
+ * int32) to EB_ERR_INVALID_ARG. */
+eb_status eb_loads_mapped(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
+                          int32_t* w, int32_t* status_dev, void* stream);
 
 /* RunSet = Schedule(S, m) for one step ([EB] §4.2, §5.2).
  * w [M, D] int32 loads; pending_mask: bit j set = j in S.

@@ -75,17 +75,20 @@ def run_episode(inp: Inputs, policy: int, m: int = 0, gemm: int = 0):
     return hidden, rows, layers, util, steps
 
 
-def oracle_loads(inp: Inputs):
+def oracle_loads(inp: Inputs, expert_rank=None):
+    if expert_rank is not None:
+        wl = inp.wl
+        return oracle.route_all(inp.logits_np, wl.k, wl.D, expert_rank=expert_rank)[3]
     if getattr(inp, "_loads", None) is None:
         wl = inp.wl
         inp._loads = oracle.route_all(inp.logits_np, wl.k, wl.D)[3]
     return inp._loads
 
 
-def oracle_episode(inp: Inputs, policy: int, m: int = 0):
+def oracle_episode(inp: Inputs, policy: int, m: int = 0, expert_rank=None):
     from oracle import native
     wl = inp.wl
-    return oracle.run_episode(oracle_loads(inp), policy, m or wl.m_default,
+    return oracle.run_episode(oracle_loads(inp, expert_rank), policy, m or wl.m_default,
                               maxutil_impl=native.maxutil if wl.M > 12 else None)
 
 

@@ -102,6 +102,49 @@ struct CtxDev {
   int use_emap;         // 0: contiguous map, experts [d E/D, (d+1) E/D) on rank d
 };
 
+// ---- programmatic dependent launch ----
+// Every kernel of a step is launched with programmatic stream serialisation
+// allowed, so it can be scheduled while the previous kernel of the stream
+// drains.  Each one calls pdl_wait() before it reads anything (griddepcontrol
+// .wait returns once the previous grid has completed and its writes are
+// visible; without a programmatic dependency it returns at once) and then
+// pdl_trigger(), which lets the next kernel be scheduled.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_enter() {
+  pdl_wait();
+  pdl_trigger();
+}
+
+// Launch with programmatic dependent launch allowed (and, cluster > 1, with
+// that cluster size along x).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[n].val.programmaticStreamSerializationAllowed = 1;
+  ++n;
+  if (cluster > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = (unsigned)cluster;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // ---- launchers (all asynchronous on `s`) ----
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
                               cudaStream_t s);

@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(256) k_gemm_simt(Dims d, const State* __restri
                                                    const int32_t* __restrict__ seg_items,
                                                    const T* __restrict__ X,
                                                    const T* __restrict__ W, T* __restrict__ out) {
+  pdl_enter();
   const int nseg = st->nseg;
   if (nseg == 0 || st->runset == 0) return;
   const int total = seg_items[nseg];
@@ -117,14 +118,14 @@ cudaError_t run(const Dims& d, const CtxDev& c, const Work& w, const void* wgu, 
                 cudaStream_t s, int which) {
   const int grid = 148 * 4;
   if (which == 1)
-    k_gemm_simt<T, true><<<grid, 256, 0, s>>>(d, c.st, w.seg_rows, w.seg_wid, w.seg_items1,
-                                              static_cast<const T*>(w.A),
-                                              static_cast<const T*>(wgu), static_cast<T*>(w.act));
-  else
-    k_gemm_simt<T, false><<<grid, 256, 0, s>>>(d, c.st, w.seg_rows, w.seg_wid, w.seg_items2,
-                                               static_cast<const T*>(w.act),
-                                               static_cast<const T*>(wdn), static_cast<T*>(w.y));
-  return cudaGetLastError();
+    return launch_pdl(k_gemm_simt<T, true>, dim3(grid), dim3(256), 0, s, 1, d, c.st,
+                      (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                      (const int32_t*)w.seg_items1, static_cast<const T*>(w.A),
+                      static_cast<const T*>(wgu), static_cast<T*>(w.act));
+  return launch_pdl(k_gemm_simt<T, false>, dim3(grid), dim3(256), 0, s, 1, d, c.st,
+                    (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                    (const int32_t*)w.seg_items2, static_cast<const T*>(w.act),
+                    static_cast<const T*>(wdn), static_cast<T*>(w.y));
 }
 
 }  // namespace

@@ -248,6 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
               __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
   using C = Cfg<GATEUP>;
   constexpr int kBN = C::kBN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -588,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
                const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
                __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
   using C = Cfg2<GATEUP>;
   constexpr int kBN = C::kBN;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -894,6 +896,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
               int32_t* __restrict__ next_item, const int32_t* __restrict__ rowmap,
               __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
   using C = CfgTM<GATEUP>;
   constexpr int Q = C::kQueue;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1287,6 +1290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
                const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
                __nv_bfloat16* __restrict__ out) {
+  pdl_enter();
   using C = CfgTM2<GATEUP>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1595,15 +1599,17 @@ cudaError_t gemm_tc_prepare() {
 cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                             int grid, cudaStream_t s, int which) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kThreads);
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (which == 1) {
     cfg.dynamicSmemBytes = CfgTM2<true>::kSmemBytes;
     cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<true>, cfg, grid / 2));
@@ -1618,33 +1624,37 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                            int grid, cudaStream_t s, int which, bool gather) {
+  const int32_t* rowmap = w.rowmap;
   if (which == 1 && gather)
-    k_gemm_tm<true, true><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
-        maps.w_gateup, maps.hidden_rows, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1, w.gemm_next,
-        w.rowmap, static_cast<__nv_bfloat16*>(w.act));
-  else if (which == 1)
-    k_gemm_tm<true, false><<<grid, kThreads, CfgTM<true>::kSmemBytes, s>>>(
-        maps.w_gateup, maps.A32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1, w.gemm_next,
-        w.rowmap, static_cast<__nv_bfloat16*>(w.act));
-  else
-    k_gemm_tm<false, false><<<grid, kThreads, CfgTM<false>::kSmemBytes, s>>>(
-        maps.w_down, maps.act32, d, c.st, w.seg_rows, w.seg_wid, w.seg_items2, w.gemm_next + 1,
-        w.rowmap, static_cast<__nv_bfloat16*>(w.y));
-  return cudaGetLastError();
+    return launch_pdl(k_gemm_tm<true, true>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes, s,
+                      1, maps.w_gateup, maps.hidden_rows, d, c.st, (const int32_t*)w.seg_rows,
+                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
+                      static_cast<__nv_bfloat16*>(w.act));
+  if (which == 1)
+    return launch_pdl(k_gemm_tm<true, false>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes,
+                      s, 1, maps.w_gateup, maps.A32, d, c.st, (const int32_t*)w.seg_rows,
+                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
+                      static_cast<__nv_bfloat16*>(w.act));
+  return launch_pdl(k_gemm_tm<false, false>, dim3(grid), dim3(kThreads), CfgTM<false>::kSmemBytes,
+                    s, 1, maps.w_down, maps.act32, d, c.st, (const int32_t*)w.seg_rows,
+                    (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowmap,
+                    static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                             int grid, cudaStream_t s, int which) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.blockDim = dim3(kThreads);
   cfg.stream = s;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (which == 1) {
     cfg.dynamicSmemBytes = Cfg2<true>::kSmemBytes;
     cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<true>, cfg, grid / 2));
@@ -1660,14 +1670,14 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
 cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                            int grid, cudaStream_t s, int which) {
   if (which == 1)
-    k_gemm_tc<true><<<grid, kThreads, Cfg<true>::kSmemBytes, s>>>(
-        maps.w_gateup, maps.A, d, c.st, w.seg_rows, w.seg_wid, w.seg_items1,
-        static_cast<__nv_bfloat16*>(w.act));
-  else
-    k_gemm_tc<false><<<grid, kThreads, Cfg<false>::kSmemBytes, s>>>(
-        maps.w_down, maps.act, d, c.st, w.seg_rows, w.seg_wid, w.seg_items2,
-        static_cast<__nv_bfloat16*>(w.y));
-  return cudaGetLastError();
+    return launch_pdl(k_gemm_tc<true>, dim3(grid), dim3(kThreads), Cfg<true>::kSmemBytes, s, 1,
+                      maps.w_gateup, maps.A, d, c.st, (const int32_t*)w.seg_rows,
+                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1,
+                      static_cast<__nv_bfloat16*>(w.act));
+  return launch_pdl(k_gemm_tc<false>, dim3(grid), dim3(kThreads), Cfg<false>::kSmemBytes, s, 1,
+                    maps.w_down, maps.act, d, c.st, (const int32_t*)w.seg_rows,
+                    (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2,
+                    static_cast<__nv_bfloat16*>(w.y));
 }
 
 }  // namespace eb

@@ -29,7 +29,6 @@ namespace {
 
 constexpr unsigned kFull = 0xffffffffu;
 constexpr int kPermThreads = 256;
-constexpr int kMaxSlots = EB_MAX_K;  // k + n_shared <= 32 (one lane per slot in the combine)
 
 __device__ __forceinline__ unsigned lanemask_lt() {
   unsigned m;
@@ -47,6 +46,7 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
                                                             const int32_t* __restrict__ prior,
                                                             int32_t* __restrict__ pos,
                                                             int32_t* __restrict__ rowmap) {
+  pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
   __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
@@ -124,6 +124,7 @@ __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const Sta
                                                                const int32_t* __restrict__ pos,
                                                                const T* __restrict__ hidden,
                                                                T* __restrict__ A) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int W = (int)(gridDim.x * (kPermThreads / 32));
   const int wid = (int)(blockIdx.x * (kPermThreads / 32) + (threadIdx.x >> 5));
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State
                                                              const float* __restrict__ gate,
                                                              const int32_t* __restrict__ pos,
                                                              const T* __restrict__ y, T* hidden) {
+  pdl_enter();
   const int lane = threadIdx.x & 31;
   const int W = (int)(gridDim.x * (kCombineThreads / 32));
   const int wid = (int)(blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5));
@@ -329,38 +331,37 @@ int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb
 
 cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                            bool copy, cudaStream_t s) {
-  k_positions<<<dim3(d.NC, d.M), kPermThreads, 0, s>>>(d, c.st, w.idx, w.chunk_hist, w.seg_rows,
-                                                      w.prior, w.pos, w.rowmap);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPermThreads), 0, s, 1, d, c.st,
+                             w.idx, w.chunk_hist, w.seg_rows, w.prior, w.pos, w.rowmap);
   if (e != cudaSuccess || !copy) return e;
   if (d.dtype == EB_DTYPE_BF16)
-    k_permute_copy<__nv_bfloat16>
-        <<<persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads, g_grid_copy_bf16),
-           kPermThreads, 0, s>>>(
-            d, c.st, w.pos, static_cast<const __nv_bfloat16*>(hidden),
-            static_cast<__nv_bfloat16*>(w.A));
-  else
-    k_permute_copy<float>
-        <<<persistent_grid((const void*)k_permute_copy<float>, kPermThreads, g_grid_copy_f32),
-           kPermThreads, 0, s>>>(d, c.st, w.pos, static_cast<const float*>(hidden),
-                                 static_cast<float*>(w.A));
-  return cudaGetLastError();
+    return launch_pdl(k_permute_copy<__nv_bfloat16>,
+                      dim3(persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads,
+                                           g_grid_copy_bf16)),
+                      dim3(kPermThreads), 0, s, 1, d, c.st, w.pos,
+                      static_cast<const __nv_bfloat16*>(hidden), static_cast<__nv_bfloat16*>(w.A));
+  return launch_pdl(k_permute_copy<float>,
+                    dim3(persistent_grid((const void*)k_permute_copy<float>, kPermThreads,
+                                         g_grid_copy_f32)),
+                    dim3(kPermThreads), 0, s, 1, d, c.st, w.pos, static_cast<const float*>(hidden),
+                    static_cast<float*>(w.A));
 }
 
 cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
                            cudaStream_t s) {
   if (d.dtype == EB_DTYPE_BF16)
-    k_combine<__nv_bfloat16>
-        <<<persistent_grid((const void*)k_combine<__nv_bfloat16>, kCombineThreads, g_grid_comb_bf16),
-           kCombineThreads, 0, s>>>(
-            d, c.st, w.gate, w.pos, static_cast<const __nv_bfloat16*>(w.y),
-            static_cast<__nv_bfloat16*>(hidden));
-  else
-    k_combine<float>
-        <<<persistent_grid((const void*)k_combine<float>, kCombineThreads, g_grid_comb_f32),
-           kCombineThreads, 0, s>>>(d, c.st, w.gate, w.pos, static_cast<const float*>(w.y),
-                                    static_cast<float*>(hidden));
-  return cudaGetLastError();
+    return launch_pdl(k_combine<__nv_bfloat16>,
+                      dim3(persistent_grid((const void*)k_combine<__nv_bfloat16>, kCombineThreads,
+                                           g_grid_comb_bf16)),
+                      dim3(kCombineThreads), 0, s, 1, d, c.st, (const float*)w.gate,
+                      (const int32_t*)w.pos, static_cast<const __nv_bfloat16*>(w.y),
+                      static_cast<__nv_bfloat16*>(hidden));
+  return launch_pdl(k_combine<float>,
+                    dim3(persistent_grid((const void*)k_combine<float>, kCombineThreads,
+                                         g_grid_comb_f32)),
+                    dim3(kCombineThreads), 0, s, 1, d, c.st, (const float*)w.gate,
+                    (const int32_t*)w.pos, static_cast<const float*>(w.y),
+                    static_cast<float*>(hidden));
 }
 
 }  // namespace eb

@@ -135,6 +135,7 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
                                                      int32_t* __restrict__ hist,
                                                      int32_t* __restrict__ wload,
                                                      const int32_t* __restrict__ emap) {
+  pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->need_route >> j) & 1u)) return;
   const int l = st->layer[j];
@@ -205,13 +206,14 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               cudaStream_t s) {
   dim3 grid(d.NC, d.M);
   const int32_t* emap = c.use_emap ? c.emap : nullptr;
+  cudaError_t e;
   switch (vpl_for(d.E)) {
-    case 1: k_route_step<1><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    case 2: k_route_step<2><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    case 4: k_route_step<4><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    default: k_route_step<8><<<grid, 1024, 0, s>>>(d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    default: e = launch_pdl(k_route_step<8>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
   }
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,

@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   __shared__ State ss;
   State* st = &ss;
   const int tid = threadIdx.x;
+  pdl_enter();
   constexpr int kStateWords = sizeof(State) / sizeof(int);
   for (int i = tid; i < kStateWords; i += blockDim.x)
     reinterpret_cast<int*>(&ss)[i] = reinterpret_cast<const int*>(c.st)[i];
@@ -550,6 +551,7 @@ __global__ void k_loads(const int32_t* __restrict__ hist, int M, int E, int D,
 }
 
 __global__ void k_reset(Dims d, CtxDev c) {
+  pdl_enter();
   State* st = c.st;
   for (int i = threadIdx.x; i < d.M * d.E; i += blockDim.x) c.hist[i] = 0;
   for (int i = threadIdx.x; i < d.M * d.D; i += blockDim.x) c.w[i] = 0;
@@ -589,8 +591,7 @@ unsigned long long maxutil_candidates(int n, int m) {
 
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
                                  int fm1, int fm2, cudaStream_t s) {
-  k_schedule_step<<<1, kThreads, 0, s>>>(d, c, w, rn1, rn2, fm1, fm2);
-  return cudaGetLastError();
+  return launch_pdl(k_schedule_step, dim3(1), dim3(kThreads), 0, s, 1, d, c, w, rn1, rn2, fm1, fm2);
 }
 
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
@@ -608,8 +609,7 @@ cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t
 }
 
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s) {
-  k_reset<<<1, 1024, 0, s>>>(d, c);
-  return cudaGetLastError();
+  return launch_pdl(k_reset, dim3(1), dim3(1024), 0, s, 1, d, c);
 }
 
 }  // namespace eb

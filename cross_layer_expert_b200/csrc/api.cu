@@ -328,12 +328,14 @@ eb_status eb_set_expert_map(eb_ctx* x, const int32_t* expert_rank) {
 }
 
 static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* wgu,
-                                 const void* wdn, cudaStream_t s, int which) {
+                                 const void* wdn, const void* hidden, cudaStream_t s, int which) {
   switch (eng) {
     case EB_GEMM_TC: return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     case EB_GEMM_TC2: return launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
-    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, false);
-    case EB_GEMM_TMG: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, true);
+    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr);
+    case EB_GEMM_TMG:
+      return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which,
+                            which == 1 ? hidden : nullptr);
     case EB_GEMM_TM2: return launch_gemm_tm2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     default: return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, which);
   }
@@ -362,10 +364,7 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   // GEMM 1 on the gathering engine reads its token rows from `hidden` itself
   // (no permuted copy)
   const bool gather = c.compute && x->eng1 == EB_GEMM_TMG;
-  if (gather && x->map_keys[3] != hidden) {
-    if (make_hidden_map(x->d, hidden, &x->maps) != cudaSuccess) return EB_ERR_UNSUPPORTED;
-    x->map_keys[3] = hidden;
-  }
+
   const int g1 = c.compute ? x->eng1 : EB_GEMM_SIMT, g2 = c.compute ? x->eng2 : EB_GEMM_SIMT;
   int rn1, fm1, rn2, fm2;
   engine_tiles(g1, 1, &rn1, &fm1);
@@ -377,9 +376,9 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     if (e == cudaSuccess)
       e = timed(x, 2, gather ? 1 : 2, s, [&] { return launch_permute(x->d, x->dev, w, hidden, !gather, s); });
     if (e == cudaSuccess) {
-      e = timed(x, 3, 1, s, [&] { return launch_engine(x, g1, w, wgu, wdn, s, 1); });
+      e = timed(x, 3, 1, s, [&] { return launch_engine(x, g1, w, wgu, wdn, hidden, s, 1); });
       if (e == cudaSuccess)
-        e = timed(x, 4, 1, s, [&] { return launch_engine(x, g2, w, wgu, wdn, s, 2); });
+        e = timed(x, 4, 1, s, [&] { return launch_engine(x, g2, w, wgu, wdn, hidden, s, 2); });
     }
     if (e == cudaSuccess)
       e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });

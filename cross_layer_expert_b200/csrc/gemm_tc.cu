@@ -114,17 +114,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Four rows y0..y3 (x .. x + box width) of a tensor whose map has a one-row
-// box, landing as four consecutive shared-memory rows at dst.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, int x, int y0,
-                                            int y1, int y2, int y3, uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(bar)
-      : "memory");
-}
-
 __device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
                    reinterpret_cast<uint64_t>(map)),
@@ -839,6 +828,8 @@ __device__ __forceinline__ SegView cache_segments(uint8_t* buf, int nseg, const 
   return {r, w, it};
 }
 
+constexpr int kGatherWarps = 4;  // row-gathering warps of the gathering GEMM 1 (one thread per row)
+constexpr int kGatherDepth = 2;  // k-blocks a gathering thread keeps in flight before signalling
 constexpr int kTmBox = 32;                    // token rows per TMA box
 constexpr int kTmBoxBytes = kTmBox * kBK * 2;  // 4 KiB
 
@@ -857,6 +848,8 @@ struct CfgTM {
   static constexpr int kQueue = 8;  // claimed items queued for the MMA issuer and the drain
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kSegCacheBytes + 1024;
   static_assert(kRows == 128 && kFeat * (GATEUP ? 2 : 1) == kN, "token-major tile shape");
+  static_assert(kGatherDepth >= 1 && kGatherDepth < kStages, "a gathering thread signals a stage before it reuses it");
+  static_assert(32 * kGatherWarps == kRows, "one gathering thread per token row");
   static_assert((2 * kStages + 4 + 2 * kQueue) * 8 + 8 + 4 * kQueue <= 1024, "barrier region");
 };
 
@@ -883,19 +876,20 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// map_x: token rows [Rcap, K] in boxes of 32 rows -- or, GATHER, the caller's
-// hidden states [M*T, H] in one-row boxes, gathered row by row through
-// rowmap (permuted row -> token) so the permuted copy is never written;
-// map_w: weights in boxes of 128 rows.  GATEUP: out = act [Rcap, F]; else
-// out = y [Rcap, H].  next_item: the step's claim counter (zero before the
-// launch).
+// map_x: token rows [Rcap, K] in boxes of 32 rows; map_w: weights in boxes
+// of 128 rows.  GATEUP: out = act [Rcap, F]; else out = y [Rcap, H].
+// next_item: the step's claim counter (zero before the launch).
+// GATHER (GEMM 1 only): the token rows are not read from a permuted copy;
+// kGatherWarps extra warps copy each chunk row straight from the hidden
+// states xsrc [M*T, H], through rowmap (permuted row -> token), into the
+// swizzled operand tile with 16-byte cp.async copies.
 template <bool GATEUP, bool GATHER>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThreads, 1)
     k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
               int32_t* __restrict__ next_item, const int32_t* __restrict__ rowmap,
-              __nv_bfloat16* __restrict__ out) {
+              const __nv_bfloat16* __restrict__ xsrc, __nv_bfloat16* __restrict__ out) {
   pdl_enter();
   using C = CfgTM<GATEUP>;
   constexpr int Q = C::kQueue;
@@ -925,7 +919,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(smem_u32(&full[i]), 1);
+      // GATHER: the weight copies' arrival plus one per gathering thread
+      mbar_init(smem_u32(&full[i]), GATHER ? 1 + 32 * kGatherWarps : 1);
       mbar_init(smem_u32(&empty[i]), 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -934,7 +929,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < Q; ++i) {
       mbar_init(smem_u32(&iready[i]), 1);
-      mbar_init(smem_u32(&ifree[i]), kEpiWarps + 1);
+      mbar_init(smem_u32(&ifree[i]), kEpiWarps + 1 + (GATHER ? kGatherWarps : 0));
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -958,82 +953,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // starts and decoded once its last k-block is issued (both off the
     // k-block path).  Claimed items go to the MMA issuer and the drain
     // through a queue in shared memory.
-    if (GATHER) {
-      // The whole warp runs the loop: lane 0 waits on the barriers, arms
-      // them and loads the weights; lane i gathers token rows 4i .. 4i + 3
-      // of the chunk (rows past the chunk repeat its last row).
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_par = 0;
-      bool ok = true;
-      int item = (int)blockIdx.x < total ? (int)blockIdx.x : -1;
-      Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item < 0 ? 0 : item);
-      for (int u = 0;; ++u) {
-        const int qs = u % Q;
-        int good = 1;
-        if (lane == 0) {
-          if (u >= Q && !mbar_wait(smem_u32(&ifree[qs]), (uint32_t)(((u / Q) - 1) & 1),
-                                   abort_flag, &st->status)) {
-            good = 0;
-          } else {
-            iq[qs] = item;
-            mbar_arrive(smem_u32(&iready[qs]));  // releases iq[qs]
-          }
-        }
-        if (!__shfl_sync(0xffffffffu, good, 0)) {
-          ok = false;
-          break;
-        }
-        if (item < 0) break;
-        int claim = 0;
-        if (lane == 0) claim = atomicAdd(next_item, 1);  // used after the k-loop
-        const int g0 = 4 * lane;
-        const bool active = g0 < it.n;
-        int y[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) y[i] = active ? __ldg(rowmap + it.r0 + min(g0 + i, it.n - 1)) : 0;
-        const uint32_t tx = (uint32_t)(((it.n + 3) / 4) * 4 * kBK * 2 + C::kBBytes);
-        const int w0 = it.wrow, w1 = GATEUP ? it.wrow + d.F : it.wrow + 128;
-        for (int kb = 0; kb < nk; ++kb) {
-          int good2 = 1;
-          if (lane == 0) good2 = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status);
-          if (!__shfl_sync(0xffffffffu, good2, 0)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = stage_base + stage * C::kStageBytes;
-          const uint32_t fb = smem_u32(&full[stage]);
-          if (lane == 0) {
-            mbar_expect_tx(fb, tx);
-            armed |= 1u << stage;
-            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          }
-          __syncwarp();
-          if (active) tma_gather4(smem_u32(sb + g0 * kBK * 2), &map_x, kb * kBK, y[0], y[1], y[2], y[3], fb);
-          if (lane == 0) {
-            tma_load_2d(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
-            tma_load_2d(smem_u32(sb + C::kABytes + C::kBBytes / 2), &map_w, kb * kBK, w1, fb);
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
-        const int nxt = (int)gridDim.x + __shfl_sync(0xffffffffu, claim, 0);
-        item = nxt < total ? nxt : -1;
-        if (item >= 0) it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
-      }
-      if (!ok && lane == 0) {  // let every issued copy land before the CTA exits
-        for (int s2 = 0; s2 < C::kStages; ++s2)
-          if ((armed >> s2) & 1u) {
-            const unsigned long long t0 = global_ns();
-            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
-                   global_ns() - t0 < kWaitLimitNs) {
-            }
-          }
-      }
-    } else if (lane == 0) {
+    if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
@@ -1051,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&iready[qs]));  // releases iq[qs]
         if (item < 0) break;
         const int claim = atomicAdd(next_item, 1);  // used after the k-loop
-        const int nbox = (it.n + kTmBox - 1) / kTmBox;
+        const int nbox = GATHER ? 0 : (it.n + kTmBox - 1) / kTmBox;
         const uint32_t tx = (uint32_t)(nbox * kTmBoxBytes + C::kBBytes);
         // weight rows of the 256-row N tile: GATEUP gate rows then up rows of
         // the feature block; else 256 consecutive output rows
@@ -1149,6 +1069,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         const unsigned long long t0 = global_ns();
         while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
         }
+      }
+    }
+  } else if (GATHER && warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ row gather
+    // Thread g copies chunk row g (128 bytes of K per k-block, eight 16-byte
+    // cp.async) to its swizzled place in the stage's token tile.  A stage's
+    // copies are signalled kGatherDepth - 1 stages later: the thread waits for
+    // its own copies (cp.async.wait_group), makes them visible to the tensor
+    // core's proxy and arrives on the stage's full barrier.
+    const int g = threadIdx.x - 32 * (2 + kEpiWarps);
+    const uint32_t row_off = (uint32_t)((g >> 3) * 1024 + (g & 7) * 128);
+    int stage = 0, pending = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    auto signal_oldest = [&](int depth_left) {
+      if (depth_left == 0) asm volatile("cp.async.wait_group 0;" ::: "memory");
+      else asm volatile("cp.async.wait_group %0;" ::"n"(kGatherDepth - 1) : "memory");
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      // unsignalled stages: stage - pending .. stage - 1 (stage already advanced)
+      const int old = (stage - pending + 4 * C::kStages) % C::kStages;
+      mbar_arrive(smem_u32(&full[old]));
+      --pending;
+    };
+    for (int u = 0; ok; ++u) {
+      const int qs = u % Q;
+      if (!mbar_wait(smem_u32(&iready[qs]), (uint32_t)((u / Q) & 1), abort_flag, &st->status)) break;
+      const int item = iq[qs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&ifree[qs]));
+      if (item < 0) break;
+      const Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
+      const bool active = g < it.n;
+      const char* src =
+          reinterpret_cast<const char*>(xsrc + (size_t)(active ? __ldg(rowmap + it.r0 + g) : 0) * d.H);
+      for (int kb = 0; kb < nk; ++kb) {
+        int good = 1;
+        if (lane == 0) good = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status);
+        if (!__shfl_sync(0xffffffffu, good, 0)) {
+          ok = false;
+          break;
+        }
+        if (active) {
+          const uint32_t dst = smem_u32(stage_base + stage * C::kStageBytes) + row_off;
+          const char* s0 = src + kb * kBK * 2;
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst + ((c ^ (g & 7)) << 4)),
+                         "l"(s0 + 16 * c)
+                         : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        ++pending;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (pending == kGatherDepth) signal_oldest(1);
+      }
+    }
+    while (pending > 0) {  // the last stages (or, on an abort, let the copies land)
+      if (ok) signal_oldest(0);
+      else {
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        pending = 0;
       }
     }
   } else {
@@ -1623,22 +1607,25 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
 }
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                           int grid, cudaStream_t s, int which, bool gather) {
+                           int grid, cudaStream_t s, int which, const void* x_rows) {
+  const bool gather = x_rows != nullptr;
   const int32_t* rowmap = w.rowmap;
+  const __nv_bfloat16* none = nullptr;
   if (which == 1 && gather)
-    return launch_pdl(k_gemm_tm<true, true>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes, s,
-                      1, maps.w_gateup, maps.hidden_rows, d, c.st, (const int32_t*)w.seg_rows,
-                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
-                      static_cast<__nv_bfloat16*>(w.act));
+    return launch_pdl(k_gemm_tm<true, true>, dim3(grid), dim3(kThreads + 32 * kGatherWarps),
+                      CfgTM<true>::kSmemBytes, s, 1, maps.w_gateup, maps.w_gateup, d, c.st,
+                      (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                      (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
+                      static_cast<const __nv_bfloat16*>(x_rows), static_cast<__nv_bfloat16*>(w.act));
   if (which == 1)
     return launch_pdl(k_gemm_tm<true, false>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes,
                       s, 1, maps.w_gateup, maps.A32, d, c.st, (const int32_t*)w.seg_rows,
                       (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
-                      static_cast<__nv_bfloat16*>(w.act));
+                      none, static_cast<__nv_bfloat16*>(w.act));
   return launch_pdl(k_gemm_tm<false, false>, dim3(grid), dim3(kThreads), CfgTM<false>::kSmemBytes,
                     s, 1, maps.w_down, maps.act32, d, c.st, (const int32_t*)w.seg_rows,
                     (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowmap,
-                    static_cast<__nv_bfloat16*>(w.y));
+                    none, static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -1720,10 +1707,6 @@ cudaError_t encode(CUtensorMap* map, const void* base, unsigned long long rows, 
 }
 
 }  // namespace
-
-cudaError_t make_hidden_map(const Dims& d, const void* hidden, TcMaps* maps) {
-  return encode(&maps->hidden_rows, hidden, (unsigned long long)d.M * d.T, d.H, 1);
-}
 
 cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
                          TcMaps* maps) {

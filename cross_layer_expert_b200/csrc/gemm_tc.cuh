@@ -18,14 +18,11 @@ struct TcMaps {
   CUtensorMap act2;
   CUtensorMap w_gateup64;  // w_gateup in boxes of 64 rows (two-SM token-major engine)
   CUtensorMap A32;       // same buffers, boxes of 32 rows (token-major engines)
-  CUtensorMap hidden_rows;  // the caller's hidden states [M*T, H], one-row boxes (gather4)
   CUtensorMap act32;
 };
 
 // Encodes the maps for these buffers; returns cudaErrorInvalidValue if the
-// driver rejects a map (alignment, strides).  make_hidden_map encodes the
-// map of the caller's hidden states that the gathering GEMM 1 reads.
-cudaError_t make_hidden_map(const Dims& d, const void* hidden, TcMaps* maps);
+// driver rejects a map (alignment, strides).
 cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, const void* w_down,
                          TcMaps* maps);
 // Opts the kernels into their dynamic shared memory (once per device).
@@ -37,10 +34,11 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
                             int grid, cudaStream_t s, int which);
 // Token-major engine: 128 token rows x 256 weight rows per MMA (GEMM 1: 128
 // features of gate and up; GEMM 2: 256 features).
-// gather (GEMM 1 only): read token rows from the hidden states through the
-// row map instead of from the permuted copy.
+// x_rows (GEMM 1 only, may be null): the hidden states [M*T, H]; when given,
+// token rows are gathered from them through the row map instead of being
+// read from the permuted copy.
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                           int grid, cudaStream_t s, int which, bool gather);
+                           int grid, cudaStream_t s, int which, const void* x_rows);
 // Two-SM token-major engine (cta_group::2): a CTA pair computes a chunk of up
 // to 256 tokens against 256 weight rows; each CTA holds half the tokens and
 // half the weight rows (M = 256 MMAs above 128 tokens, M = 128 below).

@@ -225,6 +225,11 @@ def run_ours(args, world, rank, local):
                        + (R * (wl.H * b + 4)).sum()),
         "combine": int((R * (wl.H * b + 8)).sum()
                        + 2 * sum(bin(int(m)).count("1") for m in rows[:, 0]) * wl.T * wl.H * b),
+        # every (micro-batch, layer) is routed once: fp32 logits in, indices
+        # and gates out, one count row per 64-token chunk
+        "route": int(wl.M * wl.L * (wl.T * (4 * wl.E + 8 * wl.k) + -(-wl.T // 64) * 4 * wl.E)),
+        # indices in, the row of every (token, slot) and the token of every row out
+        "positions": int((R * (4 + 4 + 4)).sum()),
     }
     flops_gemm = int((R * 6 * wl.H * wl.F).sum())
 
@@ -267,8 +272,10 @@ def run_ours(args, world, rank, local):
     gemm_ms = prof["gemm_gateup"][0] + prof["gemm_down"][0]
     kernels = {k: {"ms_per_episode": round(v[0] / args.steps, 4), "launches": v[1]}
                for k, v in prof.items()}
-    for k in ("gemm_gateup", "gemm_down", "permute", "combine"):
-        kernels[k]["GBps"] = round(alg[k] * args.steps / (prof[k][0] / 1e3) / 1e9, 1)
+    for k in ("route", "positions", "permute", "gemm_gateup", "gemm_down", "combine"):
+        if prof[k][0] > 0:
+            kernels[k]["GBps"] = round(alg[k] * args.steps / (prof[k][0] / 1e3) / 1e9, 1)
+            kernels[k]["frac_of_hbm"] = round(kernels[k]["GBps"] / peak, 4)
     kernels["gemm_tflops"] = round(flops_gemm * args.steps / (gemm_ms / 1e3) / 1e12, 2)
 
     # end to end: host buffers, copies inside the timed region

@@ -37,7 +37,8 @@ EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_crea
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
             "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped"]
 
-PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine")
+PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine",
+                "positions")
 
 
 class EbError(RuntimeError):

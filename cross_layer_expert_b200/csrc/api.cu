@@ -374,7 +374,9 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
   if (c.compute) {
     if (e == cudaSuccess)
-      e = timed(x, 2, gather ? 1 : 2, s, [&] { return launch_permute(x->d, x->dev, w, hidden, !gather, s); });
+      e = timed(x, 6, 1, s, [&] { return launch_positions(x->d, x->dev, w, s); });
+    if (e == cudaSuccess && !gather)
+      e = timed(x, 2, 1, s, [&] { return launch_permute_copy(x->d, x->dev, w, hidden, s); });
     if (e == cudaSuccess) {
       e = timed(x, 3, 1, s, [&] { return launch_engine(x, g1, w, wgu, wdn, hidden, s, 1); });
       if (e == cudaSuccess)

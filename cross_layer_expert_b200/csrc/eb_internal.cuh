@@ -162,10 +162,12 @@ cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int 
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
                          int32_t* w, int32_t* status, cudaStream_t s);
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
-// Rows of every (token, slot) of the RunSet (pos, rowmap); with `copy`, also
-// the permuted copy A of the token rows.
-cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
-                           bool copy, cudaStream_t s);
+// Rows of every (token, slot) of the RunSet (pos) and the token of every row
+// (rowmap).
+cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s);
+// The permuted copy A of the RunSet's token rows (after launch_positions).
+cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
+                                cudaStream_t s);
 cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
                            cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) on the CUDA cores.

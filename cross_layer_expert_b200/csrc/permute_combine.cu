@@ -329,11 +329,14 @@ int persistent_grid(const void* kernel, int threads, int& cache) {
 
 int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb_f32 = 0;
 
-cudaError_t launch_permute(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
-                           bool copy, cudaStream_t s) {
-  cudaError_t e = launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPermThreads), 0, s, 1, d, c.st,
-                             w.idx, w.chunk_hist, w.seg_rows, w.prior, w.pos, w.rowmap);
-  if (e != cudaSuccess || !copy) return e;
+cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s) {
+  return launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPermThreads), 0, s, 1, d, c.st,
+                    (const int32_t*)w.idx, (const int32_t*)w.chunk_hist,
+                    (const int32_t*)w.seg_rows, (const int32_t*)w.prior, w.pos, w.rowmap);
+}
+
+cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
+                                cudaStream_t s) {
   if (d.dtype == EB_DTYPE_BF16)
     return launch_pdl(k_permute_copy<__nv_bfloat16>,
                       dim3(persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads,

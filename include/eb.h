@@ -207,10 +207,11 @@ eb_status eb_trace(eb_ctx* ctx, int64_t* rows, int32_t* layers, int max_steps, i
  * enqueues with CUDA events on the launching stream (eb_profile(ctx, 0) stops;
  * both drop earlier marks).  eb_profile_read waits for them and returns, per
  * kernel, the summed milliseconds and the number of launches since, then
- * clears the marks.  Kernel order: route, schedule+plan, permute, GEMM 1
- * (gate/up + SwiGLU), GEMM 2 (down), combine.  eb_launch_count returns the
- * kernels the context has enqueued since eb_create. */
-#define EB_PROF_KERNELS 6
+ * clears the marks.  Kernel order: route, schedule+plan, permute (the row
+ * copy), GEMM 1 (gate/up + SwiGLU), GEMM 2 (down), combine, positions (the
+ * rows of every token slot).  eb_launch_count returns the kernels the
+ * context has enqueued since eb_create. */
+#define EB_PROF_KERNELS 7
 eb_status eb_profile(eb_ctx* ctx, int enable);
 eb_status eb_profile_read(eb_ctx* ctx, double* ms, int64_t* launches);
 eb_status eb_launch_count(eb_ctx* ctx, int64_t* n);

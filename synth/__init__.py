@@ -32,6 +32,12 @@ Logit recipes (noise is always N(0,1) per (micro-batch, layer, token, expert)):
                      positions: the hot set moves by one virtual rank every
                      4 layers.
 
+Router weights (for stacks whose logits are projected from the hidden state):
+row e of layer l is N(0, (s_{l,e} / sqrt(H))^2) with s_{l,e} = 0.5 + 2.5
+pi_{l,e} / max_e pi_{l,e} and pi_l ~ Dir(alpha) per layer, so experts with
+larger rows win more often -- a per-layer routing skew -- while the scores
+stay O(1) for hidden states of unit scale.
+
 Weights: ``w_init="normal"`` draws N(0, w_std^2) (the stated N(0, 0.02) of
 the tiny and Moonlight-shaped stacks); ``w_init="fan_in"`` draws
 N(0, 1 / (3 fan_in)) per matrix -- the variance of a linear layer's default
@@ -48,7 +54,7 @@ import numpy as np
 BASE_SEED = 20260808
 
 # stream tags keep the draws of different tensors independent
-_TAG_LOGITS, _TAG_HIDDEN, _TAG_WEIGHTS, _TAG_PROFILE, _TAG_PROFILE_PICK = 1, 2, 3, 4, 5
+_TAG_LOGITS, _TAG_HIDDEN, _TAG_WEIGHTS, _TAG_PROFILE, _TAG_PROFILE_PICK, _TAG_ROUTER = 1, 2, 3, 4, 5, 6
 
 
 @dataclasses.dataclass(frozen=True)
@@ -231,3 +237,20 @@ def weights_torch(w: Workload, device="cpu"):
         dn[l] = (torch.randn((Et, w.H, w.F), generator=g, device=device,
                              dtype=torch.float32) * std_dn).to(dt)
     return gu, dn
+
+
+def router_torch(w: Workload, device="cpu"):
+    """Router weights [L, E, H] in the workload's storage type (see the module
+    docstring); each layer from its own generator seeded by (seed, layer)."""
+    import torch
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    pis = _profile_pis(w, [w.alpha])[0]  # [L, E]
+    out = torch.empty((w.L, w.E, w.H), dtype=dt, device=device)
+    for l in range(w.L):
+        s = 0.5 + 2.5 * pis[l] / pis[l].max()
+        g = torch.Generator(device=device)
+        g.manual_seed((w.seed * 1000003 + _TAG_ROUTER * 7919 + l) & 0x7FFFFFFFFFFF)
+        rows = torch.randn((w.E, w.H), generator=g, device=device, dtype=torch.float32)
+        scale = torch.tensor(s / np.sqrt(w.H), dtype=torch.float32, device=device)[:, None]
+        out[l] = (rows * scale).to(dt)
+    return out

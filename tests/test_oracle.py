@@ -440,3 +440,46 @@ def test_native_maxutil_matches_python():
             continue
         w = {j: [int(x) for x in v.split()] for j, v in enumerate(ws.split(";"))}
         assert native.maxutil(sorted(w), w, int(m)) == [int(x) for x in want.split()]
+
+
+# ------------------------------------------------------------ router projection
+
+def test_router_projection_pins():
+    """The router projection: written-out loops on a small case, one-hot
+    router rows pick hidden columns exactly, a zero router gives equal scores
+    (so the top-k falls back to experts 0..k-1 with equal gates), and the
+    routed chain with identical experts equals the dense SwiGLU chain."""
+    from oracle import router as orouter
+    rng = np.random.default_rng(40)
+    h = omoe.round_bf16(rng.standard_normal((5, 24)))
+    w = omoe.round_bf16(rng.standard_normal((6, 24)) * 0.3)
+    assert np.allclose(orouter.router_logits(h, w), orouter.router_logits_loops(h, w),
+                       rtol=0, atol=1e-12)
+    cols = [3, 0, 23, 7, 7, 11]
+    onehot = np.zeros((6, 24))
+    onehot[np.arange(6), cols] = 1.0
+    assert np.array_equal(orouter.router_logits(h, onehot), h[:, cols])
+    zero = orouter.router_logits(h, np.zeros((6, 24)))
+    idx, gate = oracle.route(zero.astype(np.float32), 3)
+    assert (idx == [0, 1, 2]).all() and np.allclose(gate, 1.0 / 3)
+    # identical experts: the MoE layer is one dense SwiGLU FFN whatever the
+    # router picks (gates sum to 1), so the routed chain is the dense chain
+    H, F, E, k, L = 24, 16, 6, 2, 3
+    wg = [omoe.round_bf16(rng.standard_normal((F, H)) * 0.2) for _ in range(L)]
+    wu = [omoe.round_bf16(rng.standard_normal((F, H)) * 0.2) for _ in range(L)]
+    wd = [omoe.round_bf16(rng.standard_normal((H, F)) * 0.2) for _ in range(L)]
+    routers = [omoe.round_bf16(rng.standard_normal((E, H))) for _ in range(L)]
+    get = lambda l, e: (wg[l], wu[l], wd[l])
+    out, seen = orouter.forward_tokens_routed(h, lambda l: routers[l], [(0, t) for t in range(5)],
+                                              L, E, k, 0, "f32", get)
+    import torch
+    x = torch.tensor(h, dtype=torch.float64)
+    for l in range(L):
+        g = x @ torch.tensor(wg[l]).T
+        u = x @ torch.tensor(wu[l]).T
+        y = (g * torch.sigmoid(g) * u) @ torch.tensor(wd[l]).T
+        x = x + y
+    assert np.allclose(out, x.numpy(), rtol=1e-5, atol=1e-5)
+    assert len(seen) == L and seen[0].dtype == np.float32
+    # the first layer's scores are the projection of h_0 itself
+    assert np.array_equal(seen[0], orouter.router_logits(h, routers[0]).astype(np.float32))

@@ -42,6 +42,8 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-under-util", action="store_true")
+    p.add_argument("--no-router-mode", action="store_true",
+                   help="skip the extra router-mode episode timing")
     p.add_argument("--layers", type=int, default=0,
                    help="override the workload's MoE layer count (small profiling cases)")
     return p.parse_args()
@@ -307,6 +309,41 @@ def run_ours(args, world, rank, local):
                "steps": k_e2e}
     ctx.close()
 
+    # router mode (the routing scores projected from the hidden states on the
+    # device, a data-dependent chain): episode time and the projection's share
+    router_mode = None
+    if not args.no_router_mode:
+        w_router = synth.router_torch(wl, device=dev)
+        rctx = eb.Context(cfg_for(policy))
+        rctx.eb_set_router(w_router)
+        for _ in range(2):
+            hidden.copy_(h0)
+            rctx.eb_episode(None, hidden, wgu, wdn)
+        barrier(world)
+        torch.cuda.synchronize()
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        k_r = max(1, args.steps // 2)
+        r0.record(stream)
+        for _ in range(k_r):
+            hidden.copy_(h0)
+            n_r = rctx.eb_episode(None, hidden, wgu, wdn)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        assert rctx.eb_sync_status() == eb.EB_OK
+        ms_r = max_over_ranks(r0.elapsed_time(r1), world)
+        rctx.eb_profile(True)
+        hidden.copy_(h0)
+        rctx.eb_episode(None, hidden, wgu, wdn)
+        rprof = rctx.eb_profile_read()
+        rctx.close()
+        del w_router
+        router_mode = {"value": round(job_throughput(wl.M * wl.T * wl.L * k_r, ms_r, world), 1),
+                       "unit": UNIT, "ms_per_step": round(ms_r / k_r, 3), "scheduler_steps": n_r,
+                       "router_ms_per_episode": round(rprof["router"][0], 4),
+                       "router_tflops": round(2.0 * wl.M * wl.T * wl.L * wl.E * wl.H
+                                              / (rprof["router"][0] / 1e3) / 1e12, 2)}
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(wl, policy, logits_np, h0, wgu, wdn)
@@ -328,6 +365,7 @@ def run_ours(args, world, rank, local):
                        "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
             "e2e": e2e, "gpu_launches": int(launches), "roofline": roof,
             "cpu_baseline": cpu, "clocks": clk, "under_util": under, "kernels": kernels,
+            "router_mode": router_mode,
         }
         print(json.dumps(line), flush=True)
 

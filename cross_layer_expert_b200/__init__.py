@@ -35,10 +35,11 @@ EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_crea
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
-            "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped"]
+            "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped", "eb_set_router",
+            "eb_router"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine",
-                "positions")
+                "positions", "router")
 
 
 class EbError(RuntimeError):
@@ -83,6 +84,8 @@ def load() -> ctypes.CDLL:
         "eb_loads": (I, [P, I, I, I, P, P]),
         "eb_loads_mapped": (I, [P, I, I, I, P, P, P, P]),
         "eb_set_expert_map": (I, [P, P]),
+        "eb_set_router": (I, [P, P, P]),
+        "eb_router": (I, [P, I, I, P, I, P, P, P]),
         "eb_schedule": (I, [P, U32, I, I, I, I, P, P, P]),
         "eb_profile": (I, [P, I]),
         "eb_profile_read": (I, [P, P, P]),
@@ -161,6 +164,14 @@ def eb_loads_mapped(hist, D: int, expert_rank, w, status=None, stream=None) -> N
            "eb_loads_mapped")
 
 
+def eb_router(hidden, w_router, scores, status=None, stream=None) -> None:
+    """hidden [n, H] bf16 x w_router [E, H] bf16 -> scores [n, E] f32."""
+    n, H = hidden.shape
+    E = w_router.shape[0]
+    _check(load().eb_router(_ptr(hidden), n, H, _ptr(w_router), E, _ptr(scores), _ptr(status),
+                            _stream(stream)), "eb_router")
+
+
 def eb_schedule(w, pending_mask: int, m: int, policy: int, runset, stats=None, stream=None) -> None:
     """w [M, D] i32 -> runset (1-element u32/i32 device tensor), stats [3] i64."""
     M, D = w.shape
@@ -215,6 +226,14 @@ class Context:
 
     def eb_reset(self, stream=None) -> None:
         _check(load().eb_reset(self.handle, _stream(stream)), "eb_reset")
+
+    def eb_set_router(self, w_router=None, scores=None) -> None:
+        """Router weights [L, E, H] bf16 on the device (kept alive by the
+        caller): steps then project their routing scores from the hidden
+        states, into `scores` [M, L, T, E] f32 if given.  None returns to
+        caller-given logits."""
+        self._router = (w_router, scores)
+        _check(load().eb_set_router(self.handle, _ptr(w_router), _ptr(scores)), "eb_set_router")
 
     def eb_set_expert_map(self, expert_rank=None) -> None:
         """Placement of the E experts on the D ranks (a sequence of ints), or

@@ -23,6 +23,11 @@ struct eb_ctx {
   int num_sms = 148;
   bool use_tc = false;
   int eng1 = EB_GEMM_SIMT, eng2 = EB_GEMM_SIMT;  // engine of GEMM 1 / GEMM 2
+  // router mode: scores projected from the hidden states (eb_set_router)
+  const void* w_router = nullptr;
+  float* router_out = nullptr;  // optional caller buffer [M, L, T, E] for the scores
+  CUtensorMap router_map_h, router_map_r;
+  const void* router_keys[2] = {nullptr, nullptr};
   cudaStream_t last_stream = nullptr;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
@@ -142,6 +147,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
     x.seg_items1 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.seg_items2 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.gemm_next = (int32_t*)take(sizeof(int32_t) * 2);
+    x.scores = (float*)take(sizeof(float) * M * T * c.E);
     x.Rcap = (long long)(M * T * d.kk);
     const size_t es = elem_size(c.dtype);
     x.A = take(es * (size_t)x.Rcap * c.H);
@@ -327,6 +333,22 @@ eb_status eb_set_expert_map(eb_ctx* x, const int32_t* expert_rank) {
   return EB_OK;
 }
 
+eb_status eb_set_router(eb_ctx* x, const void* w_router, float* scores) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  if (w_router) {
+    const eb_config& c = x->cfg;
+    if (!c.compute || c.dtype != EB_DTYPE_BF16 || c.E % 16 != 0 || c.E > 256 || c.H % 64 != 0)
+      return EB_ERR_UNSUPPORTED;
+    if (((uintptr_t)w_router & 15u) != 0) return EB_ERR_INVALID_ARG;
+    if (gemm_tc_prepare() != cudaSuccess) return EB_ERR_CUDA;
+  }
+  if (scores && ((uintptr_t)scores & 15u) != 0) return EB_ERR_INVALID_ARG;
+  x->w_router = w_router;
+  x->router_out = w_router ? scores : nullptr;
+  x->router_keys[1] = nullptr;
+  return EB_OK;
+}
+
 static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* wgu,
                                  const void* wdn, const void* hidden, cudaStream_t s, int which) {
   switch (eng) {
@@ -345,7 +367,8 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
                               const void* wdn, void* workspace, size_t ws_bytes,
                               cudaStream_t s) {
   const eb_config& c = x->cfg;
-  if (!logits || !workspace) return EB_ERR_INVALID_ARG;
+  if ((!logits && !x->w_router) || !workspace) return EB_ERR_INVALID_ARG;
+  if (x->w_router && !hidden) return EB_ERR_INVALID_ARG;
   if (((uintptr_t)workspace & (kAlign - 1)) != 0) return EB_ERR_INVALID_ARG;
   if (c.compute && (!hidden || !wgu || !wdn)) return EB_ERR_INVALID_ARG;
   if (c.compute && (!aligned16(hidden) || !aligned16(wgu) || !aligned16(wdn)))
@@ -369,7 +392,35 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   int rn1, fm1, rn2, fm2;
   engine_tiles(g1, 1, &rn1, &fm1);
   engine_tiles(g2, 2, &rn2, &fm2);
-  cudaError_t e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, logits, s); });
+  cudaError_t e = cudaSuccess;
+  if (x->w_router) {  // project this step's router scores from the hidden states
+    if (x->router_keys[0] != hidden || x->router_keys[1] != x->w_router) {
+      if (make_router_maps(hidden, (long long)c.M * c.T, c.H, x->w_router, c.L, c.E,
+                           &x->router_map_h, &x->router_map_r) != cudaSuccess)
+        return EB_ERR_UNSUPPORTED;
+      x->router_keys[0] = hidden;
+      x->router_keys[1] = x->w_router;
+    }
+  }
+  // where routing reads each micro-batch's rows: the caller's logits, the
+  // caller's score buffer (router mode) or the workspace (router mode)
+  const long long TE = (long long)c.T * c.E;
+  const float* rsrc = logits;
+  long long mbs = (long long)c.L * TE, ls = TE;
+  if (x->w_router) {
+    float* dst = x->router_out ? x->router_out : w.scores;
+    if (!x->router_out) {
+      mbs = TE;
+      ls = 0;
+    }
+    rsrc = dst;
+    e = timed(x, 7, 1, s, [&] {
+      return launch_router(x->router_map_h, x->router_map_r, c.T, c.H, c.E, c.M, x->dev.st, dst,
+                           mbs, ls, &x->dev.st->status, s);
+    });
+  }
+  if (e == cudaSuccess)
+    e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, s); });
   if (e == cudaSuccess)
     e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
   if (c.compute) {
@@ -534,6 +585,23 @@ eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* s
   if (M < 0 || E < 1 || D < 1 || E % D != 0) return EB_ERR_INVALID_ARG;
   if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
   return cuda_status(launch_loads(hist, M, E, D, nullptr, w, nullptr, (cudaStream_t)stream));
+}
+
+eb_status eb_router(const void* hidden, int n, int H, const void* w_router, int E, float* scores,
+                    int32_t* status_dev, void* stream) {
+  if (n < 0 || H < 1 || E < 1 || (n > 0 && (!hidden || !w_router || !scores)))
+    return EB_ERR_INVALID_ARG;
+  if (E % 16 != 0 || E > 256 || H % 64 != 0) return EB_ERR_UNSUPPORTED;
+  if (((uintptr_t)hidden & 15u) != 0 || ((uintptr_t)w_router & 15u) != 0 ||
+      ((uintptr_t)scores & 15u) != 0)
+    return EB_ERR_INVALID_ARG;
+  if (n == 0) return EB_OK;
+  if (gemm_tc_prepare() != cudaSuccess) return EB_ERR_CUDA;
+  CUtensorMap mh, mr;
+  if (make_router_maps(hidden, n, H, w_router, 1, E, &mh, &mr) != cudaSuccess)
+    return EB_ERR_UNSUPPORTED;
+  return cuda_status(launch_router(mh, mr, n, H, E, 1, nullptr, scores, 0, 0, status_dev,
+                                   (cudaStream_t)stream));
 }
 
 eb_status eb_loads_mapped(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,

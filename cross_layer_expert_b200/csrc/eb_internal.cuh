@@ -85,6 +85,7 @@ struct Work {
   int32_t* seg_items1; // [M*Etot + 1]
   int32_t* seg_items2; // [M*Etot + 1]
   int32_t* gemm_next;  // [2]: next dynamically claimed item of GEMM 1 / GEMM 2 (zeroed by the plan)
+  float* scores;       // [M][T][E]: router scores of the step (router mode)
   void* A;             // [Rcap][H] permuted tokens
   void* act;           // [Rcap][F] SwiGLU activations
   void* y;             // [Rcap][H] expert outputs
@@ -146,8 +147,11 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 // ---- launchers (all asynchronous on `s`) ----
+// Micro-batch j's rows at layer l start at logits + j * mb_stride + l *
+// layer_stride (elements): (L T E, T E) for the caller's [M, L, T, E] logits,
+// (T E, 0) for router scores of the step kept as [M, T, E].
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
-                              cudaStream_t s);
+                              long long mb_stride, long long layer_stride, cudaStream_t s);
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
                               float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
 // rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm1 / fm2:

@@ -1519,6 +1519,169 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Router projection: scores = h W_r^T in float32 for the micro-batches that
+// route this step, each with the router of its current layer ([EB] §2.1:
+// W_l, I_l = topk(G(h'_l)), with a linear scorer).  One CTA per (micro-batch,
+// 128-token chunk): 128 tokens are the MMA's M side, the E router rows its N
+// side (E a multiple of 16, at most 256), K = H in 64-element k-blocks fed by
+// TMA through a 4-stage ring; the accumulator (128 lanes x E columns) is
+// drained to [token][expert] float32 rows.
+// ---------------------------------------------------------------------------
+
+constexpr int kRouterThreads = 192;  // producer, MMA issuer, 4 drain warps
+constexpr int kRouterStages = 4;
+constexpr int kRouterABytes = 128 * kBK * 2;                 // 16 KiB
+constexpr int kRouterStageBytes = kRouterABytes + 256 * kBK * 2;  // room for E = 256
+constexpr int kRouterSmemBytes = kRouterStages * kRouterStageBytes + 1024 + 1024;
+
+// map_h: hidden rows [rows, H] in boxes of 128 rows; map_r: router rows
+// [layers * E, H] in boxes of E rows.  st == nullptr: stand-alone call, one
+// block of T rows at layer 0; else the micro-batches in st->need_route at
+// st->layer[j].  Row t of micro-batch j at layer l goes to out + j * mb_stride
+// + l * layer_stride + t * E.
+__global__ void __launch_bounds__(kRouterThreads, 1)
+    k_router(const __grid_constant__ CUtensorMap map_h, const __grid_constant__ CUtensorMap map_r,
+             int T, int H, int E, const State* __restrict__ st, float* __restrict__ out,
+             long long mb_stride, long long layer_stride, int* __restrict__ status) {
+  pdl_enter();
+  const int c = blockIdx.x, j = blockIdx.y;
+  int l = 0;
+  if (st) {
+    if (!((st->need_route >> j) & 1u)) return;
+    l = st->layer[j];
+  }
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kRouterStages * kRouterStageBytes);
+  uint64_t* full = bars;                  // [kRouterStages]
+  uint64_t* empty = bars + kRouterStages;  // [kRouterStages]
+  uint64_t* done = bars + 2 * kRouterStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = H / kBK;
+  const uint32_t tmem_cols = E <= 32 ? 32 : E <= 64 ? 64 : E <= 128 ? 128 : 256;
+  int dummy = 0;
+  int* stat = status ? status : &dummy;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kRouterStages; ++i) {
+      mbar_init(smem_u32(&full[i]), 1);
+      mbar_init(smem_u32(&empty[i]), 1);
+    }
+    mbar_init(smem_u32(done), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(tmem_cols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const int row0 = j * T + c * 128;  // first hidden row of the chunk
+  const uint32_t tx = (uint32_t)(kRouterABytes + E * kBK * 2);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t armed = 0, armed_par = 0;
+      bool ok = true;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, stat)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sb = smem + stage * kRouterStageBytes;
+        const uint32_t fb = smem_u32(&full[stage]);
+        mbar_expect_tx(fb, tx);
+        tma_load_2d(smem_u32(sb), &map_h, kb * kBK, row0, fb);
+        tma_load_2d(smem_u32(sb + kRouterABytes), &map_r, kb * kBK, l * E, fb);
+        armed |= 1u << stage;
+        armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == kRouterStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (!ok) {
+        for (int s2 = 0; s2 < kRouterStages; ++s2)
+          if ((armed >> s2) & 1u) {
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
+                   global_ns() - t0 < kWaitLimitNs) {
+            }
+          }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued = false;
+      uint32_t last_bar = 0, last_par = 0;
+      const uint32_t idesc = idesc_bf16(128, E);
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, stat)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * kRouterStageBytes);
+#pragma unroll
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          mma_bf16(tmem, sdesc(sa + ks * 32), sdesc(sa + kRouterABytes + ks * 32), idesc,
+                   (kb | ks) != 0);
+        mma_commit(smem_u32(&empty[stage]));
+        last_bar = smem_u32(&empty[stage]);
+        last_par = phase;
+        issued = true;
+        if (++stage == kRouterStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (ok) mma_commit(smem_u32(done));
+      else if (issued) {
+        const unsigned long long t0 = global_ns();
+        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else {
+    // drain: warp w reads TMEM lanes 32 (w % 4) .. +31 = tokens of the chunk
+    const int q = warp & 3;
+    if (mbar_wait(smem_u32(done), 0, abort_flag, stat)) {
+      tc_fence_after();
+      const int t = c * 128 + q * 32 + lane;
+      float* orow = out + (size_t)j * mb_stride + (size_t)l * layer_stride + (size_t)t * E;
+      for (int cb = 0; cb < E; cb += 32) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(q * 32) << 16) + cb, v);
+        if (t < T) {
+          const int n = min(32, E - cb);  // E is a multiple of 16
+          for (int i = 0; i < n; i += 4)
+            *reinterpret_cast<float4*>(orow + cb + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                 "r"(tmem_cols));
+  }
+}
+
 // CTA pairs of `kernel` that fit on the device at once (one CTA per SM; an
 // SM pair must sit in one GPC, so an odd SM count per GPC leaves SMs out).
 // Queried once per device and kernel.
@@ -1571,6 +1734,9 @@ cudaError_t gemm_tc_prepare() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_gemm_tm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kRouterSmemBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_gemm_tm2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM2<true>::kSmemBytes);
@@ -1626,6 +1792,14 @@ cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const 
                     s, 1, maps.w_down, maps.act32, d, c.st, (const int32_t*)w.seg_rows,
                     (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowmap,
                     none, static_cast<__nv_bfloat16*>(w.y));
+}
+
+cudaError_t launch_router(const CUtensorMap& map_h, const CUtensorMap& map_r, int T, int H, int E,
+                          int n_mb, const State* st, float* out, long long mb_stride,
+                          long long layer_stride, int* status, cudaStream_t s) {
+  return launch_pdl(k_router, dim3((T + 127) / 128, n_mb), dim3(kRouterThreads),
+                    (size_t)kRouterSmemBytes, s, 1, map_h, map_r, T, H, E, st, out, mb_stride,
+                    layer_stride, status);
 }
 
 cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -1720,6 +1894,13 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   if (e == cudaSuccess) e = encode(&maps->w_gateup64, w_gateup, experts * 2 * d.F, d.H, 64);
   if (e == cudaSuccess) e = encode(&maps->A32, w.A, (unsigned long long)w.Rcap, d.H, kTmBox);
   if (e == cudaSuccess) e = encode(&maps->act32, w.act, (unsigned long long)w.Rcap, d.F, kTmBox);
+  return e;
+}
+
+cudaError_t make_router_maps(const void* hidden, long long rows, int H, const void* w_router,
+                             int layers, int E, CUtensorMap* map_h, CUtensorMap* map_r) {
+  cudaError_t e = encode(map_h, hidden, (unsigned long long)rows, H, 128);
+  if (e == cudaSuccess) e = encode(map_r, w_router, (unsigned long long)layers * E, H, E);
   return e;
 }
 

@@ -44,6 +44,17 @@ cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const 
 // half the weight rows (M = 256 MMAs above 128 tokens, M = 128 below).
 cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                             int grid, cudaStream_t s, int which);
+// Router projection (float32 scores = h W_r^T): maps of the hidden rows
+// [rows, H] (boxes of 128 rows) and of the routers [layers * E, H] (boxes of
+// E rows), and the launch: n_mb blocks of T rows; st == nullptr routes one
+// block at layer 0, else the micro-batches in st->need_route at their layer;
+// row t of micro-batch j at layer l lands at out + j mb_stride + l
+// layer_stride + t E.
+cudaError_t make_router_maps(const void* hidden, long long rows, int H, const void* w_router,
+                             int layers, int E, CUtensorMap* map_h, CUtensorMap* map_r);
+cudaError_t launch_router(const CUtensorMap& map_h, const CUtensorMap& map_r, int T, int H, int E,
+                          int n_mb, const State* st, float* out, long long mb_stride,
+                          long long layer_stride, int* status, cudaStream_t s);
 // Runs the GEMM's bounded mbarrier wait on a barrier nothing arrives on.
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) of a step; grid = persistent

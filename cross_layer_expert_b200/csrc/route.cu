@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
                                                      int32_t* __restrict__ chunk_hist,
                                                      int32_t* __restrict__ hist,
                                                      int32_t* __restrict__ wload,
-                                                     const int32_t* __restrict__ emap) {
+                                                     const int32_t* __restrict__ emap,
+                                                     long long mb_stride, long long layer_stride) {
   pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->need_route >> j) & 1u)) return;
@@ -146,7 +147,9 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
   for (int r = threadIdx.x; r < d.D; r += blockDim.x) w_s[r] = 0;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
-  const float* blk = logits + ((size_t)j * d.L + l) * (size_t)d.T * d.E;
+  // rows of micro-batch j at layer l: the caller's logits [M, L, T, E], or
+  // the router's scores of this step (see launch_route_step)
+  const float* blk = logits + (size_t)j * mb_stride + (size_t)l * layer_stride;
   const int t0 = c * kChunk, t1 = min(d.T, t0 + kChunk);
   bool nonfinite = false;
   route_chunk<VPL>(blk, t0, t1, d.E, d.k, d.renorm, idx + (size_t)j * d.T * d.k,
@@ -203,15 +206,15 @@ int vpl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 }  // namespace
 
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
-                              cudaStream_t s) {
+                              long long mb_stride, long long layer_stride, cudaStream_t s) {
   dim3 grid(d.NC, d.M);
   const int32_t* emap = c.use_emap ? c.emap : nullptr;
   cudaError_t e;
   switch (vpl_for(d.E)) {
-    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
-    default: e = launch_pdl(k_route_step<8>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap); break;
+    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
+    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
+    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
+    default: e = launch_pdl(k_route_step<8>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
   }
   return e;
 }

@@ -133,6 +133,20 @@ eb_status eb_destroy(eb_ctx* ctx);
  * zeroed accumulators and trace.  Enqueued on `stream`. */
 eb_status eb_reset(eb_ctx* ctx, void* stream);
 
+/* Router mode ([EB] §2.1, W_l, I_l = topk(G(h'_l)) with a linear scorer):
+ * w_router (DEVICE, bf16 [L, E, H], 16-byte aligned, caller-owned) makes
+ * every step project the routing scores itself -- scores = h W_r[l]^T in
+ * float32 for each micro-batch that routes, from its current hidden state
+ * and the router of its layer -- instead of reading the caller's logits,
+ * so the chain becomes data-dependent; eb_moe_step / eb_episode may then
+ * get logits = NULL.  scores (optional DEVICE float32 [M, L, T, E], 16-byte
+ * aligned, caller-owned) receives every step's scores at (j, l_j), where the
+ * routing then reads them; with scores = NULL they stay in the workspace.
+ * w_router = NULL returns to caller-given logits.  Needs compute, bf16, E a
+ * multiple of 16 (at most 256) and H a multiple of 64 (EB_ERR_UNSUPPORTED
+ * otherwise). */
+eb_status eb_set_router(eb_ctx* ctx, const void* w_router, float* scores);
+
 /* Expert placement used to fold expert counts into rank loads.  By default
  * rank d holds experts [d E/D, (d+1) E/D) ([EB] §5 Models, "evenly
  * distributed").  expert_rank (HOST array of cfg.E int32, each in
@@ -209,9 +223,10 @@ eb_status eb_trace(eb_ctx* ctx, int64_t* rows, int32_t* layers, int max_steps, i
  * kernel, the summed milliseconds and the number of launches since, then
  * clears the marks.  Kernel order: route, schedule+plan, permute (the row
  * copy), GEMM 1 (gate/up + SwiGLU), GEMM 2 (down), combine, positions (the
- * rows of every token slot).  eb_launch_count returns the kernels the
- * context has enqueued since eb_create. */
-#define EB_PROF_KERNELS 7
+ * rows of every token slot), router projection (router mode).
+ * eb_launch_count returns the kernels the context has enqueued since
+ * eb_create. */
+#define EB_PROF_KERNELS 8
 eb_status eb_profile(eb_ctx* ctx, int enable);
 eb_status eb_profile_read(eb_ctx* ctx, double* ms, int64_t* launches);
 eb_status eb_launch_count(eb_ctx* ctx, int64_t* n);
@@ -244,6 +259,14 @@ eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t
 /* Virtual-rank loads under the contiguous map: w[j][d] = sum of hist[j][e]
  * over e in [d E/D, (d+1) E/D).  hist [M, E] int32 -> w [M, D] int32. */
 eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream);
+
+/* Router scores for n token rows: scores [n, E] float32 = hidden [n, H] bf16
+ * times w_router [E, H] bf16 transposed (float32 accumulation on the tensor
+ * cores).  DEVICE pointers, 16-byte aligned.  E a multiple of 16 (<= 256), H a
+ * multiple of 64, else EB_ERR_UNSUPPORTED.  status_dev (optional device
+ * int32) gets EB_ERR_TIMEOUT if a bounded device wait expires. */
+eb_status eb_router(const void* hidden, int n, int H, const void* w_router, int E, float* scores,
+                    int32_t* status_dev, void* stream);
 
 /* Virtual-rank loads under an arbitrary placement: w[j][d] = sum of
  * hist[j][e] over the experts e with expert_rank[e] == d.  expert_rank is a

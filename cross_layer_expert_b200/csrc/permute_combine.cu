@@ -238,7 +238,7 @@ constexpr int kCombineThreads = 256;
 
 // Persistent: warp w combines tokens w, w + W, ... of the RunSet.
 template <typename T>
-__global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State* __restrict__ st,
+__global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, const State* __restrict__ st,
                                                              const float* __restrict__ gate,
                                                              const int32_t* __restrict__ pos,
                                                              const T* __restrict__ y, T* hidden) {
@@ -256,7 +256,8 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State
     const int my_row = lane < kk ? __ldg(pos + tok * kk + lane) : 0;
     const float my_gate = lane < k ? __ldg(gate + tok * k + lane) : 0.f;
     T* out = hidden + tok * d.H;
-    // two 16-byte vectors per lane per pass: 2 * kk loads in flight
+    // two 16-byte vectors per lane per pass, slots loaded four at a time
+    // (registers for three CTAs per SM)
     for (int v0 = lane; v0 < nvec; v0 += 64) {
       const int v1 = v0 + 32;
       const bool has1 = v1 < nvec;
@@ -268,10 +269,10 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State
 #pragma unroll
         for (int i = 0; i < VE; ++i) acc0[i] = acc1[i] = 0.f;
       }
-      for (int s0 = 0; s0 < kk; s0 += 8) {
-        uint4 r0[8], r1[8];
+      for (int s0 = 0; s0 < kk; s0 += 4) {
+        uint4 r0[4], r1[4];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           const int row = __shfl_sync(kFull, my_row, (s0 + q) & 31);
           if (s0 + q < kk) {
             const uint4* yrow = reinterpret_cast<const uint4*>(y + (size_t)row * d.H);
@@ -280,7 +281,7 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(Dims d, const State
           }
         }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
+        for (int q = 0; q < 4; ++q) {
           const int s = s0 + q;
           const float g = __shfl_sync(kFull, my_gate, s & 31);
           if (s >= kk) break;

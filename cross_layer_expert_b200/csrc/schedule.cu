@@ -237,50 +237,54 @@ __device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint3
   return sm.result;
 }
 
-// ---------------------------------------------------------------- block scan
-// Exclusive scan of v[0..n) in place (all threads); returns the total.
-// Each thread owns a contiguous run; run totals are scanned with warp
-// shuffles, then across the warps.
-__device__ int block_exclusive_scan(int* v, int n, int* tmp /* >= 33 ints */) {
-  const int per = (n + blockDim.x - 1) / blockDim.x;
-  const int b = threadIdx.x * per, e = min(n, b + per);
+
+struct PlanSmem {
+  int3 tmp3[33];
+};
+
+// Expert counts of the RunSet's micro-batches kept in shared memory by the
+// plan when nr * E fits (32 KiB).
+constexpr int kPlanHistCache = 8192;
+
+// Exclusive block-wide scan of per-thread int3 values: returns this thread's
+// offsets; tmp[32] receives the block totals.  All threads must call it.
+__device__ int3 block_exclusive_scan3(int3 v, int3* tmp /* >= 33 */) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int local = 0;
-  for (int i = b; i < e; ++i) local += v[i];
-  int incl = local;
+  int3 incl = v;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += y;
+    const int yx = __shfl_up_sync(0xffffffffu, incl.x, off);
+    const int yy = __shfl_up_sync(0xffffffffu, incl.y, off);
+    const int yz = __shfl_up_sync(0xffffffffu, incl.z, off);
+    if (lane >= off) {
+      incl.x += yx;
+      incl.y += yy;
+      incl.z += yz;
+    }
   }
   if (lane == 31) tmp[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int x = lane < nw ? tmp[lane] : 0;
-    int xi = x;
+    const int3 x = lane < nw ? tmp[lane] : make_int3(0, 0, 0);
+    int3 xi = x;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, xi, off);
-      if (lane >= off) xi += y;
+      const int yx = __shfl_up_sync(0xffffffffu, xi.x, off);
+      const int yy = __shfl_up_sync(0xffffffffu, xi.y, off);
+      const int yz = __shfl_up_sync(0xffffffffu, xi.z, off);
+      if (lane >= off) {
+        xi.x += yx;
+        xi.y += yy;
+        xi.z += yz;
+      }
     }
-    if (lane < nw) tmp[lane] = xi - x;  // exclusive warp offsets
-    if (lane == 31) tmp[32] = xi;       // block total
+    if (lane < nw) tmp[lane] = make_int3(xi.x - x.x, xi.y - x.y, xi.z - x.z);
+    if (lane == 31) tmp[32] = xi;
   }
   __syncthreads();
-  int run = tmp[warp] + incl - local;
-  for (int i = b; i < e; ++i) {
-    const int t = v[i];
-    v[i] = run;
-    run += t;
-  }
-  const int total = tmp[32];
-  __syncthreads();
-  return total;
+  const int3 w = tmp[warp];
+  return make_int3(w.x + incl.x - v.x, w.y + incl.y - v.y, w.z + incl.z - v.z);
 }
-
-struct PlanSmem {
-  int tmp[33];
-};
 
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
                                                              int rn2, int fm1, int fm2) {
@@ -415,32 +419,57 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   }
   __syncthreads();
   // 5. segment plan: rows of (group, expert) are counted into seg_rows and
-  //    scanned in place; GEMM work items per segment likewise.
+  //    scanned in place; GEMM work items per segment likewise.  The RunSet's
+  //    expert counts are staged in shared memory when they fit (the counts
+  //    and the prior table below read them several times).
   const int G = st->n_groups, nr = st->n_run, Et = d.Etot, nseg = G * Et;
   const int mb1 = d.F / fm1, mb2 = d.H / fm2;
   __shared__ int s_nonempty;
+  __shared__ int s_hist[kPlanHistCache];
+  const bool cached = nr * d.E <= kPlanHistCache;
   if (tid == 0) s_nonempty = 0;
+  if (cached)
+    for (int i = tid; i < nr * d.E; i += blockDim.x)
+      s_hist[i] = c.hist[st->run_list[i / d.E] * d.E + i % d.E];
   __syncthreads();
+  // counts of RunSet member a (position in run_list) for expert e
+  auto count_of = [&](int a, int e) -> int {
+    if (e >= d.E) return d.T;  // shared expert: every token
+    return cached ? s_hist[a * d.E + e] : c.hist[st->run_list[a] * d.E + e];
+  };
   int my_nonempty = 0;
-  for (int i = tid; i < nseg; i += blockDim.x) {
+  int3 local = make_int3(0, 0, 0);  // this thread's sums of rows, items1, items2
+  const int per = (nseg + blockDim.x - 1) / blockDim.x;
+  const int sb = tid * per, se = min(nseg, sb + per);
+  for (int i = sb; i < se; ++i) {
     const int g = i / Et, e = i % Et;
     int cnt = 0;
-    for (int a = 0; a < nr; ++a) {
-      const int j = st->run_list[a];
-      if (st->group_of[j] != g) continue;
-      cnt += (e < d.E) ? c.hist[j * d.E + e] : d.T;
-    }
+    for (int a = 0; a < nr; ++a)
+      if (st->group_of[st->run_list[a]] == g) cnt += count_of(a, e);
     my_nonempty += cnt > 0;
+    const int i1 = (cnt + rn1 - 1) / rn1 * mb1, i2 = (cnt + rn2 - 1) / rn2 * mb2;
     wk.seg_rows[i] = cnt;
-    wk.seg_items1[i] = (cnt + rn1 - 1) / rn1 * mb1;
-    wk.seg_items2[i] = (cnt + rn2 - 1) / rn2 * mb2;
+    wk.seg_items1[i] = i1;
+    wk.seg_items2[i] = i2;
     wk.seg_wid[i] = st->group_layer[g] * Et + e;
+    local.x += cnt;
+    local.y += i1;
+    local.z += i2;
   }
   if (my_nonempty) atomicAdd(&s_nonempty, my_nonempty);
-  __syncthreads();
-  const int rows = block_exclusive_scan(wk.seg_rows, nseg, pl.tmp);
-  const int it1 = block_exclusive_scan(wk.seg_items1, nseg, pl.tmp);
-  const int it2 = block_exclusive_scan(wk.seg_items2, nseg, pl.tmp);
+  // one block-wide exclusive scan of the three running sums
+  const int3 base = block_exclusive_scan3(local, pl.tmp3);
+  int3 acc3 = base;
+  for (int i = sb; i < se; ++i) {
+    const int a = wk.seg_rows[i], b = wk.seg_items1[i], cc = wk.seg_items2[i];
+    wk.seg_rows[i] = acc3.x;
+    wk.seg_items1[i] = acc3.y;
+    wk.seg_items2[i] = acc3.z;
+    acc3.x += a;
+    acc3.y += b;
+    acc3.z += cc;
+  }
+  const int rows = pl.tmp3[32].x, it1 = pl.tmp3[32].y, it2 = pl.tmp3[32].z;
   if (tid == 0) {
     wk.seg_rows[nseg] = rows;
     wk.seg_items1[nseg] = it1;
@@ -463,10 +492,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     const int a = i / Et, e = i % Et;
     const int j = st->run_list[a], g = st->group_of[j];
     int prior = 0;
-    for (int b = 0; b < a; ++b) {
-      const int jb = st->run_list[b];
-      if (st->group_of[jb] == g) prior += (e < d.E) ? c.hist[jb * d.E + e] : d.T;
-    }
+    for (int b = 0; b < a; ++b)
+      if (st->group_of[st->run_list[b]] == g) prior += count_of(b, e);
     wk.prior[j * Et + e] = prior;
   }
   __syncthreads();

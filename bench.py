@@ -83,6 +83,16 @@ def max_over_ranks(x: float, world: int) -> float:
     return float(t.item())
 
 
+def bench_config(wl, args, world: int) -> dict:
+    """The workload description both arms print (same keys and values)."""
+    return {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
+                        f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",
+            "policy": args.policy, "m": wl.m_default, "step": "one Algorithm-1 episode",
+            "tokens_per_step": wl.M * wl.T * wl.L,
+            "l2": "inputs larger than L2 (58 GB of expert weights streamed per episode)",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
 def job_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
     """Whole-job throughput: the units every rank processed over the slowest
     rank's time (replicas do equal work, so weak scaling)."""
@@ -357,12 +367,7 @@ def run_ours(args, world, rank, local):
             "data": ("synthetic (seeded routing skew: " + wl.profile + "; random-init weights "
                      + ("N(0, 1/(3 fan_in))" if wl.w_init == "fan_in" else f"N(0, {wl.w_std}^2)") + ")"),
             "workload_layers": wl.L,
-            "config": {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
-                                   f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",
-                       "policy": args.policy, "m": wl.m_default, "step": "one Algorithm-1 episode",
-                       "tokens_per_step": wl.M * wl.T * wl.L, "scheduler_steps": n_steps,
-                       "l2": "inputs larger than L2 (58 GB of expert weights streamed per episode)",
-                       "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+            "config": bench_config(wl, args, world), "scheduler_steps": n_steps,
             "e2e": e2e, "gpu_launches": int(launches), "roofline": roof,
             "cpu_baseline": cpu, "clocks": clk, "under_util": under, "kernels": kernels,
             "router_mode": router_mode,
@@ -481,8 +486,7 @@ def run_reference(args, world, rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(per_tl * wl.M * wl.T * wl.L * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": {"workload": wl.name, "policy": args.policy,
-                                            "m": wl.m_default},
+            "data": "synthetic", "config": bench_config(wl, args, 1),
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _blas_threads(),
                              "kind": "oracle", "sample": detail + " (host-drawn weights)"},
             "e2e": {"value": round(value, 2), "unit": UNIT, "h2d_bytes_per_step": 0,

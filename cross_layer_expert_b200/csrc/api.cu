@@ -141,7 +141,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   if (c.compute) {
     x.prior = (int32_t*)take(sizeof(int32_t) * M * d.Etot);
     x.pos = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
-    x.rowmap = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
+    x.rowslot = (int32_t*)take(sizeof(int32_t) * M * T * d.kk);
     x.seg_rows = (int32_t*)take(sizeof(int32_t) * (nseg + 1));
     x.seg_wid = (int32_t*)take(sizeof(int32_t) * nseg);
     x.seg_items1 = (int32_t*)take(sizeof(int32_t) * (nseg + 1));

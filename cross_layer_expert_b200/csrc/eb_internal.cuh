@@ -79,7 +79,7 @@ struct Work {
   int32_t* chunk_hist; // [M][NC][E]: counts of each 64-token chunk
   int32_t* prior;      // [M][Etot]: rows of (j's segment, expert) taken by earlier RunSet members
   int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
-  int32_t* rowmap;     // [Rcap]: token (j * T + t) of each permuted row
+  int32_t* rowslot;    // [Rcap]: slot (j * T + t) * kk + s of each permuted row
   int32_t* seg_rows;   // [M*Etot + 1]
   int32_t* seg_wid;    // [M*Etot]: layer * Etot + expert
   int32_t* seg_items1; // [M*Etot + 1]
@@ -88,7 +88,7 @@ struct Work {
   float* scores;       // [M][T][E]: router scores of the step (router mode)
   void* A;             // [Rcap][H] permuted tokens
   void* act;           // [Rcap][F] SwiGLU activations
-  void* y;             // [Rcap][H] expert outputs
+  void* y;             // [M*T*kk][H] expert outputs, at each row's (token, slot) position
   long long Rcap;
 };
 
@@ -166,8 +166,8 @@ cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int 
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
                          int32_t* w, int32_t* status, cudaStream_t s);
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
-// Rows of every (token, slot) of the RunSet (pos) and the token of every row
-// (rowmap).
+// Rows of every (token, slot) of the RunSet (pos) and the (token, slot) of
+// every row (rowslot).
 cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s);
 // The permuted copy A of the RunSet's token rows (after launch_positions).
 cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,

@@ -35,14 +35,17 @@ __device__ __forceinline__ int find_segment(const int32_t* items, int nseg, int 
 }
 
 // GATEUP: X = A [R][H], W = w_gateup, out = act [R][F] (SwiGLU epilogue).
-// DOWN:   X = act [R][F], W = w_down,  out = y [R][H].
+// DOWN:   X = act [R][F], W = w_down,  out = y [M*T*kk][H], row r stored at
+//         its (token, slot) position rowslot[r].
 template <typename T, bool GATEUP>
 __global__ void __launch_bounds__(256) k_gemm_simt(Dims d, const State* __restrict__ st,
                                                    const int32_t* __restrict__ seg_rows,
                                                    const int32_t* __restrict__ seg_wid,
                                                    const int32_t* __restrict__ seg_items,
                                                    const T* __restrict__ X,
-                                                   const T* __restrict__ W, T* __restrict__ out) {
+                                                   const T* __restrict__ W,
+                                                   const int32_t* __restrict__ rowslot,
+                                                   T* __restrict__ out) {
   pdl_enter();
   const int nseg = st->nseg;
   if (nseg == 0 || st->runset == 0) return;
@@ -107,7 +110,9 @@ __global__ void __launch_bounds__(256) k_gemm_simt(Dims d, const State* __restri
         if (f >= NOUT) continue;
         float v = accg[a][b];
         if (GATEUP) v = v / (1.f + expf(-v)) * accu[a][b];
-        from_f(v, out + (size_t)(r0 + r) * NOUT + f);
+        // GEMM 2 stores each row at its (token, slot) position
+        const size_t orow = GATEUP ? (size_t)(r0 + r) : (size_t)__ldg(rowslot + r0 + r);
+        from_f(v, out + orow * NOUT + f);
       }
     }
   }
@@ -121,11 +126,11 @@ cudaError_t run(const Dims& d, const CtxDev& c, const Work& w, const void* wgu, 
     return launch_pdl(k_gemm_simt<T, true>, dim3(grid), dim3(256), 0, s, 1, d, c.st,
                       (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
                       (const int32_t*)w.seg_items1, static_cast<const T*>(w.A),
-                      static_cast<const T*>(wgu), static_cast<T*>(w.act));
+                      static_cast<const T*>(wgu), (const int32_t*)w.rowslot, static_cast<T*>(w.act));
   return launch_pdl(k_gemm_simt<T, false>, dim3(grid), dim3(256), 0, s, 1, d, c.st,
                     (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
                     (const int32_t*)w.seg_items2, static_cast<const T*>(w.act),
-                    static_cast<const T*>(wdn), static_cast<T*>(w.y));
+                    static_cast<const T*>(wdn), (const int32_t*)w.rowslot, static_cast<T*>(w.y));
 }
 
 }  // namespace

@@ -236,7 +236,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-              __nv_bfloat16* __restrict__ out) {
+              const int32_t* __restrict__ rowslot, __nv_bfloat16* __restrict__ out) {
   pdl_enter();
   using C = Cfg<GATEUP>;
   constexpr int kBN = C::kBN;
@@ -426,10 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(a);
             }
           }
-        } else {
+        } else {  // y rows at their (token, slot) positions
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (cb + i < it.n) orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(g[i]);
+            if (cb + i < it.n)
+              out[(size_t)__ldg(rowslot + it.r0 + cb + i) * NOUT + (orow - out) % NOUT] =
+                  __float2bfloat16_rn(g[i]);
         }
       }
       tc_fence_before();
@@ -577,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tc2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
                const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-               __nv_bfloat16* __restrict__ out) {
+               const int32_t* __restrict__ rowslot, __nv_bfloat16* __restrict__ out) {
   pdl_enter();
   using C = Cfg2<GATEUP>;
   constexpr int kBN = C::kBN;
@@ -759,10 +761,12 @@ __global__ void __launch_bounds__(kThreads, 1)
               orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(a);
             }
           }
-        } else {
+        } else {  // y rows at their (token, slot) positions
 #pragma unroll
           for (int i = 0; i < 32; ++i)
-            if (cb + i < it.n) orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(g[i]);
+            if (cb + i < it.n)
+              out[(size_t)__ldg(rowslot + it.r0 + cb + i) * NOUT + (orow - out) % NOUT] =
+                  __float2bfloat16_rn(g[i]);
         }
       }
       tc_fence_before();
@@ -881,14 +885,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // next_item: the step's claim counter (zero before the launch).
 // GATHER (GEMM 1 only): the token rows are not read from a permuted copy;
 // kGatherWarps extra warps copy each chunk row straight from the hidden
-// states xsrc [M*T, H], through rowmap (permuted row -> token), into the
-// swizzled operand tile with 16-byte cp.async copies.
+// states xsrc [M*T, H], through rowslot (permuted row -> (token, slot)), into
+// the swizzled operand tile with 16-byte cp.async copies.  GEMM 2 stores each
+// output row at its (token, slot) position rowslot[row].
 template <bool GATEUP, bool GATHER>
 __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThreads, 1)
     k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-              int32_t* __restrict__ next_item, const int32_t* __restrict__ rowmap,
+              int32_t* __restrict__ next_item, const int32_t* __restrict__ rowslot,
               const __nv_bfloat16* __restrict__ xsrc, __nv_bfloat16* __restrict__ out) {
   pdl_enter();
   using C = CfgTM<GATEUP>;
@@ -1102,7 +1107,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
       const Item it = decode_tm<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
       const bool active = g < it.n;
       const char* src =
-          reinterpret_cast<const char*>(xsrc + (size_t)(active ? __ldg(rowmap + it.r0 + g) : 0) * d.H);
+          reinterpret_cast<const char*>(xsrc + (size_t)(active ? __ldg(rowslot + it.r0 + g) / d.kk : 0) * d.H);
       for (int kb = 0; kb < nk; ++kb) {
         int good = 1;
         if (lane == 0) good = mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status);
@@ -1158,7 +1163,9 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
       const int row = q * 32 + lane;  // token row within the item
       const bool live = row < it.n;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      __nv_bfloat16* orow = out + (size_t)(it.r0 + row) * NOUT + it.f0;
+      // GEMM 2 stores each row at its (token, slot) position
+      const int orow_idx = GATEUP ? it.r0 + row : (live ? __ldg(rowslot + it.r0 + row) : 0);
+      __nv_bfloat16* orow = out + (size_t)orow_idx * NOUT + it.f0;
       // a lane quarter past the chunk's last token has nothing to drain
       const int b_end = q * 32 < it.n ? kBlocks : 0;
       for (int b = cgrp; b < b_end; b += kGroups) {
@@ -1273,7 +1280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_gemm_tm2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
                Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
                const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-               __nv_bfloat16* __restrict__ out) {
+               const int32_t* __restrict__ rowslot, __nv_bfloat16* __restrict__ out) {
   pdl_enter();
   using C = CfgTM2<GATEUP>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -1469,7 +1476,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int fbase = wide ? 0 : (q >> 1) * (C::kFeat / 2);
       const int nblk = (wide ? C::kFeat : C::kFeat / 2) / 32;
       const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      __nv_bfloat16* orow = out + (size_t)(it.r0 + first + tok) * NOUT + it.f0 + fbase;
+      const int orow_idx =
+          GATEUP ? it.r0 + first + tok : (live ? __ldg(rowslot + it.r0 + first + tok) : 0);
+      __nv_bfloat16* orow = out + (size_t)orow_idx * NOUT + it.f0 + fbase;
       // a lane quarter whose tokens are all past the share has nothing to drain
       const int b_end = ((wide ? q * 32 : (q & 1) * 32) < cnt) ? nblk : 0;
       for (int b = cgrp; b < b_end; b += kGroups) {
@@ -1764,33 +1773,35 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
     cfg.dynamicSmemBytes = CfgTM2<true>::kSmemBytes;
     cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<true>, cfg, grid / 2));
     return cudaLaunchKernelEx(&cfg, k_gemm_tm2<true>, maps.w_gateup64, maps.A32, d, c.st, w.seg_rows,
-                              w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
+                              w.seg_wid, w.seg_items1, (const int32_t*)w.rowslot,
+                              static_cast<__nv_bfloat16*>(w.act));
   }
   cfg.dynamicSmemBytes = CfgTM2<false>::kSmemBytes;
   cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<false>, cfg, grid / 2));
   return cudaLaunchKernelEx(&cfg, k_gemm_tm2<false>, maps.w_down, maps.act32, d, c.st, w.seg_rows,
-                            w.seg_wid, w.seg_items2, static_cast<__nv_bfloat16*>(w.y));
+                            w.seg_wid, w.seg_items2, (const int32_t*)w.rowslot,
+                            static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                            int grid, cudaStream_t s, int which, const void* x_rows) {
   const bool gather = x_rows != nullptr;
-  const int32_t* rowmap = w.rowmap;
+  const int32_t* rowslot = w.rowslot;
   const __nv_bfloat16* none = nullptr;
   if (which == 1 && gather)
     return launch_pdl(k_gemm_tm<true, true>, dim3(grid), dim3(kThreads + 32 * kGatherWarps),
                       CfgTM<true>::kSmemBytes, s, 1, maps.w_gateup, maps.w_gateup, d, c.st,
                       (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
-                      (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
+                      (const int32_t*)w.seg_items1, w.gemm_next, rowslot,
                       static_cast<const __nv_bfloat16*>(x_rows), static_cast<__nv_bfloat16*>(w.act));
   if (which == 1)
     return launch_pdl(k_gemm_tm<true, false>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes,
                       s, 1, maps.w_gateup, maps.A32, d, c.st, (const int32_t*)w.seg_rows,
-                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowmap,
+                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowslot,
                       none, static_cast<__nv_bfloat16*>(w.act));
   return launch_pdl(k_gemm_tm<false, false>, dim3(grid), dim3(kThreads), CfgTM<false>::kSmemBytes,
                     s, 1, maps.w_down, maps.act32, d, c.st, (const int32_t*)w.seg_rows,
-                    (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowmap,
+                    (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowslot,
                     none, static_cast<__nv_bfloat16*>(w.y));
 }
 
@@ -1820,12 +1831,14 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
     cfg.dynamicSmemBytes = Cfg2<true>::kSmemBytes;
     cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<true>, cfg, grid / 2));
     return cudaLaunchKernelEx(&cfg, k_gemm_tc2<true>, maps.w_gateup, maps.A2, d, c.st, w.seg_rows,
-                              w.seg_wid, w.seg_items1, static_cast<__nv_bfloat16*>(w.act));
+                              w.seg_wid, w.seg_items1, (const int32_t*)w.rowslot,
+                              static_cast<__nv_bfloat16*>(w.act));
   }
   cfg.dynamicSmemBytes = Cfg2<false>::kSmemBytes;
   cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<false>, cfg, grid / 2));
   return cudaLaunchKernelEx(&cfg, k_gemm_tc2<false>, maps.w_down, maps.act2, d, c.st, w.seg_rows,
-                            w.seg_wid, w.seg_items2, static_cast<__nv_bfloat16*>(w.y));
+                            w.seg_wid, w.seg_items2, (const int32_t*)w.rowslot,
+                            static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -1834,11 +1847,11 @@ cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const 
     return launch_pdl(k_gemm_tc<true>, dim3(grid), dim3(kThreads), Cfg<true>::kSmemBytes, s, 1,
                       maps.w_gateup, maps.A, d, c.st, (const int32_t*)w.seg_rows,
                       (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1,
-                      static_cast<__nv_bfloat16*>(w.act));
+                      (const int32_t*)w.rowslot, static_cast<__nv_bfloat16*>(w.act));
   return launch_pdl(k_gemm_tc<false>, dim3(grid), dim3(kThreads), Cfg<false>::kSmemBytes, s, 1,
                     maps.w_down, maps.act, d, c.st, (const int32_t*)w.seg_rows,
                     (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2,
-                    static_cast<__nv_bfloat16*>(w.y));
+                    (const int32_t*)w.rowslot, static_cast<__nv_bfloat16*>(w.y));
 }
 
 }  // namespace eb

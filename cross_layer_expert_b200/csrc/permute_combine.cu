@@ -5,16 +5,18 @@
 // weighted sum of Eq. (1).  On one GPU the "dispatch" is a permutation of the
 // RunSet's token rows into contiguous segments, one per (layer, expert) --
 // micro-batches at the same layer share a segment --, and the "combine" is
-//   out[j,t] = (h[j,t] +) sum_{s<k} gate[j,t,s] * y[pos(j,t,s)]
-//              (+ sum over shared experts of y[pos(j,t,k+s')])
+//   out[j,t] = (h[j,t] +) sum_{s<k} gate[j,t,s] * y[j,t,s]
+//              (+ sum over shared experts of y[j,t,k+s'])
 // summed in slot order in fp32 and rounded once to the storage type.
 // [EB-read] §2.1: scheduling may change neither the expert set, the gates nor
 // the aggregation order -- the slot order here is fixed.
 //
 // The permutation is two launches: k_positions computes every (token, slot)
-// row of the RunSet and its inverse, the token of every row (a light pass
-// over the routing indices); k_permute_copy then moves the rows -- unless
-// GEMM 1 gathers them from the hidden states itself.  The copy and the combine are HBM-bound and
+// row of the RunSet and its inverse, the (token, slot) of every row (a light
+// pass over the routing indices); k_permute_copy then moves the rows --
+// unless GEMM 1 gathers them from the hidden states itself.  GEMM 2 writes
+// each row's output at its (token, slot) position, so the combine reads a
+// token's k + n_shared outputs from one contiguous run.  The copy and the combine are HBM-bound and
 // persistent: a grid of resident CTAs sized to the SM count strides over the
 // RunSet's tokens, one warp per token row with 16-byte vector loads and
 // stores, so the work spreads evenly over the SMs whatever the RunSet size
@@ -45,7 +47,7 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
                                                             const int32_t* __restrict__ seg_rows,
                                                             const int32_t* __restrict__ prior,
                                                             int32_t* __restrict__ pos,
-                                                            int32_t* __restrict__ rowmap) {
+                                                            int32_t* __restrict__ rowslot) {
   pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
   if (!((st->runset >> j) & 1u)) return;
@@ -100,14 +102,14 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
     if (e >= 0) {
       const int row = bj[e] + cnt[warp][e] + rank;
       pos_c[(p / k) * kk + p % k] = row;
-      rowmap[row] = j * d.T + t0 + p / k;
+      rowslot[row] = (j * d.T + t0 + p / k) * kk + p % k;
     }
     __syncthreads();
   }
   for (int i = tid; i < nt * d.n_shared; i += kPermThreads) {
     const int t = i / d.n_shared, s = i % d.n_shared;
     pos_c[t * kk + k + s] = bj[E + s] + t;
-    rowmap[bj[E + s] + t] = j * d.T + t0 + t;
+    rowslot[bj[E + s] + t] = (j * d.T + t0 + t) * kk + k + s;
   }
 }
 
@@ -252,8 +254,9 @@ __global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, const St
   const int nvec = d.H / VE;
   for (int u = wid; u < units; u += W) {
     const size_t tok = runset_token(st, d.T, u);
-    // slot rows and gates, one per lane
-    const int my_row = lane < kk ? __ldg(pos + tok * kk + lane) : 0;
+    // the token's expert outputs sit at its slots (tok * kk + s); gates, one
+    // per lane
+    const int my_row = lane < kk ? (int)(tok * kk + lane) : 0;
     const float my_gate = lane < k ? __ldg(gate + tok * k + lane) : 0.f;
     T* out = hidden + tok * d.H;
     // two 16-byte vectors per lane per pass, slots loaded four at a time
@@ -333,7 +336,7 @@ int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb
 cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s) {
   return launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPermThreads), 0, s, 1, d, c.st,
                     (const int32_t*)w.idx, (const int32_t*)w.chunk_hist,
-                    (const int32_t*)w.seg_rows, (const int32_t*)w.prior, w.pos, w.rowmap);
+                    (const int32_t*)w.seg_rows, (const int32_t*)w.prior, w.pos, w.rowslot);
 }
 
 cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,

@@ -81,7 +81,7 @@ typedef int eb_status;
 #define EB_GEMM_TM2 5
 #define EB_GEMM_TMG 6
 
-/* Limits of this build. */
+/* Compile-time limits of the library. */
 #define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */
 #define EB_MAX_D 64   /* virtual ranks                                   */
 #define EB_MAX_ETOT 256 /* routed + shared experts per layer            */

@@ -33,7 +33,7 @@ struct eb_ctx {
   cudaEvent_t events[8] = {};
   // cached TMA maps (rebuilt when a pointer changes)
   TcMaps maps;
-  const void* map_keys[4] = {nullptr, nullptr, nullptr, nullptr};
+  const void* map_keys[3] = {nullptr, nullptr, nullptr};
   // kernel launches enqueued since create, and optional per-kernel event timing
   long long launches = 0;
   bool prof = false;

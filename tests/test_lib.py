@@ -89,3 +89,17 @@ def test_stage_argument_errors_return_before_launch(lib):
     assert lib.eb_schedule(None, 0xF, 4, 2, 2, 0, P, None, None) == eb.EB_ERR_INVALID_ARG
     assert lib.eb_destroy(None) == eb.EB_ERR_INVALID_ARG
     assert lib.eb_reset(None, None) == eb.EB_ERR_INVALID_ARG
+    # placement: a map is required; E need not be a multiple of D
+    assert lib.eb_loads_mapped(P, 4, 10, 3, None, P, None, None) == eb.EB_ERR_INVALID_ARG
+    assert lib.eb_loads_mapped(None, 4, 10, 3, P, P, None, None) == eb.EB_ERR_INVALID_ARG
+    assert lib.eb_loads_mapped(P, 0, 10, 3, P, P, None, None) == eb.EB_OK  # nothing to do
+    assert lib.eb_set_expert_map(None, None) == eb.EB_ERR_INVALID_ARG
+    # router projection: E a multiple of 16 (<= 256), H a multiple of 64,
+    # 16-byte aligned pointers; n = 0 is a no-op
+    assert lib.eb_router(P, 8, 2048, P, 12, P, None, None) == eb.EB_ERR_UNSUPPORTED
+    assert lib.eb_router(P, 8, 2048, P, 512, P, None, None) == eb.EB_ERR_UNSUPPORTED
+    assert lib.eb_router(P, 8, 100, P, 128, P, None, None) == eb.EB_ERR_UNSUPPORTED
+    assert lib.eb_router(ctypes.c_void_p(8), 8, 2048, P, 128, P, None, None) == eb.EB_ERR_INVALID_ARG
+    assert lib.eb_router(None, 8, 2048, P, 128, P, None, None) == eb.EB_ERR_INVALID_ARG
+    assert lib.eb_router(None, 0, 2048, None, 128, None, None, None) == eb.EB_OK
+    assert lib.eb_set_router(None, P, None) == eb.EB_ERR_INVALID_ARG

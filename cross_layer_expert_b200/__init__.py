@@ -29,14 +29,14 @@ EB_ERR_TOO_LARGE = -7
 
 CUMUTIL, MAXUTIL, LOCKSTEP, DIFFPEAK = 0, 1, 2, 3
 DTYPE_F32, DTYPE_BF16 = 0, 1
-GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TC2, GEMM_TM, GEMM_TM2, GEMM_TMG = 0, 1, 2, 3, 4, 5, 6
+GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TC2, GEMM_TM, GEMM_TM2, GEMM_TMG, GEMM_TMC = range(8)
 
 EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_create", "eb_destroy",
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
             "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped", "eb_set_router",
-            "eb_router"]
+            "eb_router", "eb_engines"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine",
                 "positions", "router")
@@ -90,6 +90,7 @@ def load() -> ctypes.CDLL:
         "eb_profile": (I, [P, I]),
         "eb_profile_read": (I, [P, P, P]),
         "eb_launch_count": (I, [P, ctypes.POINTER(ctypes.c_int64)]),
+        "eb_engines": (I, [P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
         "eb_route_loads_static": (I, [P, I, I, I, I, I, I, P, P, P, P, P]),
         "eb_selftest_timeout": (I, [ctypes.c_int64, P, P]),
     }
@@ -295,3 +296,10 @@ class Context:
         n = ctypes.c_int64(0)
         _check(load().eb_launch_count(self.handle, ctypes.byref(n)), "eb_launch_count")
         return n.value
+
+    def eb_engines(self):
+        """(GEMM 1 engine, GEMM 2 engine) as GEMM_* values, after AUTO and the
+        shape fallbacks are resolved."""
+        g1, g2 = ctypes.c_int(0), ctypes.c_int(0)
+        _check(load().eb_engines(self.handle, ctypes.byref(g1), ctypes.byref(g2)), "eb_engines")
+        return g1.value, g2.value

@@ -54,8 +54,7 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool use_tc_for(const eb_config& c) {
   if (c.dtype != EB_DTYPE_BF16) return false;
-  return c.gemm == EB_GEMM_AUTO || c.gemm == EB_GEMM_TC || c.gemm == EB_GEMM_TC2 ||
-         c.gemm == EB_GEMM_TM || c.gemm == EB_GEMM_TM2 || c.gemm == EB_GEMM_TMG;
+  return c.gemm != EB_GEMM_SIMT;
 }
 
 // Engine of each GEMM.  AUTO takes the one-SM token-major engine for every
@@ -75,10 +74,13 @@ void choose_engines(const eb_config& c, bool use_tc, int num_sms, int* g1, int* 
       case EB_GEMM_TM: return nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
       case EB_GEMM_TMG: return which == 1 && nout % kTmFeat1 == 0;
       case EB_GEMM_TM2: return pair_ok && nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
+      case EB_GEMM_TMC: return which == 2 && nout % kTmFeat2 == 0;
       default: return false;
     }
   };
-  *g1 = fits(want, 1) ? want : EB_GEMM_TC;
+  // TMC fuses the combine into GEMM 2; its GEMM 1 is the token-major one
+  const int want1 = want == EB_GEMM_TMC ? EB_GEMM_TM : want;
+  *g1 = fits(want1, 1) ? want1 : EB_GEMM_TC;
   // TMG gathers GEMM 1's input; its GEMM 2 is the token-major one
   const int want2 = want == EB_GEMM_TMG ? EB_GEMM_TM : want;
   *g2 = fits(want2, 2) ? want2 : EB_GEMM_TC;
@@ -97,6 +99,7 @@ void engine_tiles(int eng, int which, int* rows, int* feats) {
       return;
     case EB_GEMM_TM:
     case EB_GEMM_TMG:
+    case EB_GEMM_TMC:
       *rows = kTmRows;
       *feats = which == 1 ? kTmFeat1 : kTmFeat2;
       return;
@@ -216,7 +219,7 @@ eb_status eb_config_check(const eb_config* c) {
   if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
   if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
   if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
-  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TMG) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TMC) return EB_ERR_INVALID_ARG;
   if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
@@ -228,8 +231,7 @@ eb_status eb_config_check(const eb_config* c) {
     const int vec = c->dtype == EB_DTYPE_BF16 ? 8 : 4;  // 16-byte rows
     if (c->H % vec != 0) return EB_ERR_UNSUPPORTED;
     if ((long long)c->M * c->T * (c->k + c->n_shared) > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
-    const bool forced_tc = c->gemm == EB_GEMM_TC || c->gemm == EB_GEMM_TC2 ||
-                           c->gemm == EB_GEMM_TM || c->gemm == EB_GEMM_TM2 || c->gemm == EB_GEMM_TMG;
+    const bool forced_tc = c->gemm != EB_GEMM_AUTO && c->gemm != EB_GEMM_SIMT;
     if (c->dtype == EB_DTYPE_F32 && forced_tc) return EB_ERR_UNSUPPORTED;
     if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
       if (forced_tc) return EB_ERR_UNSUPPORTED;
@@ -266,9 +268,13 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   const size_t n_trace = align_up(sizeof(long long) * kTraceCols * x->d.max_steps);
   const size_t n_tl = align_up(sizeof(int32_t) * c->M * (size_t)x->d.max_steps);
   const size_t n_map = align_up(sizeof(int32_t) * c->E);
+  // arrival counters of the fused combine, one per (token, 256-feature block)
+  const size_t n_arrive =
+      x->eng2 == EB_GEMM_TMC ? align_up(sizeof(int32_t) * (size_t)c->M * c->T * (c->H / kTmFeat2)) : 0;
+  const size_t n_all = n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive;
   char* p = nullptr;
-  if (e == cudaSuccess) e = cudaMalloc(&p, n_state + n_hist + n_w + n_trace + n_tl + n_map);
-  if (e == cudaSuccess) e = cudaMemset(p, 0, n_state + n_hist + n_w + n_trace + n_tl + n_map);
+  if (e == cudaSuccess) e = cudaMalloc(&p, n_all);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, n_all);
   if (e == cudaSuccess) {
     x->dev_alloc = p;
     x->dev.st = (State*)p;
@@ -278,6 +284,8 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->dev.trace_layers = (int32_t*)(p + n_state + n_hist + n_w + n_trace);
     x->dev.emap = (int32_t*)(p + n_state + n_hist + n_w + n_trace + n_tl);
     x->dev.use_emap = 0;
+    x->dev.arrive = n_arrive ? (int32_t*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map) : nullptr;
+    x->dev.arrive_bytes = n_arrive;
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
   for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
@@ -314,7 +322,12 @@ eb_status eb_reset(eb_ctx* x, void* stream) {
   cudaStream_t s = (cudaStream_t)stream;
   x->last_stream = s;
   x->launches += 1;
-  return cuda_status(launch_reset(x->d, x->dev, s));
+  cudaError_t e = launch_reset(x->d, x->dev, s);
+  // the fused combine leaves its counters at zero; a step that gave up on a
+  // bounded wait may not have, so a reset clears them
+  if (e == cudaSuccess && x->dev.arrive)
+    e = cudaMemsetAsync(x->dev.arrive, 0, x->dev.arrive_bytes, s);
+  return cuda_status(e);
 }
 
 eb_status eb_set_expert_map(eb_ctx* x, const int32_t* expert_rank) {
@@ -354,10 +367,14 @@ static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* 
   switch (eng) {
     case EB_GEMM_TC: return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     case EB_GEMM_TC2: return launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
-    case EB_GEMM_TM: return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr);
+    case EB_GEMM_TM:
+      return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr, nullptr);
     case EB_GEMM_TMG:
       return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which,
-                            which == 1 ? hidden : nullptr);
+                            which == 1 ? hidden : nullptr, nullptr);
+    case EB_GEMM_TMC:  // GEMM 2 only (GEMM 1 of TMC is TM)
+      return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr,
+                            const_cast<void*>(hidden));
     case EB_GEMM_TM2: return launch_gemm_tm2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     default: return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, which);
   }
@@ -433,7 +450,8 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
       if (e == cudaSuccess)
         e = timed(x, 4, 1, s, [&] { return launch_engine(x, g2, w, wgu, wdn, hidden, s, 2); });
     }
-    if (e == cudaSuccess)
+    // the fused engine combines inside GEMM 2
+    if (e == cudaSuccess && g2 != EB_GEMM_TMC)
       e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });
   }
   return cuda_status(e);
@@ -554,6 +572,13 @@ eb_status eb_profile_read(eb_ctx* x, double* ms, int64_t* launches) {
 eb_status eb_launch_count(eb_ctx* x, int64_t* n) {
   if (!x || !n) return EB_ERR_INVALID_ARG;
   *n = x->launches;
+  return EB_OK;
+}
+
+eb_status eb_engines(const eb_ctx* x, int* gemm1, int* gemm2) {
+  if (!x || !gemm1 || !gemm2) return EB_ERR_INVALID_ARG;
+  *gemm1 = x->eng1;
+  *gemm2 = x->eng2;
   return EB_OK;
 }
 

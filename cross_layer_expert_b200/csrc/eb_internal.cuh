@@ -101,6 +101,8 @@ struct CtxDev {
   int32_t* trace_layers;  // [max_steps][M]
   int32_t* emap;        // [E]: rank of each expert (a custom placement)
   int use_emap;         // 0: contiguous map, experts [d E/D, (d+1) E/D) on rank d
+  int32_t* arrive;      // [M*T][H/256]: fused-combine arrival counts (engine TMC), else null
+  size_t arrive_bytes;
 };
 
 // ---- programmatic dependent launch ----

@@ -880,6 +880,62 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// One token's combine over 256 features, by one warp (lane: features
+// f + 8 lane .. + 7): h (if residual) + sum over slots s of gate_s y_s (shared
+// slots s >= k with weight 1), in slot order, rounded once to bf16 into
+// hidden.  The same arithmetic, element for element, as the stand-alone
+// combine kernel, so the fused and unfused steps agree bit for bit.  The
+// token's y rows were stored by other CTAs of this launch: they are read
+// through L2 (ld.global.cg), after the acquiring fence of the caller.
+__device__ __forceinline__ void combine_token(const Dims& d, int tok, int f, int lane,
+                                              const float* __restrict__ gate,
+                                              const __nv_bfloat16* y, __nv_bfloat16* hidden) {
+  const int k = d.k, kk = d.kk;
+  const float my_gate = lane < k ? __ldg(gate + (size_t)tok * k + lane) : 0.f;
+  uint4* hp = reinterpret_cast<uint4*>(hidden + (size_t)tok * d.H + f + 8 * lane);
+  float acc[8];
+  if (d.residual) {
+    const uint4 h = __ldcg(hp);
+    const __nv_bfloat162* hb = reinterpret_cast<const __nv_bfloat162*>(&h);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 v = __bfloat1622float2(hb[i]);
+      acc[2 * i] = v.x;
+      acc[2 * i + 1] = v.y;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  }
+  const __nv_bfloat16* yt = y + (size_t)tok * kk * d.H + f + 8 * lane;
+  for (int s0 = 0; s0 < kk; s0 += 4) {
+    uint4 r[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (s0 + q < kk) r[q] = __ldcg(reinterpret_cast<const uint4*>(yt + (size_t)(s0 + q) * d.H));
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int s = s0 + q;
+      const float g = __shfl_sync(0xffffffffu, my_gate, s & 31);
+      if (s >= kk) break;
+      const __nv_bfloat162* yb = reinterpret_cast<const __nv_bfloat162*>(&r[q]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 v = __bfloat1622float2(yb[i]);
+        if (s < k) {
+          acc[2 * i] = fmaf(g, v.x, acc[2 * i]);
+          acc[2 * i + 1] = fmaf(g, v.y, acc[2 * i + 1]);
+        } else {
+          acc[2 * i] += v.x;
+          acc[2 * i + 1] += v.y;
+        }
+      }
+    }
+  }
+  *hp = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                   pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+}
+
 // map_x: token rows [Rcap, K] in boxes of 32 rows; map_w: weights in boxes
 // of 128 rows.  GATEUP: out = act [Rcap, F]; else out = y [Rcap, H].
 // next_item: the step's claim counter (zero before the launch).
@@ -888,13 +944,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // states xsrc [M*T, H], through rowslot (permuted row -> (token, slot)), into
 // the swizzled operand tile with 16-byte cp.async copies.  GEMM 2 stores each
 // output row at its (token, slot) position rowslot[row].
-template <bool GATEUP, bool GATHER>
+// COMBINE (GEMM 2 only): the combine runs in the drain.  Each drain thread
+// that has stored its share of a row of y counts it in arrive[token][feature
+// block] (after a fence); the thread that brings the count to kk * kGroups
+// (every slot of the token, every column group) resets it to zero and its
+// warp combines the token's 256 features of that block into hidden.
+// Nothing waits: a token is combined by whichever drain finishes it last.
+template <bool GATEUP, bool GATHER, bool COMBINE>
 __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThreads, 1)
     k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
               int32_t* __restrict__ next_item, const int32_t* __restrict__ rowslot,
-              const __nv_bfloat16* __restrict__ xsrc, __nv_bfloat16* __restrict__ out) {
+              const __nv_bfloat16* __restrict__ xsrc, __nv_bfloat16* out,
+              int32_t* __restrict__ arrive, const float* __restrict__ gate,
+              __nv_bfloat16* hidden) {
+  static_assert(!COMBINE || (!GATEUP && !GATHER), "the combine follows GEMM 2");
   pdl_enter();
   using C = CfgTM<GATEUP>;
   constexpr int Q = C::kQueue;
@@ -1198,6 +1263,29 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
       if (++acc == C::kAccBufs) {
         acc = 0;
         acc_phase ^= 1;
+      }
+      if constexpr (COMBINE) {
+        // the accumulator is released; count this thread's stored share
+        int tok = 0;
+        bool last = false;
+        if (live) {
+          tok = orow_idx / d.kk;
+          int32_t* cnt = arrive + (size_t)tok * (d.H / C::kFeat) + it.f0 / C::kFeat;
+          __threadfence();  // the stores of y above before the count
+          last = atomicAdd(cnt, 1) == d.kk * kGroups - 1;
+          if (last) *cnt = 0;  // no other arrival on it in this launch
+        }
+        unsigned lm = __ballot_sync(0xffffffffu, last);
+        if (lm) {
+          __syncwarp();
+          __threadfence();  // every counted share before the reads of y
+          while (lm) {
+            const int src = __ffs(lm) - 1;
+            lm &= lm - 1;
+            const int t = __shfl_sync(0xffffffffu, tok, src);
+            combine_token(d, t, it.f0, lane, gate, out, hidden);
+          }
+        }
       }
     }
   }
@@ -1735,13 +1823,16 @@ cudaError_t gemm_tc_prepare() {
     e = cudaFuncSetAttribute(k_gemm_tc2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg2<false>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemm_tm<true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<true>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemm_tm<true, true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<true>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    e = cudaFuncSetAttribute(k_gemm_tm<false, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             CfgTM<false>::kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(k_gemm_tm<false, false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<false>::kSmemBytes);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1784,25 +1875,38 @@ cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const
 }
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                           int grid, cudaStream_t s, int which, const void* x_rows) {
+                           int grid, cudaStream_t s, int which, const void* x_rows, void* combine_into) {
   const bool gather = x_rows != nullptr;
   const int32_t* rowslot = w.rowslot;
   const __nv_bfloat16* none = nullptr;
+  int32_t* no_count = nullptr;
+  const float* no_gate = nullptr;
+  __nv_bfloat16* no_hidden = nullptr;
   if (which == 1 && gather)
-    return launch_pdl(k_gemm_tm<true, true>, dim3(grid), dim3(kThreads + 32 * kGatherWarps),
+    return launch_pdl(k_gemm_tm<true, true, false>, dim3(grid), dim3(kThreads + 32 * kGatherWarps),
                       CfgTM<true>::kSmemBytes, s, 1, maps.w_gateup, maps.w_gateup, d, c.st,
                       (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
                       (const int32_t*)w.seg_items1, w.gemm_next, rowslot,
-                      static_cast<const __nv_bfloat16*>(x_rows), static_cast<__nv_bfloat16*>(w.act));
+                      static_cast<const __nv_bfloat16*>(x_rows), static_cast<__nv_bfloat16*>(w.act),
+                      no_count, no_gate, no_hidden);
   if (which == 1)
-    return launch_pdl(k_gemm_tm<true, false>, dim3(grid), dim3(kThreads), CfgTM<true>::kSmemBytes,
-                      s, 1, maps.w_gateup, maps.A32, d, c.st, (const int32_t*)w.seg_rows,
-                      (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items1, w.gemm_next, rowslot,
-                      none, static_cast<__nv_bfloat16*>(w.act));
-  return launch_pdl(k_gemm_tm<false, false>, dim3(grid), dim3(kThreads), CfgTM<false>::kSmemBytes,
-                    s, 1, maps.w_down, maps.act32, d, c.st, (const int32_t*)w.seg_rows,
-                    (const int32_t*)w.seg_wid, (const int32_t*)w.seg_items2, w.gemm_next + 1, rowslot,
-                    none, static_cast<__nv_bfloat16*>(w.y));
+    return launch_pdl(k_gemm_tm<true, false, false>, dim3(grid), dim3(kThreads),
+                      CfgTM<true>::kSmemBytes, s, 1, maps.w_gateup, maps.A32, d, c.st,
+                      (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                      (const int32_t*)w.seg_items1, w.gemm_next, rowslot, none,
+                      static_cast<__nv_bfloat16*>(w.act), no_count, no_gate, no_hidden);
+  if (combine_into)
+    return launch_pdl(k_gemm_tm<false, false, true>, dim3(grid), dim3(kThreads),
+                      CfgTM<false>::kSmemBytes, s, 1, maps.w_down, maps.act32, d, c.st,
+                      (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                      (const int32_t*)w.seg_items2, w.gemm_next + 1, rowslot, none,
+                      static_cast<__nv_bfloat16*>(w.y), c.arrive, (const float*)w.gate,
+                      static_cast<__nv_bfloat16*>(combine_into));
+  return launch_pdl(k_gemm_tm<false, false, false>, dim3(grid), dim3(kThreads),
+                    CfgTM<false>::kSmemBytes, s, 1, maps.w_down, maps.act32, d, c.st,
+                    (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
+                    (const int32_t*)w.seg_items2, w.gemm_next + 1, rowslot, none,
+                    static_cast<__nv_bfloat16*>(w.y), no_count, no_gate, no_hidden);
 }
 
 cudaError_t launch_router(const CUtensorMap& map_h, const CUtensorMap& map_r, int T, int H, int E,

@@ -37,8 +37,13 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
 // x_rows (GEMM 1 only, may be null): the hidden states [M*T, H]; when given,
 // token rows are gathered from them through the row map instead of being
 // read from the permuted copy.
+// combine_into (GEMM 2 only, may be null): the hidden states [M*T, H]; when
+// given, GEMM 2 also combines every RunSet token into them (the step needs no
+// combine kernel) using the arrival counters c.arrive, which must be zero
+// before the launch and are zero again after it.
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                           int grid, cudaStream_t s, int which, const void* x_rows);
+                           int grid, cudaStream_t s, int which, const void* x_rows,
+                           void* combine_into);
 // Two-SM token-major engine (cta_group::2): a CTA pair computes a chunk of up
 // to 256 tokens against 256 weight rows; each CTA holds half the tokens and
 // half the weight rows (M = 256 MMAs above 128 tokens, M = 128 below).

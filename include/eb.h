@@ -68,11 +68,17 @@ typedef int eb_status;
  *         dynamically, so CTAs finish together whatever the segment sizes.
  *   TM2   token-major over an SM pair (cta_group::2): 256 tokens x 256 weight
  *         rows per MMA, each SM holding 128 tokens and half the weight rows.
- *   TMG   as TM, but GEMM 1 reads its token rows straight from `hidden` with
- *         TMA gather4 (four rows per copy) instead of from a permuted copy,
- *         which is then not written.
- * TM and TM2 need F a multiple of 128 (gate/up) and H a multiple of 256
- * (down); a GEMM they do not fit runs on TC. */
+ *   TMG   as TM, but GEMM 1 reads its token rows straight from `hidden`
+ *         (extra warps copy each row into the operand tile with 16-byte
+ *         cp.async) instead of from a permuted copy, which is then not
+ *         written.
+ *   TMC   as TM, with the combine fused into GEMM 2: each token is combined
+ *         into `hidden` by the GEMM 2 drain that stores its last expert
+ *         output row, and the step launches no combine kernel.  Bit-identical
+ *         to TM.  The context then holds M*T*H/256 int32 arrival counters.
+ * TM, TM2 and TMC need F a multiple of 128 (gate/up) and H a multiple of 256
+ * (down); a GEMM they do not fit runs on TC (and TMC's step then runs the
+ * combine kernel). */
 #define EB_GEMM_AUTO 0
 #define EB_GEMM_TC 1
 #define EB_GEMM_SIMT 2
@@ -80,6 +86,7 @@ typedef int eb_status;
 #define EB_GEMM_TM 4
 #define EB_GEMM_TM2 5
 #define EB_GEMM_TMG 6
+#define EB_GEMM_TMC 7
 
 /* Compile-time limits of the library. */
 #define EB_MAX_M 32   /* micro-batches (RunSets are 32-bit masks)        */
@@ -225,11 +232,16 @@ eb_status eb_trace(eb_ctx* ctx, int64_t* rows, int32_t* layers, int max_steps, i
  * copy), GEMM 1 (gate/up + SwiGLU), GEMM 2 (down), combine, positions (the
  * rows of every token slot), router projection (router mode).
  * eb_launch_count returns the kernels the context has enqueued since
- * eb_create. */
+ * eb_create.  eb_engines returns the EB_GEMM_* engine that runs GEMM 1 and
+ * GEMM 2 (after AUTO and the shape fallbacks above are resolved; SIMT for
+ * f32); with EB_GEMM_TMC as GEMM 2 the step launches no combine kernel and
+ * the combine's time is in GEMM 2's.  Host only: EB_ERR_INVALID_ARG for a
+ * null argument. */
 #define EB_PROF_KERNELS 8
 eb_status eb_profile(eb_ctx* ctx, int enable);
 eb_status eb_profile_read(eb_ctx* ctx, double* ms, int64_t* launches);
 eb_status eb_launch_count(eb_ctx* ctx, int64_t* n);
+eb_status eb_engines(const eb_ctx* ctx, int* gemm1, int* gemm2);
 
 /* Failure-detection self-test (the pages describe no failure handling).  Every
  * device-side wait of the tensor-core GEMMs is bounded; when one expires the

@@ -1,7 +1,8 @@
 """Degenerate and boundary cases of the step against the oracle: one token,
 one micro-batch, one rank (u = 1), every expert per token (k = E), one
 expert per rank (D = E), m = M (MaxUtil reduces to lock-step), and a ragged
-token count -- on the default tensor-core engine and on SIMT."""
+token count -- on the default tensor-core engine, on SIMT and with the
+combine fused into GEMM 2."""
 import numpy as np
 import pytest
 
@@ -33,7 +34,7 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("gemm", [0, 2])
+@pytest.mark.parametrize("gemm", [0, 2, 7])
 @pytest.mark.parametrize("case", sorted(CASES))
 def test_edge_case_episode_matches_oracle(torch, case, gemm):
     wl = synth.get("small_bf16", L=3, **CASES[case])

@@ -164,15 +164,16 @@ def small_expected(small_inputs):
 
 @pytest.mark.parametrize("name", SMALL)
 @pytest.mark.parametrize("policy", [0, 1, 2, 3])
-@pytest.mark.parametrize("gemm", [0, 1, 2, 3, 5, 6])
+@pytest.mark.parametrize("gemm", [0, 1, 2, 3, 5, 6, 7])
 def test_small_episode_matches_oracle(small_inputs, small_expected, name, policy, gemm):
     """gemm 0: default engine (one-SM token-major tensor-core engine for bf16,
     SIMT for fp32); 1: one-SM weight-major; 2: SIMT; 3: two-SM weight-major;
     5: two-SM token-major; 6: token-major with GEMM 1 gathering its rows
-    from the hidden states (the tensor-core engines take bf16 only)."""
+    from the hidden states; 7: token-major with the combine fused into GEMM 2
+    (the tensor-core engines take bf16 only)."""
     inp = small_inputs[name]
     wl = inp.wl
-    if wl.dtype == "f32" and gemm in (1, 3, 5, 6):
+    if wl.dtype == "f32" and gemm in (1, 3, 5, 6, 7):
         pytest.skip("the tensor-core engines take bf16 operands")
     if gemm == 3 and (wl.H % 256 or wl.F % 256):
         pytest.skip("the two-SM weight-major engine needs H and F multiples of 256")
@@ -191,6 +192,29 @@ def test_scheduled_equals_lockstep_bitwise(small_inputs, name):
     for policy in (0, 1, 3):
         h = run_episode(inp, policy)[0].cpu()
         assert torch.equal(h.view(torch.int16), lock.view(torch.int16)), policy
+
+
+@pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16"])
+@pytest.mark.parametrize("policy", [0, 1])
+def test_fused_combine_bitwise_equals_unfused(small_inputs, name, policy):
+    """The combine fused into GEMM 2 (engine 7) does the stand-alone combine's
+    arithmetic in the same slot order, so whole episodes agree bit for bit
+    with the token-major engine (4).  Two episodes on one context agree too:
+    the arrival counters are back at zero after every step."""
+    import torch
+    import cross_layer_expert_b200 as eb
+    from _common import lib_config
+    inp = small_inputs[name]
+    ref = run_episode(inp, policy, gemm=4)[0].cpu()
+    ctx = eb.Context(lib_config(inp.wl, policy, gemm=7))
+    try:
+        for rep in range(2):
+            hidden = inp.h0.clone()
+            ctx.eb_episode(inp.logits, hidden, inp.w_gateup, inp.w_down)
+            assert ctx.eb_sync_status() == eb.EB_OK
+            assert torch.equal(hidden.cpu().view(torch.int16), ref.view(torch.int16)), rep
+    finally:
+        ctx.close()
 
 
 @pytest.mark.parametrize("m", [1, 2, 4])

@@ -49,17 +49,20 @@ def _cfg(**kw):
 def test_config_check(lib):
     assert eb.eb_config_check(_cfg()) == eb.EB_OK
     bad = [dict(E=15), dict(k=17), dict(m=5), dict(m=0), dict(T=0), dict(L=0), dict(M=0),
-           dict(policy=7), dict(dtype=5), dict(D=0), dict(n_shared=-1), dict(gemm=7), dict(gemm=-1)]
+           dict(policy=7), dict(dtype=5), dict(D=0), dict(n_shared=-1), dict(gemm=8), dict(gemm=-1)]
     for b in bad:
         assert eb.eb_config_check(_cfg(**b)) == eb.EB_ERR_INVALID_ARG, b
     unsup = [dict(M=33, m=3), dict(D=64, E=128 * 3), dict(k=20, n_shared=13, E=64),
              dict(H=130), dict(gemm=eb.GEMM_TC), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TC, H=192),
              dict(gemm=eb.GEMM_TM), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TM, F=192),
              dict(gemm=eb.GEMM_TM2), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TM2, H=192),
+             dict(gemm=eb.GEMM_TMC), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TMC, H=192),
              dict(M=32, m=8, policy=eb.MAXUTIL)]
     for u in unsup:
         assert eb.eb_config_check(_cfg(**u)) == eb.EB_ERR_UNSUPPORTED, u
     assert eb.eb_config_check(_cfg(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TM)) == eb.EB_OK
+    # H = 384 is not a multiple of 256: TMC's GEMM 2 then runs weight-major
+    assert eb.eb_config_check(_cfg(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TMC, H=384)) == eb.EB_OK
     # routing-only configs need no hidden / FFN sizes
     assert eb.eb_config_check(_cfg(compute=0, H=0, F=0)) == eb.EB_OK
     # MaxUtil at M = 32 with m = 24 enumerates ~15M complements: supported
@@ -88,6 +91,8 @@ def test_stage_argument_errors_return_before_launch(lib):
     assert lib.eb_schedule(P, 0xF, 4, 2, 2, 9, P, None, None) == eb.EB_ERR_INVALID_ARG
     assert lib.eb_schedule(None, 0xF, 4, 2, 2, 0, P, None, None) == eb.EB_ERR_INVALID_ARG
     assert lib.eb_destroy(None) == eb.EB_ERR_INVALID_ARG
+    g1, g2 = ctypes.c_int(-1), ctypes.c_int(-1)
+    assert lib.eb_engines(None, ctypes.byref(g1), ctypes.byref(g2)) == eb.EB_ERR_INVALID_ARG
     assert lib.eb_reset(None, None) == eb.EB_ERR_INVALID_ARG
     # placement: a map is required; E need not be a multiple of D
     assert lib.eb_loads_mapped(P, 4, 10, 3, None, P, None, None) == eb.EB_ERR_INVALID_ARG

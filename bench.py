@@ -8,6 +8,7 @@ loads, the RunSet choice, permutation, the two grouped expert GEMMs and the
 combine.  Throughput counts token-layer passes: M * T * L per episode.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --sweep [--impl reference]   # routing + scheduling sweep, D x M
 
 N > 1 (launched with torchrun) runs one independent replica per GPU: the path
 has no exchange step on one GPU ("replicas only"); value = all ranks' tokens /
@@ -48,6 +49,16 @@ def parse():
                    help="skip the extra router-mode episode timing")
     p.add_argument("--layers", type=int, default=0,
                    help="override the workload's MoE layer count (small profiling cases)")
+    p.add_argument("--sweep", action="store_true",
+                   help="instead of the step benchmark: the routing + scheduling sweep at the "
+                        "Qwen3-30B shape (D in 8..64, M in 4..32), 1-u per policy and the "
+                        "routing / scheduler kernel time per step (one GPU, one JSON line)")
+    p.add_argument("--sweep-episodes", type=int, default=4,
+                   help="episodes per sweep point (the workload defines 43, about 2048 "
+                        "lock-step steps; each episode's logits are drawn on the host)")
+    p.add_argument("--sweep-episodes-m32", type=int, default=1,
+                   help="episodes of the MaxUtil points at M = 32, whose exhaustive search "
+                        "covers about 15.3M subsets per step")
     return p.parse_args()
 
 
@@ -503,8 +514,123 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+SWEEP_M = (4, 8, 16, 32)
+SWEEP_D = (8, 16, 32, 64)
+SWEEP_NOTE = ("routing + scheduling only, Qwen3-30B shape: L=48 E=128 k=8 T=256, "
+              "13 task profiles switching every 16 lock-step steps")
+
+
+def sweep_jobs(args):
+    """(M, D, policy, episodes) of the routing + scheduling sweep, in order.
+    1 - u of a point pools its episodes: numerators and denominators are
+    summed over them."""
+    jobs = []
+    for M in SWEEP_M:
+        for D in SWEEP_D:
+            for pol in POLICY_NAMES:
+                n = args.sweep_episodes_m32 if (M == 32 and pol == 1) else args.sweep_episodes
+                jobs.append((M, D, pol, n))
+    return jobs
+
+
+def sweep_line(M, D, pol, n_ep, num, den, den_sep, steps, extra):
+    line = {"M": M, "D": D, "policy": POLICY_NAMES[pol], "episodes": n_ep, "steps": steps,
+            "under_util": round(1 - num / den, 6), "separate": round(1 - num / den_sep, 6),
+            "num": num, "den": den, "den_sep": den_sep}
+    line.update(extra)
+    print(json.dumps(line), flush=True)
+
+
+def run_sweep(args):
+    """The sweep on the GPU: for every (M, D) and policy, the exact 1 - u over
+    the point's episodes, the no-balancing 1 - u (every micro-batch run
+    separately) and the CUDA-event time per launch of the routing and
+    scheduler kernels.  One JSON line per point, as it completes."""
+    import torch
+
+    import cross_layer_expert_b200 as eb
+    import synth
+    from cross_layer_expert_b200 import build
+
+    build.build()
+    eb.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    print(json.dumps({"sweep": SWEEP_NOTE, "impl": "ours", "gpu": torch.cuda.get_device_name(dev),
+                      "unit_time": "us per launch (CUDA events on the launching stream)"}),
+          flush=True)
+    t0 = time.time()
+    cache_M, episodes = None, []
+    for M, D, pol, n_ep in sweep_jobs(args):
+        base = synth.get("sweep", M=M)
+        if cache_M != M:
+            episodes = [torch.from_numpy(synth.logits(base, episode=r)).to(dev)
+                        for r in range(max(args.sweep_episodes, args.sweep_episodes_m32))]
+            cache_M = M
+        wl = base.replace(D=D)
+        ctx = eb.Context(eb.make_config(L=wl.L, E=wl.E, k=wl.k, H=wl.H, F=wl.F, D=wl.D, M=wl.M,
+                                        T=wl.T, dtype=eb.DTYPE_BF16, policy=pol,
+                                        m=wl.m_default, compute=0))
+        ctx.eb_profile(True)
+        num = den = den_sep = steps = 0
+        for lg in episodes[:n_ep]:
+            steps += ctx.eb_episode(lg, None, None, None)
+            a, b, c = ctx.eb_utilization()
+            num, den, den_sep = num + a, den + b, den_sep + c
+        prof = ctx.eb_profile_read()
+        ctx.eb_profile(False)
+        assert ctx.eb_sync_status() == eb.EB_OK
+        ctx.close()
+        rt, sc = prof["route"], prof["schedule"]
+        sweep_line(M, D, pol, n_ep, num, den, den_sep, steps,
+                   {"route_us": round(1e3 * rt[0] / max(1, rt[1]), 2),
+                    "schedule_us": round(1e3 * sc[0] / max(1, sc[1]), 2)})
+    print(json.dumps({"sweep_done": True, "wall_s": round(time.time() - t0, 1)}), flush=True)
+
+
+def _oracle_sweep_job(job):
+    """One sweep point on the host with the oracle (a worker of a spawn pool)."""
+    sys.path.insert(0, ROOT)
+    import oracle
+    import synth
+    from oracle import native
+    M, D, pol, n_ep = job
+    wl = synth.get("sweep", M=M, D=D)
+    t = time.time()
+    num = den = den_sep = steps = 0
+    for r in range(n_ep):
+        hist = oracle.route_all(synth.logits(wl, episode=r), wl.k, D)[2]
+        ep = oracle.run_episode(oracle.loads(hist, D), pol, wl.m_default,
+                                maxutil_impl=native.maxutil if M > 12 else None)
+        num, den, den_sep = num + ep["num"], den + ep["den"], den_sep + ep["den_sep"]
+        steps += len(ep["steps"])
+    return job, (num, den, den_sep, steps, time.time() - t)
+
+
+def run_reference_sweep(args):
+    """The same sweep with the CPU oracle (routing, loads and Algorithm 1 in
+    float64 / exact integers; the exhaustive MaxUtil in plain C), one point
+    per worker of a spawn pool over the host's cores."""
+    import multiprocessing as mproc
+    cores = os.cpu_count() or 1
+    print(json.dumps({"sweep": SWEEP_NOTE, "impl": "reference", "kind": "oracle", "cores": cores,
+                      "unit_time": "s of one core per point"}), flush=True)
+    from oracle import native
+    native.build()
+    t0 = time.time()
+    # the heaviest points first, so the pool's tail is short
+    jobs = sorted(sweep_jobs(args), key=lambda j: (j[0] == 32 and j[2] == 1, j[1]), reverse=True)
+    with mproc.get_context("spawn").Pool(cores) as pool:
+        for (M, D, pol, n_ep), (num, den, den_sep, steps, sec) in pool.imap_unordered(
+                _oracle_sweep_job, jobs):
+            sweep_line(M, D, pol, n_ep, num, den, den_sep, steps, {"oracle_s": round(sec, 2)})
+    print(json.dumps({"sweep_done": True, "wall_s": round(time.time() - t0, 1)}), flush=True)
+
+
 def main():
     args = parse()
+    if args.sweep:
+        (run_reference_sweep if args.impl == "reference" else run_sweep)(args)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -1,0 +1,36 @@
+"""Host-side parts of bench.py that need no GPU: the routing + scheduling
+sweep's job list and one of its points computed by the oracle (the sweep's
+reference arm), checked against what Algorithm 1 and Eq. (3) fix."""
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+class _Args:
+    sweep_episodes = 2
+    sweep_episodes_m32 = 1
+
+
+def test_sweep_jobs_cover_every_point_and_policy():
+    import bench
+    jobs = bench.sweep_jobs(_Args)
+    assert len(jobs) == len(bench.SWEEP_M) * len(bench.SWEEP_D) * len(bench.POLICY_NAMES)
+    assert len(set(jobs)) == len(jobs)
+    for M, D, pol, n in jobs:
+        assert n == (1 if (M == 32 and pol == 1) else 2)
+
+
+def test_oracle_sweep_point_invariants():
+    """M = 4, D = 8, CumUtil, two episodes: every (micro-batch, layer) runs
+    once, so num = episodes * M * L * T * k; 1/D <= u <= 1; scheduling never
+    does worse than running each micro-batch separately (den <= den_sep);
+    L <= steps per episode <= M * L."""
+    import bench
+    (M, D, pol, n), (num, den, den_sep, steps, _) = bench._oracle_sweep_job((4, 8, 0, 2))
+    L, T, k = 48, 256, 8
+    assert num == n * M * L * T * k
+    assert num <= den <= D * num
+    assert den <= den_sep
+    assert n * L <= steps <= n * M * L

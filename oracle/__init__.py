@@ -4,9 +4,11 @@ TEST INFRASTRUCTURE ONLY.  This package is a plain, slow, float64 / exact-
 integer restatement of what the cross-layer MoE step computes, written from
 the paper "EasyBalance: Cross-Layer Load Balancing in Distributed MoE
 Inference" (Wu, Gao, Li, Wu) and the pages that restate it.  Only the tests,
-``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
-it.  It shares no code with the CUDA library (``cross_layer_expert_b200``) and
-imports nothing from it; both take their inputs from ``synth``.
+``__graft_entry__.smoke()`` and two parts of ``bench.py`` may import it: the
+CPU-baseline leg and the reference arm (``--impl reference``, the sweep's
+included).  It shares no code with the CUDA library
+(``cross_layer_expert_b200``) and imports nothing from it; both take their
+inputs from ``synth``.
 
 Modules:
   routing   top-k gating, per-expert histograms T_e, virtual-rank loads w

@@ -1,7 +1,8 @@
 """Oracle: SwiGLU experts, the gated combine and whole-stack token trajectories.
 
-Test infrastructure only (parity checks, the smoke check and the CPU baseline
-timing); nothing in the library's product path calls it.
+Test infrastructure only (parity checks, the smoke check, and the CPU
+baseline and reference arm of the benchmark); nothing in the library's
+product path calls it.
 
 [EB] is the paper "EasyBalance: Cross-Layer Load Balancing in Distributed MoE
 Inference".  All arithmetic is float64; values are rounded to the storage type

@@ -1,7 +1,8 @@
 """Oracle: router top-k, per-expert histograms and virtual-rank loads.
 
-Test infrastructure only (parity checks, the smoke check and the CPU baseline
-timing); nothing in the library's product path calls it.
+Test infrastructure only (parity checks, the smoke check, and the CPU
+baseline and reference arm of the benchmark); nothing in the library's
+product path calls it.
 
 Citations name the paper "EasyBalance: Cross-Layer Load Balancing in
 Distributed MoE Inference" (Wu, Gao, Li, Wu) as [EB], the deep-read page

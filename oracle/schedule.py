@@ -1,7 +1,8 @@
 """Oracle: effective workload, utilisation and the RunSet schedulers.
 
-Test infrastructure only (parity checks, the smoke check and the CPU baseline
-timing); nothing in the library's product path calls it.
+Test infrastructure only (parity checks, the smoke check, and the CPU
+baseline and reference arm of the benchmark); nothing in the library's
+product path calls it.
 
 [EB] is the paper "EasyBalance: Cross-Layer Load Balancing in Distributed MoE
 Inference"; [EB-read] the deep-read page "EasyBalance：分布式 MoE 推理的跨层负载均衡".

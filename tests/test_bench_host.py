@@ -34,3 +34,35 @@ def test_oracle_sweep_point_invariants():
     assert num <= den <= D * num
     assert den <= den_sep
     assert n * L <= steps <= n * M * L
+
+
+def test_reference_arm_prints_the_contract_line():
+    """The reference arm (the oracle on the host) prints one JSON line with the
+    step benchmark's keys, its own cpu_baseline and an e2e with no copies."""
+    import contextlib
+    import io
+    import json
+
+    import bench
+
+    class A:
+        workload, policy, steps, warmup, gpus = "tiny_f32", "cumutil", 1, 0, 1
+        layers = 0
+
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        bench.run_reference(A, 1, 0)
+    lines = [ln for ln in buf.getvalue().splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == bench.UNIT
+    assert d["metric"] == bench.METRIC and d["higher_is_better"] is True
+    assert "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}

@@ -58,7 +58,7 @@ def parse():
                         "lock-step steps; each episode's logits are drawn on the host)")
     p.add_argument("--sweep-episodes-m32", type=int, default=1,
                    help="episodes of the MaxUtil points at M = 32, whose exhaustive search "
-                        "covers about 15.3M subsets per step")
+                        "covers about 15.3M subsets per step (0: skip those points)")
     return p.parse_args()
 
 
@@ -529,7 +529,8 @@ def sweep_jobs(args):
         for D in SWEEP_D:
             for pol in POLICY_NAMES:
                 n = args.sweep_episodes_m32 if (M == 32 and pol == 1) else args.sweep_episodes
-                jobs.append((M, D, pol, n))
+                if n > 0:
+                    jobs.append((M, D, pol, n))
     return jobs
 
 

@@ -22,6 +22,14 @@ def test_sweep_jobs_cover_every_point_and_policy():
         assert n == (1 if (M == 32 and pol == 1) else 2)
 
 
+    class NoM32(_Args):
+        sweep_episodes_m32 = 0
+
+    skipped = bench.sweep_jobs(NoM32)
+    assert len(skipped) == len(jobs) - len(bench.SWEEP_D)
+    assert not any(M == 32 and pol == 1 for M, _, pol, _ in skipped)
+
+
 def test_oracle_sweep_point_invariants():
     """M = 4, D = 8, CumUtil, two episodes: every (micro-batch, layer) runs
     once, so num = episodes * M * L * T * k; 1/D <= u <= 1; scheduling never

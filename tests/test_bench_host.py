@@ -74,3 +74,17 @@ def test_reference_arm_prints_the_contract_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_oracle_sweep_pairs_policies_on_one_workload():
+    """The sweep's loads do not depend on the schedule, so every policy sees
+    the same work: num (all token-expert pairs) and den_sep (every micro-batch
+    run separately) agree across policies.  On this point MaxUtil's u is also
+    at least lock-step's (MaxUtil is greedy per step, so this is checked on
+    the point, not claimed in general)."""
+    import bench
+    out = {pol: bench._oracle_sweep_job((4, 16, pol, 1))[1] for pol in bench.POLICY_NAMES}
+    assert len({o[0] for o in out.values()}) == 1
+    assert len({o[2] for o in out.values()}) == 1
+    num, den_max = out[1][0], out[1][1]
+    assert num / den_max >= num / out[2][1]  # u(MaxUtil) >= u(lock-step)

@@ -137,7 +137,10 @@ eb_status eb_destroy(eb_ctx* ctx);
 
 /* Algorithm 1 initialisation ([EB] §4.2): l_j = 0 for all j, S_0 = all
  * micro-batches, RunSet_0 = all (every micro-batch routes at step 1), and
- * zeroed accumulators and trace.  Enqueued on `stream`. */
+ * zeroed accumulators and trace.  With EB_GEMM_TMC it also zeroes the fused
+ * combine's arrival counters, which a step that gave up on a bounded wait
+ * (EB_ERR_TIMEOUT) may have left non-zero: after such an error, reset before
+ * the next step.  Enqueued on `stream`. */
 eb_status eb_reset(eb_ctx* ctx, void* stream);
 
 /* Router mode ([EB] §2.1, W_l, I_l = topk(G(h'_l)) with a linear scorer):

@@ -9,9 +9,16 @@
  *
  * This is the same definition as oracle/schedule.py's maxutil, in plain C so
  * that pending sets of 32 micro-batches (about 15 million admissible subsets
- * at m = 24) finish in seconds.  Every admissible S is visited as the
- * complement C = P \ S with |C| <= n - m, C running over all combinations in
- * lexicographic order; W is recomputed from scratch for every S.
+ * at m = 24) finish in seconds.  Two enumerations of it:
+ *   oracle_maxutil_plain  every bitmask S over the n pending positions, in
+ *                         increasing order, skipping |S| < m; W summed from
+ *                         the member rows.  2^n masks: n <= 24 in practice.
+ *   oracle_maxutil        every admissible S visited as its complement
+ *                         C = P \ S with |C| <= n - m, C running over all
+ *                         combinations in lexicographic order; W recomputed
+ *                         from the totals minus the rows of C.  For large n
+ *                         with m close to n (n = 32, m = 24).
+ * They share nothing but the U comparison, so each pins the other.
  */
 #include <stdint.h>
 #include <string.h>
@@ -74,6 +81,50 @@ uint32_t oracle_maxutil(const int64_t* w, const int32_t* ids, int n, int D, int 
       if (i < 0) break;
       ++comb[i];
       for (int k = i + 1; k < c; ++k) comb[k] = comb[k - 1] + 1;
+    }
+  }
+  return best_mask;
+}
+
+/* Forward enumeration: every mask over the n positions with at least m set
+ * bits; W_d = sum of the member rows; the same order of candidates. */
+uint32_t oracle_maxutil_plain(const int64_t* w, const int32_t* ids, int n, int D, int m) {
+  uint32_t all = 0;
+  for (int i = 0; i < n; ++i) all |= 1u << ids[i];
+  if (n <= m) return all;
+  int have = 0, best_size = 0;
+  int64_t best_sum = 0, best_max = 0;
+  uint32_t best_mask = 0;
+  const uint64_t count = (uint64_t)1 << n;
+  for (uint64_t s = 1; s < count; ++s) {
+    int size = 0;
+    uint32_t mask = 0;
+    for (int i = 0; i < n; ++i)
+      if ((s >> i) & 1u) {
+        ++size;
+        mask |= 1u << ids[i];
+      }
+    if (size < m) continue;
+    int64_t sum = 0, mx = 0;
+    for (int d = 0; d < D; ++d) {
+      int64_t W = 0;
+      for (int i = 0; i < n; ++i)
+        if ((s >> i) & 1u) W += w[i * D + d];
+      sum += W;
+      if (W > mx) mx = W;
+    }
+    int better = !have;
+    if (have) {
+      if (u_greater(sum, mx, best_sum, best_max)) better = 1;
+      else if (u_equal(sum, mx, best_sum, best_max))
+        better = size > best_size || (size == best_size && mask < best_mask);
+    }
+    if (better) {
+      have = 1;
+      best_sum = sum;
+      best_max = mx;
+      best_size = size;
+      best_mask = mask;
     }
   }
   return best_mask;

@@ -85,11 +85,20 @@ def oracle_loads(inp: Inputs, expert_rank=None):
     return inp._loads
 
 
-def oracle_episode(inp: Inputs, policy: int, m: int = 0, expert_rank=None):
+def maxutil_impl(M: int):
+    """The oracle's MaxUtil for M micro-batches: the Python enumeration up to
+    12, the plain-C forward enumeration over every bitmask up to 20, and the
+    plain-C complement enumeration (pinned against the forward one) beyond."""
     from oracle import native
+    if M <= 12:
+        return None
+    return native.maxutil_plain if M <= 20 else native.maxutil
+
+
+def oracle_episode(inp: Inputs, policy: int, m: int = 0, expert_rank=None):
     wl = inp.wl
     return oracle.run_episode(oracle_loads(inp, expert_rank), policy, m or wl.m_default,
-                              maxutil_impl=native.maxutil if wl.M > 12 else None)
+                              maxutil_impl=maxutil_impl(wl.M))
 
 
 def check_schedule(rows, layers, util, steps, ref, M: int):

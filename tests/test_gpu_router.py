@@ -1,9 +1,10 @@
 """Router mode: routing scores projected from the hidden states on the
 device ([EB] §2.1 topk(G(h'_l)) with a linear scorer), so the chain is
 data-dependent.  The projection is checked against the oracle's float64
-product; episodes against the oracle's routed chain, and -- the property the
-method rests on -- scheduling still moves only timing: MaxUtil's final hidden
-states equal the lock-step run's bit for bit."""
+product; episodes against the oracle's own routed chain -- the oracle computes
+its own scores from its own hidden states and takes every routing decision on
+them -- and, the property the method rests on, scheduling still moves only
+timing: MaxUtil's final hidden states equal the lock-step run's bit for bit."""
 import numpy as np
 import pytest
 
@@ -58,30 +59,97 @@ def _episode(eb, torch, wl, inp, router, policy):
     return hidden, rows, layers, util, n, scores.cpu().numpy()
 
 
+# Near-tie bound for a router score: the device projection was measured within
+# 1e-4 abs + 1e-4 rel of the float64 product on identical inputs (above); a
+# later layer's input also differs from the oracle's chain by the rounding of
+# the bf16 hidden state (one unit in the last place in a few elements, each
+# contributing about 2^-8 |h_i| |w_i| to a score).  TAU covers both with a
+# margin; the test prints the largest deviation it saw.
+TAU_ABS, TAU_REL = 2e-3, 2e-3
+
+
+def _topk_sets(scores, k):
+    """Top-k expert sets of score rows [n, E] (descending score, lower index
+    first on equal scores), as sorted index arrays [n, k]."""
+    order = np.argsort(-np.asarray(scores, dtype=np.float32), axis=1, kind="stable")
+    return np.sort(order[:, :k], axis=1)
+
+
+def _oracle_chain(wl, inp, routers, gpu_scores):
+    """The routed chain of every token on the oracle's side: each layer's
+    scores are the float64 projection of the oracle's own hidden states
+    (decided in float32), routed by oracle.route, then the oracle's MoE layer.
+
+    The device's scores are used only to see which experts the device chose.
+    Where the oracle's own k-th and (k+1)-th scores lie within 2 tau(s) of each
+    other (a near tie: both choices are correct within the projection error),
+    the device's choice is accepted if it is a valid top-k of the oracle's
+    scores within that bound, and the oracle continues with it; everywhere
+    else the device must have chosen exactly the oracle's set.
+
+    Returns (final hidden [M*T, H], loads [M, L, D], near-tie count, adopted
+    count, largest |device score - oracle score| over tokens)."""
+    M, L, T, E, k = wl.M, wl.L, wl.T, wl.E, wl.k
+    h = inp.h0_np.reshape(M * T, wl.H).copy()
+    loads = np.zeros((M, L, wl.D), dtype=np.int64)
+    near = adopted = 0
+    worst = 0.0
+    for l in range(L):
+        osc = orouter.router_logits(h, routers[l]).astype(np.float32)
+        gsc = gpu_scores[:, l].reshape(M * T, E)
+        dev = np.abs(gsc.astype(np.float64) - osc)
+        tau = TAU_ABS + TAU_REL * np.abs(osc.astype(np.float64))
+        worst = max(worst, float(dev.max()))
+        assert np.all(dev <= tau), (l, float(dev.max()))
+        idx, gate = oracle.route(osc, k)
+        # near ties of the oracle's own decision
+        srt = -np.sort(-osc.astype(np.float64), axis=1)
+        gap = srt[:, k - 1] - srt[:, k] if k < E else np.full(M * T, np.inf)
+        tie = gap <= 2 * (TAU_ABS + TAU_REL * np.abs(srt[:, k - 1]))
+        near += int(tie.sum())
+        want = np.sort(idx, axis=1)
+        got = _topk_sets(gsc, k)
+        same = np.all(got == want, axis=1)
+        assert np.all(same | tie), f"layer {l}: {int((~same & ~tie).sum())} tokens routed " \
+                                   "differently away from a near tie"
+        for t in np.nonzero(~same)[0]:
+            # valid under the oracle's scores within the bound: every chosen
+            # expert scores at least every unchosen one, less 2 tau
+            sel = np.zeros(E, dtype=bool)
+            sel[got[t]] = True
+            lo = osc[t, sel].astype(np.float64).min()
+            hi = osc[t, ~sel].astype(np.float64).max()
+            assert lo >= hi - 2 * (TAU_ABS + TAU_REL * abs(hi)), (l, t)
+            # the device's set, slots and renormalised gates as the oracle
+            # forms them over that set (experts outside it masked far below)
+            masked = np.where(sel, osc[t], np.float32(-1e30)).astype(np.float32)
+            i1, g1 = oracle.route(masked[None], k)
+            idx[t], gate[t] = i1[0], g1[0]
+            adopted += 1
+        hist = np.stack([oracle.histogram(idx[j * T:(j + 1) * T], E) for j in range(M)])
+        loads[:, l] = oracle.loads(hist, wl.D)
+        h = omoe.moe_layer(h, idx, gate, l, inp.expert, E, wl.n_shared, wl.dtype)
+    return h, loads, near, adopted, worst
+
+
 def _check_router_episode(torch, wl, inp, router, toks, policies):
-    """The top-k decisions are taken on the kernel's float32 scores on both
-    sides (a float decides an integer): the oracle routes the scores the GPU
-    computed.  Then (1) the schedule, trace and utilisation match the oracle
-    bit for bit; (2) the final hidden states of `toks` match the oracle's
-    chain within the bf16 tolerance; (3) every step's scores match the
-    projection of the oracle's own hidden states; (4) MaxUtil equals
-    lock-step bit for bit."""
+    """The oracle runs its own routed chain (above) and so decides every
+    routing on its own scores.  Then (1) every device score is within the
+    near-tie bound of the oracle's; (2) routing equals the oracle's except at
+    counted near ties, where the device's choice is valid under the oracle's
+    scores; (3) the schedule, trace and utilisation equal the oracle's episode
+    on that routing bit for bit; (4) the final hidden states of `toks` match
+    the oracle's chain within the bf16 tolerance; (5) MaxUtil equals lock-step
+    bit for bit."""
     import cross_layer_expert_b200 as eb
     routers = [router[l].float().cpu().numpy().astype(np.float64) for l in range(wl.L)]
     lock = _episode(eb, torch, wl, inp, router, osch.LOCKSTEP)
     sc = lock[5]
     assert np.isfinite(sc).all()
-    loads = oracle.route_all(sc, wl.k, wl.D)[3]
-    h0 = np.stack([inp.h0_np[j, t] for (j, t) in toks])
-    want = omoe.forward_tokens(h0, lambda j, l: sc[j, l], toks, wl.L, wl.E, wl.k, wl.n_shared,
-                               wl.dtype, inp.expert)
-    # the scores are the projection of the hidden states: against the oracle's
-    # own chain (which drifts from the GPU's by bf16 rounding only)
-    _, seen = orouter.forward_tokens_routed(h0, lambda l: routers[l], toks, wl.L, wl.E, wl.k,
-                                            wl.n_shared, wl.dtype, inp.expert)
-    for l in range(wl.L):
-        got = np.stack([sc[j, l, t] for (j, t) in toks]).astype(np.float64)
-        assert np.all(np.abs(got - seen[l]) <= 5e-2 + 5e-2 * np.abs(seen[l])), l
+    final, loads, near, adopted, worst = _oracle_chain(wl, inp, routers, sc)
+    print(f"router chain {wl.name} L={wl.L}: {near} near ties, {adopted} routed by the device's "
+          f"valid choice, largest score deviation {worst:.3g}")
+    want = np.stack([final[j * wl.T + t] for (j, t) in toks])
     for policy in policies:
         hidden, rows, layers, util, n, sc2 = _episode(eb, torch, wl, inp, router, policy)
         # routing scores of a (micro-batch, layer) do not depend on the schedule
@@ -102,13 +170,14 @@ def test_small_router_episode_matches_oracle(torch):
 
 
 def test_qwen3_shape_router_episode(torch):
-    """Qwen3 per-layer sizes, 3 layers, sampled tokens."""
-    wl = synth.get("qwen3_bf16").replace(L=3)
+    """Qwen3 per-layer sizes (E = 128, k = 8, H = 2048, F = 768, D = 8, M = 8),
+    3 layers of 256 tokens per micro-batch: the oracle's chain covers every
+    token, so every routing decision and every output is checked."""
+    wl = synth.get("qwen3_bf16").replace(L=3, T=256)
     inp = Inputs(wl)
     router = synth.router_torch(wl, device="cuda")
-    rng = np.random.default_rng(41)
-    toks = [(j, int(rng.integers(0, wl.T))) for j in range(wl.M)] + [(0, 0), (wl.M - 1, wl.T - 1)]
-    _check_router_episode(torch, wl, inp, router, toks, (osch.MAXUTIL,))
+    toks = [(j, t) for j in range(wl.M) for t in range(wl.T)]
+    _check_router_episode(torch, wl, inp, router, toks, (osch.MAXUTIL, osch.CUMUTIL))
 
 
 def test_router_mode_rejects_unsupported_shapes(torch):

@@ -442,6 +442,37 @@ def test_native_maxutil_matches_python():
         assert native.maxutil(sorted(w), w, int(m)) == [int(x) for x in want.split()]
 
 
+def test_native_maxutil_plain_pins_the_complement_enumeration():
+    """The forward enumeration over every bitmask (oracle_maxutil_plain) is
+    pinned against the Python enumeration of [EB] §4.2's candidate subsets up
+    to 16 pending micro-batches; the complement enumeration (used for pending
+    sets of 32) is pinned against the forward one up to 20, with many equal-U
+    ties (small loads) and pending sets with holes."""
+    from oracle import native
+    rng = np.random.default_rng(1620)
+    for trial in range(200):
+        M = int(rng.integers(1, 13))
+        D = int(rng.integers(1, 9))
+        pending = sorted(rng.choice(M, size=int(rng.integers(1, M + 1)), replace=False).tolist())
+        hi = int(rng.choice([2, 4, 60]))
+        w = {j: [int(x) for x in rng.integers(0, hi, size=D)] for j in pending}
+        m = int(rng.integers(1, M + 1))
+        assert native.maxutil_plain(pending, w, m) == osch.maxutil(pending, w, m), (pending, w, m)
+    for trial in range(2):  # 16 pending micro-batches: 65 536 subsets in Python
+        pending = list(range(16))
+        w = {j: [int(x) for x in rng.integers(0, 6, size=4)] for j in pending}
+        assert native.maxutil_plain(pending, w, 12) == osch.maxutil(pending, w, 12)
+    for trial in range(120):
+        M = int(rng.integers(12, 21))
+        D = int(rng.choice([1, 3, 8, 16, 64]))
+        pending = sorted(rng.choice(32, size=M, replace=False).tolist())
+        hi = int(rng.choice([2, 3, 1000]))
+        w = {j: [int(x) for x in rng.integers(0, hi, size=D)] for j in pending}
+        m = int(rng.integers(max(1, M - 6), M + 1)) if trial % 3 else int(rng.integers(1, M + 1))
+        a, b = native.maxutil(pending, w, m), native.maxutil_plain(pending, w, m)
+        assert a == b, (pending, m, a, b)
+
+
 # ------------------------------------------------------------ router projection
 
 def test_router_projection_pins():

@@ -4,9 +4,10 @@ eb_route_loads_static is for callers that cannot allocate device memory (a
 serving process whose memory is fixed at start-up, or one that must not call
 cudaMalloc because it can synchronise the device).  Its counts live in the
 library's fixed device array; this test calls it through the C ABI twice in a
-row -- a large call, then a smaller one that leaves stale counts of the first
-call in the array -- and checks each result against eb_route on every
-micro-batch followed by eb_loads.  It is collected last so that a failure here
+row -- a large call, then smaller ones that leave stale counts of the earlier
+calls in the array -- and checks each result against eb_route on every
+micro-batch followed by eb_loads, and against the CPU oracle's routing and
+loads.  It is collected last so that a failure here
 stops a `-x` run only after every other test has run, and it passes both alone
 in a fresh process and after the other tests.
 """
@@ -54,13 +55,28 @@ def _static(torch, lib, logits, k, renorm, D):
     return idx, gate, w, status
 
 
+def _oracle(x, k, renorm, D):
+    """idx, gate and loads of every micro-batch from the CPU oracle."""
+    import oracle
+    ridx, rgate, w = [], [], []
+    for j in range(x.shape[0]):
+        i, g = oracle.route(x[j], k, renorm)
+        ridx.append(i)
+        rgate.append(g)
+        w.append(oracle.loads(oracle.histogram(i, x.shape[2]), D))
+    return np.stack(ridx), np.stack(rgate), np.stack(w)
+
+
 def test_no_alloc_route_loads_matches_allocating_entry_points(lib):
     import torch
     import cross_layer_expert_b200 as eb
     rng = np.random.default_rng(2026)
-    cases = [  # (n_mb, T, E, k, D, renorm): large first, then smaller with ragged T
+    cases = [  # (n_mb, T, E, k, D, renorm): large first, then smaller ones whose
+        # counts leave stale entries of the earlier calls in the array
         (8, 1024, 128, 8, 8, True),
         (3, 200, 64, 6, 4, False),
+        (2, 70, 40, 40, 8, True),  # E not a multiple of 32 (padded lanes), k = E
+        (1, 17, 16, 2, 4, True),   # one micro-batch shorter than a 64-token chunk
     ]
     for (n_mb, T, E, k, D, renorm) in cases:
         x = rng.standard_normal((n_mb, T, E)).astype(np.float32)
@@ -70,11 +86,39 @@ def test_no_alloc_route_loads_matches_allocating_entry_points(lib):
         ridx, rgate, rw = _reference(torch, eb, logits, k, renorm, D)
         torch.cuda.synchronize()
         assert int(status.item()) == 0
+        # against the allocating entry points (same kernels' arithmetic) ...
         assert torch.equal(idx, ridx)
         assert torch.equal(w, rw)
         g, rg = gate.double().cpu().numpy(), rgate.double().cpu().numpy()
         assert np.all(np.abs(g - rg) <= 1e-6 * np.abs(rg) + 1e-12)
+        # ... and against the CPU oracle, independently of any CUDA path
+        oidx, ogate, ow = _oracle(x, k, renorm, D)
+        assert np.array_equal(idx.cpu().numpy(), oidx)
+        assert np.array_equal(w.cpu().numpy(), ow)
+        assert np.all(np.abs(g - ogate) <= 1e-6 * np.abs(ogate) + 1e-12)
         assert int(w.sum().item()) == n_mb * T * k
+
+
+def test_no_alloc_reports_nonfinite_logits(lib):
+    """A NaN logit sets EB_ERR_NONFINITE in status_dev; the row is routed
+    among the finite experts as eb_route does, and every count still lands."""
+    import torch
+    import cross_layer_expert_b200 as eb
+    rng = np.random.default_rng(7)
+    x = rng.standard_normal((2, 90, 32)).astype(np.float32)
+    x[1, 65, 3] = np.nan
+    logits = torch.from_numpy(x).cuda()
+    idx, gate, w, status = _static(torch, lib, logits, 4, True, 4)
+    ridx, rgate, rw = _reference(torch, eb, logits, 4, True, 4)
+    torch.cuda.synchronize()
+    assert int(status.item()) == eb.EB_ERR_NONFINITE
+    assert torch.equal(idx, ridx)
+    assert torch.equal(w, rw)
+    assert int(w.sum().item()) == 2 * 90 * 4
+    # the finite micro-batch agrees with the oracle
+    oidx, _, ow = _oracle(x[:1], 4, True, 4)
+    assert np.array_equal(idx[:1].cpu().numpy(), oidx)
+    assert np.array_equal(w[:1].cpu().numpy(), ow)
 
 
 def test_no_alloc_rejects_sizes_beyond_its_capacity(lib):

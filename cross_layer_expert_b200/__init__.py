@@ -29,14 +29,14 @@ EB_ERR_TOO_LARGE = -7
 
 CUMUTIL, MAXUTIL, LOCKSTEP, DIFFPEAK = 0, 1, 2, 3
 DTYPE_F32, DTYPE_BF16 = 0, 1
-GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TC2, GEMM_TM, GEMM_TM2, GEMM_TMG, GEMM_TMC = range(8)
+GEMM_AUTO, GEMM_TC, GEMM_SIMT, GEMM_TM, GEMM_TMG, GEMM_TMC = 0, 1, 2, 4, 6, 7
 
 EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_create", "eb_destroy",
             "eb_reset", "eb_moe_step", "eb_episode", "eb_utilization", "eb_trace",
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
             "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped", "eb_set_router",
-            "eb_router", "eb_engines"]
+            "eb_router", "eb_engines", "eb_inject_status"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine",
                 "positions", "router")
@@ -93,6 +93,7 @@ def load() -> ctypes.CDLL:
         "eb_engines": (I, [P, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]),
         "eb_route_loads_static": (I, [P, I, I, I, I, I, I, P, P, P, P, P]),
         "eb_selftest_timeout": (I, [ctypes.c_int64, P, P]),
+        "eb_inject_status": (I, [P, I, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -280,6 +281,12 @@ class Context:
 
     def eb_sync_status(self) -> int:
         return load().eb_sync_status(self.handle)
+
+    def eb_inject_status(self, status: int, stream=None) -> None:
+        """Test hook: records `status` in the context's device status word
+        (EB_ERR_TIMEOUT also dirties the fused combine's arrival counters)."""
+        _check(load().eb_inject_status(self.handle, int(status), _stream(stream)),
+               "eb_inject_status")
 
     def eb_profile(self, enable: bool) -> None:
         _check(load().eb_profile(self.handle, int(enable)), "eb_profile")

@@ -29,6 +29,9 @@ struct eb_ctx {
   CUtensorMap router_map_h, router_map_r;
   const void* router_keys[2] = {nullptr, nullptr};
   cudaStream_t last_stream = nullptr;
+  // set once the host has seen EB_ERR_TIMEOUT in the status word; steps are
+  // refused until eb_reset
+  bool timed_out = false;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
   // cached TMA maps (rebuilt when a pointer changes)
@@ -57,23 +60,20 @@ bool use_tc_for(const eb_config& c) {
   return c.gemm != EB_GEMM_SIMT;
 }
 
-// Engine of each GEMM.  AUTO takes the one-SM token-major engine for every
-// GEMM whose tile shape fits (GEMM 1: F a multiple of 128; GEMM 2: H a
-// multiple of 256) and the one-SM weight-major engine otherwise; an explicit
-// choice that does not fit one GEMM runs that GEMM on the weight-major engine.
-void choose_engines(const eb_config& c, bool use_tc, int num_sms, int* g1, int* g2) {
+// Engine of each GEMM.  AUTO takes the token-major engine for every GEMM
+// whose tile shape fits (GEMM 1: F a multiple of 128; GEMM 2: H a multiple of
+// 256) and the weight-major engine otherwise; an explicit choice that does not
+// fit one GEMM runs that GEMM on the weight-major engine.
+void choose_engines(const eb_config& c, bool use_tc, int* g1, int* g2) {
   *g1 = *g2 = EB_GEMM_SIMT;
   if (!use_tc) return;
-  const bool pair_ok = num_sms >= 2;
   const int want = c.gemm == EB_GEMM_AUTO ? EB_GEMM_TM : c.gemm;
   auto fits = [&](int eng, int which) {
     const int nout = which == 1 ? c.F : c.H;
     switch (eng) {
       case EB_GEMM_TC: return true;
-      case EB_GEMM_TC2: return pair_ok && nout % kTc2Feat == 0;
       case EB_GEMM_TM: return nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
       case EB_GEMM_TMG: return which == 1 && nout % kTmFeat1 == 0;
-      case EB_GEMM_TM2: return pair_ok && nout % (which == 1 ? kTmFeat1 : kTmFeat2) == 0;
       case EB_GEMM_TMC: return which == 2 && nout % kTmFeat2 == 0;
       default: return false;
     }
@@ -93,18 +93,10 @@ void engine_tiles(int eng, int which, int* rows, int* feats) {
       *rows = which == 1 ? kTcRows1 : kTcRows2;
       *feats = kTcFeat;
       return;
-    case EB_GEMM_TC2:
-      *rows = which == 1 ? kTc2Rows1 : kTc2Rows2;
-      *feats = kTc2Feat;
-      return;
     case EB_GEMM_TM:
     case EB_GEMM_TMG:
     case EB_GEMM_TMC:
       *rows = kTmRows;
-      *feats = which == 1 ? kTmFeat1 : kTmFeat2;
-      return;
-    case EB_GEMM_TM2:
-      *rows = 2 * kTmRows;
       *feats = which == 1 ? kTmFeat1 : kTmFeat2;
       return;
     default:
@@ -219,7 +211,8 @@ eb_status eb_config_check(const eb_config* c) {
   if (c->E % c->D != 0) return EB_ERR_INVALID_ARG;
   if (c->policy < EB_SCHED_CUMUTIL || c->policy > EB_SCHED_DIFFPEAK) return EB_ERR_INVALID_ARG;
   if (c->dtype != EB_DTYPE_F32 && c->dtype != EB_DTYPE_BF16) return EB_ERR_INVALID_ARG;
-  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TMC) return EB_ERR_INVALID_ARG;
+  if (c->gemm < EB_GEMM_AUTO || c->gemm > EB_GEMM_TMC || c->gemm == 3 || c->gemm == 5)
+    return EB_ERR_INVALID_ARG;  // 3 and 5 were retired engines
   if (c->M > EB_MAX_M || c->D > EB_MAX_D || c->E + c->n_shared > EB_MAX_ETOT ||
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
@@ -236,7 +229,6 @@ eb_status eb_config_check(const eb_config* c) {
     if (use_tc_for(*c) && (c->H % 128 != 0 || c->F % 128 != 0)) {
       if (forced_tc) return EB_ERR_UNSUPPORTED;
     }
-    if (c->gemm == EB_GEMM_TC2 && (c->H % 256 != 0 || c->F % 256 != 0)) return EB_ERR_UNSUPPORTED;
   }
   return EB_OK;
 }
@@ -260,8 +252,7 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   x->use_tc = use_tc_for(*c) && c->H % 128 == 0 && c->F % 128 == 0;
   cudaError_t e = cudaGetDevice(&x->device);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&x->num_sms, cudaDevAttrMultiProcessorCount, x->device);
-  // the two-SM engine covers 256 output features per item
-  if (e == cudaSuccess) choose_engines(*c, x->use_tc, x->num_sms, &x->eng1, &x->eng2);
+  if (e == cudaSuccess) choose_engines(*c, x->use_tc, &x->eng1, &x->eng2);
   const size_t n_state = align_up(sizeof(State));
   const size_t n_hist = align_up(sizeof(int32_t) * c->M * c->E);
   const size_t n_w = align_up(sizeof(int32_t) * c->M * c->D);
@@ -271,7 +262,10 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   // arrival counters of the fused combine, one per (token, 256-feature block)
   const size_t n_arrive =
       x->eng2 == EB_GEMM_TMC ? align_up(sizeof(int32_t) * (size_t)c->M * c->T * (c->H / kTmFeat2)) : 0;
-  const size_t n_all = n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive;
+  // MaxUtil search grid results, when one CTA would search too many subsets
+  const bool grid_search = c->policy == EB_SCHED_MAXUTIL && maxutil_uses_grid(c->M, c->m);
+  const size_t n_slots = grid_search ? align_up(kSearchCtas * kSearchSlotBytes) : 0;
+  const size_t n_all = n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots;
   char* p = nullptr;
   if (e == cudaSuccess) e = cudaMalloc(&p, n_all);
   if (e == cudaSuccess) e = cudaMemset(p, 0, n_all);
@@ -286,6 +280,8 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->dev.use_emap = 0;
     x->dev.arrive = n_arrive ? (int32_t*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map) : nullptr;
     x->dev.arrive_bytes = n_arrive;
+    x->dev.search_slots =
+        n_slots ? (void*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive) : nullptr;
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
   for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
@@ -320,8 +316,10 @@ eb_status eb_destroy(eb_ctx* x) {
 eb_status eb_reset(eb_ctx* x, void* stream) {
   if (!x) return EB_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   x->last_stream = s;
   x->launches += 1;
+  x->timed_out = false;
   cudaError_t e = launch_reset(x->d, x->dev, s);
   // the fused combine leaves its counters at zero; a step that gave up on a
   // bounded wait may not have, so a reset clears them
@@ -366,7 +364,6 @@ static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* 
                                  const void* wdn, const void* hidden, cudaStream_t s, int which) {
   switch (eng) {
     case EB_GEMM_TC: return launch_gemm_tc(x->d, x->dev, w, x->maps, x->num_sms, s, which);
-    case EB_GEMM_TC2: return launch_gemm_tc2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     case EB_GEMM_TM:
       return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr, nullptr);
     case EB_GEMM_TMG:
@@ -375,7 +372,6 @@ static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* 
     case EB_GEMM_TMC:  // GEMM 2 only (GEMM 1 of TMC is TM)
       return launch_gemm_tm(x->d, x->dev, w, x->maps, x->num_sms, s, which, nullptr,
                             const_cast<void*>(hidden));
-    case EB_GEMM_TM2: return launch_gemm_tm2(x->d, x->dev, w, x->maps, x->num_sms, s, which);
     default: return launch_gemm_simt(x->d, x->dev, w, wgu, wdn, s, which);
   }
 }
@@ -384,6 +380,7 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
                               const void* wdn, void* workspace, size_t ws_bytes,
                               cudaStream_t s) {
   const eb_config& c = x->cfg;
+  if (x->timed_out) return EB_ERR_TIMEOUT;
   if ((!logits && !x->w_router) || !workspace) return EB_ERR_INVALID_ARG;
   if (x->w_router && !hidden) return EB_ERR_INVALID_ARG;
   if (((uintptr_t)workspace & (kAlign - 1)) != 0) return EB_ERR_INVALID_ARG;
@@ -393,6 +390,7 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   Work w;
   const size_t need = layout(c, (char*)workspace, &w);
   if (ws_bytes < need) return EB_ERR_WORKSPACE;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   x->last_stream = s;
   const bool tc = c.compute && x->use_tc;
   if (tc && (x->map_keys[0] != wgu || x->map_keys[1] != wdn || x->map_keys[2] != workspace)) {
@@ -439,7 +437,8 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   if (e == cudaSuccess)
     e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, s); });
   if (e == cudaSuccess)
-    e = timed(x, 1, 1, s, [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
+    e = timed(x, 1, x->dev.search_slots ? 2 : 1, s,
+              [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
   if (c.compute) {
     if (e == cudaSuccess)
       e = timed(x, 6, 1, s, [&] { return launch_positions(x->d, x->dev, w, s); });
@@ -467,8 +466,15 @@ eb_status eb_moe_step(eb_ctx* x, const float* logits, void* hidden, const void* 
   if (runset_host) {
     cudaError_t e = cudaMemcpyAsync(runset_host, &x->dev.st->runset, sizeof(uint32_t),
                                     cudaMemcpyDeviceToHost, s);
+    int status = EB_OK;
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(&status, &x->dev.st->status, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
-    return cuda_status(e);
+    if (e != cudaSuccess) return EB_ERR_CUDA;
+    if (status == EB_ERR_TIMEOUT) {
+      x->timed_out = true;
+      return EB_ERR_TIMEOUT;
+    }
   }
   return EB_OK;
 }
@@ -498,10 +504,15 @@ eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* w
     }
   }
   if (cudaStreamSynchronize(s) != cudaSuccess) return EB_ERR_CUDA;
-  int steps = 0;
-  if (cudaMemcpy(&steps, &x->dev.st->n_steps, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+  int steps = 0, status = EB_OK;
+  if (cudaMemcpy(&steps, &x->dev.st->n_steps, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      cudaMemcpy(&status, &x->dev.st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return EB_ERR_CUDA;
   if (n_steps) *n_steps = steps;
+  if (status == EB_ERR_TIMEOUT) {
+    x->timed_out = true;
+    return EB_ERR_TIMEOUT;
+  }
   return EB_OK;
 }
 
@@ -588,11 +599,25 @@ eb_status eb_sync_status(eb_ctx* x) {
   int status = 0;
   if (cudaMemcpy(&status, &x->dev.st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
     return EB_ERR_CUDA;
+  if (status == EB_ERR_TIMEOUT) x->timed_out = true;
   return status;
+}
+
+eb_status eb_inject_status(eb_ctx* x, eb_status status, void* stream) {
+  if (!x || status > 0 || status < EB_ERR_TOO_LARGE) return EB_ERR_INVALID_ARG;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
+  x->last_stream = s;
+  cudaError_t e = launch_set_status(x->dev.st, status, s);
+  // the partial arrival counts a fused GEMM 2 that gave up part-way leaves
+  if (e == cudaSuccess && status == EB_ERR_TIMEOUT && x->dev.arrive)
+    e = cudaMemsetAsync(x->dev.arrive, 1, x->dev.arrive_bytes, s);
+  return cuda_status(e);
 }
 
 eb_status eb_selftest_timeout(int64_t limit_ns, int32_t* status_dev, void* stream) {
   if (!status_dev || limit_ns < 1000 || limit_ns > 2000000000ll) return EB_ERR_INVALID_ARG;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   return cuda_status(launch_selftest_wait((unsigned long long)limit_ns, status_dev,
                                           (cudaStream_t)stream));
 }
@@ -609,6 +634,8 @@ eb_status eb_route(const float* logits, int n, int E, int k, int renorm, int32_t
 eb_status eb_loads(const int32_t* hist, int M, int E, int D, int32_t* w, void* stream) {
   if (M < 0 || E < 1 || D < 1 || E % D != 0) return EB_ERR_INVALID_ARG;
   if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
+  if (M == 0) return EB_OK;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   return cuda_status(launch_loads(hist, M, E, D, nullptr, w, nullptr, (cudaStream_t)stream));
 }
 
@@ -621,6 +648,7 @@ eb_status eb_router(const void* hidden, int n, int H, const void* w_router, int 
       ((uintptr_t)scores & 15u) != 0)
     return EB_ERR_INVALID_ARG;
   if (n == 0) return EB_OK;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   if (gemm_tc_prepare() != cudaSuccess) return EB_ERR_CUDA;
   CUtensorMap mh, mr;
   if (make_router_maps(hidden, n, H, w_router, 1, E, &mh, &mr) != cudaSuccess)
@@ -633,6 +661,8 @@ eb_status eb_loads_mapped(const int32_t* hist, int M, int E, int D, const int32_
                           int32_t* w, int32_t* status_dev, void* stream) {
   if (M < 0 || E < 1 || D < 1 || !expert_rank) return EB_ERR_INVALID_ARG;
   if (M > 0 && (!hist || !w)) return EB_ERR_INVALID_ARG;
+  if (M == 0) return EB_OK;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
   return cuda_status(
       launch_loads(hist, M, E, D, expert_rank, w, status_dev, (cudaStream_t)stream));
 }
@@ -646,8 +676,21 @@ eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int
   if (policy == EB_SCHED_MAXUTIL && maxutil_candidates(__builtin_popcount(pending_mask), m) >
                                         kMaxUtilCandidateCap)
     return EB_ERR_UNSUPPORTED;
-  return cuda_status(launch_schedule_once(w, pending_mask, M, D, m, policy, runset_mask,
-                                          (long long*)step_stats, (cudaStream_t)stream));
+  if (cuda_error_pending()) return EB_ERR_CUDA;
+  cudaStream_t s = (cudaStream_t)stream;
+  // a large MaxUtil search runs on a grid whose per-CTA results need a few KB
+  // of scratch: stream-ordered, freed on the same stream
+  void* slots = nullptr;
+  if (policy == EB_SCHED_MAXUTIL && maxutil_uses_grid(__builtin_popcount(pending_mask), m) &&
+      cudaMallocAsync(&slots, kSearchCtas * kSearchSlotBytes, s) != cudaSuccess)
+    return EB_ERR_CUDA;
+  cudaError_t e = launch_schedule_once(w, pending_mask, M, D, m, policy, runset_mask,
+                                       (long long*)step_stats, slots, s);
+  if (slots) {
+    const cudaError_t f = cudaFreeAsync(slots, s);
+    if (e == cudaSuccess) e = f;
+  }
+  return cuda_status(e);
 }
 
 }  // extern "C"

@@ -26,10 +26,6 @@ constexpr int kChunk = 64;
 #endif
 constexpr int kTcRows1 = EB_TC_ROWS1;
 constexpr int kTcRows2 = EB_TC_ROWS2;
-// Two-SM tiles: 256 features x kTc2Rows tokens per CTA pair.
-constexpr int kTc2Rows1 = 128;
-constexpr int kTc2Rows2 = 256;
-constexpr int kTc2Feat = 256;
 constexpr int kTcFeat = 128;
 // Token-major tiles: 128 tokens x (128 gate/up features | 256 down features).
 constexpr int kTmRows = 128;
@@ -103,6 +99,8 @@ struct CtxDev {
   int use_emap;         // 0: contiguous map, experts [d E/D, (d+1) E/D) on rank d
   int32_t* arrive;      // [M*T][H/256]: fused-combine arrival counts (engine TMC), else null
   size_t arrive_bytes;
+  void* search_slots;   // [kSearchCtas] MaxUtil search results (MaxUtil with a large
+                        // candidate count), else null
 };
 
 // ---- programmatic dependent launch ----
@@ -148,6 +146,13 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// A launch error that something else left pending is not this library's:
+// every entry point checks cudaPeekAtLastError() right before its first
+// launch and, if an error is pending, returns EB_ERR_CUDA without launching
+// and without clearing it.  The cudaGetLastError() after its own launches
+// then reports only errors of those launches.
+inline bool cuda_error_pending() { return cudaPeekAtLastError() != cudaSuccess; }
+
 // ---- launchers (all asynchronous on `s`) ----
 // Micro-batch j's rows at layer l start at logits + j * mb_stride + l *
 // layer_stride (elements): (L T E, T E) for the caller's [M, L, T, E] logits,
@@ -157,17 +162,23 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
                               float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
 // rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm1 / fm2:
-// output features per item.
+// output features per item.  With c.search_slots set, the MaxUtil search
+// grid runs first (two launches).
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
                                  int fm1, int fm2, cudaStream_t s);
+// slots: kSearchCtas * kSearchSlotBytes of device scratch for the MaxUtil
+// search grid, or null to search in the scheduler's CTA.
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
-                                 int policy, uint32_t* runset, long long* stats, cudaStream_t s);
+                                 int policy, uint32_t* runset, long long* stats, void* slots,
+                                 cudaStream_t s);
 // expert_rank: device [E] placement, or nullptr for the contiguous map;
 // status (device, may be nullptr) gets EB_ERR_INVALID_ARG for a rank outside
 // [0, D) (that expert's count is then dropped).
 cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t* expert_rank,
                          int32_t* w, int32_t* status, cudaStream_t s);
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s);
+// Records `status` in the step state's status word (stream-ordered).
+cudaError_t launch_set_status(State* st, int status, cudaStream_t s);
 // Rows of every (token, slot) of the RunSet (pos) and the (token, slot) of
 // every row (rowslot).
 cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s);
@@ -184,5 +195,11 @@ cudaError_t launch_gemm_simt(const Dims& d, const CtxDev& c, const Work& w, cons
 // count a single step may need (sum_{c <= M-m} C(M, c)).
 constexpr unsigned long long kMaxUtilCandidateCap = 1ull << 25;
 unsigned long long maxutil_candidates(int n, int m);
+// Above a candidate count that one CTA searches quickly, MaxUtil runs a
+// search grid of kSearchCtas CTAs first; each leaves its best candidate in
+// a slot of kSearchSlotBytes bytes, which the scheduler then reduces.
+constexpr int kSearchCtas = 296;
+constexpr size_t kSearchSlotBytes = 24;
+bool maxutil_uses_grid(int n, int m);
 
 }  // namespace eb

@@ -160,9 +160,9 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// 32 lanes x 32 columns of 32-bit accumulator -> 32 registers per thread.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-  uint32_t r[32];
+// 32 lanes x 32 columns of 32-bit accumulator -> 32 registers per thread,
+// issued without waiting (tmem_wait() makes the registers valid).
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
       "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
@@ -174,9 +174,32 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
       : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+  uint32_t r[32];
+  tmem_ld32_issue(taddr, r);
+  tmem_wait();
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Two 32-column loads in flight together, one wait.
+__device__ __forceinline__ void tmem_ld32x2(uint32_t taddr0, uint32_t taddr1, float* v0,
+                                            float* v1) {
+  uint32_t r0[32], r1[32];
+  tmem_ld32_issue(taddr0, r0);
+  tmem_ld32_issue(taddr1, r1);
+  tmem_wait();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    v0[i] = __uint_as_float(r0[i]);
+    v1[i] = __uint_as_float(r1[i]);
+  }
 }
 
 __device__ __forceinline__ int find_segment(const int32_t* items, int nseg, int item) {
@@ -466,326 +489,6 @@ __global__ void k_selftest_wait(unsigned long long limit_ns, int* status) {
   __syncthreads();
   if (threadIdx.x == 0 && mbar_wait(smem_u32(&bar), 0, &abort_flag, status, limit_ns))
     atomicExch(status, EB_OK);  // not reached: nothing arrives on the barrier
-}
-
-
-// ---------------------------------------------------------------------------
-// Two-SM variant (tcgen05 cta_group::2).  A cluster of two CTAs on an SM pair
-// computes one 256-feature x N-token tile: CTA r holds weight rows
-// [f0 + 128 r, f0 + 128 r + 128) and token rows [r0 + r N/2, r0 + (r+1) N/2)
-// of the operands, the leader CTA (rank 0) issues the M = 256 MMAs, and each
-// CTA's TMEM receives its 128 feature rows x all N tokens.  Each SM therefore
-// fetches only half of the token tile: per output, 1.2x (gate/up) to 1.5x
-// (down) fewer bytes cross L2 -> SM than the one-SM kernel.
-//
-// Barriers: the leader arms its full barrier with both CTAs' bytes and both
-// CTAs' TMA loads complete on it; the leader's commits arrive on the empty
-// and accumulator-full barriers of both CTAs (multicast commit); each CTA's
-// drain warps arrive on the leader's accumulator-empty barrier.
-// ---------------------------------------------------------------------------
-
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t cluster_id() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ uint32_t num_clusters() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
-  return r;
-}
-// Address of the same shared-memory location in CTA `rank` of the cluster.
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
-  uint32_t out;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
-  return out;
-}
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
-               : "memory");
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-// TMA load into this CTA's shared memory whose completion is counted on the
-// leader CTA's barrier (bar = that barrier's shared::cluster address).
-__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
-                                                 uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-__device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t a, uint64_t b,
-                                              uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-      "l"(a), "l"(b), "r"(idesc), "r"(accumulate));
-}
-// Arrives on the barrier at this shared-memory offset in both CTAs of the pair
-// once the leader's earlier MMAs have completed.
-__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
-  const uint16_t mask = 0x3;
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
-      " [%0], %1;" ::"r"(bar),
-      "h"(mask)
-      : "memory");
-}
-
-template <bool GATEUP>
-struct Cfg2 {
-  static constexpr int kBN = GATEUP ? kTc2Rows1 : kTc2Rows2;  // token rows per pair item
-  static constexpr int kBNc = kBN / 2;                         // token rows per CTA
-  static constexpr int kXBytes = kBNc * kBK * 2;
-  static constexpr int kStageBytes = (GATEUP ? 2 : 1) * kTileBytes + kXBytes;  // per CTA
-  static constexpr int kStages = (204800 / kStageBytes) < 8 ? (204800 / kStageBytes) : 8;
-  static constexpr int kAccCols = (GATEUP ? 2 : 1) * kBN;
-  static constexpr int kAccBufs = 2 * kAccCols <= 512 ? 2 : 1;
-  static constexpr int kTmemCols = kAccBufs * kAccCols;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + 1024;
-};
-
-// One pair item: (segment, 256-feature block, chunk of kBN tokens).
-template <bool GATEUP>
-__device__ __forceinline__ Item decode2(const Dims& d, const int32_t* seg_rows,
-                                        const int32_t* seg_wid, const int32_t* seg_items, int nseg,
-                                        int item) {
-  constexpr int kBN = Cfg2<GATEUP>::kBN;
-  const int s = find_segment(seg_items, nseg, item);
-  const int local = item - seg_items[s];
-  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
-  const int nch = (cnt + kBN - 1) / kBN;
-  const int chunk = local % nch, mb = local / nch;
-  Item it;
-  it.r0 = rb + chunk * kBN;
-  it.n = min(kBN, cnt - chunk * kBN);
-  it.f0 = mb * 256;
-  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
-  return it;
-}
-
-template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tc2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
-               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-               const int32_t* __restrict__ rowslot, __nv_bfloat16* __restrict__ out) {
-  pdl_enter();
-  using C = Cfg2<GATEUP>;
-  constexpr int kBN = C::kBN;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* full = bars;                    // [kStages], used in the leader
-  uint64_t* empty = bars + C::kStages;      // [kStages]
-  uint64_t* tfull = bars + 2 * C::kStages;  // [2]
-  uint64_t* tempty = tfull + 2;             // [2], used in the leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const bool leader = rank == 0;
-  const int pair = (int)cluster_id(), npairs = (int)num_clusters();
-  const int nseg = st->nseg;
-  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
-  if (total == 0) return;  // both CTAs of a pair read the same value
-  const int K = GATEUP ? d.H : d.F;
-  const int nk = K / kBK;
-  const int NOUT = GATEUP ? d.F : d.H;
-  constexpr uint32_t kTxBytes = 2u * (uint32_t)C::kStageBytes;  // both CTAs' loads
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 2 * kEpiWarps);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"((uint32_t)C::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-  }
-  tc_fence_before();
-  cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_par = 0;
-      bool ok = true;
-      for (int item = pair; item < total && ok; item += npairs) {
-        const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
-        const int N = ((it.n + 15) / 16) * 16;
-        const int wrow = it.wrow + (int)rank * 128;
-        const int xrow = it.r0 + (int)rank * (N / 2);
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = stage_base + stage * C::kStageBytes;
-          const uint32_t fb_local = smem_u32(&full[stage]);
-          const uint32_t fb = map_to_rank(fb_local, 0);
-          if (leader) {
-            mbar_expect_tx(fb_local, kTxBytes);
-            armed |= 1u << stage;
-            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          }
-          tma_load_2d_pair(smem_u32(sb), &map_w, kb * kBK, wrow, fb);
-          if (GATEUP) tma_load_2d_pair(smem_u32(sb + kTileBytes), &map_w, kb * kBK, wrow + d.F, fb);
-          tma_load_2d_pair(smem_u32(sb + (GATEUP ? 2 : 1) * kTileBytes), &map_x, kb * kBK, xrow, fb);
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      if (!ok && leader) {  // the leader's barriers count both CTAs' copies
-        for (int s2 = 0; s2 < C::kStages; ++s2)
-          if ((armed >> s2) & 1u) {
-            const unsigned long long t0 = global_ns();
-            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
-                   global_ns() - t0 < kWaitLimitNs) {
-            }
-          }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      uint32_t last_bar = 0, last_par = 0;
-      bool ok = true, issued = false;
-      for (int item = pair; item < total && ok; item += npairs) {
-        const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
-        const int N = ((it.n + 15) / 16) * 16;
-        const uint32_t idesc = idesc_bf16(256, N);
-        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t d_gate = tmem + acc * C::kAccCols;
-        const uint32_t d_up = d_gate + kBN;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sb = smem_u32(stage_base + stage * C::kStageBytes);
-          const uint32_t sx = sb + (GATEUP ? 2 : 1) * kTileBytes;
-#pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks) {
-            const uint32_t koff = ks * 32;
-            const uint32_t acc_flag = (kb | ks) != 0;
-            mma_bf16_pair(d_gate, sdesc(sb + koff), sdesc(sx + koff), idesc, acc_flag);
-            if (GATEUP)
-              mma_bf16_pair(d_up, sdesc(sb + kTileBytes + koff), sdesc(sx + koff), idesc, acc_flag);
-          }
-          mma_commit_pair(smem_u32(&empty[stage]));
-          last_bar = smem_u32(&empty[stage]);
-          last_par = phase;
-          issued = true;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-        if (!ok) break;
-        mma_commit_pair(smem_u32(&tfull[acc]));
-        last_bar = smem_u32(&tfull[acc]);
-        last_par = acc_phase;
-        if (++acc == C::kAccBufs) {
-          acc = 0;
-          acc_phase ^= 1;
-        }
-      }
-      if (!ok && issued) {
-        const unsigned long long t0 = global_ns();
-        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ drain (both CTAs)
-    const int q = warp & 3;
-    const int frow = q * 32 + lane;
-    const int cgrp = (warp - 2) >> 2;
-    constexpr int kColStep = 32 * (kEpiWarps / 4);
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int item = pair; item < total; item += npairs) {
-      const Item it = decode2<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
-      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
-      tc_fence_after();
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      __nv_bfloat16* orow = out + (size_t)it.r0 * NOUT + it.f0 + (int)rank * 128 + frow;
-      for (int cb = cgrp * 32; cb < it.n; cb += kColStep) {
-        float g[32];
-        tmem_ld32(tbase + cb, g);
-        if (GATEUP) {
-          float u[32];
-          tmem_ld32(tbase + kBN + cb, u);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            if (cb + i < it.n) {
-              const float a = g[i] / (1.f + expf(-g[i])) * u[i];
-              orow[(size_t)(cb + i) * NOUT] = __float2bfloat16_rn(a);
-            }
-          }
-        } else {  // y rows at their (token, slot) positions
-#pragma unroll
-          for (int i = 0; i < 32; ++i)
-            if (cb + i < it.n)
-              out[(size_t)__ldg(rowslot + it.r0 + cb + i) * NOUT + (orow - out) % NOUT] =
-                  __float2bfloat16_rn(g[i]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
-      if (++acc == C::kAccBufs) {
-        acc = 0;
-        acc_phase ^= 1;
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // neither CTA leaves while the pair's MMAs or signals may touch it
-  tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"((uint32_t)C::kTmemCols));
-  }
 }
 
 
@@ -1235,11 +938,10 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
       const int b_end = q * 32 < it.n ? kBlocks : 0;
       for (int b = cgrp; b < b_end; b += kGroups) {
         float g[32];
-        tmem_ld32(tbase + b * 32, g);
         uint32_t packed[16];
         if (GATEUP) {
           float uu[32];
-          tmem_ld32(tbase + 128 + b * 32, uu);
+          tmem_ld32x2(tbase + b * 32, tbase + 128 + b * 32, g, uu);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float a0 = g[2 * i] / (1.f + expf(-g[2 * i])) * uu[2 * i];
@@ -1247,6 +949,7 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
             packed[i] = pack_bf16x2(a0, a1);
           }
         } else {
+          tmem_ld32(tbase + b * 32, g);
 #pragma unroll
           for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
         }
@@ -1298,323 +1001,6 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
   }
 }
 
-
-// ---------------------------------------------------------------------------
-// Two-SM token-major variant (cta_group::2).  A CTA pair computes one chunk
-// of up to 256 tokens against 256 weight rows.  The weight tile is split
-// between the pair's shared memories (B operand halves), so each SM loads
-// half of it; the chunk's tokens are split too (A operand halves):
-//  - more than 128 tokens: an M = 256 MMA, 128 tokens per CTA;
-//  - up to 128 tokens: an M = 128 MMA, 64 tokens per CTA.
-// Both shapes run at the tensor pipe's full rate, so a small segment costs a
-// pair no more SM time than the one-SM engine and half the shared-memory
-// bytes per SM.
-//
-// B half of CTA r: GEMM 1: gate rows f0 + 64 r .. + 63 then the matching up
-// rows (two 64-row boxes); GEMM 2: output rows f0 + 128 r .. + 127.  With this
-// order every accumulator lane holds the gate and up values of the same
-// features side by side (SwiGLU stays in one thread), for both MMA shapes:
-//  - M = 256: lane l is token 128 r + l; columns [128 G, 128 G + 64) are the
-//    gate and [128 G + 64, 128 G + 128) the up values of features
-//    f0 + 64 G .. (GEMM 1, G = 0, 1); columns 0..255 are features f0..f0+255
-//    (GEMM 2).
-//  - M = 128: lane l < 64 is token 64 r + l with columns 0..127 = the pair's
-//    N columns 0..127; lane 64 + l is the same token with N columns 128..255.
-// ---------------------------------------------------------------------------
-
-template <bool GATEUP>
-struct CfgTM2 {
-  static constexpr int kRows = 2 * kTmRows;          // token rows per pair item (at most)
-  static constexpr int kFeat = GATEUP ? kTmFeat1 : kTmFeat2;
-  static constexpr int kABytes = kTmRows * kBK * 2;  // 16 KiB: this CTA's tokens (at most)
-  static constexpr int kBBytes = 128 * kBK * 2;      // 16 KiB: this CTA's weight rows
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = 196608 / kStageBytes;  // 6
-  static constexpr int kAccCols = 256;
-  static constexpr int kAccBufs = 2;
-  static constexpr int kTmemCols = kAccBufs * kAccCols;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kSegCacheBytes + 1024;
-};
-
-template <bool GATEUP>
-__device__ __forceinline__ Item decode_tm2(const Dims& d, const int32_t* seg_rows,
-                                           const int32_t* seg_wid, const int32_t* seg_items,
-                                           int nseg, int item) {
-  using C = CfgTM2<GATEUP>;
-  const int s = find_segment(seg_items, nseg, item);
-  const int local = item - seg_items[s];
-  const int rb = seg_rows[s], cnt = seg_rows[s + 1] - rb;
-  const int nch = (cnt + C::kRows - 1) / C::kRows;
-  const int chunk = local % nch, mb = local / nch;
-  Item it;
-  it.r0 = rb + chunk * C::kRows;
-  it.n = min(C::kRows, cnt - chunk * C::kRows);
-  it.f0 = mb * C::kFeat;
-  it.wrow = seg_wid[s] * (GATEUP ? 2 * d.F : d.H) + it.f0;
-  return it;
-}
-
-// Tokens of a pair item held by CTA `rank`, and where they start in the item.
-__device__ __forceinline__ void pair_split(int n, uint32_t rank, int* first, int* count) {
-  const int per = n > kTmRows ? kTmRows : kTmRows / 2;  // tokens per CTA: M / 2
-  *first = (int)rank * per;
-  *count = min(max(n - *first, 0), per);
-}
-
-// map_w: GATEUP w_gateup in boxes of 64 rows, else w_down in boxes of 128
-// rows; map_x: token rows in boxes of 32 rows.
-template <bool GATEUP>
-__global__ void __launch_bounds__(kThreads, 1)
-    k_gemm_tm2(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
-               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
-               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
-               const int32_t* __restrict__ rowslot, __nv_bfloat16* __restrict__ out) {
-  pdl_enter();
-  using C = CfgTM2<GATEUP>;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
-  uint8_t* stage_base = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kStages * C::kStageBytes);
-  uint64_t* full = bars;                    // [kStages], used in the leader
-  uint64_t* empty = bars + C::kStages;      // [kStages]
-  uint64_t* tfull = bars + 2 * C::kStages;  // [2]
-  uint64_t* tempty = tfull + 2;             // [2], used in the leader
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  uint8_t* seg_buf = reinterpret_cast<uint8_t*>(bars) + 1024;
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_rank();
-  const bool leader = rank == 0;
-  const int pair = (int)cluster_id(), npairs = (int)num_clusters();
-  const int nseg = st->nseg;
-  const int total = (nseg > 0 && st->runset != 0) ? seg_items[nseg] : 0;
-  if (total == 0) return;  // both CTAs of a pair read the same value
-  const int K = GATEUP ? d.H : d.F;
-  const int nk = K / kBK;
-  const int NOUT = GATEUP ? d.F : d.H;
-
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
-      mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&tfull[i]), 1);
-      mbar_init(smem_u32(&tempty[i]), 2 * kEpiWarps);
-    }
-    *abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  const SegView sv = cache_segments(seg_buf, nseg, seg_rows, seg_wid, seg_items);
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"((uint32_t)C::kTmemCols));
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
-  }
-  tc_fence_before();
-  cluster_sync_all();  // both CTAs' barriers exist before anyone signals them
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer (both CTAs)
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t armed = 0, armed_par = 0;
-      bool ok = true;
-      Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, pair < total ? pair : 0);
-      for (int item = pair; item < total && ok; item += npairs) {
-        int first0, cnt0, first1, cnt1, first, cnt;
-        pair_split(it.n, 0, &first0, &cnt0);
-        pair_split(it.n, 1, &first1, &cnt1);
-        pair_split(it.n, rank, &first, &cnt);
-        const int nbox = (cnt + kTmBox - 1) / kTmBox;
-        const uint32_t tx = (uint32_t)(((cnt0 + kTmBox - 1) / kTmBox + (cnt1 + kTmBox - 1) / kTmBox) *
-                                           kTmBoxBytes +
-                                       2 * C::kBBytes);
-        const int xrow = it.r0 + first;
-        // this CTA's B half (see the layout note above)
-        const int w0 = GATEUP ? it.wrow + 64 * (int)rank : it.wrow + 128 * (int)rank;
-        const int w1 = it.wrow + d.F + 64 * (int)rank;  // GATEUP only: the up rows
-        const int next = item + npairs;
-        Item nx = it;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sb = stage_base + stage * C::kStageBytes;
-          const uint32_t fb_local = smem_u32(&full[stage]);
-          const uint32_t fb = map_to_rank(fb_local, 0);
-          if (leader) {
-            mbar_expect_tx(fb_local, tx);
-            armed |= 1u << stage;
-            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
-          }
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d_pair(smem_u32(sb + b * kTmBoxBytes), &map_x, kb * kBK, xrow + b * kTmBox, fb);
-          if (GATEUP) {
-            tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
-            tma_load_2d_pair(smem_u32(sb + C::kABytes + C::kBBytes / 2), &map_w, kb * kBK, w1, fb);
-          } else {
-            tma_load_2d_pair(smem_u32(sb + C::kABytes), &map_w, kb * kBK, w0, fb);
-          }
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-          // decode the next item while this item's copies are in flight
-          if (kb == 0 && next < total) nx = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, next);
-        }
-        it = nx;
-      }
-      if (!ok && leader) {  // the leader's barriers count both CTAs' copies
-        for (int s2 = 0; s2 < C::kStages; ++s2)
-          if ((armed >> s2) & 1u) {
-            const unsigned long long t0 = global_ns();
-            while (!mbar_try(smem_u32(&full[s2]), (armed_par >> s2) & 1u) &&
-                   global_ns() - t0 < kWaitLimitNs) {
-            }
-          }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader)
-    if (lane == 0 && leader) {
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
-      uint32_t last_bar = 0, last_par = 0;
-      bool ok = true, issued = false;
-      Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, pair < total ? pair : 0);
-      for (int item = pair; item < total && ok; item += npairs) {
-        const uint32_t idesc = idesc_bf16(it.n > kTmRows ? 256 : 128, 256);
-        const int next = item + npairs;
-        Item nx = it;
-        if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1, abort_flag, &st->status)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t dcol = tmem + acc * C::kAccCols;
-        for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag, &st->status)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t sa = smem_u32(stage_base + stage * C::kStageBytes);
-          const uint32_t sb = sa + C::kABytes;
-#pragma unroll
-          for (int ks = 0; ks < kBK / 16; ++ks) {
-            const uint32_t koff = ks * 32;
-            mma_bf16_pair(dcol, sdesc(sa + koff), sdesc(sb + koff), idesc, (kb | ks) != 0);
-          }
-          mma_commit_pair(smem_u32(&empty[stage]));
-          last_bar = smem_u32(&empty[stage]);
-          last_par = phase;
-          issued = true;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-          if (kb == 0 && next < total) nx = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, next);
-        }
-        if (!ok) break;
-        mma_commit_pair(smem_u32(&tfull[acc]));
-        last_bar = smem_u32(&tfull[acc]);
-        last_par = acc_phase;
-        if (++acc == C::kAccBufs) {
-          acc = 0;
-          acc_phase ^= 1;
-        }
-        it = nx;
-      }
-      if (!ok && issued) {
-        const unsigned long long t0 = global_ns();
-        while (!mbar_try(last_bar, last_par) && global_ns() - t0 < kWaitLimitNs) {
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------ drain (both CTAs)
-    // warp w reads TMEM lanes 32 (w % 4) .. +31; the two warps sharing a lane
-    // quarter split its 32-feature blocks.
-    const int q = warp & 3;
-    const int cgrp = (warp - 2) >> 2;
-    constexpr int kGroups = kEpiWarps / 4;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int item = pair; item < total; item += npairs) {
-      const Item it = decode_tm2<GATEUP>(d, sv.rows, sv.wid, sv.items, nseg, item);
-      if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag, &st->status)) break;
-      tc_fence_after();
-      int first, cnt;
-      pair_split(it.n, rank, &first, &cnt);
-      const bool wide = it.n > kTmRows;  // M = 256
-      // token of this lane within the CTA's share, the features it holds and
-      // the 32-feature blocks that cover them
-      const int tok = wide ? q * 32 + lane : (q & 1) * 32 + lane;
-      const bool live = tok < cnt;
-      const int fbase = wide ? 0 : (q >> 1) * (C::kFeat / 2);
-      const int nblk = (wide ? C::kFeat : C::kFeat / 2) / 32;
-      const uint32_t tbase = tmem + ((uint32_t)(q * 32) << 16) + acc * C::kAccCols;
-      const int orow_idx =
-          GATEUP ? it.r0 + first + tok : (live ? __ldg(rowslot + it.r0 + first + tok) : 0);
-      __nv_bfloat16* orow = out + (size_t)orow_idx * NOUT + it.f0 + fbase;
-      // a lane quarter whose tokens are all past the share has nothing to drain
-      const int b_end = ((wide ? q * 32 : (q & 1) * 32) < cnt) ? nblk : 0;
-      for (int b = cgrp; b < b_end; b += kGroups) {
-        float g[32];
-        uint32_t packed[16];
-        if (GATEUP) {
-          // features 64 G + 32 h of this lane's range: gate at column 128 G + 32 h,
-          // up 64 columns further
-          const int G = b >> 1, h = b & 1;
-          float u[32];
-          tmem_ld32(tbase + 128 * G + 32 * h, g);
-          tmem_ld32(tbase + 128 * G + 64 + 32 * h, u);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float a0 = g[2 * i] / (1.f + expf(-g[2 * i])) * u[2 * i];
-            const float a1 = g[2 * i + 1] / (1.f + expf(-g[2 * i + 1])) * u[2 * i + 1];
-            packed[i] = pack_bf16x2(a0, a1);
-          }
-        } else {
-          tmem_ld32(tbase + 32 * b, g);
-#pragma unroll
-          for (int i = 0; i < 16; ++i) packed[i] = pack_bf16x2(g[2 * i], g[2 * i + 1]);
-        }
-        if (live) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + b * 32);
-#pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(map_to_rank(smem_u32(&tempty[acc]), 0));
-      if (++acc == C::kAccBufs) {
-        acc = 0;
-        acc_phase ^= 1;
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  cluster_sync_all();  // neither CTA leaves while the pair's MMAs or signals may touch it
-  tc_fence_after();
-  if (warp == 1) {
-    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                 "r"((uint32_t)C::kTmemCols));
-  }
-}
 
 // ---------------------------------------------------------------------------
 // Router projection: scores = h W_r^T in float32 for the micro-batches that
@@ -1779,26 +1165,6 @@ __global__ void __launch_bounds__(kRouterThreads, 1)
   }
 }
 
-// CTA pairs of `kernel` that fit on the device at once (one CTA per SM; an
-// SM pair must sit in one GPC, so an odd SM count per GPC leaves SMs out).
-// Queried once per device and kernel.
-template <typename Kernel>
-int resident_pairs(Kernel kernel, cudaLaunchConfig_t cfg, int fallback) {
-  static std::atomic<int> cache[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fallback;
-  int n = cache[dev].load(std::memory_order_relaxed);
-  if (n > 0) return n;
-  cfg.gridDim = dim3(2 * (unsigned)fallback);
-  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
-    (void)cudaGetLastError();
-    n = fallback;
-  }
-  n = n < fallback ? n : fallback;
-  cache[dev].store(n, std::memory_order_relaxed);
-  return n;
-}
-
 }  // namespace
 
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, int* status, cudaStream_t s) {
@@ -1817,12 +1183,6 @@ cudaError_t gemm_tc_prepare() {
     e = cudaFuncSetAttribute(k_gemm_tc<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              Cfg<false>::kSmemBytes);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tc2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg2<true>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tc2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             Cfg2<false>::kSmemBytes);
-  if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_gemm_tm<true, false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              CfgTM<true>::kSmemBytes);
   if (e == cudaSuccess)
@@ -1837,41 +1197,7 @@ cudaError_t gemm_tc_prepare() {
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(k_router, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              kRouterSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm2<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CfgTM2<true>::kSmemBytes);
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(k_gemm_tm2<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             CfgTM2<false>::kSmemBytes);
   return e;
-}
-
-cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                            int grid, cudaStream_t s, int which) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  if (which == 1) {
-    cfg.dynamicSmemBytes = CfgTM2<true>::kSmemBytes;
-    cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<true>, cfg, grid / 2));
-    return cudaLaunchKernelEx(&cfg, k_gemm_tm2<true>, maps.w_gateup64, maps.A32, d, c.st, w.seg_rows,
-                              w.seg_wid, w.seg_items1, (const int32_t*)w.rowslot,
-                              static_cast<__nv_bfloat16*>(w.act));
-  }
-  cfg.dynamicSmemBytes = CfgTM2<false>::kSmemBytes;
-  cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tm2<false>, cfg, grid / 2));
-  return cudaLaunchKernelEx(&cfg, k_gemm_tm2<false>, maps.w_down, maps.act32, d, c.st, w.seg_rows,
-                            w.seg_wid, w.seg_items2, (const int32_t*)w.rowslot,
-                            static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -1915,34 +1241,6 @@ cudaError_t launch_router(const CUtensorMap& map_h, const CUtensorMap& map_r, in
   return launch_pdl(k_router, dim3((T + 127) / 128, n_mb), dim3(kRouterThreads),
                     (size_t)kRouterSmemBytes, s, 1, map_h, map_r, T, H, E, st, out, mb_stride,
                     layer_stride, status);
-}
-
-cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                            int grid, cudaStream_t s, int which) {
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.blockDim = dim3(kThreads);
-  cfg.stream = s;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  if (which == 1) {
-    cfg.dynamicSmemBytes = Cfg2<true>::kSmemBytes;
-    cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<true>, cfg, grid / 2));
-    return cudaLaunchKernelEx(&cfg, k_gemm_tc2<true>, maps.w_gateup, maps.A2, d, c.st, w.seg_rows,
-                              w.seg_wid, w.seg_items1, (const int32_t*)w.rowslot,
-                              static_cast<__nv_bfloat16*>(w.act));
-  }
-  cfg.dynamicSmemBytes = Cfg2<false>::kSmemBytes;
-  cfg.gridDim = dim3(2 * (unsigned)resident_pairs(k_gemm_tc2<false>, cfg, grid / 2));
-  return cudaLaunchKernelEx(&cfg, k_gemm_tc2<false>, maps.w_down, maps.act2, d, c.st, w.seg_rows,
-                            w.seg_wid, w.seg_items2, (const int32_t*)w.rowslot,
-                            static_cast<__nv_bfloat16*>(w.y));
 }
 
 cudaError_t launch_gemm_tc(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
@@ -2006,9 +1304,6 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
   if (e == cudaSuccess) e = encode(&maps->w_down, w_down, experts * d.H, d.F, kBM);
   if (e == cudaSuccess) e = encode(&maps->A, w.A, (unsigned long long)w.Rcap, d.H, kTcRows1);
   if (e == cudaSuccess) e = encode(&maps->act, w.act, (unsigned long long)w.Rcap, d.F, kTcRows2);
-  if (e == cudaSuccess) e = encode(&maps->A2, w.A, (unsigned long long)w.Rcap, d.H, kTc2Rows1 / 2);
-  if (e == cudaSuccess) e = encode(&maps->act2, w.act, (unsigned long long)w.Rcap, d.F, kTc2Rows2 / 2);
-  if (e == cudaSuccess) e = encode(&maps->w_gateup64, w_gateup, experts * 2 * d.F, d.H, 64);
   if (e == cudaSuccess) e = encode(&maps->A32, w.A, (unsigned long long)w.Rcap, d.H, kTmBox);
   if (e == cudaSuccess) e = encode(&maps->act32, w.act, (unsigned long long)w.Rcap, d.F, kTmBox);
   return e;

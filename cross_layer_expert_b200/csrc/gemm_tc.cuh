@@ -14,9 +14,6 @@ struct TcMaps {
   CUtensorMap w_down;    // [L*Etot*H rows, F cols]
   CUtensorMap A;         // [Rcap rows, H cols]
   CUtensorMap act;       // [Rcap rows, F cols]
-  CUtensorMap A2;        // same buffers, boxes of half a pair's token tile
-  CUtensorMap act2;
-  CUtensorMap w_gateup64;  // w_gateup in boxes of 64 rows (two-SM token-major engine)
   CUtensorMap A32;       // same buffers, boxes of 32 rows (token-major engines)
   CUtensorMap act32;
 };
@@ -28,10 +25,6 @@ cudaError_t make_tc_maps(const Dims& d, const Work& w, const void* w_gateup, con
 // Opts the kernels into their dynamic shared memory (once per device).
 cudaError_t gemm_tc_prepare();
 int gemm_tc_smem_bytes(bool gateup);
-// Two-SM (cta_group::2) version of launch_gemm_tc: clusters of two CTAs, one
-// per SM pair; each item covers 256 output features.
-cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                            int grid, cudaStream_t s, int which);
 // Token-major engine: 128 token rows x 256 weight rows per MMA (GEMM 1: 128
 // features of gate and up; GEMM 2: 256 features).
 // x_rows (GEMM 1 only, may be null): the hidden states [M*T, H]; when given,
@@ -44,11 +37,6 @@ cudaError_t launch_gemm_tc2(const Dims& d, const CtxDev& c, const Work& w, const
 cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
                            int grid, cudaStream_t s, int which, const void* x_rows,
                            void* combine_into);
-// Two-SM token-major engine (cta_group::2): a CTA pair computes a chunk of up
-// to 256 tokens against 256 weight rows; each CTA holds half the tokens and
-// half the weight rows (M = 256 MMAs above 128 tokens, M = 128 below).
-cudaError_t launch_gemm_tm2(const Dims& d, const CtxDev& c, const Work& w, const TcMaps& maps,
-                            int grid, cudaStream_t s, int which);
 // Router projection (float32 scores = h W_r^T): maps of the hidden rows
 // [rows, H] (boxes of 128 rows) and of the routers [layers * E, H] (boxes of
 // E rows), and the launch: n_mb blocks of T rows; st == nullptr routes one

@@ -15,7 +15,12 @@
 // MaxUtil enumerates the complements C of the pending set P with
 // |C| <= |P| - m (so every candidate S = P \ C has |S| >= m): the threads
 // split the candidate ranks, unrank a first complement in colexicographic
-// order and walk on with Gosper's next-combination step.
+// order and walk on with Gosper's next-combination step.  Up to
+// kBlockSearchMax candidates the scheduler's own CTA searches them; above
+// that a grid of kSearchCtas CTAs (k_maxutil_search) each searches a
+// contiguous rank range and leaves its best candidate in a slot, and the
+// scheduler reduces the slots.  The order on candidates is total, so the
+// split never changes the RunSet.
 #include "eb_internal.cuh"
 
 namespace eb {
@@ -36,12 +41,20 @@ struct BinomTable {
 };
 __constant__ BinomTable kBinom = BinomTable();
 
+// A MaxUtil candidate S = P \ C: (sum_d W_d, max_d W_d, |S|, C as a mask over
+// positions in P).  size < 0 marks "no candidate".
 struct Cand {
   long long sum, mx;
   int size;
-  uint32_t mask;
+  uint32_t cmask;
 };
 
+static_assert(sizeof(Cand) == kSearchSlotBytes, "search slot layout");
+
+// Higher U first, then the larger set, then the smaller bitmask of
+// micro-batch ids.  P lists ids in ascending order and C is a subset of P,
+// so the RunSet's id mask is smaller exactly when its complement's position
+// mask is larger.
 __device__ __forceinline__ bool cand_better(const Cand& a, const Cand& b) {
   if (a.mx == 0 || b.mx == 0) {
     if (a.mx != b.mx) return a.mx != 0;  // a set with work beats one without
@@ -50,12 +63,24 @@ __device__ __forceinline__ bool cand_better(const Cand& a, const Cand& b) {
     if (l != r) return l > r;
   }
   if (a.size != b.size) return a.size > b.size;
-  return a.mask < b.mask;
+  return a.cmask > b.cmask;
 }
+
+// a beats b, where either may be "no candidate"
+__device__ __forceinline__ bool cand_wins(const Cand& a, const Cand& b) {
+  return a.size >= 0 && (b.size < 0 || cand_better(a, b));
+}
+
+// Row stride of the load rows in shared memory: odd, so threads reading the
+// same rank of different micro-batches' rows hit different banks.
+constexpr int kWStride = EB_MAX_D + 1;
+
+// Candidate counts up to this are searched by the scheduler's own CTA.
+constexpr unsigned long long kBlockSearchMax = 32768;
 
 // Shared-memory workspace of the scheduler.
 struct SchedSmem {
-  int w[EB_MAX_M][EB_MAX_D];  // loads of pending micro-batches, by position in P
+  int w[EB_MAX_M][kWStride];  // loads of pending micro-batches, by position in P
   long long wsum[EB_MAX_M];
   long long tot[EB_MAX_D];
   long long totsum;
@@ -91,10 +116,23 @@ __device__ Cand eval_complement(const SchedSmem& sm, int D, uint32_t cm) {
     for (uint32_t b = cm; b; b &= b - 1) Wd -= sm.w[__ffs(b) - 1][dd];
     mx = Wd > mx ? Wd : mx;
   }
+  return Cand{sum, mx, sm.n - __popc(cm), cm};
+}
+
+// RunSet id mask of a candidate.
+__device__ uint32_t cand_runset(const SchedSmem& sm, const Cand& c) {
   uint32_t mask = 0;
   for (int i = 0; i < sm.n; ++i)
-    if (!((cm >> i) & 1u)) mask |= 1u << sm.P[i];
-  return Cand{sum, mx, sm.n - __popc(cm), mask};
+    if (!((c.cmask >> i) & 1u)) mask |= 1u << sm.P[i];
+  return mask;
+}
+
+// Number of MaxUtil candidates of n pending micro-batches: complements of
+// size 0 .. n - m.
+__device__ unsigned long long candidate_count(int n, int m) {
+  unsigned long long N = 0;
+  for (int c = 0; c <= n - m; ++c) N += kBinom.v[n][c];
+  return N;
 }
 
 __device__ Cand shfl_cand(const Cand& c, int off) {
@@ -102,21 +140,48 @@ __device__ Cand shfl_cand(const Cand& c, int off) {
   o.sum = __shfl_xor_sync(0xffffffffu, c.sum, off);
   o.mx = __shfl_xor_sync(0xffffffffu, c.mx, off);
   o.size = __shfl_xor_sync(0xffffffffu, c.size, off);
-  o.mask = __shfl_xor_sync(0xffffffffu, c.mask, off);
+  o.cmask = __shfl_xor_sync(0xffffffffu, c.cmask, off);
   return o;
 }
 
-// All threads of the block: MaxUtil over complements of size <= n - m.
-__device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
-  const int n = sm.n, cmax = n - m;
-  unsigned long long N = 0;
+// All threads of the block: the best of every thread's `best` (threads
+// without one pass size = -1).  Returns it to every thread.
+__device__ Cand block_best(Cand best, Cand* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int off = 16; off; off >>= 1) {
+    const Cand o = shfl_cand(best, off);
+    if (cand_wins(o, best)) best = o;
+  }
+  if (lane == 0) red[warp] = best;
+  __syncthreads();
+  if (warp == 0) {
+    best = lane < (int)(blockDim.x >> 5) ? red[lane] : Cand{0, 0, -1, 0};
+    for (int off = 16; off; off >>= 1) {
+      const Cand o = shfl_cand(best, off);
+      if (cand_wins(o, best)) best = o;
+    }
+    if (lane == 0) red[0] = best;
+  }
+  __syncthreads();
+  best = red[0];
+  __syncthreads();  // red may be reused
+  return best;
+}
+
+// This thread's best candidate over the complement ranks [r_lo, r_hi)
+// (sizes ascending, colexicographic order within a size), the range split
+// evenly over the block's threads.
+__device__ Cand search_ranks(const SchedSmem& sm, int D, int m, unsigned long long r_lo,
+                             unsigned long long r_hi) {
+  const int n = sm.n;
   const uint32_t (*B)[33] = kBinom.v;
-  for (int c = 0; c <= cmax; ++c) N += B[n][c];
+  const unsigned long long N = r_hi > r_lo ? r_hi - r_lo : 0;
   const unsigned long long per = (N + blockDim.x - 1) / blockDim.x;
-  unsigned long long r = per * threadIdx.x;
-  const unsigned long long r_end = r + per < N ? r + per : N;
-  Cand best{0, 0, -1, 0xffffffffu};
+  unsigned long long r = r_lo + per * threadIdx.x;
+  const unsigned long long r_end = r + per < r_hi ? r + per : r_hi;
+  Cand best{0, 0, -1, 0};
   bool have = false;
+  (void)m;
   if (r < r_end) {
     int c = 0;
     unsigned long long q = r;
@@ -140,24 +205,23 @@ __device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
       }
     }
   }
-  // block reduction; threads without candidates carry size = -1 (never wins)
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int off = 16; off; off >>= 1) {
-    const Cand o = shfl_cand(best, off);
-    if (o.size >= 0 && (best.size < 0 || cand_better(o, best))) best = o;
+  return best;
+}
+
+// All threads of the block: MaxUtil over all complements of size <= n - m.
+__device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
+  const Cand best = block_best(search_ranks(sm, D, m, 0, candidate_count(sm.n, m)), sm.red);
+  return cand_runset(sm, best);
+}
+
+// All threads of the block: the best of the search grid's slots.
+__device__ uint32_t maxutil_slots(SchedSmem& sm, const Cand* __restrict__ slots, int n_slots) {
+  Cand best{0, 0, -1, 0};
+  for (int i = threadIdx.x; i < n_slots; i += blockDim.x) {
+    const Cand c = slots[i];
+    if (cand_wins(c, best)) best = c;
   }
-  if (lane == 0) sm.red[warp] = best;
-  __syncthreads();
-  if (warp == 0) {
-    best = lane < (int)(blockDim.x >> 5) ? sm.red[lane] : Cand{0, 0, -1, 0xffffffffu};
-    for (int off = 16; off; off >>= 1) {
-      const Cand o = shfl_cand(best, off);
-      if (o.size >= 0 && (best.size < 0 || cand_better(o, best))) best = o;
-    }
-    if (lane == 0) sm.result = best.mask;
-  }
-  __syncthreads();
-  return sm.result;
+  return cand_runset(sm, block_best(best, sm.red));
 }
 
 // Thread 0 only: CumUtil (policy 0) or DiffPeak (policy 3), padded to m.
@@ -210,8 +274,9 @@ __device__ uint32_t scan_policy(const SchedSmem& sm, int D, int m, int policy) {
 }
 
 // All threads: loads w[j][:] of the pending set must be in sm.w (by position);
-// returns the RunSet mask (over micro-batch ids).
-__device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending) {
+// returns the RunSet mask (over micro-batch ids).  slots: the MaxUtil search
+// grid's results for this pending set (null: search here).
+__device__ void prepare_totals(SchedSmem& sm, int D) {
   const int tid = threadIdx.x;
   for (int dd = tid; dd < D; dd += blockDim.x) {
     long long t = 0;
@@ -230,9 +295,15 @@ __device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint3
     sm.totsum = ts;
   }
   __syncthreads();
+}
+
+__device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending,
+                                  const Cand* slots = nullptr) {
+  prepare_totals(sm, D);
   if (policy == EB_SCHED_LOCKSTEP || sm.n <= m) return pending;
-  if (policy == EB_SCHED_MAXUTIL) return maxutil_block(sm, D, m);
-  if (tid == 0) sm.result = scan_policy(sm, D, m, policy);
+  if (policy == EB_SCHED_MAXUTIL)
+    return slots ? maxutil_slots(sm, slots, kSearchCtas) : maxutil_block(sm, D, m);
+  if (threadIdx.x == 0) sm.result = scan_policy(sm, D, m, policy);
   __syncthreads();
   return sm.result;
 }
@@ -286,6 +357,45 @@ __device__ int3 block_exclusive_scan3(int3 v, int3* tmp /* >= 33 */) {
   return make_int3(w.x + incl.x - v.x, w.y + incl.y - v.y, w.z + incl.z - v.z);
 }
 
+constexpr int kSearchThreads = 512;
+
+// MaxUtil search grid: CTA b searches complement ranks [N b / G, N (b+1) / G)
+// of the pending set (N candidates, G = gridDim.x) and writes its best
+// candidate (or "none") to slots[b].  The pending set and loads are the
+// step state's (st != null; nothing is searched while a timed-out step
+// awaits a reset) or the caller's (pending_arg, w).
+__global__ void __launch_bounds__(kSearchThreads) k_maxutil_search(int M, int D, int m,
+                                                                   const State* __restrict__ st,
+                                                                   uint32_t pending_arg,
+                                                                   const int32_t* __restrict__ w,
+                                                                   Cand* __restrict__ slots) {
+  __shared__ SchedSmem sm;
+  pdl_enter();
+  const int tid = threadIdx.x;
+  if (tid == 0) {
+    const uint32_t pending =
+        st ? (st->status == EB_ERR_TIMEOUT ? 0u : st->pending) : pending_arg;
+    int n = 0;
+    for (int j = 0; j < M; ++j)
+      if ((pending >> j) & 1u) sm.P[n++] = j;
+    sm.n = n;
+  }
+  __syncthreads();
+  Cand best{0, 0, -1, 0};
+  if (sm.n > m) {
+    for (int i = tid; i < sm.n * D; i += blockDim.x) {
+      const int p = i / D, dd = i % D;
+      sm.w[p][dd] = w[sm.P[p] * D + dd];
+    }
+    __syncthreads();
+    prepare_totals(sm, D);
+    const unsigned long long N = candidate_count(sm.n, m), G = gridDim.x;
+    best = search_ranks(sm, D, m, N * blockIdx.x / G, N * (blockIdx.x + 1) / G);
+  }
+  best = block_best(best, sm.red);
+  if (tid == 0) slots[blockIdx.x] = best;
+}
+
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
                                                              int rn2, int fm1, int fm2) {
   __shared__ SchedSmem sm;
@@ -305,6 +415,24 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
     for (int i = tid; i < kStateWords; i += blockDim.x)
       reinterpret_cast<int*>(c.st)[i] = reinterpret_cast<const int*>(&ss)[i];
   };
+  // A context whose status word holds EB_ERR_TIMEOUT (a bounded wait of an
+  // earlier step expired, so its state may be partial) runs no further step
+  // until eb_reset: the step does nothing and reports S as empty.
+  if (ss.status == EB_ERR_TIMEOUT) {
+    if (tid == 0) {
+      st->pending = 0;
+      st->runset = 0;
+      st->n_run = 0;
+      st->need_route = 0;
+      st->nseg = 0;
+      st->items1 = 0;
+      st->items2 = 0;
+      st->rows = 0;
+      for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
+    }
+    write_back();
+    return;
+  }
   // 1. hist[j][:] and w[j][:] of the micro-batches routed for this step were
   //    accumulated by the routing kernel
   // 2. pending set
@@ -336,7 +464,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   }
   __syncthreads();
   // 3. RunSet
-  const uint32_t run = choose_runset(sm, d.D, d.m, d.policy, pending);
+  const uint32_t run = choose_runset(sm, d.D, d.m, d.policy, pending,
+                                     static_cast<const Cand*>(c.search_slots));
   // 4. accounting, trace and Algorithm 1 bookkeeping (thread 0)
   if (tid == 0) {
     long long sumW = 0, maxW = 0, summax = 0;
@@ -510,7 +639,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __res
                                                              uint32_t pending, int M, int D,
                                                              int m, int policy,
                                                              uint32_t* __restrict__ runset_out,
-                                                             long long* __restrict__ stats) {
+                                                             long long* __restrict__ stats,
+                                                             const Cand* __restrict__ slots) {
   __shared__ SchedSmem sm;
   const int tid = threadIdx.x;
   if (tid == 0) {
@@ -532,7 +662,7 @@ __global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __res
     sm.w[p][dd] = w[sm.P[p] * D + dd];
   }
   __syncthreads();
-  const uint32_t run = choose_runset(sm, D, m, policy, pending);
+  const uint32_t run = choose_runset(sm, D, m, policy, pending, slots);
   if (tid == 0) {
     *runset_out = run;
     if (stats) {
@@ -616,14 +746,30 @@ unsigned long long maxutil_candidates(int n, int m) {
   return total;
 }
 
+bool maxutil_uses_grid(int n, int m) { return maxutil_candidates(n, m) > kBlockSearchMax; }
+
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
                                  int fm1, int fm2, cudaStream_t s) {
+  if (c.search_slots) {
+    const cudaError_t e = launch_pdl(k_maxutil_search, dim3(kSearchCtas), dim3(kSearchThreads), 0,
+                                     s, 1, d.M, d.D, d.m, (const State*)c.st, 0u,
+                                     (const int32_t*)c.w, static_cast<Cand*>(c.search_slots));
+    if (e != cudaSuccess) return e;
+  }
   return launch_pdl(k_schedule_step, dim3(1), dim3(kThreads), 0, s, 1, d, c, w, rn1, rn2, fm1, fm2);
 }
 
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
-                                 int policy, uint32_t* runset, long long* stats, cudaStream_t s) {
-  k_schedule_once<<<1, kThreads, 0, s>>>(w, pending, M, D, m, policy, runset, stats);
+                                 int policy, uint32_t* runset, long long* stats, void* slots,
+                                 cudaStream_t s) {
+  if (slots) {
+    k_maxutil_search<<<kSearchCtas, kSearchThreads, 0, s>>>(M, D, m, nullptr, pending, w,
+                                                           static_cast<Cand*>(slots));
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  k_schedule_once<<<1, kThreads, 0, s>>>(w, pending, M, D, m, policy, runset, stats,
+                                         static_cast<const Cand*>(slots));
   return cudaGetLastError();
 }
 
@@ -633,6 +779,15 @@ cudaError_t launch_loads(const int32_t* hist, int M, int E, int D, const int32_t
   if (n == 0) return cudaSuccess;
   k_loads<<<(n + 255) / 256, 256, 0, s>>>(hist, M, E, D, expert_rank, w, status);
   return cudaGetLastError();
+}
+
+__global__ void k_set_status(State* st, int status) {
+  pdl_enter();
+  st->status = status;
+}
+
+cudaError_t launch_set_status(State* st, int status, cudaStream_t s) {
+  return launch_pdl(k_set_status, dim3(1), dim3(1), 0, s, 1, st, status);
 }
 
 cudaError_t launch_reset(const Dims& d, const CtxDev& c, cudaStream_t s) {

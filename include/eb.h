@@ -18,7 +18,11 @@
  *     and returned as a negative eb_status; nothing runs in that case.
  *   - Errors the device detects (a non-finite router logit, an expired
  *     bounded wait) are recorded in the context's status word and returned by
- *     eb_sync_status().
+ *     eb_sync_status().  After EB_ERR_TIMEOUT the context's state may be
+ *     partial, so it runs no further step until eb_reset (see eb_moe_step).
+ *   - A CUDA error that something else left pending (cudaPeekAtLastError)
+ *     makes a call return EB_ERR_CUDA before it launches anything; the error
+ *     stays pending for its owner.
  *   - There is no CPU fallback: a shape the kernels do not support returns
  *     EB_ERR_UNSUPPORTED.
  *   - A context is not thread-safe; its calls must be ordered on one stream.
@@ -61,13 +65,9 @@ typedef int eb_status;
  *   TC    one SM per tile; weight rows are the MMA's M side (128 features),
  *         tokens its N side.
  *   SIMT  CUDA cores (any shape, f32 or bf16).
- *   TC2   as TC over an SM pair (cta_group::2, 256 features); F and H
- *         multiples of 256.
  *   TM    token-major, one SM: 128 tokens x 256 weight rows per MMA (gate/up:
  *         128 features of each; down: 256 features); work items are claimed
  *         dynamically, so CTAs finish together whatever the segment sizes.
- *   TM2   token-major over an SM pair (cta_group::2): 256 tokens x 256 weight
- *         rows per MMA, each SM holding 128 tokens and half the weight rows.
  *   TMG   as TM, but GEMM 1 reads its token rows straight from `hidden`
  *         (extra warps copy each row into the operand tile with 16-byte
  *         cp.async) instead of from a permuted copy, which is then not
@@ -76,15 +76,14 @@ typedef int eb_status;
  *         into `hidden` by the GEMM 2 drain that stores its last expert
  *         output row, and the step launches no combine kernel.  Bit-identical
  *         to TM.  The context then holds M*T*H/256 int32 arrival counters.
- * TM, TM2 and TMC need F a multiple of 128 (gate/up) and H a multiple of 256
+ * TM and TMC need F a multiple of 128 (gate/up) and H a multiple of 256
  * (down); a GEMM they do not fit runs on TC (and TMC's step then runs the
- * combine kernel). */
+ * combine kernel).  Values 3 and 5 (two-SM engines, measured slower than TM)
+ * are retired and rejected as EB_ERR_INVALID_ARG. */
 #define EB_GEMM_AUTO 0
 #define EB_GEMM_TC 1
 #define EB_GEMM_SIMT 2
-#define EB_GEMM_TC2 3
 #define EB_GEMM_TM 4
-#define EB_GEMM_TM2 5
 #define EB_GEMM_TMG 6
 #define EB_GEMM_TMC 7
 
@@ -183,6 +182,13 @@ eb_status eb_set_expert_map(eb_ctx* ctx, const int32_t* expert_rank);
  *   4. l_j += 1 for the RunSet; finished micro-batches leave S.
  * Once S is empty a step does nothing.
  *
+ * After a step that gave up on a bounded wait (status EB_ERR_TIMEOUT) the
+ * context refuses to step until eb_reset: on the device every later step
+ * does nothing and reports S as empty; once the host has seen the status
+ * (eb_sync_status, eb_episode, or a step with runset_host) eb_moe_step
+ * returns EB_ERR_TIMEOUT at once.  With runset_host the call also returns
+ * EB_ERR_TIMEOUT when the status word holds it after the step.
+ *
  * logits    [M, L, T, E] float32: the router logits of micro-batch j at
  *           layer l; only the blocks (j, l_j) of routed micro-batches are read.
  * hidden    [M, T, H] cfg.dtype, updated in place for RunSet micro-batches.
@@ -204,7 +210,8 @@ eb_status eb_moe_step(eb_ctx* ctx, const float* logits, void* hidden, const void
 /* A whole episode: eb_reset, then eb_moe_step until S is empty.  Steps are
  * enqueued a few ahead of the host's completion check, so the GPU never waits
  * for the host; steps enqueued after S became empty do nothing.  Returns the
- * number of steps that ran in *n_steps (host).  Waits for completion. */
+ * number of steps that ran in *n_steps (host).  Waits for completion; returns
+ * EB_ERR_TIMEOUT if a bounded device wait expired during the episode. */
 eb_status eb_episode(eb_ctx* ctx, const float* logits, void* hidden, const void* w_gateup,
                      const void* w_down, void* workspace, size_t workspace_bytes, void* stream,
                      int* n_steps);
@@ -256,6 +263,16 @@ eb_status eb_selftest_timeout(int64_t limit_ns, int32_t* status_dev, void* strea
 
 /* Waits for the context's work and returns the device-side status. */
 eb_status eb_sync_status(eb_ctx* ctx);
+
+/* Failure-injection hook for tests (the pages describe no failure handling):
+ * records `status` (EB_OK or one of the EB_ERR_* codes) in the context's
+ * device status word, stream-ordered, as a failing kernel would.  With
+ * EB_ERR_TIMEOUT and the fused-combine engine (EB_GEMM_TMC) it also leaves
+ * every arrival counter non-zero, the partial counts a GEMM 2 that gave up
+ * part-way can leave, so a test can check that the context refuses to step
+ * and that eb_reset restores it.  Nothing on the GPU waits, traps or faults.
+ * EB_ERR_INVALID_ARG for an unknown code. */
+eb_status eb_inject_status(eb_ctx* ctx, eb_status status, void* stream);
 
 /* ---------------------------------------------------------------------------
  * Stand-alone stages (stateless; device pointers; async on `stream`).
@@ -317,8 +334,11 @@ eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int
  * n_mb * ceil(T / 64) * E above 2^20 returns EB_ERR_TOO_LARGE before any
  * launch.  The call allocates nothing (no cudaMalloc, cudaFree or allocating
  * library routine).  Its first call on a device looks the array's device
- * address up (cudaGetSymbolAddress) and caches it: make that first call
- * before any stream capture.  Every call shares the one array: calls that
+ * address up (cudaGetSymbolAddress) and caches it with the CUDA context it
+ * belongs to: make that first call before any stream capture.  If the
+ * context changes (cudaDeviceReset() ends the primary context; the next
+ * call runs in a new one), the next call looks the address up again, and
+ * that call too should come before any stream capture.  Every call shares the one array: calls that
  * overlap on the GPU (other streams, other threads) race on it, so order
  * them on one stream.  Each call writes every count it reads, so stale
  * contents from an earlier call never leak into a result.

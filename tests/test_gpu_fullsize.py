@@ -149,7 +149,7 @@ def test_full_shape_chain(torch_mod, name):
         _free()
 
 
-@pytest.mark.parametrize("gemm", [0, 1, 3, 5, 6, 7])
+@pytest.mark.parametrize("gemm", [0, 1, 6, 7])
 @pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16", "qwen3_bf16",
                                   "moonlight_bf16", "longctx_bf16"])
 def test_single_step_expert_outputs(torch_mod, name, gemm):

@@ -49,13 +49,13 @@ def _cfg(**kw):
 def test_config_check(lib):
     assert eb.eb_config_check(_cfg()) == eb.EB_OK
     bad = [dict(E=15), dict(k=17), dict(m=5), dict(m=0), dict(T=0), dict(L=0), dict(M=0),
-           dict(policy=7), dict(dtype=5), dict(D=0), dict(n_shared=-1), dict(gemm=8), dict(gemm=-1)]
+           dict(policy=7), dict(dtype=5), dict(D=0), dict(n_shared=-1), dict(gemm=8), dict(gemm=-1),
+           dict(gemm=3), dict(gemm=5)]  # 3 and 5: retired two-SM engines
     for b in bad:
         assert eb.eb_config_check(_cfg(**b)) == eb.EB_ERR_INVALID_ARG, b
     unsup = [dict(M=33, m=3), dict(D=64, E=128 * 3), dict(k=20, n_shared=13, E=64),
              dict(H=130), dict(gemm=eb.GEMM_TC), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TC, H=192),
              dict(gemm=eb.GEMM_TM), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TM, F=192),
-             dict(gemm=eb.GEMM_TM2), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TM2, H=192),
              dict(gemm=eb.GEMM_TMC), dict(dtype=eb.DTYPE_BF16, gemm=eb.GEMM_TMC, H=192),
              dict(M=32, m=8, policy=eb.MAXUTIL)]
     for u in unsup:

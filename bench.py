@@ -5,7 +5,8 @@ workload (48 MoE layers, 128 experts, top-8, hidden 2048, expert FFN 768,
 D = 8 virtual ranks, M = 8 micro-batches x 1024 tokens): from reset until every
 micro-batch has passed all 48 layers, each scheduler step running routing,
 loads, the RunSet choice, permutation, the two grouped expert GEMMs and the
-combine.  Throughput counts token-layer passes: M * T * L per episode.
+combine.  Throughput counts token-layer passes: M * T * L per episode (the
+model-level rate, M * T tokens per episode, is printed beside it).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --sweep [--impl reference]   # routing + scheduling sweep, D x M
@@ -28,7 +29,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "cross-layer MoE step tokens/s at Qwen3-30B shape (1 B200); under-util 1−u"
-UNIT = "tokens/s"
+UNIT = "token-layer passes/s"
 POLICY_NAMES = {0: "cumutil", 1: "maxutil", 2: "lockstep", 3: "diffpeak"}
 
 
@@ -47,6 +48,8 @@ def parse():
     p.add_argument("--no-under-util", action="store_true")
     p.add_argument("--no-router-mode", action="store_true",
                    help="skip the extra router-mode episode timing")
+    p.add_argument("--no-policy-times", action="store_true",
+                   help="skip timing an episode of every scheduling policy")
     p.add_argument("--layers", type=int, default=0,
                    help="override the workload's MoE layer count (small profiling cases)")
     p.add_argument("--sweep", action="store_true",
@@ -56,7 +59,7 @@ def parse():
     p.add_argument("--sweep-episodes", type=int, default=4,
                    help="episodes per sweep point (the workload defines 43, about 2048 "
                         "lock-step steps; each episode's logits are drawn on the host)")
-    p.add_argument("--sweep-episodes-m32", type=int, default=1,
+    p.add_argument("--sweep-episodes-m32", type=int, default=0,
                    help="episodes of the MaxUtil points at M = 32, whose exhaustive search "
                         "covers about 15.3M subsets per step (0: skip those points)")
     return p.parse_args()
@@ -98,11 +101,14 @@ def max_over_ranks(x: float, world: int) -> float:
 
 def bench_config(wl, args, world: int) -> dict:
     """The workload description both arms print (same keys and values)."""
+    weights = wl.L * wl.E_tot * 3 * wl.F * wl.H * (2 if wl.dtype == "bf16" else 4)
     return {"workload": f"{wl.name}: Qwen3-30B-A3B shape L={wl.L} E={wl.E} k={wl.k} "
                         f"H={wl.H} F={wl.F} D={wl.D} M={wl.M} T={wl.T}",
             "policy": args.policy, "m": wl.m_default, "step": "one Algorithm-1 episode",
-            "tokens_per_step": wl.M * wl.T * wl.L,
-            "l2": "inputs larger than L2 (58 GB of expert weights streamed per episode)",
+            "tokens_per_step": wl.M * wl.T * wl.L, "model_tokens_per_step": wl.M * wl.T,
+            "l2": (f"inputs larger than L2: {weights / 1e9:.0f} GB of expert weights resident; "
+                   "each scheduler step streams the weights of every (layer, expert) it touches "
+                   "(per-episode GEMM bytes in `kernels`)"),
             "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
 
 
@@ -159,12 +165,15 @@ class ClockSampler:
 
 
 def measured_peaks():
+    """(HBM GB/s, dense bf16 TFLOP/s burst, sustained, source): the pool's
+    measured figures when present, else the profiling recipe's fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return d.get("hbm_gbs", 6650.0), "measured"
-    return 6650.0, "fallback"
+        return (d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0),
+                d.get("bf16_tflops_sustained", 1400.0), "measured")
+    return 6650.0, 1590.0, 1400.0, "fallback"
 
 
 def ncu_traffic(name: str, alg_bytes_per_launch: float):
@@ -256,7 +265,9 @@ def run_ours(args, world, rank, local):
         # indices in, the row of every (token, slot) and the token of every row out
         "positions": int((R * (4 + 4 + 4)).sum()),
     }
-    flops_gemm = int((R * 6 * wl.H * wl.F).sum())
+    # useful FLOPs of the expert GEMMs (rows x 2 H F per output pair)
+    flops = {"gemm_gateup": int((R * 4 * wl.H * wl.F).sum()),
+             "gemm_down": int((R * 2 * wl.H * wl.F).sum())}
     fused = ctx.eb_engines()[1] == eb.GEMM_TMC
     if fused:
         # GEMM 2 also combines: its bytes are the down GEMM's and the
@@ -264,9 +275,9 @@ def run_ours(args, world, rank, local):
         # as far as the design goes)
         alg["gemm_down"] += alg.pop("combine") - int((R * wl.H * b).sum())
 
+    # the headline: whole episodes, nothing between the kernels
     clocks = ClockSampler(local)
     launches0 = ctx.eb_launch_count()
-    ctx.eb_profile(True)
     barrier(world)
     torch.cuda.synchronize()
     clocks.start()
@@ -281,34 +292,93 @@ def run_ours(args, world, rank, local):
     barrier(world)
     clk = clocks.stop()
     ms_total = t_start.elapsed_time(t_stop)
-    prof = ctx.eb_profile_read()
-    ctx.eb_profile(False)
     launches = ctx.eb_launch_count() - launches0
     assert ctx.eb_sync_status() == eb.EB_OK
     ms_max = max_over_ranks(ms_total, world)
     value = job_throughput(wl.M * wl.T * wl.L * args.steps, ms_max, world)
 
-    # roofline of the dominant kernel
+    # per-kernel times: a separate pass with CUDA events around every kernel
+    k_prof = max(2, args.steps // 2)
+    ctx.eb_profile(True)
+    for _ in range(k_prof):
+        hidden.copy_(h0)
+        ctx.eb_episode(logits, hidden, wgu, wdn)
+    prof = ctx.eb_profile_read()
+    ctx.eb_profile(False)
+    hbm, tf_burst, tf_sust, peak_src = measured_peaks()
+
+    def floor_bound(k):
+        """The binding roofline of kernel k: whichever of its bytes at the HBM
+        peak and its useful FLOPs at the sustained tensor peak takes longer."""
+        if k in flops and flops[k] / (tf_sust * 1e12) > alg[k] / (hbm * 1e9):
+            return "tensor"
+        return "hbm"
+
     kern = max((k for k in ("gemm_gateup", "gemm_down", "permute", "combine") if k in alg),
                key=lambda k: prof[k][0])
     kms, kl = prof[kern]
-    peak, peak_src = measured_peaks()
-    achieved = alg[kern] * args.steps / (kms / 1e3) / 1e9
-    alg_launch = alg[kern] * args.steps / max(1, kl)
-    roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1), "peak": peak,
-            "unit": "GB/s", "frac": round(achieved / peak, 4), "traffic": ncu_traffic(kern, alg_launch),
-            "peak_source": peak_src + " (MEASURED_PEAKS.json hbm_gbs)" if peak_src == "measured"
-            else "fallback 6650 GB/s",
-            "alg_bytes_per_launch": int(alg_launch),
-            "avg_launch_ms": round(kms / max(1, kl), 5)}
-    gemm_ms = prof["gemm_gateup"][0] + prof["gemm_down"][0]
-    kernels = {k: {"ms_per_episode": round(v[0] / args.steps, 4), "launches": v[1]}
+    alg_launch = alg[kern] * k_prof / max(1, kl)
+    bound = floor_bound(kern)
+    if bound == "tensor":
+        achieved = flops[kern] * k_prof / (kms / 1e3) / 1e12
+        roof = {"kernel": kern, "bound": "tensor", "achieved": round(achieved, 1), "peak": tf_sust,
+                "unit": "TFLOP/s", "frac": round(achieved / tf_sust, 4),
+                "peak_source": (peak_src + " dense bf16, sustained (the kernel runs inside a "
+                                "long step)"),
+                "flops_per_launch": int(flops[kern] * k_prof / max(1, kl)),
+                "hbm_frac": round(alg[kern] * k_prof / (kms / 1e3) / 1e9 / hbm, 4)}
+    else:
+        achieved = alg[kern] * k_prof / (kms / 1e3) / 1e9
+        roof = {"kernel": kern, "bound": "hbm", "achieved": round(achieved, 1), "peak": hbm,
+                "unit": "GB/s", "frac": round(achieved / hbm, 4),
+                "peak_source": (peak_src + " HBM copy bandwidth" if peak_src == "measured"
+                                else "fallback 6650 GB/s")}
+    roof.update({"traffic": ncu_traffic(kern, alg_launch), "alg_bytes_per_launch": int(alg_launch),
+                 "avg_launch_ms": round(kms / max(1, kl), 5), "of": peak_src})
+    kernels = {k: {"ms_per_episode": round(v[0] / k_prof, 4), "launches": v[1]}
                for k, v in prof.items()}
     for k in ("route", "positions", "permute", "gemm_gateup", "gemm_down", "combine"):
         if k in alg and prof[k][0] > 0:
-            kernels[k]["GBps"] = round(alg[k] * args.steps / (prof[k][0] / 1e3) / 1e9, 1)
-            kernels[k]["frac_of_hbm"] = round(kernels[k]["GBps"] / peak, 4)
-    kernels["gemm_tflops"] = round(flops_gemm * args.steps / (gemm_ms / 1e3) / 1e12, 2)
+            kernels[k]["GB_per_episode"] = round(alg[k] / 1e9, 3)
+            kernels[k]["GBps"] = round(alg[k] * k_prof / (prof[k][0] / 1e3) / 1e9, 1)
+            kernels[k]["frac_of_hbm"] = round(kernels[k]["GBps"] / hbm, 4)
+            if k in flops:
+                tfs = flops[k] * k_prof / (prof[k][0] / 1e3) / 1e12
+                kernels[k]["useful_TFLOPs"] = round(tfs, 1)
+                kernels[k]["frac_of_tensor_sustained"] = round(tfs / tf_sust, 4)
+                kernels[k]["bound"] = floor_bound(k)
+    kernels["note"] = ("per-kernel times from a separate pass with CUDA events around every "
+                       "kernel; the headline pass has none")
+
+    # every policy's episode time and GEMM weight bytes on the same inputs
+    # ([EB] Table 3 / Fig. 2 compare policies by time): on one GPU a step
+    # streams the weights of every (layer, expert) its RunSet touches, so the
+    # schedule with the best 1 - u may move more bytes
+    policy_ms = {}
+    if not args.no_policy_times:
+        for pol, name in POLICY_NAMES.items():
+            pc = ctx if pol == policy else eb.Context(cfg_for(pol))
+            hidden.copy_(h0)
+            pc.eb_episode(logits, hidden, wgu, wdn)
+            prow, _ = pc.eb_trace()
+            reps = max(1, args.steps // 3)
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                hidden.copy_(h0)
+                pc.eb_episode(logits, hidden, wgu, wdn)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms_p = max_over_ranks(e0.elapsed_time(e1) / reps, world)
+            num, den, _ = pc.eb_utilization()
+            pt = prow[:, 5].astype(np.int64)
+            policy_ms[name] = {"ms_per_episode": round(ms_p, 3), "scheduler_steps": int(prow.shape[0]),
+                               "gemm_weight_GB": round(float((pt * 3 * wl.F * wl.H * b).sum()) / 1e9, 2),
+                               "under_util": round(1 - num / den, 6)}
+            if pc is not ctx:
+                pc.close()
 
     # end to end: host buffers, copies inside the timed region
     e2e = None
@@ -336,7 +406,8 @@ def run_ours(args, world, rank, local):
                "unit": UNIT,
                "h2d_bytes_per_step": int(lg_host.numel() * 4 + h_host.numel() * h_host.element_size()),
                "d2h_bytes_per_step": int(out_host.numel() * out_host.element_size()),
-               "steps": k_e2e}
+               "steps": k_e2e,
+               "model_tokens_per_s": round(job_throughput(wl.M * wl.T * k_e2e, ms_e2e, world), 1)}
     ctx.close()
 
     # router mode (the routing scores projected from the hidden states on the
@@ -381,6 +452,7 @@ def run_ours(args, world, rank, local):
     if rank == 0:
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world,
+            "model_tokens_per_s": round(value / wl.L, 1),
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms_max / args.steps, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
@@ -390,7 +462,7 @@ def run_ours(args, world, rank, local):
             "config": bench_config(wl, args, world), "scheduler_steps": n_steps,
             "e2e": e2e, "gpu_launches": int(launches), "roofline": roof,
             "cpu_baseline": cpu, "clocks": clk, "under_util": under, "kernels": kernels,
-            "router_mode": router_mode,
+            "policy_ms": policy_ms, "router_mode": router_mode,
         }
         print(json.dumps(line), flush=True)
 
@@ -452,8 +524,8 @@ def oracle_sample(wl, policy, logits_np, h0_np, fetch_expert, n_tokens: int, rou
     detail = (f"oracle on a bounded sample: routing+loads of {route_tokens} tokens x {wl.L} layers "
               f"({t_route:.2f}s), the full-episode schedule ({t_sched:.2f}s), expert FFN + combine "
               f"of {n_tokens} token(s) through {ffn_layers} layers ({t_ffn:.2f}s); time per "
-              f"token-layer = sum of the three per-unit costs")
-    return per_tl, detail
+              f"token-layer = sum of the three per-unit costs, extrapolated to the workload")
+    return per_tl, detail, t_route + t_sched + t_ffn
 
 
 def make_fetch(wgu, wdn, F):
@@ -466,8 +538,8 @@ def make_fetch(wgu, wdn, F):
 def cpu_baseline(wl, policy, logits_np, h0, wgu, wdn, n_tokens=4, ffn_layers=8):
     import numpy as np
     h0_np = h0.float().cpu().numpy().astype(np.float64)
-    per_tl, detail = oracle_sample(wl, policy, logits_np, h0_np, make_fetch(wgu, wdn, wl.F),
-                                   n_tokens, 256, episode_loads(wl, logits_np), ffn_layers)
+    per_tl, detail, _ = oracle_sample(wl, policy, logits_np, h0_np, make_fetch(wgu, wdn, wl.F),
+                                      n_tokens, 256, episode_loads(wl, logits_np), ffn_layers)
     return {"value": round(1.0 / per_tl, 2), "unit": UNIT, "cores": _blas_threads(),
             "kind": "oracle", "sample": detail + " (expert weights copied from the device)"}
 
@@ -494,17 +566,23 @@ def run_reference(args, world, rank):
         dn = (torch.randn((wl.H, wl.F), generator=g) * sd).to(torch.bfloat16).float().numpy()
         return gu[:wl.F], gu[wl.F:], dn
 
-    times, detail = [], ""
+    times, sample_s, detail = [], [], ""
     full_loads = episode_loads(wl, logits_np)
     for i in range(args.warmup + args.steps):
-        per_tl, detail = oracle_sample(wl, policy, logits_np, h0_np, fetch, 1, 64, full_loads, 4)
+        per_tl, detail, sec = oracle_sample(wl, policy, logits_np, h0_np, fetch, 1, 64, full_loads, 4)
         if i >= args.warmup:
             times.append(per_tl)
+            sample_s.append(sec)
     per_tl = statistics.median(times)
     value = 1.0 / per_tl
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 2), "unit": UNIT,
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            # one step of the workload (a whole episode) is far beyond a
+            # bounded CPU run: each timed step is a sample, and the step time
+            # below is extrapolated from the sample's per-unit costs
             "ms_per_step": round(per_tl * wl.M * wl.T * wl.L * 1e3, 1),
+            "ms_per_step_extrapolated": True,
+            "sample_s_per_step": round(statistics.median(sample_s), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": bench_config(wl, args, 1),
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": _blas_threads(),

@@ -101,6 +101,11 @@ WORKLOADS = {
     "moonlight_bf16": Workload("moonlight_bf16", L=26, E=64, k=6, H=2048, F=1408, D=8,
                                M=8, T=512, n_shared=2, profile="dirichlet_layer",
                                alpha=0.3),
+    # Moonlight-16B-A3B shape with weights scaled by fan-in (N(0, 1/(3 fan_in))),
+    # so that the full 26-layer chain stays finite in bf16
+    "moonlight_fanin_bf16": Workload("moonlight_fanin_bf16", L=26, E=64, k=6, H=2048, F=1408,
+                                     D=8, M=8, T=512, n_shared=2, profile="dirichlet_layer",
+                                     alpha=0.3, w_init="fan_in"),
     # Qwen3-30B-A3B shape: the throughput workload
     "qwen3_bf16": Workload("qwen3_bf16", L=48, E=128, k=8, H=2048, F=768, D=8, M=8,
                            T=1024, profile="task_profiles", alpha=0.2, w_init="fan_in"),

@@ -119,6 +119,39 @@ def test_full_size_episode(torch_mod, name, policy):
         _free()
 
 
+def test_moonlight_fanin_chain(torch_mod):
+    """The Moonlight-16B-A3B shape (64 routed experts top-6, 2 shared experts,
+    H = 2048, F = 1408) with fan-in-scaled weights: the full 26-layer episode
+    stays finite and equals lock-step bit for bit, and an 8-layer cross-layer
+    chain (MaxUtil) matches the oracle on sampled tokens through every
+    layer."""
+    wl = synth.get("moonlight_fanin_bf16")
+    inp = Inputs(wl)
+    try:
+        hidden = run_episode(inp, osch.MAXUTIL)[0]
+        assert bool(torch_mod.isfinite(hidden.float()).all())
+        lock = run_episode(inp, osch.LOCKSTEP)[0]
+        assert torch_mod.equal(lock.view(torch_mod.int16), hidden.view(torch_mod.int16))
+        del lock, hidden
+    finally:
+        del inp
+        _free()
+    wl = wl.replace(L=8)
+    inp = Inputs(wl)
+    try:
+        hidden, rows, layers, util, steps = run_episode(inp, osch.MAXUTIL)
+        check_schedule(rows, layers, util, steps, oracle_episode(inp, osch.MAXUTIL), wl.M)
+        rng = np.random.default_rng(13)
+        toks = [(j, int(rng.integers(0, wl.T))) for j in range(wl.M)] + [(wl.M - 1, wl.T - 1), (0, 0)]
+        want = oracle_hidden(inp, toks)
+        assert np.abs(want).mean() > 0.2
+        got = np.stack([hidden[j, t].float().cpu().numpy() for (j, t) in toks])
+        assert_close(got, want, "bf16", "moonlight fan-in 8-layer chain")
+    finally:
+        del inp
+        _free()
+
+
 @pytest.mark.parametrize("name", ["qwen3_bf16", "moonlight_bf16", "longctx_bf16"])
 def test_full_shape_chain(torch_mod, name):
     """Every per-layer size at full scale (M, T, E, k, H, F, D, shared

@@ -113,26 +113,44 @@ __device__ __forceinline__ void route_token(const float* row, int E, int k, int 
   }
   const float vmax = key_value(top[0]);
   float ex[KMAX];
-  float denom = 0.f;
 #pragma unroll
-  for (int i = 0; i < KMAX; ++i) {
-    ex[i] = i < k ? expf(key_value(top[i]) - vmax) : 0.f;
-    denom += ex[i];
+  for (int i = 0; i < KMAX; ++i) ex[i] = i < k ? expf(key_value(top[i]) - vmax) : 0.f;
+  float denom;
+  if (renorm) {
+    // pairwise sum of the k terms (a tree keeps the rounding error at
+    // log2(k) additions)
+    float t[KMAX];
+#pragma unroll
+    for (int i = 0; i < KMAX; ++i) t[i] = ex[i];
+#pragma unroll
+    for (int w = KMAX / 2; w >= 1; w /= 2)
+#pragma unroll
+      for (int i = 0; i < w; ++i) t[i] += t[i + w];
+    denom = t[0];
+  } else {
+    // softmax over all E: eight interleaved partial sums, then a tree
+    float part[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) part[i] = 0.f;
+    for (int e0 = 0; e0 < E; e0 += 8)
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (e0 + i < E) {
+          const float x = row[e0 + i];
+          part[i] += expf((isfinite(x) ? x : -INFINITY) - vmax);
+        }
+#pragma unroll
+    for (int w = 4; w >= 1; w /= 2)
+#pragma unroll
+      for (int i = 0; i < w; ++i) part[i] += part[i + w];
+    denom = part[0];
   }
-  if (!renorm) {
-    denom = 0.f;
-    for (int e = 0; e < E; ++e) {
-      const float x = row[e];
-      denom += expf((isfinite(x) ? x : -INFINITY) - vmax);
-    }
-  }
-  const float inv = 1.f / denom;
 #pragma unroll
   for (int i = 0; i < KMAX; ++i)
     if (i < k) {
       const int e = key_expert(top[i]);
       idx[i] = e;
-      gate[i] = ex[i] * inv;
+      gate[i] = ex[i] / denom;
       atomicAdd(&hist_s[e], 1);
     }
 }

@@ -59,13 +59,19 @@ def _episode(eb, torch, wl, inp, router, policy):
     return hidden, rows, layers, util, n, scores.cpu().numpy()
 
 
-# Near-tie bound for a router score: the device projection was measured within
-# 1e-4 abs + 1e-4 rel of the float64 product on identical inputs (above); a
-# later layer's input also differs from the oracle's chain by the rounding of
-# the bf16 hidden state (one unit in the last place in a few elements, each
-# contributing about 2^-8 |h_i| |w_i| to a score).  TAU covers both with a
-# margin; the test prints the largest deviation it saw.
-TAU_ABS, TAU_REL = 2e-3, 2e-3
+# Bound on |device score - oracle score| at layer l: tau_l(s) = (TAU0 + TAU_L
+# l) (1 + |s|).  At layer 0 both sides project the same hidden states, and
+# the device projection was measured within 1e-4 + 1e-4 |s| of the float64
+# product (above).  Each later layer's input also carries the rounding of the
+# bf16 hidden state: the two chains round the same values, but a value close
+# to a rounding boundary can land one unit in the last place apart, and the
+# next layer carries that on; TAU_L per layer covers it (the largest
+# deviation seen per layer is printed).
+TAU0, TAU_L = 1e-4, 3e-3
+
+
+def _tau(s, l):
+    return (TAU0 + TAU_L * l) * (1.0 + np.abs(np.asarray(s, dtype=np.float64)))
 
 
 def _topk_sets(scores, k):
@@ -88,24 +94,23 @@ def _oracle_chain(wl, inp, routers, gpu_scores):
     else the device must have chosen exactly the oracle's set.
 
     Returns (final hidden [M*T, H], loads [M, L, D], near-tie count, adopted
-    count, largest |device score - oracle score| over tokens)."""
+    count, the largest |device score - oracle score| of each layer)."""
     M, L, T, E, k = wl.M, wl.L, wl.T, wl.E, wl.k
     h = inp.h0_np.reshape(M * T, wl.H).copy()
     loads = np.zeros((M, L, wl.D), dtype=np.int64)
     near = adopted = 0
-    worst = 0.0
+    worst = []
     for l in range(L):
         osc = orouter.router_logits(h, routers[l]).astype(np.float32)
         gsc = gpu_scores[:, l].reshape(M * T, E)
         dev = np.abs(gsc.astype(np.float64) - osc)
-        tau = TAU_ABS + TAU_REL * np.abs(osc.astype(np.float64))
-        worst = max(worst, float(dev.max()))
-        assert np.all(dev <= tau), (l, float(dev.max()))
+        worst.append(float(dev.max()))
+        assert np.all(dev <= _tau(osc, l)), (l, float(dev.max()))
         idx, gate = oracle.route(osc, k)
         # near ties of the oracle's own decision
         srt = -np.sort(-osc.astype(np.float64), axis=1)
         gap = srt[:, k - 1] - srt[:, k] if k < E else np.full(M * T, np.inf)
-        tie = gap <= 2 * (TAU_ABS + TAU_REL * np.abs(srt[:, k - 1]))
+        tie = gap <= 2 * _tau(srt[:, k - 1], l)
         near += int(tie.sum())
         want = np.sort(idx, axis=1)
         got = _topk_sets(gsc, k)
@@ -119,7 +124,7 @@ def _oracle_chain(wl, inp, routers, gpu_scores):
             sel[got[t]] = True
             lo = osc[t, sel].astype(np.float64).min()
             hi = osc[t, ~sel].astype(np.float64).max()
-            assert lo >= hi - 2 * (TAU_ABS + TAU_REL * abs(hi)), (l, t)
+            assert lo >= hi - 2 * _tau(hi, l), (l, t)
             # the device's set, slots and renormalised gates as the oracle
             # forms them over that set (experts outside it masked far below)
             masked = np.where(sel, osc[t], np.float32(-1e30)).astype(np.float32)
@@ -148,7 +153,8 @@ def _check_router_episode(torch, wl, inp, router, toks, policies):
     assert np.isfinite(sc).all()
     final, loads, near, adopted, worst = _oracle_chain(wl, inp, routers, sc)
     print(f"router chain {wl.name} L={wl.L}: {near} near ties, {adopted} routed by the device's "
-          f"valid choice, largest score deviation {worst:.3g}")
+          f"valid choice, largest score deviation per layer "
+          + " ".join(f"{x:.3g}" for x in worst))
     want = np.stack([final[j * wl.T + t] for (j, t) in toks])
     for policy in policies:
         hidden, rows, layers, util, n, sc2 = _episode(eb, torch, wl, inp, router, policy)

@@ -75,7 +75,8 @@ def test_no_alloc_route_loads_matches_allocating_entry_points(lib):
         # counts leave stale entries of the earlier calls in the array
         (8, 1024, 128, 8, 8, True),
         (3, 200, 64, 6, 4, False),
-        (2, 70, 40, 40, 8, True),  # E not a multiple of 32 (padded lanes), k = E
+        (2, 70, 24, 24, 8, True),  # k = E (every expert), E not a multiple of 32
+        (2, 70, 40, 32, 8, False),  # the largest k, E not a multiple of 32
         (1, 17, 16, 2, 4, True),   # one micro-batch shorter than a 64-token chunk
     ]
     for (n_mb, T, E, k, D, renorm) in cases:

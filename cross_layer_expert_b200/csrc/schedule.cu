@@ -357,13 +357,84 @@ __device__ int3 block_exclusive_scan3(int3 v, int3* tmp /* >= 33 */) {
   return make_int3(w.x + incl.x - v.x, w.y + incl.y - v.y, w.z + incl.z - v.z);
 }
 
-constexpr int kSearchThreads = 512;
+constexpr int kSearchThreads = 256;
+
+// The same search as search_ranks, for the grid: each thread keeps its
+// current complement's W_d (d < D <= DMAX) in registers and updates it by
+// the rows that enter or leave the complement between neighbours in
+// Gosper's order (about two rows per step), instead of re-summing every
+// member's row for every candidate.  W_d <= sum of all loads < 2^31.
+template <int DMAX>
+__device__ Cand search_ranks_inc(const SchedSmem& sm, int D, unsigned long long r_lo,
+                                 unsigned long long r_hi) {
+  const int n = sm.n;
+  const uint32_t (*B)[33] = kBinom.v;
+  const unsigned long long N = r_hi > r_lo ? r_hi - r_lo : 0;
+  const unsigned long long per = (N + blockDim.x - 1) / blockDim.x;
+  unsigned long long r = r_lo + per * threadIdx.x;
+  const unsigned long long r_end = r + per < r_hi ? r + per : r_hi;
+  Cand best{0, 0, -1, 0};
+  if (r >= r_end) return best;
+  int c = 0;
+  unsigned long long q = r;
+  while (q >= B[n][c]) {
+    q -= B[n][c];
+    ++c;
+  }
+  uint32_t cm = c == 0 ? 0u : unrank_colex((uint32_t)q, c, B);
+  int W[DMAX];
+  long long sum;
+  auto load_full = [&]() {  // W and sum of the complement cm from scratch
+    sum = sm.totsum;
+#pragma unroll
+    for (int d = 0; d < DMAX; ++d) W[d] = d < D ? (int)sm.tot[d] : 0;
+    for (uint32_t b = cm; b; b &= b - 1) {
+      const int i = __ffs(b) - 1;
+      sum -= sm.wsum[i];
+#pragma unroll
+      for (int d = 0; d < DMAX; ++d)
+        if (d < D) W[d] -= sm.w[i][d];
+    }
+  };
+  load_full();
+  bool have = false;
+  for (;;) {
+    int mx = 0;
+#pragma unroll
+    for (int d = 0; d < DMAX; ++d) mx = W[d] > mx ? W[d] : mx;
+    const Cand cd{sum, (long long)mx, n - c, cm};
+    if (!have || cand_better(cd, best)) {
+      best = cd;
+      have = true;
+    }
+    if (++r == r_end) break;
+    if (++q == B[n][c]) {  // next size: its first combination, from scratch
+      ++c;
+      q = 0;
+      cm = (1u << c) - 1u;
+      load_full();
+    } else {
+      const uint32_t nx = (uint32_t)gosper_next(cm);
+      for (uint32_t b = cm ^ nx; b; b &= b - 1) {
+        const int i = __ffs(b) - 1;
+        const int sgn = ((nx >> i) & 1u) ? -1 : 1;  // enters the complement: leaves S
+        sum += sgn * sm.wsum[i];
+#pragma unroll
+        for (int d = 0; d < DMAX; ++d)
+          if (d < D) W[d] += sgn * sm.w[i][d];
+      }
+      cm = nx;
+    }
+  }
+  return best;
+}
 
 // MaxUtil search grid: CTA b searches complement ranks [N b / G, N (b+1) / G)
 // of the pending set (N candidates, G = gridDim.x) and writes its best
 // candidate (or "none") to slots[b].  The pending set and loads are the
 // step state's (st != null; nothing is searched while a timed-out step
 // awaits a reset) or the caller's (pending_arg, w).
+template <int DMAX>
 __global__ void __launch_bounds__(kSearchThreads) k_maxutil_search(int M, int D, int m,
                                                                    const State* __restrict__ st,
                                                                    uint32_t pending_arg,
@@ -390,7 +461,7 @@ __global__ void __launch_bounds__(kSearchThreads) k_maxutil_search(int M, int D,
     __syncthreads();
     prepare_totals(sm, D);
     const unsigned long long N = candidate_count(sm.n, m), G = gridDim.x;
-    best = search_ranks(sm, D, m, N * blockIdx.x / G, N * (blockIdx.x + 1) / G);
+    best = search_ranks_inc<DMAX>(sm, D, N * blockIdx.x / G, N * (blockIdx.x + 1) / G);
   }
   best = block_best(best, sm.red);
   if (tid == 0) slots[blockIdx.x] = best;
@@ -751,9 +822,15 @@ bool maxutil_uses_grid(int n, int m) { return maxutil_candidates(n, m) > kBlockS
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
                                  int fm1, int fm2, cudaStream_t s) {
   if (c.search_slots) {
-    const cudaError_t e = launch_pdl(k_maxutil_search, dim3(kSearchCtas), dim3(kSearchThreads), 0,
-                                     s, 1, d.M, d.D, d.m, (const State*)c.st, 0u,
-                                     (const int32_t*)c.w, static_cast<Cand*>(c.search_slots));
+    auto go = [&](auto kernel) {
+      return launch_pdl(kernel, dim3(kSearchCtas), dim3(kSearchThreads), 0, s, 1, d.M, d.D, d.m,
+                        (const State*)c.st, 0u, (const int32_t*)c.w,
+                        static_cast<Cand*>(c.search_slots));
+    };
+    const cudaError_t e = d.D <= 8    ? go(k_maxutil_search<8>)
+                          : d.D <= 16 ? go(k_maxutil_search<16>)
+                          : d.D <= 32 ? go(k_maxutil_search<32>)
+                                      : go(k_maxutil_search<64>);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(k_schedule_step, dim3(1), dim3(kThreads), 0, s, 1, d, c, w, rn1, rn2, fm1, fm2);
@@ -763,8 +840,14 @@ cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int 
                                  int policy, uint32_t* runset, long long* stats, void* slots,
                                  cudaStream_t s) {
   if (slots) {
-    k_maxutil_search<<<kSearchCtas, kSearchThreads, 0, s>>>(M, D, m, nullptr, pending, w,
-                                                           static_cast<Cand*>(slots));
+    auto go = [&](auto kernel) {
+      kernel<<<kSearchCtas, kSearchThreads, 0, s>>>(M, D, m, nullptr, pending, w,
+                                                     static_cast<Cand*>(slots));
+    };
+    if (D <= 8) go(k_maxutil_search<8>);
+    else if (D <= 16) go(k_maxutil_search<16>);
+    else if (D <= 32) go(k_maxutil_search<32>);
+    else go(k_maxutil_search<64>);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }

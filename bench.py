@@ -635,7 +635,11 @@ def run_sweep(args):
     eb.load()
     dev = torch.device("cuda", torch.cuda.current_device())
     print(json.dumps({"sweep": SWEEP_NOTE, "impl": "ours", "gpu": torch.cuda.get_device_name(dev),
-                      "unit_time": "us per launch (CUDA events on the launching stream)"}),
+                      "unit_time": "step_us: whole steps (routing + scheduling; the host's "
+                                   "per-episode completion checks included), CUDA events "
+                                   "around the episodes; route_us / "
+                                   "schedule_us: each kernel alone, CUDA events around every "
+                                   "launch (launch gaps included)"}),
           flush=True)
     t0 = time.time()
     cache_M, episodes = None, []
@@ -649,10 +653,23 @@ def run_sweep(args):
         ctx = eb.Context(eb.make_config(L=wl.L, E=wl.E, k=wl.k, H=wl.H, F=wl.F, D=wl.D, M=wl.M,
                                         T=wl.T, dtype=eb.DTYPE_BF16, policy=pol,
                                         m=wl.m_default, compute=0))
-        ctx.eb_profile(True)
-        num = den = den_sep = steps = 0
+        ctx.eb_episode(episodes[0], None, None, None)  # warm-up
+        # whole steps, no events between the kernels
+        stream = torch.cuda.current_stream()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        steps = 0
+        e0.record(stream)
         for lg in episodes[:n_ep]:
             steps += ctx.eb_episode(lg, None, None, None)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        step_us = 1e3 * e0.elapsed_time(e1) / max(1, steps)
+        # each kernel alone (events around every launch), and the exact
+        # utilisation of every episode (the same episodes again)
+        num = den = den_sep = 0
+        ctx.eb_profile(True)
+        for lg in episodes[:n_ep]:
+            ctx.eb_episode(lg, None, None, None)
             a, b, c = ctx.eb_utilization()
             num, den, den_sep = num + a, den + b, den_sep + c
         prof = ctx.eb_profile_read()
@@ -661,7 +678,8 @@ def run_sweep(args):
         ctx.close()
         rt, sc = prof["route"], prof["schedule"]
         sweep_line(M, D, pol, n_ep, num, den, den_sep, steps,
-                   {"route_us": round(1e3 * rt[0] / max(1, rt[1]), 2),
+                   {"step_us": round(step_us, 2),
+                    "route_us": round(1e3 * rt[0] / max(1, rt[1]), 2),
                     "schedule_us": round(1e3 * sc[0] / max(1, sc[1]), 2)})
     print(json.dumps({"sweep_done": True, "wall_s": round(time.time() - t0, 1)}), flush=True)
 

@@ -536,6 +536,13 @@ __device__ __forceinline__ SegView cache_segments(uint8_t* buf, int nseg, const 
 }
 
 constexpr int kGatherWarps = 4;  // row-gathering warps of the gathering GEMM 1 (one thread per row)
+// The fused combine (GEMM 2, engine TMC): the drain hands every completed
+// (token, 256-feature block) to kCombineWarps extra warps through a ring of
+// kCombineQueue entries in shared memory, so the drain never waits on the
+// combine's loads.
+constexpr int kCombineWarps = 8;
+constexpr int kCombineQueue = 512;
+constexpr int kCombineBytes = (kCombineQueue + 4) * 4;
 constexpr int kGatherDepth = 2;  // k-blocks a gathering thread keeps in flight before signalling
 constexpr int kTmBox = 32;                    // token rows per TMA box
 constexpr int kTmBoxBytes = kTmBox * kBK * 2;  // 4 KiB
@@ -553,7 +560,8 @@ struct CfgTM {
   static constexpr int kAccBufs = 2;
   static constexpr int kTmemCols = kAccBufs * kAccCols;  // 512
   static constexpr int kQueue = 8;  // claimed items queued for the MMA issuer and the drain
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 + kSegCacheBytes + 1024;
+  static constexpr int kSmemBytes =
+      kStages * kStageBytes + 1024 + kSegCacheBytes + (GATEUP ? 0 : kCombineBytes) + 1024;
   static_assert(kRows == 128 && kFeat * (GATEUP ? 2 : 1) == kN, "token-major tile shape");
   static_assert(kGatherDepth >= 1 && kGatherDepth < kStages, "a gathering thread signals a stage before it reuses it");
   static_assert(32 * kGatherWarps == kRows, "one gathering thread per token row");
@@ -654,7 +662,10 @@ __device__ __forceinline__ void combine_token(const Dims& d, int tok, int f, int
 // warp combines the token's 256 features of that block into hidden.
 // Nothing waits: a token is combined by whichever drain finishes it last.
 template <bool GATEUP, bool GATHER, bool COMBINE>
-__global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThreads, 1)
+__global__ void __launch_bounds__(GATHER    ? kThreads + 32 * kGatherWarps
+                                  : COMBINE ? kThreads + 32 * kCombineWarps
+                                            : kThreads,
+                                  1)
     k_gemm_tm(const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_x,
               Dims d, State* __restrict__ st, const int32_t* __restrict__ seg_rows,
               const int32_t* __restrict__ seg_wid, const int32_t* __restrict__ seg_items,
@@ -681,6 +692,10 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* iq = const_cast<int*>(abort_flag) + 1;  // [Q] claimed items, -1 ends the sequence
   uint8_t* seg_buf = reinterpret_cast<uint8_t*>(bars) + 1024;
+  // fused combine: ring of (token, feature block) entries (-1: empty), then
+  // the push and pop counters and the count of drain warps that finished
+  volatile int* cq = reinterpret_cast<volatile int*>(seg_buf + kSegCacheBytes);
+  int* cq_ctl = const_cast<int*>(cq) + kCombineQueue;  // [0] pushed [1] popped [2] drains done
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nseg = st->nseg;
@@ -706,6 +721,10 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
     }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if constexpr (COMBINE) {
+    for (int i = threadIdx.x; i < kCombineQueue; i += blockDim.x) cq[i] = -1;
+    if (threadIdx.x < 3) cq_ctl[threadIdx.x] = 0;
   }
   const SegView sv = cache_segments(seg_buf, nseg, seg_rows, seg_wid, seg_items);
   if (warp == 1) {
@@ -908,6 +927,44 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
         pending = 0;
       }
     }
+  } else if (COMBINE && warp >= 2 + kEpiWarps) {
+    // ------------------------------------------------------------ combine
+    // Each warp pops (token, feature block) entries in order and combines
+    // that block of the token into hidden.  It stops once every drain warp
+    // has finished and the ring holds nothing more.
+    const unsigned long long t_begin = global_ns();
+    for (;;) {
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(&cq_ctl[1], 1);
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      int v = -1;
+      if (lane == 0) {
+        const unsigned long long t0 = global_ns();
+        for (uint32_t it_ = 1;; ++it_) {
+          v = cq[slot % kCombineQueue];
+          if (v >= 0) {
+            cq[slot % kCombineQueue] = -1;  // frees the entry for the push kCombineQueue later
+            break;
+          }
+          // every push happens before its drain warp counts itself done, so
+          // with all drains done the pushed count is final
+          if (*(volatile int*)&cq_ctl[2] == kEpiWarps && *(volatile int*)&cq_ctl[0] <= slot) break;
+          if ((it_ & 255) == 0 && (*abort_flag || global_ns() - t0 > kWaitLimitNs)) {
+            if (!*abort_flag) {
+              *abort_flag = 1;
+              atomicCAS(&st->status, EB_OK, EB_ERR_TIMEOUT);
+            }
+            break;
+          }
+        }
+      }
+      v = __shfl_sync(0xffffffffu, v, 0);
+      if (v < 0) break;
+      __threadfence();  // the arrivals the drain counted before the reads of y
+      const int nfb = d.H / C::kFeat;
+      combine_token(d, v / nfb, (v % nfb) * C::kFeat, lane, gate, out, hidden);
+    }
+    (void)t_begin;
   } else {
     // ------------------------------------------------------------ drain
     // warp w reads TMEM lanes (tokens) 32 (w % 4) .. +31; with 8 warps two
@@ -978,18 +1035,26 @@ __global__ void __launch_bounds__(GATHER ? kThreads + 32 * kGatherWarps : kThrea
           last = atomicAdd(cnt, 1) == d.kk * kGroups - 1;
           if (last) *cnt = 0;  // no other arrival on it in this launch
         }
-        unsigned lm = __ballot_sync(0xffffffffu, last);
-        if (lm) {
-          __syncwarp();
-          __threadfence();  // every counted share before the reads of y
-          while (lm) {
-            const int src = __ffs(lm) - 1;
-            lm &= lm - 1;
-            const int t = __shfl_sync(0xffffffffu, tok, src);
-            combine_token(d, t, it.f0, lane, gate, out, hidden);
-          }
+        if (last) {  // hand the block to the combine warps
+          __threadfence();  // every counted share before the hand-over
+          const int slot = atomicAdd(&cq_ctl[0], 1);
+          const unsigned long long t0 = global_ns();
+          for (uint32_t it_ = 1; cq[slot % kCombineQueue] >= 0; ++it_)  // ring full: wait
+            if ((it_ & 255) == 0 && (*abort_flag || global_ns() - t0 > kWaitLimitNs)) {
+              if (!*abort_flag) {
+                *abort_flag = 1;
+                atomicCAS(&st->status, EB_OK, EB_ERR_TIMEOUT);
+              }
+              break;
+            }
+          cq[slot % kCombineQueue] = tok * (d.H / C::kFeat) + it.f0 / C::kFeat;
         }
       }
+    }
+    if constexpr (COMBINE) {  // this drain warp pushes nothing more
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) atomicAdd(&cq_ctl[2], 1);
     }
   }
   tc_fence_before();
@@ -1222,7 +1287,7 @@ cudaError_t launch_gemm_tm(const Dims& d, const CtxDev& c, const Work& w, const 
                       (const int32_t*)w.seg_items1, w.gemm_next, rowslot, none,
                       static_cast<__nv_bfloat16*>(w.act), no_count, no_gate, no_hidden);
   if (combine_into)
-    return launch_pdl(k_gemm_tm<false, false, true>, dim3(grid), dim3(kThreads),
+    return launch_pdl(k_gemm_tm<false, false, true>, dim3(grid), dim3(kThreads + 32 * kCombineWarps),
                       CfgTM<false>::kSmemBytes, s, 1, maps.w_down, maps.act32, d, c.st,
                       (const int32_t*)w.seg_rows, (const int32_t*)w.seg_wid,
                       (const int32_t*)w.seg_items2, w.gemm_next + 1, rowslot, none,

@@ -217,6 +217,8 @@ eb_status eb_config_check(const eb_config* c) {
       c->k + c->n_shared > EB_MAX_K)
     return EB_ERR_UNSUPPORTED;
   if ((long long)c->M * c->L * c->T * c->E > (1ll << 40)) return EB_ERR_UNSUPPORTED;
+  // a RunSet's rank loads sum at most M T k token slots: int32 throughout
+  if ((long long)c->M * c->T * c->k > (1ll << 31) - 1) return EB_ERR_UNSUPPORTED;
   if (c->policy == EB_SCHED_MAXUTIL && maxutil_candidates(c->M, c->m) > kMaxUtilCandidateCap)
     return EB_ERR_UNSUPPORTED;
   if (c->compute) {

@@ -38,60 +38,76 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
+constexpr int kPosThreads = 512;
+
 // CTA (c, j): chunk c of RunSet micro-batch j.  Row of (t, s) = base of
 // (j, c, expert) + number of earlier (t', s') of this chunk with the same
 // expert, so rows follow (micro-batch, token, slot) order inside a segment.
-__global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State* __restrict__ st,
-                                                            const int32_t* __restrict__ idx,
-                                                            const int32_t* __restrict__ chunk_hist,
-                                                            const int32_t* __restrict__ seg_rows,
-                                                            const int32_t* __restrict__ prior,
-                                                            int32_t* __restrict__ pos,
-                                                            int32_t* __restrict__ rowslot) {
+// The base is the segment's first row + the rows of earlier RunSet members
+// of the segment (prior) + this micro-batch's rows in chunks 0..c-1.  Every
+// load that does not depend on the step state (the chunk's routing indices,
+// prior, the earlier chunks' counts) is issued before the state is read.
+__global__ void __launch_bounds__(kPosThreads) k_positions(Dims d, const State* __restrict__ st,
+                                                           const int32_t* __restrict__ idx,
+                                                           const int32_t* __restrict__ chunk_hist,
+                                                           const int32_t* __restrict__ seg_rows,
+                                                           const int32_t* __restrict__ prior,
+                                                           int32_t* __restrict__ pos,
+                                                           int32_t* __restrict__ rowslot) {
+  constexpr int kWarps = kPosThreads / 32;
   pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
-  if (!((st->runset >> j) & 1u)) return;
-  __shared__ int cnt[kPermThreads / 32][EB_MAX_ETOT];
+  __shared__ int cnt[kWarps][EB_MAX_ETOT];
   __shared__ int running[EB_MAX_ETOT];
   __shared__ int bj[EB_MAX_ETOT];  // first row of (j, this chunk, expert)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int t0 = c * kChunk, nt = min(kChunk, d.T - t0);
   const int k = d.k, kk = d.kk, E = d.E, Et = d.Etot;
-  const int g = st->group_of[j];
-  for (int e = tid; e < Et; e += kPermThreads) {
-    int b = seg_rows[g * Et + e] + prior[j * Et + e];
-    if (e < E) {
-      const int32_t* ch = chunk_hist + (size_t)j * d.NC * E + e;
-      int cc = 0;
-      for (; cc + 8 <= c; cc += 8) {  // eight independent loads in flight
-        int part[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) part[u] = __ldg(ch + (size_t)(cc + u) * E);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) b += part[u];
-      }
-      for (; cc < c; ++cc) b += __ldg(ch + (size_t)cc * E);
-    } else {
-      b += c * kChunk;
-    }
-    bj[e] = b;
-  }
-  for (int e = tid; e < E; e += kPermThreads) running[e] = 0;
   const int npairs = nt * k;
   const int32_t* idx_c = idx + ((size_t)j * d.T + t0) * k;
   int32_t* pos_c = pos + ((size_t)j * d.T + t0) * kk;
-  for (int r0 = 0; r0 < npairs; r0 += kPermThreads) {
-    for (int i = tid; i < (kPermThreads / 32) * E; i += kPermThreads) cnt[i / E][i % E] = 0;
-    __syncthreads();
+  // state-independent loads: the first round's expert, and for expert
+  // e = tid % Et the counts of chunks part, part + parts, ... below c
+  // (parts = threads per expert) plus, in part 0, prior
+  int e_next = tid < npairs ? __ldg(idx_c + tid) : -1;
+  const int parts = kPosThreads / Et, part = tid / Et, pe = tid % Et;
+  int partial = 0;
+  if (part < parts) {
+    if (pe < E) {
+      const int32_t* ch = chunk_hist + (size_t)j * d.NC * E + pe;
+      int cc = part;
+      for (; cc + 7 * parts < c; cc += 8 * parts) {  // eight independent loads in flight
+        int v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(ch + (size_t)(cc + u * parts) * E);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) partial += v[u];
+      }
+      for (; cc < c; cc += parts) partial += __ldg(ch + (size_t)cc * E);
+    } else if (part == 0) {
+      partial = c * kChunk;  // shared expert: every token of the earlier chunks
+    }
+    if (part == 0) partial += __ldg(prior + j * Et + pe);
+  }
+  for (int i = tid; i < kWarps * E; i += kPosThreads) cnt[i / E][i % E] = 0;
+  for (int e = tid; e < E; e += kPosThreads) running[e] = 0;
+  if (!((st->runset >> j) & 1u)) return;
+  const int g = st->group_of[j];
+  if (part == 0) bj[pe] = partial + seg_rows[g * Et + pe];
+  __syncthreads();
+  if (part > 0 && part < parts && partial) atomicAdd(&bj[pe], partial);
+  for (int r0 = 0; r0 < npairs; r0 += kPosThreads) {
     const int p = r0 + tid;
-    const int e = p < npairs ? idx_c[p] : -1;
+    const int e = e_next;
     const unsigned peers = __match_any_sync(kFull, e);
     const int rank = __popc(peers & lanemask_lt());
     if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] = __popc(peers);
+    if (p + kPosThreads < npairs) e_next = idx_c[p + kPosThreads];
+    else e_next = -1;
     __syncthreads();
-    for (int ee = tid; ee < E; ee += kPermThreads) {
+    for (int ee = tid; ee < E; ee += kPosThreads) {
       int run = running[ee];
-      for (int w = 0; w < kPermThreads / 32; ++w) {
+      for (int w = 0; w < kWarps; ++w) {
         const int t = cnt[w][ee];
         cnt[w][ee] = run;
         run += t;
@@ -104,9 +120,13 @@ __global__ void __launch_bounds__(kPermThreads) k_positions(Dims d, const State*
       pos_c[(p / k) * kk + p % k] = row;
       rowslot[row] = (j * d.T + t0 + p / k) * kk + p % k;
     }
-    __syncthreads();
+    if (r0 + kPosThreads < npairs) {
+      __syncthreads();
+      for (int i = tid; i < kWarps * E; i += kPosThreads) cnt[i / E][i % E] = 0;
+      __syncthreads();
+    }
   }
-  for (int i = tid; i < nt * d.n_shared; i += kPermThreads) {
+  for (int i = tid; i < nt * d.n_shared; i += kPosThreads) {
     const int t = i / d.n_shared, s = i % d.n_shared;
     pos_c[t * kk + k + s] = bj[E + s] + t;
     rowslot[bj[E + s] + t] = (j * d.T + t0 + t) * kk + k + s;
@@ -334,7 +354,7 @@ int persistent_grid(const void* kernel, int threads, int& cache) {
 int g_grid_copy_bf16 = 0, g_grid_copy_f32 = 0, g_grid_comb_bf16 = 0, g_grid_comb_f32 = 0;
 
 cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cudaStream_t s) {
-  return launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPermThreads), 0, s, 1, d, c.st,
+  return launch_pdl(k_positions, dim3(d.NC, d.M), dim3(kPosThreads), 0, s, 1, d, c.st,
                     (const int32_t*)w.idx, (const int32_t*)w.chunk_hist,
                     (const int32_t*)w.seg_rows, (const int32_t*)w.prior, w.pos, w.rowslot);
 }

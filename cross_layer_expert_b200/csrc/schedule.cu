@@ -71,6 +71,12 @@ __device__ __forceinline__ bool cand_wins(const Cand& a, const Cand& b) {
   return a.size >= 0 && (b.size < 0 || cand_better(a, b));
 }
 
+// Candidate counts up to this are searched by warp 0 alone; up to
+// kMaskEnumMax pending micro-batches warp 0's lanes walk every complement
+// bitmask directly instead of ranking the candidates.
+constexpr unsigned long long kWarpSearchMax = 1024;
+constexpr int kMaskEnumMax = 12;
+
 // Row stride of the load rows in shared memory: odd, so threads reading the
 // same rank of different micro-batches' rows hit different banks.
 constexpr int kWStride = EB_MAX_D + 1;
@@ -87,7 +93,6 @@ struct SchedSmem {
   int P[EB_MAX_M];            // pending micro-batch ids, ascending
   int n;
   Cand red[kThreads / 32];
-  uint32_t result;
 };
 
 __device__ __forceinline__ uint64_t gosper_next(uint64_t v) {
@@ -135,31 +140,46 @@ __device__ unsigned long long candidate_count(int n, int m) {
   return N;
 }
 
+// Loads and their sums stay below 2^31 (the configuration check bounds
+// M * T * k), so a candidate crosses lanes as four 32-bit words.
 __device__ Cand shfl_cand(const Cand& c, int off) {
   Cand o;
-  o.sum = __shfl_xor_sync(0xffffffffu, c.sum, off);
-  o.mx = __shfl_xor_sync(0xffffffffu, c.mx, off);
+  o.sum = __shfl_xor_sync(0xffffffffu, (int)c.sum, off);
+  o.mx = __shfl_xor_sync(0xffffffffu, (int)c.mx, off);
   o.size = __shfl_xor_sync(0xffffffffu, c.size, off);
   o.cmask = __shfl_xor_sync(0xffffffffu, c.cmask, off);
   return o;
+}
+
+// The scheduler kernel runs once per step from a cold instruction cache:
+// its time follows the size of the code it runs more than the arithmetic, so
+// the steps it repeats are single out-of-line copies with rolled loops.
+
+// All lanes: the best of the warp's candidates, returned to every lane.
+__device__ __noinline__ Cand warp_best(Cand best) {
+#pragma unroll 1
+  for (int off = 16; off; off >>= 1) {
+    const Cand o = shfl_cand(best, off);
+    if (cand_wins(o, best)) best = o;
+  }
+  return best;
+}
+
+// best := the better of best and the candidate S = P \ cm.
+__device__ __noinline__ void consider(const SchedSmem& sm, int D, uint32_t cm, Cand& best) {
+  const Cand cd = eval_complement(sm, D, cm);
+  if (cand_wins(cd, best)) best = cd;
 }
 
 // All threads of the block: the best of every thread's `best` (threads
 // without one pass size = -1).  Returns it to every thread.
 __device__ Cand block_best(Cand best, Cand* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int off = 16; off; off >>= 1) {
-    const Cand o = shfl_cand(best, off);
-    if (cand_wins(o, best)) best = o;
-  }
+  best = warp_best(best);
   if (lane == 0) red[warp] = best;
   __syncthreads();
   if (warp == 0) {
-    best = lane < (int)(blockDim.x >> 5) ? red[lane] : Cand{0, 0, -1, 0};
-    for (int off = 16; off; off >>= 1) {
-      const Cand o = shfl_cand(best, off);
-      if (cand_wins(o, best)) best = o;
-    }
+    best = warp_best(lane < (int)(blockDim.x >> 5) ? red[lane] : Cand{0, 0, -1, 0});
     if (lane == 0) red[0] = best;
   }
   __syncthreads();
@@ -170,18 +190,17 @@ __device__ Cand block_best(Cand best, Cand* red) {
 
 // This thread's best candidate over the complement ranks [r_lo, r_hi)
 // (sizes ascending, colexicographic order within a size), the range split
-// evenly over the block's threads.
-__device__ Cand search_ranks(const SchedSmem& sm, int D, int m, unsigned long long r_lo,
-                             unsigned long long r_hi) {
+// evenly over `parts` searchers of which this is number `part`.
+__device__ Cand search_ranks(const SchedSmem& sm, int D, unsigned long long r_lo,
+                             unsigned long long r_hi, int part, int parts) {
   const int n = sm.n;
   const uint32_t (*B)[33] = kBinom.v;
   const unsigned long long N = r_hi > r_lo ? r_hi - r_lo : 0;
-  const unsigned long long per = (N + blockDim.x - 1) / blockDim.x;
-  unsigned long long r = r_lo + per * threadIdx.x;
+  const unsigned long long per = (N + parts - 1) / parts;
+  unsigned long long r = r_lo + per * part;
   const unsigned long long r_end = r + per < r_hi ? r + per : r_hi;
   Cand best{0, 0, -1, 0};
   bool have = false;
-  (void)m;
   if (r < r_end) {
     int c = 0;
     unsigned long long q = r;
@@ -208,10 +227,19 @@ __device__ Cand search_ranks(const SchedSmem& sm, int D, int m, unsigned long lo
   return best;
 }
 
-// All threads of the block: MaxUtil over all complements of size <= n - m.
+// All threads of the block: MaxUtil over all complements of size <= n - m
+// (up to kMaskEnumMax pending micro-batches each thread walks the bitmasks
+// tid, tid + blockDim, ...; above, the candidate ranks are split).
 __device__ uint32_t maxutil_block(SchedSmem& sm, int D, int m) {
-  const Cand best = block_best(search_ranks(sm, D, m, 0, candidate_count(sm.n, m)), sm.red);
-  return cand_runset(sm, best);
+  const int n = sm.n;
+  Cand mine{0, 0, -1, 0};
+  if (n <= kMaskEnumMax) {
+    for (uint32_t cm = threadIdx.x; cm < (1u << n); cm += blockDim.x)
+      if (__popc(cm) <= n - m) consider(sm, D, cm, mine);
+  } else {
+    mine = search_ranks(sm, D, 0, candidate_count(n, m), threadIdx.x, blockDim.x);
+  }
+  return cand_runset(sm, block_best(mine, sm.red));
 }
 
 // All threads of the block: the best of the search grid's slots.
@@ -224,138 +252,226 @@ __device__ uint32_t maxutil_slots(SchedSmem& sm, const Cand* __restrict__ slots,
   return cand_runset(sm, block_best(best, sm.red));
 }
 
-// Thread 0 only: CumUtil (policy 0) or DiffPeak (policy 3), padded to m.
-__device__ uint32_t scan_policy(const SchedSmem& sm, int D, int m, int policy) {
-  const int n = sm.n;
-  long long W[EB_MAX_D];
-  for (int dd = 0; dd < D; ++dd) W[dd] = sm.w[0][dd];
-  long long sum = sm.wsum[0], mx = 0;
-  for (int dd = 0; dd < D; ++dd) mx = W[dd] > mx ? W[dd] : mx;
-  uint32_t chosen = 1u;  // positions in P
-  unsigned long long peaks = 0;
-  auto peak_of = [&](int i) {
-    int best = 0;
-    for (int dd = 1; dd < D; ++dd)
-      if (sm.w[i][dd] > sm.w[i][best]) best = dd;
-    return best;
-  };
-  if (policy == EB_SCHED_DIFFPEAK) peaks = 1ull << peak_of(0);
-  for (int i = 1; i < n; ++i) {
-    if (policy == EB_SCHED_DIFFPEAK) {
-      const int p = peak_of(i);
-      if (!((peaks >> p) & 1ull)) {
-        peaks |= 1ull << p;
-        chosen |= 1u << i;
-      }
-      continue;
-    }
-    long long nmx = 0;
-    for (int dd = 0; dd < D; ++dd) {
-      const long long v = W[dd] + sm.w[i][dd];
-      nmx = v > nmx ? v : nmx;
-    }
-    const long long nsum = sum + sm.wsum[i];
-    // U(S u {i}) > U(S) <=> nsum * mx > sum * nmx; a set without work has U = 0
-    bool gain;
-    if (nmx == 0 || mx == 0) gain = (nmx != 0 && mx == 0);
-    else gain = nsum * mx > sum * nmx;
-    if (gain) {
-      chosen |= 1u << i;
-      for (int dd = 0; dd < D; ++dd) W[dd] += sm.w[i][dd];
-      sum = nsum;
-      mx = nmx;
-    }
-  }
-  for (int i = 0; i < n && __popc(chosen) < m; ++i) chosen |= 1u << i;
-  uint32_t mask = 0;
-  for (int i = 0; i < n; ++i)
-    if ((chosen >> i) & 1u) mask |= 1u << sm.P[i];
-  return mask;
+__device__ __forceinline__ long long warp_sum_ll(long long x) {
+#pragma unroll
+  for (int off = 16; off; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
 }
 
-// All threads: loads w[j][:] of the pending set must be in sm.w (by position);
-// returns the RunSet mask (over micro-batch ids).  slots: the MaxUtil search
-// grid's results for this pending set (null: search here).
-__device__ void prepare_totals(SchedSmem& sm, int D) {
-  const int tid = threadIdx.x;
-  for (int dd = tid; dd < D; dd += blockDim.x) {
+// Warp 0: tot[d] = sum_i w_i[d], wsum[i] = sum_d w_i[d] and their total,
+// lanes over ranks and over pending positions (n <= 32).
+__device__ void warp_totals(SchedSmem& sm, int D) {
+  const int lane = threadIdx.x & 31, n = sm.n;
+  for (int dd = lane; dd < D; dd += 32) {
     long long t = 0;
-    for (int i = 0; i < sm.n; ++i) t += sm.w[i][dd];
+    for (int i = 0; i < n; ++i) t += sm.w[i][dd];
     sm.tot[dd] = t;
   }
-  for (int i = tid; i < sm.n; i += blockDim.x) {
-    long long t = 0;
-    for (int dd = 0; dd < D; ++dd) t += sm.w[i][dd];
-    sm.wsum[i] = t;
+  long long ws = 0;
+  if (lane < n) {
+    for (int dd = 0; dd < D; ++dd) ws += sm.w[lane][dd];
+    sm.wsum[lane] = ws;
   }
-  __syncthreads();
-  if (tid == 0) {
-    long long ts = 0;
-    for (int i = 0; i < sm.n; ++i) ts += sm.wsum[i];
-    sm.totsum = ts;
-  }
+  ws = warp_sum_ll(ws);
+  if (lane == 0) sm.totsum = ws;
+  __syncwarp();
+}
+
+// All threads: the totals (warp 0), visible to the block.
+__device__ void prepare_totals(SchedSmem& sm, int D) {
+  if ((threadIdx.x >> 5) == 0) warp_totals(sm, D);
   __syncthreads();
 }
 
-__device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending,
-                                  const Cand* slots = nullptr) {
-  prepare_totals(sm, D);
-  if (policy == EB_SCHED_LOCKSTEP || sm.n <= m) return pending;
-  if (policy == EB_SCHED_MAXUTIL)
-    return slots ? maxutil_slots(sm, slots, kSearchCtas) : maxutil_block(sm, D, m);
-  if (threadIdx.x == 0) sm.result = scan_policy(sm, D, m, policy);
-  __syncthreads();
-  return sm.result;
-}
-
-
-struct PlanSmem {
-  int3 tmp3[33];
-};
-
-// Expert counts of the RunSet's micro-batches kept in shared memory by the
-// plan when nr * E fits (32 KiB).
-constexpr int kPlanHistCache = 8192;
-
-// Exclusive block-wide scan of per-thread int3 values: returns this thread's
-// offsets; tmp[32] receives the block totals.  All threads must call it.
-__device__ int3 block_exclusive_scan3(int3 v, int3* tmp /* >= 33 */) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int3 incl = v;
+// Warp 0: the RunSet (micro-batch ids) of a policy that needs no block-wide
+// search, with the totals in place.  CumUtil walks the positions in order
+// with the candidate's W_d spread over the lanes (d = lane, lane + 32); a
+// step adds position i iff U(S u {i}) > U(S), compared exactly
+// (nsum * mx > sum * nmx; a set without work has U = 0).  DiffPeak adds i
+// iff its peak rank (lowest index of max_d w_i[d]) is the first occurrence
+// of that rank among positions 0..i.  Both then pad to m with the lowest
+// positions not taken.  MaxUtil splits the candidate ranks over the lanes.
+// Warp 0, n <= kMaskEnumMax and D <= 32: MaxUtil over every complement
+// bitmask with at most n - m bits, lane-strided; each candidate's W_d
+// (d < D <= DMAX) is summed in registers, so a complement's rows are read
+// with independent loads.
+template <int DMAX>
+__device__ __noinline__ Cand warp_maxutil_masks(const SchedSmem& sm, int D, int m) {
+  const int lane = threadIdx.x & 31, n = sm.n, cmax = n - m;
+  Cand best{0, 0, -1, 0};
+  for (uint32_t cm = lane; cm < (1u << n); cm += 32) {
+    if (__popc(cm) > cmax) continue;
+    int W[DMAX];
+    long long sum = sm.totsum;
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int yx = __shfl_up_sync(0xffffffffu, incl.x, off);
-    const int yy = __shfl_up_sync(0xffffffffu, incl.y, off);
-    const int yz = __shfl_up_sync(0xffffffffu, incl.z, off);
-    if (lane >= off) {
-      incl.x += yx;
-      incl.y += yy;
-      incl.z += yz;
+    for (int d = 0; d < DMAX; ++d) W[d] = d < D ? (int)sm.tot[d] : 0;
+    for (uint32_t b = cm; b; b &= b - 1) {
+      const int i = __ffs(b) - 1;
+      sum -= sm.wsum[i];
+#pragma unroll
+      for (int d = 0; d < DMAX; ++d)
+        if (d < D) W[d] -= sm.w[i][d];
     }
-  }
-  if (lane == 31) tmp[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    const int3 x = lane < nw ? tmp[lane] : make_int3(0, 0, 0);
-    int3 xi = x;
+    int mx = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int yx = __shfl_up_sync(0xffffffffu, xi.x, off);
-      const int yy = __shfl_up_sync(0xffffffffu, xi.y, off);
-      const int yz = __shfl_up_sync(0xffffffffu, xi.z, off);
-      if (lane >= off) {
-        xi.x += yx;
-        xi.y += yy;
-        xi.z += yz;
+    for (int d = 0; d < DMAX; ++d) mx = W[d] > mx ? W[d] : mx;
+    const Cand cd{sum, (long long)mx, n - __popc(cm), cm};
+    if (cand_wins(cd, best)) best = cd;
+  }
+  return warp_best(best);
+}
+
+__device__ uint32_t warp_choose(SchedSmem& sm, int D, int m, int policy, uint32_t pending) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31, n = sm.n;
+  if (policy == EB_SCHED_LOCKSTEP || n <= m) return pending;
+  if (policy == EB_SCHED_MAXUTIL) {
+    warp_totals(sm, D);
+    Cand best{0, 0, -1, 0};
+    if (n <= kMaskEnumMax && D <= 32) {
+      best = D <= 8    ? warp_maxutil_masks<8>(sm, D, m)
+             : D <= 16 ? warp_maxutil_masks<16>(sm, D, m)
+                       : warp_maxutil_masks<32>(sm, D, m);
+    } else if (n <= kMaskEnumMax) {
+      for (uint32_t cm = lane; cm < (1u << n); cm += 32)
+        if (__popc(cm) <= n - m) consider(sm, D, cm, best);
+      best = warp_best(best);
+    } else {
+      best = warp_best(search_ranks(sm, D, 0, candidate_count(n, m), lane, 32));
+    }
+    return cand_runset(sm, best);
+  }
+  uint32_t chosen;  // positions in P
+  if (policy == EB_SCHED_DIFFPEAK) {
+    int peak = -1 - lane;  // distinct keys for lanes without a position
+    if (lane < n) {
+      peak = 0;
+      for (int dd = 1; dd < D; ++dd)
+        if (sm.w[lane][dd] > sm.w[lane][peak]) peak = dd;
+    }
+    const unsigned same = __match_any_sync(kFull, peak);
+    chosen = __ballot_sync(kFull, lane < n && (__ffs(same) - 1) == lane);
+  } else {
+    warp_totals(sm, D);
+    const int d0 = lane, d1 = lane + 32;
+    int W0 = d0 < D ? sm.w[0][d0] : 0, W1 = d1 < D ? sm.w[0][d1] : 0;
+    long long sum = sm.wsum[0];
+    long long mx = __reduce_max_sync(kFull, W0 > W1 ? W0 : W1);
+    chosen = 1u;
+    // the next row's loads are issued one step ahead
+    int x0 = n > 1 && d0 < D ? sm.w[1][d0] : 0, x1 = n > 1 && d1 < D ? sm.w[1][d1] : 0;
+    long long xs = n > 1 ? sm.wsum[1] : 0;
+    for (int i = 1; i < n; ++i) {
+      const int c0 = x0, c1 = x1;
+      const long long cs = xs;
+      if (i + 1 < n) {
+        x0 = d0 < D ? sm.w[i + 1][d0] : 0;
+        x1 = d1 < D ? sm.w[i + 1][d1] : 0;
+        xs = sm.wsum[i + 1];
+      }
+      const int v0 = W0 + c0, v1 = W1 + c1;
+      const long long nmx = __reduce_max_sync(kFull, v0 > v1 ? v0 : v1);
+      const long long nsum = sum + cs;
+      bool gain;
+      if (nmx == 0 || mx == 0) gain = (nmx != 0 && mx == 0);
+      else gain = nsum * mx > sum * nmx;
+      if (gain) {
+        chosen |= 1u << i;
+        W0 = v0;
+        W1 = v1;
+        sum = nsum;
+        mx = nmx;
       }
     }
-    if (lane < nw) tmp[lane] = make_int3(xi.x - x.x, xi.y - x.y, xi.z - x.z);
-    if (lane == 31) tmp[32] = xi;
   }
-  __syncthreads();
-  const int3 w = tmp[warp];
-  return make_int3(w.x + incl.x - v.x, w.y + incl.y - v.y, w.z + incl.z - v.z);
+  const uint32_t posmask = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+  const int need = m - __popc(chosen);
+  if (need > 0 && lane < n && !((chosen >> lane) & 1u) &&
+      __popc(~chosen & posmask & ((1u << lane) - 1u)) < need)
+    chosen |= 1u << lane;
+  chosen = __reduce_or_sync(kFull, chosen);
+  return __reduce_or_sync(kFull, (lane < n && ((chosen >> lane) & 1u)) ? 1u << sm.P[lane] : 0u);
 }
+
+
+// All threads, with sm.P, sm.n and the pending rows sm.w (by position) in
+// place.  Returns the RunSet (micro-batch ids) to warp 0; the other threads'
+// return value is unspecified.  slots: the MaxUtil search grid's results for
+// this pending set (null: search here).  Only a large MaxUtil search uses
+// the whole block.
+__device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending,
+                                  const Cand* slots) {
+  const int n = sm.n;
+  if (policy == EB_SCHED_MAXUTIL && n > m &&
+      (slots != nullptr || candidate_count(n, m) > kWarpSearchMax)) {
+    prepare_totals(sm, D);
+    return slots ? maxutil_slots(sm, slots, kSearchCtas) : maxutil_block(sm, D, m);
+  }
+  if ((threadIdx.x >> 5) != 0) return 0u;
+  return warp_choose(sm, D, m, policy, pending);
+}
+
+// Warp 0: the step's exact accounting -- sum_d W_d, max_d W_d of the RunSet
+// and the sum over its members of their own peaks (Eq. (3) numerator and
+// the scheduled and separate denominators / D).
+__device__ void warp_account(const SchedSmem& sm, int D, uint32_t run, long long& sumW,
+                             long long& maxW, long long& summax) {
+  constexpr unsigned kFull = 0xffffffffu;
+  const int lane = threadIdx.x & 31, n = sm.n;
+  // positions in P of the RunSet's members
+  const uint32_t rpos = __ballot_sync(kFull, lane < n && ((run >> sm.P[lane]) & 1u));
+  unsigned s = 0;
+  int mxw = 0;
+  for (int dd = lane; dd < D; dd += 32) {
+    int Wd = 0;
+    for (uint32_t b = rpos; b; b &= b - 1) Wd += sm.w[__ffs(b) - 1][dd];
+    s += (unsigned)Wd;
+    mxw = Wd > mxw ? Wd : mxw;
+  }
+  unsigned own = 0;
+  if ((rpos >> lane) & 1u) {
+    int mx = 0;
+    for (int dd = 0; dd < D; ++dd) mx = sm.w[lane][dd] > mx ? sm.w[lane][dd] : mx;
+    own = (unsigned)mx;
+  }
+  sumW = __reduce_add_sync(kFull, s);
+  maxW = __reduce_max_sync(kFull, mxw);
+  summax = __reduce_add_sync(kFull, own);
+}
+
+// All threads: sm.P / sm.n from the pending mask, and the pending rows of
+// sm.w (loaded by micro-batch id) moved to their positions (P ascending,
+// so row p reads row P[p] >= p; every thread reads before any writes).
+// Blocks of kThreads threads.
+__device__ void compact_rows(SchedSmem& sm, uint32_t pending, int M, int D) {
+  constexpr int kPer = (EB_MAX_M * EB_MAX_D) / 1024;
+  const int tid = threadIdx.x;
+  int val[kPer], dst[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int i = tid + q * kThreads;
+    dst[q] = -1;
+    if (i < M * D) {
+      const int j = i / D, dd = i % D;
+      if ((pending >> j) & 1u) {
+        dst[q] = __popc(pending & ((1u << j) - 1u)) * kWStride + dd;
+        val[q] = sm.w[j][dd];
+      }
+    }
+  }
+  if (tid < M && ((pending >> tid) & 1u)) sm.P[__popc(pending & ((1u << tid) - 1u))] = tid;
+  if (tid == 0) sm.n = __popc(pending);
+  __syncthreads();
+#pragma unroll
+  for (int q = 0; q < kPer; ++q)
+    if (dst[q] >= 0) (&sm.w[0][0])[dst[q]] = val[q];
+  __syncthreads();
+}
+
+
+// Expert counts of every micro-batch, kept in shared memory by the plan
+// (M * E <= EB_MAX_M * EB_MAX_ETOT int32: 32 KiB).
+constexpr int kPlanHistCache = EB_MAX_M * EB_MAX_ETOT;
 
 constexpr int kSearchThreads = 256;
 
@@ -467,242 +583,259 @@ __global__ void __launch_bounds__(kSearchThreads) k_maxutil_search(int M, int D,
   if (tid == 0) slots[blockIdx.x] = best;
 }
 
+// Work items of a segment of n rows: ceil(n / rows per item) * feature blocks.
+__device__ __noinline__ int items_of(int n, int rn, int mb) { return (n + rn - 1) / rn * mb; }
+
+// All threads: zero the counts and loads of the micro-batches routed at
+// the next step (warp j clears row j).
+__device__ void zero_next(const Dims& d, const CtxDev& c, uint32_t next) {
+  const int lane = threadIdx.x & 31;
+  for (int j = threadIdx.x >> 5; j < d.M; j += kThreads / 32)
+    if ((next >> j) & 1u) {
+      for (int e = lane; e < d.E; e += 32) c.hist[j * d.E + e] = 0;
+      for (int r = lane; r < d.D; r += 32) c.w[j * d.D + r] = 0;
+    }
+}
+
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
                                                              int rn2, int fm1, int fm2) {
   __shared__ SchedSmem sm;
-  __shared__ PlanSmem pl;
-  // the step state lives in shared memory for the whole kernel (thread 0's
-  // bookkeeping would otherwise be a chain of dependent global loads)
+  // the step state lives in shared memory for the whole kernel
   __shared__ State ss;
+  __shared__ int s_hist[kPlanHistCache];  // hist[j][e] of every micro-batch, by id
   State* st = &ss;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   pdl_enter();
+  // 1. one round of global loads: the state, the loads w[j][:] of every
+  //    micro-batch (by id) and, for the plan, the expert counts hist[j][:]
+  //    accumulated by the routing kernel
   constexpr int kStateWords = sizeof(State) / sizeof(int);
-  for (int i = tid; i < kStateWords; i += blockDim.x)
+  for (int i = tid; i < kStateWords; i += kThreads)
     reinterpret_cast<int*>(&ss)[i] = reinterpret_cast<const int*>(c.st)[i];
+  for (int i = tid; i < d.M * d.D; i += kThreads) sm.w[i / d.D][i % d.D] = c.w[i];
+  if (d.compute)
+    for (int i = tid; i < d.M * d.E; i += kThreads) s_hist[i] = c.hist[i];
   __syncthreads();
   auto write_back = [&]() {
     __syncthreads();
-    for (int i = tid; i < kStateWords; i += blockDim.x)
+    for (int i = tid; i < kStateWords; i += kThreads)
       reinterpret_cast<int*>(c.st)[i] = reinterpret_cast<const int*>(&ss)[i];
+  };
+  auto finish_empty = [&]() {
+    if (tid == 0) {
+      st->pending = ss.status == EB_ERR_TIMEOUT ? 0u : st->pending;
+      st->runset = 0;
+      st->n_run = 0;
+      st->need_route = 0;
+      st->nseg = 0;
+      st->items1 = 0;
+      st->items2 = 0;
+      st->rows = 0;
+      for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
+    }
+    write_back();
   };
   // A context whose status word holds EB_ERR_TIMEOUT (a bounded wait of an
   // earlier step expired, so its state may be partial) runs no further step
-  // until eb_reset: the step does nothing and reports S as empty.
-  if (ss.status == EB_ERR_TIMEOUT) {
-    if (tid == 0) {
-      st->pending = 0;
-      st->runset = 0;
-      st->n_run = 0;
-      st->need_route = 0;
-      st->nseg = 0;
-      st->items1 = 0;
-      st->items2 = 0;
-      st->rows = 0;
-      for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
-    }
-    write_back();
+  // until eb_reset: the step does nothing and reports S as empty.  A step
+  // with S empty (episode finished) does nothing either.
+  const uint32_t pending = ss.pending;
+  if (ss.status == EB_ERR_TIMEOUT || pending == 0u) {
+    finish_empty();
     return;
   }
-  // 1. hist[j][:] and w[j][:] of the micro-batches routed for this step were
-  //    accumulated by the routing kernel
-  // 2. pending set
-  const uint32_t pending = st->pending;
-  if (tid == 0) {
-    int n = 0;
-    for (int j = 0; j < d.M; ++j)
-      if ((pending >> j) & 1u) sm.P[n++] = j;
-    sm.n = n;
-  }
-  __syncthreads();
-  if (sm.n == 0) {  // episode finished: this step does nothing
-    if (tid == 0) {
-      st->runset = 0;
-      st->n_run = 0;
-      st->need_route = 0;
-      st->nseg = 0;
-      st->items1 = 0;
-      st->items2 = 0;
-      st->rows = 0;
-      for (int j = 0; j < d.M; ++j) st->step_layer[j] = -1;
-    }
-    write_back();
-    return;
-  }
-  for (int i = tid; i < sm.n * d.D; i += blockDim.x) {
-    const int p = i / d.D, dd = i % d.D;
-    sm.w[p][dd] = c.w[sm.P[p] * d.D + dd];
-  }
-  __syncthreads();
-  // 3. RunSet
+  // 2. pending set: positions in P and the pending rows of w by position
+  compact_rows(sm, pending, d.M, d.D);
+  // 3. RunSet (in warp 0)
   const uint32_t run = choose_runset(sm, d.D, d.m, d.policy, pending,
                                      static_cast<const Cand*>(c.search_slots));
-  // 4. accounting, trace and Algorithm 1 bookkeeping (thread 0)
-  if (tid == 0) {
-    long long sumW = 0, maxW = 0, summax = 0;
-    for (int dd = 0; dd < d.D; ++dd) {
-      long long Wd = 0;
-      for (int p = 0; p < sm.n; ++p)
-        if ((run >> sm.P[p]) & 1u) Wd += sm.w[p][dd];
-      sumW += Wd;
-      maxW = Wd > maxW ? Wd : maxW;
-    }
-    for (int p = 0; p < sm.n; ++p)
-      if ((run >> sm.P[p]) & 1u) {
-        long long mx = 0;
-        for (int dd = 0; dd < d.D; ++dd) mx = sm.w[p][dd] > mx ? sm.w[p][dd] : mx;
-        summax += mx;
-      }
-    st->num += sumW;
-    st->den += (long long)d.D * maxW;
-    st->den_sep += (long long)d.D * summax;
+  // 4. accounting, trace and Algorithm 1 bookkeeping (warp 0: lane j is
+  //    micro-batch j, M <= 32)
+  __shared__ int s_group_run[EB_MAX_M];  // group of RunSet member a
+  if (warp == 0) {
+    long long sumW, maxW, summax;
+    warp_account(sm, d.D, run, sumW, maxW, summax);
     const int step = st->n_steps;
+    const int j = lane;
+    const bool inrun = j < d.M && ((run >> j) & 1u);
+    const int lj = j < d.M ? st->layer[j] : 0;  // l_j before this step
     if (step < d.max_steps) {
-      c.trace[step * kTraceCols + 0] = run;
-      c.trace[step * kTraceCols + 1] = sumW;
-      c.trace[step * kTraceCols + 2] = maxW;
-      c.trace[step * kTraceCols + 3] = summax;
-      c.trace[step * kTraceCols + 4] = 0;
-      c.trace[step * kTraceCols + 5] = 0;
-      for (int j = 0; j < d.M; ++j)
-        c.trace_layers[step * d.M + j] = ((run >> j) & 1u) ? st->layer[j] : -1;
-    }
-    st->n_steps = step + 1;
-    int nr = 0;
-    uint32_t still = 0;
-    for (int j = 0; j < d.M; ++j) {
-      if ((run >> j) & 1u) {
-        st->step_layer[j] = st->layer[j];
-        st->run_list[nr++] = j;
-        st->layer[j] += 1;
-      } else {
-        st->step_layer[j] = -1;
+      if (lane == 0) {
+        c.trace[step * kTraceCols + 0] = run;
+        c.trace[step * kTraceCols + 1] = sumW;
+        c.trace[step * kTraceCols + 2] = maxW;
+        c.trace[step * kTraceCols + 3] = summax;
+        c.trace[step * kTraceCols + 4] = 0;
+        c.trace[step * kTraceCols + 5] = 0;
       }
-      if (st->layer[j] < d.L) still |= 1u << j;
+      if (j < d.M) c.trace_layers[step * d.M + j] = inrun ? lj : -1;
     }
-    st->n_run = nr;
-    st->runset = run;
-    st->pending = still;
-    st->need_route = run & still;
-    // segment groups: distinct layers of the RunSet, ascending
-    int G = 0;
-    for (int a = 0; a < nr; ++a) {
-      const int l = st->step_layer[st->run_list[a]];
-      bool seen = false;
-      for (int g = 0; g < G; ++g) seen |= (st->group_layer[g] == l);
-      if (!seen) {
-        int g = G++;
-        while (g > 0 && st->group_layer[g - 1] > l) {
-          st->group_layer[g] = st->group_layer[g - 1];
-          --g;
-        }
-        st->group_layer[g] = l;
-      }
+    const int nl = lj + (inrun ? 1 : 0);
+    const uint32_t still = __ballot_sync(0xffffffffu, j < d.M && nl < d.L);
+    // segment groups: the distinct layers of the RunSet, ascending; lane j's
+    // group is the number of distinct RunSet layers below l_j
+    const unsigned same = __match_any_sync(0xffffffffu, inrun ? lj : -1 - lane);
+    const bool leader = inrun && (__ffs(same) - 1) == lane;
+    const uint32_t leaders = __ballot_sync(0xffffffffu, leader);
+    int g = 0;
+    for (uint32_t b = leaders; b; b &= b - 1) {
+      const int li = __shfl_sync(0xffffffffu, lj, __ffs(b) - 1);
+      g += li < lj;
     }
-    for (int a = 0; a < nr; ++a) {
-      const int j = st->run_list[a];
-      for (int g = 0; g < G; ++g)
-        if (st->group_layer[g] == st->step_layer[j]) st->group_of[j] = g;
+    __syncwarp();  // every lane has read n_steps and l_j before they change
+    if (j < d.M) {
+      st->step_layer[j] = inrun ? lj : -1;
+      st->layer[j] = nl;
     }
-    st->n_groups = G;
-    st->nseg = G * d.Etot;
+    if (inrun) {
+      const int a = __popc(run & ((1u << j) - 1u));
+      st->run_list[a] = j;
+      st->group_of[j] = g;
+      s_group_run[a] = g;
+    }
+    if (leader) st->group_layer[g] = lj;
+    if (lane == 0) {
+      st->num += sumW;
+      st->den += (long long)d.D * maxW;
+      st->den_sep += (long long)d.D * summax;
+      st->n_steps = step + 1;
+      st->n_run = __popc(run);
+      st->runset = run;
+      st->pending = still;
+      st->need_route = run & still;
+      st->n_groups = __popc(leaders);
+      st->nseg = __popc(leaders) * d.Etot;
+    }
   }
+  __syncthreads();
   if (!d.compute) {
-    __syncthreads();
-    const uint32_t next = st->need_route;
-    for (int i = tid; i < d.M * d.E; i += blockDim.x)
-      if ((next >> (i / d.E)) & 1u) c.hist[i] = 0;
-    for (int i = tid; i < d.M * d.D; i += blockDim.x)
-      if ((next >> (i / d.D)) & 1u) c.w[i] = 0;
+    zero_next(d, c, st->need_route);
     write_back();
     return;
   }
-  __syncthreads();
-  // 5. segment plan: rows of (group, expert) are counted into seg_rows and
-  //    scanned in place; GEMM work items per segment likewise.  The RunSet's
-  //    expert counts are staged in shared memory when they fit (the counts
-  //    and the prior table below read them several times).
+  // 5. segment plan, one warp per segment group (G <= 32 warps).  Lane l of
+  //    warp g holds the segments (g, e) for e in [l Q, (l + 1) Q), Q =
+  //    ceil(Et / 32).  The warp walks the group's members in RunSet order:
+  //    prior[j][e] is the running count before member j and the final count
+  //    is the segment's rows.  Items per segment follow, a warp scan gives
+  //    the offsets inside the group's row, and after one barrier a scan of
+  //    the G row totals gives each row's base.  The kernel runs once per
+  //    step from a cold instruction cache, so its loops stay rolled: code
+  //    size, not arithmetic, sets the time of this single-CTA kernel.
   const int G = st->n_groups, nr = st->n_run, Et = d.Etot, nseg = G * Et;
   const int mb1 = d.F / fm1, mb2 = d.H / fm2;
-  __shared__ int s_nonempty;
-  __shared__ int s_hist[kPlanHistCache];
-  const bool cached = nr * d.E <= kPlanHistCache;
-  if (tid == 0) s_nonempty = 0;
-  if (cached)
-    for (int i = tid; i < nr * d.E; i += blockDim.x)
-      s_hist[i] = c.hist[st->run_list[i / d.E] * d.E + i % d.E];
+  constexpr int kQ = EB_MAX_ETOT / 32;
+  const int Q = (Et + 31) / 32, e0 = lane * Q;
+  __shared__ int4 s_rowtot[EB_MAX_M];  // rows, items1, items2, non-empty segments of each group
+  int cnt[kQ];
+  int3 mine = make_int3(0, 0, 0);  // this lane's sums of rows, items1, items2
+  if (warp < G) {
+#pragma unroll 1
+    for (int q = 0; q < Q; ++q) cnt[q] = 0;
+    for (int a = 0; a < nr; ++a) {
+      if (s_group_run[a] != warp) continue;  // warp-uniform
+      const int j = st->run_list[a];
+      const int* hj = s_hist + j * d.E;
+      int32_t* pj = wk.prior + j * Et;
+#pragma unroll 1
+      for (int q = 0; q < Q; ++q) {
+        const int e = e0 + q;
+        if (e < Et) {
+          pj[e] = cnt[q];
+          cnt[q] += e < d.E ? hj[e] : d.T;  // a shared expert takes every token
+        }
+      }
+    }
+    int nonempty = 0;
+#pragma unroll 1
+    for (int q = 0; q < Q; ++q) {
+      const int e = e0 + q;
+      if (e < Et) {
+        mine.x += cnt[q];
+        mine.y += items_of(cnt[q], rn1, mb1);
+        mine.z += items_of(cnt[q], rn2, mb2);
+        nonempty += cnt[q] > 0;
+        wk.seg_wid[warp * Et + e] = st->group_layer[warp] * Et + e;
+      }
+    }
+    // inclusive warp scan of the lanes' sums; lane 31 holds the row's totals
+    int3 inc = mine;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, inc.x, off);
+      const int y = __shfl_up_sync(0xffffffffu, inc.y, off);
+      const int z = __shfl_up_sync(0xffffffffu, inc.z, off);
+      if (lane >= off) {
+        inc.x += x;
+        inc.y += y;
+        inc.z += z;
+      }
+    }
+    nonempty = __reduce_add_sync(0xffffffffu, nonempty);
+    if (lane == 31) s_rowtot[warp] = make_int4(inc.x, inc.y, inc.z, nonempty);
+    mine = make_int3(inc.x - mine.x, inc.y - mine.y, inc.z - mine.z);  // exclusive
+  }
   __syncthreads();
-  // counts of RunSet member a (position in run_list) for expert e
-  auto count_of = [&](int a, int e) -> int {
-    if (e >= d.E) return d.T;  // shared expert: every token
-    return cached ? s_hist[a * d.E + e] : c.hist[st->run_list[a] * d.E + e];
-  };
-  int my_nonempty = 0;
-  int3 local = make_int3(0, 0, 0);  // this thread's sums of rows, items1, items2
-  const int per = (nseg + blockDim.x - 1) / blockDim.x;
-  const int sb = tid * per, se = min(nseg, sb + per);
-  for (int i = sb; i < se; ++i) {
-    const int g = i / Et, e = i % Et;
-    int cnt = 0;
-    for (int a = 0; a < nr; ++a)
-      if (st->group_of[st->run_list[a]] == g) cnt += count_of(a, e);
-    my_nonempty += cnt > 0;
-    const int i1 = (cnt + rn1 - 1) / rn1 * mb1, i2 = (cnt + rn2 - 1) / rn2 * mb2;
-    wk.seg_rows[i] = cnt;
-    wk.seg_items1[i] = i1;
-    wk.seg_items2[i] = i2;
-    wk.seg_wid[i] = st->group_layer[g] * Et + e;
-    local.x += cnt;
-    local.y += i1;
-    local.z += i2;
-  }
-  if (my_nonempty) atomicAdd(&s_nonempty, my_nonempty);
-  // one block-wide exclusive scan of the three running sums
-  const int3 base = block_exclusive_scan3(local, pl.tmp3);
-  int3 acc3 = base;
-  for (int i = sb; i < se; ++i) {
-    const int a = wk.seg_rows[i], b = wk.seg_items1[i], cc = wk.seg_items2[i];
-    wk.seg_rows[i] = acc3.x;
-    wk.seg_items1[i] = acc3.y;
-    wk.seg_items2[i] = acc3.z;
-    acc3.x += a;
-    acc3.y += b;
-    acc3.z += cc;
-  }
-  const int rows = pl.tmp3[32].x, it1 = pl.tmp3[32].y, it2 = pl.tmp3[32].z;
-  if (tid == 0) {
-    wk.seg_rows[nseg] = rows;
-    wk.seg_items1[nseg] = it1;
-    wk.seg_items2[nseg] = it2;
-    st->rows = rows;
-    st->items1 = it1;
-    st->items2 = it2;
-    wk.gemm_next[0] = 0;
-    wk.gemm_next[1] = 0;
-    const int step = st->n_steps - 1;  // the row written above
-    if (step < d.max_steps) {
-      c.trace[step * kTraceCols + 4] = rows;
-      c.trace[step * kTraceCols + 5] = s_nonempty;
+  if (warp < G) {
+    // base of row g: the totals of rows 0..g-1 (lane r holds row r's)
+    int4 t = lane < G ? s_rowtot[lane] : make_int4(0, 0, 0, 0);
+    int4 inc = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, inc.x, off);
+      const int y = __shfl_up_sync(0xffffffffu, inc.y, off);
+      const int z = __shfl_up_sync(0xffffffffu, inc.z, off);
+      const int w = __shfl_up_sync(0xffffffffu, inc.w, off);
+      if (lane >= off) {
+        inc.x += x;
+        inc.y += y;
+        inc.z += z;
+        inc.w += w;
+      }
+    }
+    const int bx = __shfl_sync(0xffffffffu, inc.x - t.x, warp);
+    const int by = __shfl_sync(0xffffffffu, inc.y - t.y, warp);
+    const int bz = __shfl_sync(0xffffffffu, inc.z - t.z, warp);
+    int3 acc3 = make_int3(bx + mine.x, by + mine.y, bz + mine.z);
+#pragma unroll 1
+    for (int q = 0; q < Q; ++q) {
+      const int e = e0 + q;
+      if (e < Et) {
+        const int i = warp * Et + e;
+        wk.seg_rows[i] = acc3.x;
+        wk.seg_items1[i] = acc3.y;
+        wk.seg_items2[i] = acc3.z;
+        acc3.x += cnt[q];
+        acc3.y += items_of(cnt[q], rn1, mb1);
+        acc3.z += items_of(cnt[q], rn2, mb2);
+      }
+    }
+    if (warp == 0) {
+      // every row's totals: lane G - 1's inclusive sums
+      const int rows = __shfl_sync(0xffffffffu, inc.x, G - 1);
+      const int it1 = __shfl_sync(0xffffffffu, inc.y, G - 1);
+      const int it2 = __shfl_sync(0xffffffffu, inc.z, G - 1);
+      const int ne = __shfl_sync(0xffffffffu, inc.w, G - 1);
+      if (lane == 0) {
+        wk.seg_rows[nseg] = rows;
+        wk.seg_items1[nseg] = it1;
+        wk.seg_items2[nseg] = it2;
+        st->rows = rows;
+        st->items1 = it1;
+        st->items2 = it2;
+        wk.gemm_next[0] = 0;
+        wk.gemm_next[1] = 0;
+        const int step = st->n_steps - 1;  // the row written above
+        if (step < d.max_steps) {
+          c.trace[step * kTraceCols + 4] = rows;
+          c.trace[step * kTraceCols + 5] = ne;
+        }
+      }
     }
   }
-  __syncthreads();
-  // rows of (j's segment, expert) taken by earlier micro-batches of its group;
-  // the permute kernel adds the earlier chunks of j itself
-  for (int i = tid; i < nr * Et; i += blockDim.x) {
-    const int a = i / Et, e = i % Et;
-    const int j = st->run_list[a], g = st->group_of[j];
-    int prior = 0;
-    for (int b = 0; b < a; ++b)
-      if (st->group_of[st->run_list[b]] == g) prior += count_of(b, e);
-    wk.prior[j * Et + e] = prior;
-  }
-  __syncthreads();
-  // the micro-batches routed at the next step start from zero counts
-  const uint32_t next = st->need_route;
-  for (int i = tid; i < d.M * d.E; i += blockDim.x)
-    if ((next >> (i / d.E)) & 1u) c.hist[i] = 0;
-  for (int i = tid; i < d.M * d.D; i += blockDim.x)
-    if ((next >> (i / d.D)) & 1u) c.w[i] = 0;
+  // the micro-batches routed at the next step start from zero counts (the
+  // counts of this step were read into shared memory above)
+  zero_next(d, c, st->need_route);
   write_back();
 }
 
@@ -714,46 +847,27 @@ __global__ void __launch_bounds__(kThreads) k_schedule_once(const int32_t* __res
                                                              const Cand* __restrict__ slots) {
   __shared__ SchedSmem sm;
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    int n = 0;
-    for (int j = 0; j < M; ++j)
-      if ((pending >> j) & 1u) sm.P[n++] = j;
-    sm.n = n;
-  }
-  __syncthreads();
-  if (sm.n == 0) {
+  if (pending == 0u) {
     if (tid == 0) {
       *runset_out = 0;
       if (stats) stats[0] = stats[1] = stats[2] = 0;
     }
     return;
   }
-  for (int i = tid; i < sm.n * D; i += blockDim.x) {
-    const int p = i / D, dd = i % D;
-    sm.w[p][dd] = w[sm.P[p] * D + dd];
-  }
+  for (int i = tid; i < M * D; i += kThreads) sm.w[i / D][i % D] = w[i];
   __syncthreads();
+  compact_rows(sm, pending, M, D);
   const uint32_t run = choose_runset(sm, D, m, policy, pending, slots);
-  if (tid == 0) {
-    *runset_out = run;
-    if (stats) {
-      long long sumW = 0, maxW = 0, summax = 0;
-      for (int dd = 0; dd < D; ++dd) {
-        long long Wd = 0;
-        for (int p = 0; p < sm.n; ++p)
-          if ((run >> sm.P[p]) & 1u) Wd += sm.w[p][dd];
-        sumW += Wd;
-        maxW = Wd > maxW ? Wd : maxW;
+  if ((tid >> 5) == 0) {
+    long long sumW, maxW, summax;
+    warp_account(sm, D, run, sumW, maxW, summax);
+    if (tid == 0) {
+      *runset_out = run;
+      if (stats) {
+        stats[0] = sumW;
+        stats[1] = maxW;
+        stats[2] = summax;
       }
-      for (int p = 0; p < sm.n; ++p)
-        if ((run >> sm.P[p]) & 1u) {
-          long long mx = 0;
-          for (int dd = 0; dd < D; ++dd) mx = sm.w[p][dd] > mx ? sm.w[p][dd] : mx;
-          summax += mx;
-        }
-      stats[0] = sumW;
-      stats[1] = maxW;
-      stats[2] = summax;
     }
   }
 }

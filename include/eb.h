@@ -102,7 +102,7 @@ typedef struct eb_config {
   int D;        /* virtual EP ranks; E % D == 0; rank d holds experts
                    [d E/D, (d+1) E/D)  ([EB] §5 Models: even mapping)     */
   int M;        /* micro-batches, 1..EB_MAX_M                            */
-  int T;        /* tokens per micro-batch, >= 1                          */
+  int T;        /* tokens per micro-batch, >= 1; M * T * k < 2^31      */
   int n_shared; /* always-on shared experts per layer (gate 1.0, not
                    counted in the workloads w)                           */
   int renorm;   /* 1: gates renormalised over the top-k                  */

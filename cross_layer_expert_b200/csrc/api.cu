@@ -32,6 +32,8 @@ struct eb_ctx {
   // set once the host has seen EB_ERR_TIMEOUT in the status word; steps are
   // refused until eb_reset
   bool timed_out = false;
+  // the previous step already enqueued this step's routing (eb_episode)
+  bool routed_ahead = false;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
   // cached TMA maps (rebuilt when a pointer changes)
@@ -130,7 +132,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   };
   Work x{};
   x.idx = (int32_t*)take(sizeof(int32_t) * M * T * c.k);
-  x.gate = (float*)take(sizeof(float) * M * T * c.k);
+  x.gate = (float*)take(sizeof(float) * 2 * M * T * c.k);
   x.chunk_hist = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
   const size_t nseg = M * (size_t)d.Etot;
   if (c.compute) {
@@ -322,6 +324,7 @@ eb_status eb_reset(eb_ctx* x, void* stream) {
   x->last_stream = s;
   x->launches += 1;
   x->timed_out = false;
+  x->routed_ahead = false;
   cudaError_t e = launch_reset(x->d, x->dev, s);
   // the fused combine leaves its counters at zero; a step that gave up on a
   // bounded wait may not have, so a reset clears them
@@ -378,9 +381,12 @@ static cudaError_t launch_engine(eb_ctx* x, int eng, const Work& w, const void* 
   }
 }
 
+// route_next: the caller enqueues the next step with the same logits
+// (eb_episode), so this step may route it ahead: after GEMM 2, whose
+// persistent CTAs it runs beside, and before the combine.
 static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
                               const void* wdn, void* workspace, size_t ws_bytes,
-                              cudaStream_t s) {
+                              cudaStream_t s, bool route_next) {
   const eb_config& c = x->cfg;
   if (x->timed_out) return EB_ERR_TIMEOUT;
   if ((!logits && !x->w_router) || !workspace) return EB_ERR_INVALID_ARG;
@@ -436,8 +442,10 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
                            mbs, ls, &x->dev.st->status, s);
     });
   }
-  if (e == cudaSuccess)
-    e = timed(x, 0, 1, s, [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, s); });
+  if (e == cudaSuccess && !x->routed_ahead)
+    e = timed(x, 0, 1, s,
+              [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, false, s); });
+  x->routed_ahead = false;
   if (e == cudaSuccess)
     e = timed(x, 1, x->dev.search_slots ? 2 : 1, s,
               [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
@@ -451,6 +459,14 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
       if (e == cudaSuccess)
         e = timed(x, 4, 1, s, [&] { return launch_engine(x, g2, w, wgu, wdn, hidden, s, 2); });
     }
+    // the next step's routing reads the caller's logits and this step's
+    // state only, so it runs beside GEMM 2 (router mode projects the scores
+    // from the hidden states this step's combine writes, so it does not)
+    if (e == cudaSuccess && route_next && !x->w_router && g2 != EB_GEMM_SIMT) {
+      e = timed(x, 0, 1, s,
+                [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, true, s); });
+      x->routed_ahead = e == cudaSuccess;
+    }
     // the fused engine combines inside GEMM 2
     if (e == cudaSuccess && g2 != EB_GEMM_TMC)
       e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });
@@ -463,7 +479,7 @@ eb_status eb_moe_step(eb_ctx* x, const float* logits, void* hidden, const void* 
                       uint32_t* runset_host) {
   if (!x) return EB_ERR_INVALID_ARG;
   cudaStream_t s = (cudaStream_t)stream;
-  const eb_status st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s);
+  const eb_status st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s, false);
   if (st != EB_OK) return st;
   if (runset_host) {
     cudaError_t e = cudaMemcpyAsync(runset_host, &x->dev.st->runset, sizeof(uint32_t),
@@ -490,7 +506,7 @@ eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* w
   if (st != EB_OK) return st;
   const int max_steps = x->d.max_steps;
   for (int i = 0; i < max_steps; ++i) {
-    st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s);
+    st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s, true);
     if (st != EB_OK) return st;
     const int slot = i % kLookahead;
     cudaError_t e = cudaMemcpyAsync(&x->host_pending[slot], &x->dev.st->pending, sizeof(uint32_t),

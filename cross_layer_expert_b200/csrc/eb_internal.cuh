@@ -56,7 +56,7 @@ struct State {
   int32_t items1;    // work items of the gate/up GEMM
   int32_t items2;    // work items of the down GEMM
   int32_t rows;      // permuted rows of this step
-  int32_t pad0;
+  uint32_t gate_buf; // bit j: which of the two gate buffers holds j's current routing
   long long num, den, den_sep;  // utilisation accumulators (Eq. (3))
 };
 
@@ -71,7 +71,7 @@ struct Dims {
 // Pointers into the caller's workspace.
 struct Work {
   int32_t* idx;        // [M][T][k]
-  float* gate;         // [M][T][k]
+  float* gate;         // [2][M][T][k]: two buffers, State::gate_buf picks one per micro-batch
   int32_t* chunk_hist; // [M][NC][E]: counts of each 64-token chunk
   int32_t* prior;      // [M][Etot]: rows of (j's segment, expert) taken by earlier RunSet members
   int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
@@ -153,12 +153,27 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // then reports only errors of those launches.
 inline bool cuda_error_pending() { return cudaPeekAtLastError() != cudaSuccess; }
 
+// Gates of token tok = j T + t of the current step.  Routing writes a
+// micro-batch's gates into the buffer its gate_buf bit does not name, and
+// the scheduler flips the bits of the micro-batches it routed, so the
+// routing of step i + 1 can run while step i's combine still reads step i's
+// gates.
+__device__ __forceinline__ const float* gates_of(const float* gate, const State* st,
+                                                 const Dims& d, long long tok) {
+  const int j = (int)(tok / d.T);
+  return gate + (size_t)((st->gate_buf >> j) & 1u) * ((size_t)d.M * d.T * d.k) + (size_t)tok * d.k;
+}
+
 // ---- launchers (all asynchronous on `s`) ----
 // Micro-batch j's rows at layer l start at logits + j * mb_stride + l *
 // layer_stride (elements): (L T E, T E) for the caller's [M, L, T, E] logits,
 // (T E, 0) for router scores of the step kept as [M, T, E].
+// early: the launch follows a kernel of the previous step that does not
+// read what routing writes (the persistent GEMM 2); the routing runs before
+// waiting for it, in smaller CTAs that fit beside it, and waits at its end.
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
-                              long long mb_stride, long long layer_stride, cudaStream_t s);
+                              long long mb_stride, long long layer_stride, bool early,
+                              cudaStream_t s);
 cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int renorm, int32_t* idx,
                               float* gate, int32_t* hist, int32_t* status, cudaStream_t s);
 // rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm1 / fm2:

@@ -604,11 +604,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 // combine kernel, so the fused and unfused steps agree bit for bit.  The
 // token's y rows were stored by other CTAs of this launch: they are read
 // through L2 (ld.global.cg), after the acquiring fence of the caller.
-__device__ __forceinline__ void combine_token(const Dims& d, int tok, int f, int lane,
-                                              const float* __restrict__ gate,
+__device__ __forceinline__ void combine_token(const Dims& d, const State* st, int tok, int f,
+                                              int lane, const float* __restrict__ gate,
                                               const __nv_bfloat16* y, __nv_bfloat16* hidden) {
   const int k = d.k, kk = d.kk;
-  const float my_gate = lane < k ? __ldg(gate + (size_t)tok * k + lane) : 0.f;
+  const float my_gate = lane < k ? __ldg(gates_of(gate, st, d, tok) + lane) : 0.f;
   uint4* hp = reinterpret_cast<uint4*>(hidden + (size_t)tok * d.H + f + 8 * lane);
   float acc[8];
   if (d.residual) {
@@ -968,7 +968,7 @@ __global__ void __launch_bounds__(GATHER    ? kThreads + 32 * kGatherWarps
       if (v < 0) break;
       __threadfence();  // the arrivals the drain counted before the reads of y
       const int nfb = d.H / C::kFeat;
-      combine_token(d, v / nfb, (v % nfb) * C::kFeat, lane, gate, out, hidden);
+      combine_token(d, st, v / nfb, (v % nfb) * C::kFeat, lane, gate, out, hidden);
     }
     (void)t_begin;
   } else {

@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, const St
     // the token's expert outputs sit at its slots (tok * kk + s); gates, one
     // per lane
     const int my_row = lane < kk ? (int)(tok * kk + lane) : 0;
-    const float my_gate = lane < k ? __ldg(gate + tok * k + lane) : 0.f;
+    const float my_gate = lane < k ? __ldg(gates_of(gate, st, d, (long long)tok) + lane) : 0.f;
     T* out = hidden + tok * d.H;
     // two 16-byte vectors per lane per pass, slots loaded four at a time
     // (registers for three CTAs per SM)

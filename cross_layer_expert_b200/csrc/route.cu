@@ -36,86 +36,113 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Routes one token row with the calling warp.  Lane s < k returns slot s.
-// Each of the k rounds takes the warp maximum of the lanes' best keys, then
-// the smallest expert index among the lanes holding it.
-template <int VPL>
-__device__ __forceinline__ void route_row(const float* __restrict__ row, int E, int k, int renorm,
-                                          int lane, int& out_e, float& out_g, bool& nonfinite) {
-  float v[VPL];
-  uint32_t key[VPL];
+// Routes R token rows with the calling warp, their k argmax rounds
+// interleaved so the rows' dependency chains overlap.  Lane s < k returns
+// slot s of each row.  Each round takes the warp maximum of the lanes' best
+// keys, then the smallest expert index among the lanes holding it.  A row
+// with valid[r] false is skipped (its outputs are unspecified).
+template <int VPL, int R>
+__device__ __forceinline__ void route_rows(const float* const (&row)[R], const bool (&valid)[R],
+                                           int E, int k, int renorm, int lane, int (&out_e)[R],
+                                           float (&out_g)[R], bool& nonfinite) {
+  float v[R][VPL];
+  uint32_t key[R][VPL];
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    const int e = i * 32 + lane;
-    float x = -INFINITY;
-    if (e < E) {
-      x = __ldg(row + e);
-      if (!isfinite(x)) {
-        nonfinite = true;
-        x = -INFINITY;  // selection stays among real experts; the call reports the error
-      }
-    }
-    v[i] = x;
-    key[i] = e < E ? order_key(x) : 0u;  // real experts (even -inf) rank above padding
-    if (e < E && key[i] == 0u) key[i] = 1u;
-  }
-  float top_v = -INFINITY, vmax = -INFINITY;
-  int top_e = 0;
-  for (int s = 0; s < k; ++s) {
-    uint32_t bk = 0;
-    int be = 0x7fffffff;
+  for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      // ascending i visits ascending expert ids of this lane: strict > keeps the lowest
-      if (key[i] > bk) {
-        bk = key[i];
-        be = i * 32 + lane;
+      const int e = i * 32 + lane;
+      float x = -INFINITY;
+      if (valid[r] && e < E) {
+        x = __ldg(row[r] + e);
+        if (!isfinite(x)) {
+          nonfinite = true;
+          x = -INFINITY;  // selection stays among real experts; the call reports the error
+        }
       }
+      v[r][i] = x;
+      key[r][i] = e < E ? order_key(x) : 0u;  // real experts (even -inf) rank above padding
+      if (e < E && key[r][i] == 0u) key[r][i] = 1u;
     }
-    const uint32_t wk = __reduce_max_sync(kFull, bk);
-    const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
-    float wv = 0.f;
+  float top_v[R], vmax[R];
+  int top_e[R];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i)
-      if (i * 32 + lane == we) {
-        wv = v[i];
-        key[i] = 0u;  // taken
+  for (int r = 0; r < R; ++r) {
+    top_v[r] = -INFINITY;
+    vmax[r] = -INFINITY;
+    top_e[r] = 0;
+  }
+  for (int s = 0; s < k; ++s) {
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      uint32_t bk = 0;
+      int be = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        // ascending i visits ascending expert ids of this lane: strict > keeps the lowest
+        if (key[r][i] > bk) {
+          bk = key[r][i];
+          be = i * 32 + lane;
+        }
       }
-    wv = __shfl_sync(kFull, wv, we & 31);
-    if (lane == s) {
-      top_v = wv;
-      top_e = we;
-    }
-    if (s == 0) vmax = wv;
-  }
-  const float ex = (lane < k) ? expf(top_v - vmax) : 0.f;
-  float denom;
-  if (renorm) {
-    denom = warp_sum(ex);
-  } else {
-    float part = 0.f;
+      const uint32_t wk = __reduce_max_sync(kFull, bk);
+      const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
+      float wv = 0.f;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i)
-      if (i * 32 + lane < E) part += expf(v[i] - vmax);
-    denom = warp_sum(part);
+      for (int i = 0; i < VPL; ++i)
+        if (i * 32 + lane == we) {
+          wv = v[r][i];
+          key[r][i] = 0u;  // taken
+        }
+      wv = __shfl_sync(kFull, wv, we & 31);
+      if (lane == s) {
+        top_v[r] = wv;
+        top_e[r] = we;
+      }
+      if (s == 0) vmax[r] = wv;
+    }
   }
-  out_e = top_e;
-  out_g = ex / denom;
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    const float ex = (lane < k) ? expf(top_v[r] - vmax[r]) : 0.f;
+    float denom;
+    if (renorm) {
+      denom = warp_sum(ex);
+    } else {
+      float part = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i * 32 + lane < E) part += expf(v[r][i] - vmax[r]);
+      denom = warp_sum(part);
+    }
+    out_e[r] = top_e[r];
+    out_g[r] = ex / denom;
+  }
 }
 
+// Tokens [t0, t1) of a block of rows: warp w routes tokens w and w + W
+// together (W warps), then w + 2W and w + 3W, ...
 template <int VPL>
 __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
                             int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
                             int* hist_s, bool& nonfinite) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = t0 + warp; t < t1; t += nwarps) {
-    int e;
-    float g;
-    route_row<VPL>(logits + (size_t)t * E, E, k, renorm, lane, e, g, nonfinite);
+  for (int t = t0 + warp; t < t1; t += 2 * nwarps) {
+    const int t2 = t + nwarps;
+    const float* rows[2] = {logits + (size_t)t * E, logits + (size_t)(t2 < t1 ? t2 : t) * E};
+    const bool valid[2] = {true, t2 < t1};
+    int e[2];
+    float g[2];
+    route_rows<VPL, 2>(rows, valid, E, k, renorm, lane, e, g, nonfinite);
     if (lane < k) {
-      idx[(size_t)t * k + lane] = e;
-      gate[(size_t)t * k + lane] = g;
-      atomicAdd(&hist_s[e], 1);
+      idx[(size_t)t * k + lane] = e[0];
+      gate[(size_t)t * k + lane] = g[0];
+      atomicAdd(&hist_s[e[0]], 1);
+      if (valid[1]) {
+        idx[(size_t)t2 * k + lane] = e[1];
+        gate[(size_t)t2 * k + lane] = g[1];
+        atomicAdd(&hist_s[e[1]], 1);
+      }
     }
   }
 }
@@ -126,6 +153,14 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
 // hist[j][:] and rank loads w[j][:], which the previous step zeroed.  The
 // loads fold the counts by the context's expert placement: contiguous
 // blocks of E/D experts, or emap[e] if one was set.
+//
+// early: launched right after the previous step's GEMM 2 (whose persistent
+// CTAs are all resident), which reads nothing routing writes -- the gates go
+// to the buffer the micro-batch's gate_buf bit does not name, while the
+// previous step's combine reads the other.  The CTA then routes first and
+// waits for GEMM 2 only at its end, so the step's combine and everything
+// after it still start after GEMM 2.  The state it reads was written by the
+// previous scheduler step, which completed before GEMM 2 started.
 template <int VPL>
 __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__ st,
                                                      const float* __restrict__ logits,
@@ -135,12 +170,19 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
                                                      int32_t* __restrict__ hist,
                                                      int32_t* __restrict__ wload,
                                                      const int32_t* __restrict__ emap,
-                                                     long long mb_stride, long long layer_stride) {
-  pdl_enter();
+                                                     long long mb_stride, long long layer_stride,
+                                                     int early) {
+  if (early) pdl_trigger();
+  else pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
   // nothing routes while a timed-out step awaits eb_reset
-  if (!((st->need_route >> j) & 1u) || st->status == EB_ERR_TIMEOUT) return;
+  if (!((st->need_route >> j) & 1u) || st->status == EB_ERR_TIMEOUT) {
+    if (early) pdl_wait();
+    return;
+  }
   const int l = st->layer[j];
+  // the gate buffer j's current routing does not use
+  float* gate_j = gate + (size_t)(((st->gate_buf >> j) & 1u) ^ 1u) * ((size_t)d.M * d.T * d.k);
   __shared__ int hist_s[EB_MAX_ETOT];
   __shared__ int w_s[EB_MAX_D];
   __shared__ int bad;
@@ -154,7 +196,7 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
   const int t0 = c * kChunk, t1 = min(d.T, t0 + kChunk);
   bool nonfinite = false;
   route_chunk<VPL>(blk, t0, t1, d.E, d.k, d.renorm, idx + (size_t)j * d.T * d.k,
-                   gate + (size_t)j * d.T * d.k, hist_s, nonfinite);
+                   gate_j + (size_t)j * d.T * d.k, hist_s, nonfinite);
   if (nonfinite) bad = 1;
   __syncthreads();
   int32_t* out = chunk_hist + ((size_t)j * d.NC + c) * d.E;
@@ -177,6 +219,7 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
     }
   }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
+  if (early) pdl_wait();
 }
 
 // Stand-alone path: rows [c*kChunk, ...) of an [n, E] block; counts summed
@@ -207,15 +250,20 @@ int vpl_for(int E) { return E <= 32 ? 1 : E <= 64 ? 2 : E <= 128 ? 4 : 8; }
 }  // namespace
 
 cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, const float* logits,
-                              long long mb_stride, long long layer_stride, cudaStream_t s) {
+                              long long mb_stride, long long layer_stride, bool early,
+                              cudaStream_t s) {
   dim3 grid(d.NC, d.M);
+  // beside GEMM 2's CTAs (one per SM, most of its registers and shared
+  // memory) an early launch uses 256-thread CTAs
+  const dim3 block(early ? 256 : 1024);
   const int32_t* emap = c.use_emap ? c.emap : nullptr;
+  const int ea = early ? 1 : 0;
   cudaError_t e;
   switch (vpl_for(d.E)) {
-    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
-    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
-    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
-    default: e = launch_pdl(k_route_step<8>, dim3(grid), dim3(1024), 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride); break;
+    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
+    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
+    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
+    default: e = launch_pdl(k_route_step<8>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
   }
   return e;
 }

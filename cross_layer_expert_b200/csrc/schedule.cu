@@ -616,6 +616,9 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   if (d.compute)
     for (int i = tid; i < d.M * d.E; i += kThreads) s_hist[i] = c.hist[i];
   __syncthreads();
+  // the micro-batches routed for this step wrote their gates into the
+  // buffers their gate_buf bits did not name: from now on those hold them
+  if (tid == 0) ss.gate_buf ^= ss.need_route;
   auto write_back = [&]() {
     __syncthreads();
     for (int i = tid; i < kStateWords; i += kThreads)
@@ -913,6 +916,7 @@ __global__ void k_reset(Dims d, CtxDev c) {
   st->n_groups = 0;
   st->n_steps = 0;
   st->status = EB_OK;
+  st->gate_buf = 0;
   st->nseg = 0;
   st->items1 = st->items2 = 0;
   st->rows = 0;

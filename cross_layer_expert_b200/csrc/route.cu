@@ -38,15 +38,19 @@ __device__ __forceinline__ uint32_t order_key(float x) {
 
 // Routes R token rows with the calling warp, their k argmax rounds
 // interleaved so the rows' dependency chains overlap.  Lane s < k returns
-// slot s of each row.  Each round takes the warp maximum of the lanes' best
-// keys, then the smallest expert index among the lanes holding it.  A row
-// with valid[r] false is skipped (its outputs are unspecified).
+// slot s of each row.  Each lane first sorts its VPL experts by (logit
+// descending, expert index ascending); a round then compares only the
+// lanes' heads: the warp maximum of the head keys, then the smallest expert
+// index among the lanes holding it, and the winning lane drops its head.
+// A row with valid[r] false is skipped (its outputs are unspecified).
 template <int VPL, int R>
 __device__ __forceinline__ void route_rows(const float* const (&row)[R], const bool (&valid)[R],
                                            int E, int k, int renorm, int lane, int (&out_e)[R],
                                            float (&out_g)[R], bool& nonfinite) {
   float v[R][VPL];
   uint32_t key[R][VPL];
+  int id[R][VPL];
+  float part[R];  // this lane's share of the full softmax denominator (renorm off)
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -63,86 +67,119 @@ __device__ __forceinline__ void route_rows(const float* const (&row)[R], const b
       v[r][i] = x;
       key[r][i] = e < E ? order_key(x) : 0u;  // real experts (even -inf) rank above padding
       if (e < E && key[r][i] == 0u) key[r][i] = 1u;
+      id[r][i] = e;
     }
-  float top_v[R], vmax[R];
+  // the first round's maximum is every lane's unsorted maximum
+  float vmax[R];
+#pragma unroll
+  for (int r = 0; r < R; ++r) {
+    uint32_t bk = 0;
+    int be = 0x7fffffff;
+    float bv = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i)
+      if (key[r][i] > bk) {
+        bk = key[r][i];
+        be = id[r][i];
+        bv = v[r][i];
+      }
+    const uint32_t wk = __reduce_max_sync(kFull, bk);
+    const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
+    vmax[r] = __shfl_sync(kFull, bv, we & 31);
+    part[r] = 0.f;
+    if (!renorm) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i * 32 + lane < E) part[r] += expf(v[r][i] - vmax[r]);
+    }
+  }
+  // sort each lane's experts: key descending, index ascending among equal keys
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int a = 0; a < VPL; ++a)
+#pragma unroll
+      for (int b = VPL - 1; b > a; --b) {
+        const bool sw = key[r][b] > key[r][b - 1] ||
+                        (key[r][b] == key[r][b - 1] && id[r][b] < id[r][b - 1]);
+        if (sw) {
+          const uint32_t tk = key[r][b];
+          key[r][b] = key[r][b - 1];
+          key[r][b - 1] = tk;
+          const int ti = id[r][b];
+          id[r][b] = id[r][b - 1];
+          id[r][b - 1] = ti;
+          const float tv = v[r][b];
+          v[r][b] = v[r][b - 1];
+          v[r][b - 1] = tv;
+        }
+      }
+  float top_v[R];
   int top_e[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     top_v[r] = -INFINITY;
-    vmax[r] = -INFINITY;
     top_e[r] = 0;
   }
   for (int s = 0; s < k; ++s) {
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      uint32_t bk = 0;
-      int be = 0x7fffffff;
+      const uint32_t wk = __reduce_max_sync(kFull, key[r][0]);
+      const int we = (int)__reduce_min_sync(kFull, key[r][0] == wk ? (uint32_t)id[r][0] : 0xffffffffu);
+      const float wv = __shfl_sync(kFull, v[r][0], we & 31);
+      if (lane == (we & 31)) {  // the winner drops its head
 #pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        // ascending i visits ascending expert ids of this lane: strict > keeps the lowest
-        if (key[r][i] > bk) {
-          bk = key[r][i];
-          be = i * 32 + lane;
+        for (int i = 0; i + 1 < VPL; ++i) {
+          key[r][i] = key[r][i + 1];
+          id[r][i] = id[r][i + 1];
+          v[r][i] = v[r][i + 1];
         }
+        key[r][VPL - 1] = 0u;
       }
-      const uint32_t wk = __reduce_max_sync(kFull, bk);
-      const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
-      float wv = 0.f;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (i * 32 + lane == we) {
-          wv = v[r][i];
-          key[r][i] = 0u;  // taken
-        }
-      wv = __shfl_sync(kFull, wv, we & 31);
       if (lane == s) {
         top_v[r] = wv;
         top_e[r] = we;
       }
-      if (s == 0) vmax[r] = wv;
     }
   }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
     const float ex = (lane < k) ? expf(top_v[r] - vmax[r]) : 0.f;
-    float denom;
-    if (renorm) {
-      denom = warp_sum(ex);
-    } else {
-      float part = 0.f;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (i * 32 + lane < E) part += expf(v[r][i] - vmax[r]);
-      denom = warp_sum(part);
-    }
+    const float denom = warp_sum(renorm ? ex : part[r]);
     out_e[r] = top_e[r];
     out_g[r] = ex / denom;
   }
 }
 
-// Tokens [t0, t1) of a block of rows: warp w routes tokens w and w + W
-// together (W warps), then w + 2W and w + 3W, ...
+// Tokens [t0, t1) of a block of rows: warp w routes tokens w, w + W, ...
+// (W warps) R at a time, R = 2 while two rows' registers fit (VPL <= 4).
 template <int VPL>
 __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
                             int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
                             int* hist_s, bool& nonfinite) {
+  constexpr int R = VPL <= 4 ? 2 : 1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = t0 + warp; t < t1; t += 2 * nwarps) {
-    const int t2 = t + nwarps;
-    const float* rows[2] = {logits + (size_t)t * E, logits + (size_t)(t2 < t1 ? t2 : t) * E};
-    const bool valid[2] = {true, t2 < t1};
-    int e[2];
-    float g[2];
-    route_rows<VPL, 2>(rows, valid, E, k, renorm, lane, e, g, nonfinite);
+  for (int t = t0 + warp; t < t1; t += R * nwarps) {
+    const float* rows[R];
+    bool valid[R];
+    int tr[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      tr[r] = t + r * nwarps;
+      valid[r] = tr[r] < t1;
+      rows[r] = logits + (size_t)(valid[r] ? tr[r] : t) * E;
+    }
+    int e[R];
+    float g[R];
+    route_rows<VPL, R>(rows, valid, E, k, renorm, lane, e, g, nonfinite);
     if (lane < k) {
-      idx[(size_t)t * k + lane] = e[0];
-      gate[(size_t)t * k + lane] = g[0];
-      atomicAdd(&hist_s[e[0]], 1);
-      if (valid[1]) {
-        idx[(size_t)t2 * k + lane] = e[1];
-        gate[(size_t)t2 * k + lane] = g[1];
-        atomicAdd(&hist_s[e[1]], 1);
-      }
+#pragma unroll
+      for (int r = 0; r < R; ++r)
+        if (valid[r]) {
+          idx[(size_t)tr[r] * k + lane] = e[r];
+          gate[(size_t)tr[r] * k + lane] = g[r];
+          atomicAdd(&hist_s[e[r]], 1);
+        }
     }
   }
 }

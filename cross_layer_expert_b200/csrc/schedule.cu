@@ -332,10 +332,6 @@ __device__ uint32_t warp_choose(SchedSmem& sm, int D, int m, int policy, uint32_
       best = D <= 8    ? warp_maxutil_masks<8>(sm, D, m)
              : D <= 16 ? warp_maxutil_masks<16>(sm, D, m)
                        : warp_maxutil_masks<32>(sm, D, m);
-    } else if (n <= kMaskEnumMax) {
-      for (uint32_t cm = lane; cm < (1u << n); cm += 32)
-        if (__popc(cm) <= n - m) consider(sm, D, cm, best);
-      best = warp_best(best);
     } else {
       best = warp_best(search_ranks(sm, D, 0, candidate_count(n, m), lane, 32));
     }
@@ -397,13 +393,13 @@ __device__ uint32_t warp_choose(SchedSmem& sm, int D, int m, int policy, uint32_
 // All threads, with sm.P, sm.n and the pending rows sm.w (by position) in
 // place.  Returns the RunSet (micro-batch ids) to warp 0; the other threads'
 // return value is unspecified.  slots: the MaxUtil search grid's results for
-// this pending set (null: search here).  Only a large MaxUtil search uses
-// the whole block.
+// this pending set (null: search here).  Only a large MaxUtil search, or
+// one over more than 32 ranks, uses the whole block.
 __device__ uint32_t choose_runset(SchedSmem& sm, int D, int m, int policy, uint32_t pending,
                                   const Cand* slots) {
   const int n = sm.n;
   if (policy == EB_SCHED_MAXUTIL && n > m &&
-      (slots != nullptr || candidate_count(n, m) > kWarpSearchMax)) {
+      (slots != nullptr || candidate_count(n, m) > kWarpSearchMax || D > 32)) {
     prepare_totals(sm, D);
     return slots ? maxutil_slots(sm, slots, kSearchCtas) : maxutil_block(sm, D, m);
   }

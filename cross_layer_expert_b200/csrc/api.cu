@@ -34,6 +34,12 @@ struct eb_ctx {
   bool timed_out = false;
   // the previous step already enqueued this step's routing (eb_episode)
   bool routed_ahead = false;
+  // the previous step's combine is enqueued by this step, beside its
+  // scheduler (eb_episode); it writes deferred_hidden
+  bool combine_deferred = false;
+  void* deferred_hidden = nullptr;
+  // steps enqueued since create; its parity picks the step's StepView slot
+  long long seq = 0;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
   // cached TMA maps (rebuilt when a pointer changes)
@@ -134,6 +140,7 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   x.idx = (int32_t*)take(sizeof(int32_t) * M * T * c.k);
   x.gate = (float*)take(sizeof(float) * 2 * M * T * c.k);
   x.chunk_hist = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
+  x.views = (StepView*)take(sizeof(StepView) * 2);
   const size_t nseg = M * (size_t)d.Etot;
   if (c.compute) {
     x.prior = (int32_t*)take(sizeof(int32_t) * M * d.Etot);
@@ -325,6 +332,7 @@ eb_status eb_reset(eb_ctx* x, void* stream) {
   x->launches += 1;
   x->timed_out = false;
   x->routed_ahead = false;
+  x->combine_deferred = false;
   cudaError_t e = launch_reset(x->d, x->dev, s);
   // the fused combine leaves its counters at zero; a step that gave up on a
   // bounded wait may not have, so a reset clears them
@@ -446,9 +454,20 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     e = timed(x, 0, 1, s,
               [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, false, s); });
   x->routed_ahead = false;
+  const int slot = (int)(x->seq & 1);
+  x->seq += 1;
   if (e == cudaSuccess)
     e = timed(x, 1, x->dev.search_slots ? 2 : 1, s,
-              [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, s); });
+              [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, slot, s); });
+  // the previous step's combine runs beside this step's scheduler: it reads
+  // the previous step's view, outputs and gates, none of which the scheduler
+  // writes, and the positions pass after it waits for both
+  if (e == cudaSuccess && x->combine_deferred) {
+    x->combine_deferred = false;
+    e = timed(x, 5, 1, s, [&] {
+      return launch_combine(x->d, w, x->deferred_hidden, slot ^ 1, true, s);
+    });
+  }
   if (c.compute) {
     if (e == cudaSuccess)
       e = timed(x, 6, 1, s, [&] { return launch_positions(x->d, x->dev, w, s); });
@@ -467,11 +486,30 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
                 [&] { return launch_route_step(x->d, x->dev, w, rsrc, mbs, ls, true, s); });
       x->routed_ahead = e == cudaSuccess;
     }
-    // the fused engine combines inside GEMM 2
-    if (e == cudaSuccess && g2 != EB_GEMM_TMC)
-      e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, x->dev, w, hidden, s); });
+    // the fused engine combines inside GEMM 2; after routing ahead the
+    // combine waits for the next step, to run beside its scheduler
+    if (e == cudaSuccess && g2 != EB_GEMM_TMC) {
+      if (x->routed_ahead) {
+        x->combine_deferred = true;
+        x->deferred_hidden = hidden;
+      } else {
+        e = timed(x, 5, 1, s, [&] { return launch_combine(x->d, w, hidden, slot, false, s); });
+      }
+    }
   }
   return cuda_status(e);
+}
+
+// The combine a step deferred to the next one, when no next step follows.
+static eb_status flush_combine(eb_ctx* x, void* workspace, cudaStream_t s) {
+  if (!x->combine_deferred) return EB_OK;
+  x->combine_deferred = false;
+  Work w;
+  layout(x->cfg, (char*)workspace, &w);
+  const int slot = (int)((x->seq - 1) & 1);
+  return cuda_status(timed(x, 5, 1, s, [&] {
+    return launch_combine(x->d, w, x->deferred_hidden, slot, false, s);
+  }));
 }
 
 eb_status eb_moe_step(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
@@ -521,6 +559,8 @@ eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* w
       if (x->host_pending[cs] == 0) break;
     }
   }
+  st = flush_combine(x, workspace, s);
+  if (st != EB_OK) return st;
   if (cudaStreamSynchronize(s) != cudaSuccess) return EB_ERR_CUDA;
   int steps = 0, status = EB_OK;
   if (cudaMemcpy(&steps, &x->dev.st->n_steps, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess ||

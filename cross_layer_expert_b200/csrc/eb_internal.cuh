@@ -60,6 +60,17 @@ struct State {
   long long num, den, den_sep;  // utilisation accumulators (Eq. (3))
 };
 
+// What a step's combine reads of the step state.  The step's scheduler
+// writes it into one of two slots (by step parity), so the next step's
+// scheduler may run while this step's combine still reads it.
+struct StepView {
+  int32_t n_run;
+  uint32_t gate_buf;  // State::gate_buf of the step
+  int32_t next;       // the combine's next unclaimed token (zeroed by the scheduler)
+  int32_t pad;
+  int32_t run_list[EB_MAX_M];
+};
+
 // Plain-old-data copy of the configuration used by kernels.
 struct Dims {
   int L, E, k, H, F, D, M, T, n_shared, Etot, renorm, dtype, policy, m, residual, compute;
@@ -81,6 +92,7 @@ struct Work {
   int32_t* seg_items1; // [M*Etot + 1]
   int32_t* seg_items2; // [M*Etot + 1]
   int32_t* gemm_next;  // [2]: next dynamically claimed item of GEMM 1 / GEMM 2 (zeroed by the plan)
+  StepView* views;     // [2]: the combine's view of a step, by step parity
   float* scores;       // [M][T][E]: router scores of the step (router mode)
   void* A;             // [Rcap][H] permuted tokens
   void* act;           // [Rcap][F] SwiGLU activations
@@ -158,10 +170,10 @@ inline bool cuda_error_pending() { return cudaPeekAtLastError() != cudaSuccess; 
 // the scheduler flips the bits of the micro-batches it routed, so the
 // routing of step i + 1 can run while step i's combine still reads step i's
 // gates.
-__device__ __forceinline__ const float* gates_of(const float* gate, const State* st,
+__device__ __forceinline__ const float* gates_of(const float* gate, uint32_t gate_buf,
                                                  const Dims& d, long long tok) {
   const int j = (int)(tok / d.T);
-  return gate + (size_t)((st->gate_buf >> j) & 1u) * ((size_t)d.M * d.T * d.k) + (size_t)tok * d.k;
+  return gate + (size_t)((gate_buf >> j) & 1u) * ((size_t)d.M * d.T * d.k) + (size_t)tok * d.k;
 }
 
 // ---- launchers (all asynchronous on `s`) ----
@@ -179,8 +191,9 @@ cudaError_t launch_route_rows(const float* logits, int n, int E, int k, int reno
 // rn1 / rn2: token rows per work item of GEMM 1 / GEMM 2; fm1 / fm2:
 // output features per item.  With c.search_slots set, the MaxUtil search
 // grid runs first (two launches).
+// slot: the StepView slot of this step (its parity).
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
-                                 int fm1, int fm2, cudaStream_t s);
+                                 int fm1, int fm2, int slot, cudaStream_t s);
 // slots: kSearchCtas * kSearchSlotBytes of device scratch for the MaxUtil
 // search grid, or null to search in the scheduler's CTA.
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,
@@ -200,7 +213,10 @@ cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cuda
 // The permuted copy A of the RunSet's token rows (after launch_positions).
 cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                                 cudaStream_t s);
-cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
+// slot: the StepView slot of the step being combined.  early: launched
+// after the next step's scheduler, which it does not depend on; it combines
+// first and waits for the scheduler only at its end.
+cudaError_t launch_combine(const Dims& d, const Work& w, void* hidden, int slot, bool early,
                            cudaStream_t s);
 // GEMM `which` (1: gate/up + SwiGLU, 2: down) on the CUDA cores.
 cudaError_t launch_gemm_simt(const Dims& d, const CtxDev& c, const Work& w, const void* w_gateup,

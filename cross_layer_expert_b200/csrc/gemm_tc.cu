@@ -608,7 +608,7 @@ __device__ __forceinline__ void combine_token(const Dims& d, const State* st, in
                                               int lane, const float* __restrict__ gate,
                                               const __nv_bfloat16* y, __nv_bfloat16* hidden) {
   const int k = d.k, kk = d.kk;
-  const float my_gate = lane < k ? __ldg(gates_of(gate, st, d, tok) + lane) : 0.f;
+  const float my_gate = lane < k ? __ldg(gates_of(gate, st->gate_buf, d, tok) + lane) : 0.f;
   uint4* hp = reinterpret_cast<uint4*>(hidden + (size_t)tok * d.H + f + 8 * lane);
   float acc[8];
   if (d.residual) {

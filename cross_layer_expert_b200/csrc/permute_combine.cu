@@ -258,26 +258,42 @@ struct Vec<__nv_bfloat16> {
 
 constexpr int kCombineThreads = 256;
 
-// Persistent: warp w combines tokens w, w + W, ... of the RunSet.
+// Tokens a combine CTA claims at a time (two per warp).
+constexpr int kCombineClaim = 2 * (kCombineThreads / 32);
+
+// Persistent: each CTA claims kCombineClaim consecutive tokens of the RunSet
+// at a time from the step view's counter, and warp w combines the claim's
+// tokens w and w + 8.  Claiming keeps a CTA that starts late (beside the
+// next step's scheduler) from holding the others up.  The step view (not
+// the live state, which the next step's scheduler may be rewriting) gives
+// the RunSet and the gate buffers.
 template <typename T>
-__global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, const State* __restrict__ st,
+__global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, StepView* __restrict__ view,
                                                              const float* __restrict__ gate,
                                                              const int32_t* __restrict__ pos,
-                                                             const T* __restrict__ y, T* hidden) {
-  pdl_enter();
-  const int lane = threadIdx.x & 31;
-  const int W = (int)(gridDim.x * (kCombineThreads / 32));
-  const int wid = (int)(blockIdx.x * (kCombineThreads / 32) + (threadIdx.x >> 5));
-  const int units = st->n_run * d.T;
+                                                             const T* __restrict__ y, T* hidden,
+                                                             int early) {
+  if (early) pdl_trigger();
+  else pdl_enter();
+  __shared__ int s_claim;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int units = view->n_run * d.T;
+  const uint32_t gate_buf = view->gate_buf;
   const int k = d.k, kk = d.kk;
   constexpr int VE = Vec<T>::n;
   const int nvec = d.H / VE;
-  for (int u = wid; u < units; u += W) {
-    const size_t tok = runset_token(st, d.T, u);
+  for (;;) {
+    __syncthreads();  // every warp has read the previous claim
+    if (threadIdx.x == 0) s_claim = atomicAdd(&view->next, kCombineClaim);
+    __syncthreads();
+    const int base = s_claim;
+    if (base >= units) break;
+  for (int u = base + warp; u < min(base + kCombineClaim, units); u += kCombineThreads / 32) {
+    const size_t tok = (size_t)view->run_list[u / d.T] * d.T + (u % d.T);
     // the token's expert outputs sit at its slots (tok * kk + s); gates, one
     // per lane
     const int my_row = lane < kk ? (int)(tok * kk + lane) : 0;
-    const float my_gate = lane < k ? __ldg(gates_of(gate, st, d, (long long)tok) + lane) : 0.f;
+    const float my_gate = lane < k ? __ldg(gates_of(gate, gate_buf, d, (long long)tok) + lane) : 0.f;
     T* out = hidden + tok * d.H;
     // two 16-byte vectors per lane per pass, slots loaded four at a time
     // (registers for three CTAs per SM)
@@ -330,6 +346,8 @@ __global__ void __launch_bounds__(kCombineThreads, 3) k_combine(Dims d, const St
       if (has1) Vec<T>::store(out, v1, acc1);
     }
   }
+  }
+  if (early) pdl_wait();
 }
 
 }  // namespace
@@ -374,21 +392,23 @@ cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, c
                     static_cast<float*>(w.A));
 }
 
-cudaError_t launch_combine(const Dims& d, const CtxDev& c, const Work& w, void* hidden,
+cudaError_t launch_combine(const Dims& d, const Work& w, void* hidden, int slot, bool early,
                            cudaStream_t s) {
+  StepView* view = w.views + slot;
+  const int ea = early ? 1 : 0;
   if (d.dtype == EB_DTYPE_BF16)
     return launch_pdl(k_combine<__nv_bfloat16>,
                       dim3(persistent_grid((const void*)k_combine<__nv_bfloat16>, kCombineThreads,
                                            g_grid_comb_bf16)),
-                      dim3(kCombineThreads), 0, s, 1, d, c.st, (const float*)w.gate,
+                      dim3(kCombineThreads), 0, s, 1, d, view, (const float*)w.gate,
                       (const int32_t*)w.pos, static_cast<const __nv_bfloat16*>(w.y),
-                      static_cast<__nv_bfloat16*>(hidden));
+                      static_cast<__nv_bfloat16*>(hidden), ea);
   return launch_pdl(k_combine<float>,
                     dim3(persistent_grid((const void*)k_combine<float>, kCombineThreads,
                                          g_grid_comb_f32)),
-                    dim3(kCombineThreads), 0, s, 1, d, c.st, (const float*)w.gate,
+                    dim3(kCombineThreads), 0, s, 1, d, view, (const float*)w.gate,
                     (const int32_t*)w.pos, static_cast<const float*>(w.y),
-                    static_cast<float*>(hidden));
+                    static_cast<float*>(hidden), ea);
 }
 
 }  // namespace eb

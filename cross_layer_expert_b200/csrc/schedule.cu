@@ -593,8 +593,10 @@ __device__ void zero_next(const Dims& d, const CtxDev& c, uint32_t next) {
     }
 }
 
+// view: this step's StepView slot, written for the step's combine.
 __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Work wk, int rn1,
-                                                             int rn2, int fm1, int fm2) {
+                                                             int rn2, int fm1, int fm2,
+                                                             StepView* __restrict__ view) {
   __shared__ SchedSmem sm;
   // the step state lives in shared memory for the whole kernel
   __shared__ State ss;
@@ -622,6 +624,8 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   };
   auto finish_empty = [&]() {
     if (tid == 0) {
+      view->n_run = 0;
+      view->next = 0;
       st->pending = ss.status == EB_ERR_TIMEOUT ? 0u : st->pending;
       st->runset = 0;
       st->n_run = 0;
@@ -691,9 +695,13 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
       st->run_list[a] = j;
       st->group_of[j] = g;
       s_group_run[a] = g;
+      view->run_list[a] = j;
     }
     if (leader) st->group_layer[g] = lj;
     if (lane == 0) {
+      view->n_run = __popc(run);
+      view->gate_buf = ss.gate_buf;
+      view->next = 0;
       st->num += sumW;
       st->den += (long long)d.D * maxW;
       st->den_sep += (long long)d.D * summax;
@@ -934,7 +942,7 @@ unsigned long long maxutil_candidates(int n, int m) {
 bool maxutil_uses_grid(int n, int m) { return maxutil_candidates(n, m) > kBlockSearchMax; }
 
 cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, int rn1, int rn2,
-                                 int fm1, int fm2, cudaStream_t s) {
+                                 int fm1, int fm2, int slot, cudaStream_t s) {
   if (c.search_slots) {
     auto go = [&](auto kernel) {
       return launch_pdl(kernel, dim3(kSearchCtas), dim3(kSearchThreads), 0, s, 1, d.M, d.D, d.m,
@@ -947,7 +955,8 @@ cudaError_t launch_schedule_step(const Dims& d, const CtxDev& c, const Work& w, 
                                       : go(k_maxutil_search<64>);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(k_schedule_step, dim3(1), dim3(kThreads), 0, s, 1, d, c, w, rn1, rn2, fm1, fm2);
+  return launch_pdl(k_schedule_step, dim3(1), dim3(kThreads), 0, s, 1, d, c, w, rn1, rn2, fm1, fm2,
+                    w.views + slot);
 }
 
 cudaError_t launch_schedule_once(const int32_t* w, uint32_t pending, int M, int D, int m,

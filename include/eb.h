@@ -211,7 +211,15 @@ eb_status eb_moe_step(eb_ctx* ctx, const float* logits, void* hidden, const void
  * enqueued a few ahead of the host's completion check, so the GPU never waits
  * for the host; steps enqueued after S became empty do nothing.  Returns the
  * number of steps that ran in *n_steps (host).  Waits for completion; returns
- * EB_ERR_TIMEOUT if a bounded device wait expired during the episode. */
+ * EB_ERR_TIMEOUT if a bounded device wait expired during the episode.
+ * Because every step reads the same logits, consecutive steps overlap (same
+ * results, bit for bit, as eb_moe_step step by step; without router mode
+ * and with a tensor-core GEMM 2):
+ *   - step i+1's routing runs beside step i's GEMM 2, into the second of the
+ *     workspace's two gate buffers;
+ *   - step i's combine runs beside step i+1's scheduler.
+ * An episode that returns an error leaves the context mid-step: call
+ * eb_reset before stepping it again. */
 eb_status eb_episode(eb_ctx* ctx, const float* logits, void* hidden, const void* w_gateup,
                      const void* w_down, void* workspace, size_t workspace_bytes, void* stream,
                      int* n_steps);

@@ -233,6 +233,39 @@ def test_fused_combine_bitwise_equals_unfused(small_inputs, name, policy):
         ctx.close()
 
 
+@pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16"])
+@pytest.mark.parametrize("gemm", [4, 7, 1])
+def test_routing_ahead_equals_step_by_step(small_inputs, name, gemm):
+    """eb_episode routes step i+1 beside step i's GEMM 2, into the gate buffer
+    the micro-batch's current routing does not use; eb_moe_step routes every
+    step at its start.  Both paths must give the same RunSets, trace,
+    utilisation and final hidden states, bit for bit, on the token-major,
+    fused-combine and weight-major engines."""
+    import torch
+    import cross_layer_expert_b200 as eb
+    from _common import lib_config
+    inp = small_inputs[name]
+    for policy in (0, 1):
+        h_ep, rows_ep, layers_ep, util_ep, steps_ep = run_episode(inp, policy, gemm=gemm)
+        ctx = eb.Context(lib_config(inp.wl, policy, gemm=gemm))
+        try:
+            hidden = inp.h0.clone()
+            ctx.eb_reset()
+            for _ in range(steps_ep):
+                assert ctx.eb_moe_step(inp.logits, hidden, inp.w_gateup, inp.w_down,
+                                       want_runset=True) != 0
+            assert ctx.eb_moe_step(inp.logits, hidden, inp.w_gateup, inp.w_down,
+                                   want_runset=True) == 0
+            assert ctx.eb_sync_status() == eb.EB_OK
+            rows, layers = ctx.eb_trace()
+            util = ctx.eb_utilization()
+        finally:
+            ctx.close()
+        assert np.array_equal(rows, rows_ep) and np.array_equal(layers, layers_ep), policy
+        assert util == util_ep, policy
+        assert torch.equal(hidden.cpu().view(torch.int16), h_ep.cpu().view(torch.int16)), policy
+
+
 @pytest.mark.parametrize("m", [1, 2, 4])
 def test_small_episode_m_sweep(small_inputs, small_expected, m):
     inp = small_inputs["small_bf16"]

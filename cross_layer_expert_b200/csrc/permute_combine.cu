@@ -17,10 +17,12 @@
 // unless GEMM 1 gathers them from the hidden states itself.  GEMM 2 writes
 // each row's output at its (token, slot) position, so the combine reads a
 // token's k + n_shared outputs from one contiguous run.  The copy and the combine are HBM-bound and
-// persistent: a grid of resident CTAs sized to the SM count strides over the
-// RunSet's tokens, one warp per token row with 16-byte vector loads and
+// persistent: a grid of resident CTAs sized to the SM count works through
+// the RunSet's tokens, one warp per token row with 16-byte vector loads and
 // stores, so the work spreads evenly over the SMs whatever the RunSet size
-// (no partial last wave).  Each row is read once and written k + n_shared
+// (no partial last wave).  The copy strides over the tokens; the combine's
+// CTAs claim them from a counter, since some of them may start late beside
+// the next step's scheduler.  Each row is read once and written k + n_shared
 // times (permute), or k + n_shared rows are read and one written (combine).
 #include <cuda_bf16.h>
 

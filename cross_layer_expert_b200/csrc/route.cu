@@ -4,16 +4,19 @@
 // weighs them.  The counts T_e per expert are what a rank's load is built
 // from ([SysLB] §1: L_r = sum_{e in E_r} T_e).
 //
-// One warp routes one token: the E logits are read coalesced (lane i holds
-// experts i, i+32, ...), the k winners come out of k rounds of a warp-wide
-// argmax under the order (logit descending, expert index ascending) -- a
-// hardware max-reduction over order-preserving integer keys, then a
-// min-reduction over the expert ids holding the maximum --, and the
-// gates exp(l_s - l_max) / sum_{s'} exp(l_s' - l_max) are formed from the
-// winners alone when renormalised (the full softmax denominator cancels).
-// Counts go to shared-memory atomics (integers, so the result is exact and
-// order-free) and are written once per (micro-batch, chunk): no global
-// atomics and no zeroing pass in the step path.
+// A warp routes token rows: the E logits are read coalesced (lane i holds
+// experts i, i+32, ...), each lane sorts its experts once, and the k winners
+// come out of k rounds over the lanes' heads under the order (logit
+// descending, expert index ascending) -- a hardware max-reduction over
+// order-preserving integer keys, then a min-reduction over the expert ids
+// holding the maximum; the winning lane drops its head.  Two rows are routed
+// together, their rounds interleaved.  The gates exp(l_s - l_max) /
+// sum_{s'} exp(l_s' - l_max) are formed from the winners alone when
+// renormalised (the full softmax denominator cancels).  Counts go to
+// shared-memory atomics (integers, so the result is exact and order-free),
+// are written once per (micro-batch, chunk) and are added to the
+// micro-batch's histogram and rank loads with one global atomic per (chunk,
+// expert) and (chunk, rank).
 #include <math.h>
 
 #include "eb_internal.cuh"

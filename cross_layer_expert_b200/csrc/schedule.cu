@@ -1,5 +1,5 @@
 // Loads, the RunSet scheduler, exact utilisation accounting and the segment
-// plan of one step -- one CTA, everything in shared memory.
+// plan of one step -- one CTA of 1024 threads, everything in shared memory.
 //
 // [EB] §2.3 Eq. (2) w_hat = max_d w_d, Eq. (3) u = sum sum w / (sum w_hat D);
 // [EB] §4.2 Algorithm 1 and the minimum RunSet size m; [EB] §5.2 CumUtil
@@ -13,14 +13,23 @@
 // with the lowest skipped indices.
 //
 // MaxUtil enumerates the complements C of the pending set P with
-// |C| <= |P| - m (so every candidate S = P \ C has |S| >= m): the threads
-// split the candidate ranks, unrank a first complement in colexicographic
-// order and walk on with Gosper's next-combination step.  Up to
-// kBlockSearchMax candidates the scheduler's own CTA searches them; above
-// that a grid of kSearchCtas CTAs (k_maxutil_search) each searches a
+// |C| <= |P| - m (so every candidate S = P \ C has |S| >= m).  Up to
+// kWarpSearchMax candidates over at most 32 ranks, warp 0 searches them:
+// with at most kMaskEnumMax pending micro-batches its lanes walk the
+// complement bitmasks directly, above that they split the candidate ranks.
+// Up to kBlockSearchMax candidates the scheduler's whole CTA splits them;
+// above that a grid of kSearchCtas CTAs (k_maxutil_search) each searches a
 // contiguous rank range and leaves its best candidate in a slot, and the
-// scheduler reduces the slots.  The order on candidates is total, so the
-// split never changes the RunSet.
+// scheduler reduces the slots.  A rank range is walked by unranking its
+// first complement in colexicographic order and stepping on with Gosper's
+// next-combination step.  The order on candidates is total, so no split
+// changes the RunSet.
+//
+// The scheduler kernel runs once per step from a cold instruction cache;
+// its time follows the size of the code it runs more than its arithmetic,
+// so warp 0 does the serial parts with lane-parallel reductions, loops stay
+// rolled, and the steps repeated per candidate or per segment are single
+// out-of-line copies.
 #include "eb_internal.cuh"
 
 namespace eb {
@@ -150,10 +159,6 @@ __device__ Cand shfl_cand(const Cand& c, int off) {
   o.cmask = __shfl_xor_sync(0xffffffffu, c.cmask, off);
   return o;
 }
-
-// The scheduler kernel runs once per step from a cold instruction cache:
-// its time follows the size of the code it runs more than the arithmetic, so
-// the steps it repeats are single out-of-line copies with rolled loops.
 
 // All lanes: the best of the warp's candidates, returned to every lane.
 __device__ __noinline__ Cand warp_best(Cand best) {

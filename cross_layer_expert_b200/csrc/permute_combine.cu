@@ -196,6 +196,111 @@ __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const Sta
   }
 }
 
+// ---- the copy by the TMA engine ----
+// Rows of up to kBulkMaxRowBytes are copied with bulk copies: a warp's lane 0
+// loads a token's row into one of its two shared-memory slots
+// (cp.async.bulk, completion on an mbarrier), then lanes s < k + n_shared
+// each store it to the row of slot s (cp.async.bulk to global, one bulk
+// group per lane per token).  Before a slot is loaded again, every lane's
+// stores that read it (two tokens back) must have read it.  The copy engine
+// moves the bytes; the warps only issue.
+constexpr int kBulkWarps = 8;
+constexpr int kBulkSlots = 2;
+constexpr int kBulkMaxRowBytes = 8192;
+constexpr unsigned long long kBulkWaitNs = 4000000000ull;  // 4 s per wait
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false after kBulkWaitNs.
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+  if (bar_try(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (bar_try(bar, parity)) return true;
+    if ((it & 63) == 0 && global_ns() - t0 > kBulkWaitNs) return false;
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State* __restrict__ st,
+                                                                  const int32_t* __restrict__ pos,
+                                                                  const T* __restrict__ hidden,
+                                                                  T* __restrict__ A) {
+  pdl_enter();
+  extern __shared__ __align__(128) uint8_t bulk_rows[];
+  __shared__ __align__(8) uint64_t bars[kBulkWarps][kBulkSlots];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int W = (int)(gridDim.x * kBulkWarps);
+  const int wid = (int)(blockIdx.x * kBulkWarps) + warp;
+  const int units = st->n_run * d.T;
+  const int kk = d.kk;
+  const uint32_t bytes = (uint32_t)(d.H * sizeof(T));
+  if (lane == 0) {
+    for (int sl = 0; sl < kBulkSlots; ++sl)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(&bars[warp][sl])));
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
+  uint32_t phases = 0;  // bit sl: parity of slot sl's next completion
+  int it = 0;
+  for (int u = wid; u < units; u += W, ++it) {
+    const int sl = it & 1;
+    uint8_t* buf = bulk_rows + (size_t)(warp * kBulkSlots + sl) * bytes;
+    const uint32_t bar = smem_u32(&bars[warp][sl]);
+    // the stores issued from this slot two tokens ago have read it
+    if (lane < kk) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    __syncwarp();
+    const size_t tok = (size_t)st->run_list[u / d.T] * d.T + (u % d.T);
+    if (lane == 0) {
+      asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                   : "memory");
+      asm volatile(
+          "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+          ::"r"(smem_u32(buf)), "l"(hidden + tok * d.H), "r"(bytes), "r"(bar)
+          : "memory");
+    }
+    const int row = lane < kk ? __ldg(pos + tok * kk + lane) : 0;
+    const bool ok = bar_wait(bar, (phases >> sl) & 1u);
+    phases ^= 1u << sl;
+    if (!__all_sync(0xffffffffu, ok)) {
+      if (lane == 0) {
+        atomicCAS(&st->status, EB_OK, EB_ERR_TIMEOUT);
+        bar_wait(bar, (phases >> sl) & 1u ^ 1u);  // give the load in flight one more bounded wait
+      }
+      break;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (lane < kk) {
+      asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                   ::"l"(A + (size_t)row * d.H), "r"(smem_u32(buf)), "r"(bytes)
+                   : "memory");
+      asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    }
+  }
+  // every store has completed (its writes are performed) before the CTA exits
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 template <typename T>
 struct Vec;
 template <>
@@ -379,8 +484,39 @@ cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cuda
                     (const int32_t*)w.seg_rows, (const int32_t*)w.prior, w.pos, w.rowslot);
 }
 
+int g_grid_bulk_bf16 = 0, g_grid_bulk_f32 = 0;
+
+template <typename T>
+cudaError_t launch_permute_bulk(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
+                                int& grid_cache, cudaStream_t s) {
+  const size_t smem = (size_t)kBulkWarps * kBulkSlots * d.H * sizeof(T);
+  if (grid_cache == 0) {
+    cudaError_t e = cudaFuncSetAttribute(k_permute_bulk<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(kBulkWarps * kBulkSlots * kBulkMaxRowBytes));
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0, per_sm = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess &&
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess &&
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_permute_bulk<T>,
+                                                      32 * kBulkWarps, smem) == cudaSuccess &&
+        sms > 0 && per_sm > 0)
+      grid_cache = sms * per_sm;
+    else
+      grid_cache = 148;
+  }
+  return launch_pdl(k_permute_bulk<T>, dim3(grid_cache), dim3(32 * kBulkWarps), smem, s, 1, d,
+                    c.st, (const int32_t*)w.pos, static_cast<const T*>(hidden),
+                    static_cast<T*>(w.A));
+}
+
 cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                                 cudaStream_t s) {
+  // rows that fit two shared-memory slots per warp go through the copy engine
+  if ((size_t)d.H * (d.dtype == EB_DTYPE_BF16 ? 2 : 4) <= (size_t)kBulkMaxRowBytes)
+    return d.dtype == EB_DTYPE_BF16
+               ? launch_permute_bulk<__nv_bfloat16>(d, c, w, hidden, g_grid_bulk_bf16, s)
+               : launch_permute_bulk<float>(d, c, w, hidden, g_grid_bulk_f32, s);
   if (d.dtype == EB_DTYPE_BF16)
     return launch_pdl(k_permute_copy<__nv_bfloat16>,
                       dim3(persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads,

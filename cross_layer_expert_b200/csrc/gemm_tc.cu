@@ -42,13 +42,6 @@ constexpr int kEpiWarps = EB_EPI_WARPS;    // 4 or 8: warps draining TMEM
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr unsigned long long kWaitLimitNs = 4000000000ull;  // 4 s per wait
 
-// Weight tiles are prefetched into L2 this many k-blocks ahead of the
-// shared-memory ring (0: off), so the ring's loads mostly hit L2.
-#ifndef EB_L2_PREFETCH
-#define EB_L2_PREFETCH 0
-#endif
-constexpr int kPrefetch = EB_L2_PREFETCH;
-
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -112,13 +105,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* map, int x, int y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(x), "r"(y)
-               : "memory");
 }
 
 // K-major operand, 128-byte swizzle: rows of 128 B, 8-row atoms 1024 B apart.
@@ -315,26 +301,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x) {
         const Item it = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item);
-        Item nx = it;
-        const bool has_next = kPrefetch > 0 && item + (int)gridDim.x < total;
-        if (has_next) nx = decode<GATEUP>(d, seg_rows, seg_wid, seg_items, nseg, item + gridDim.x);
-        if (kPrefetch > 0 && item == (int)blockIdx.x) {
-          for (int p = 0; p < kPrefetch && p < nk; ++p) {
-            tma_prefetch_2d(&map_w, p * kBK, it.wrow);
-            if (GATEUP) tma_prefetch_2d(&map_w, p * kBK, it.wrow + d.F);
-          }
-        }
         for (int kb = 0; kb < nk; ++kb) {
-          if (kPrefetch > 0) {
-            const int pk = kb + kPrefetch;
-            if (pk < nk) {
-              tma_prefetch_2d(&map_w, pk * kBK, it.wrow);
-              if (GATEUP) tma_prefetch_2d(&map_w, pk * kBK, it.wrow + d.F);
-            } else if (has_next && pk - nk < nk) {
-              tma_prefetch_2d(&map_w, (pk - nk) * kBK, nx.wrow);
-              if (GATEUP) tma_prefetch_2d(&map_w, (pk - nk) * kBK, nx.wrow + d.F);
-            }
-          }
           if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1, abort_flag, &st->status)) {
             ok = false;
             break;

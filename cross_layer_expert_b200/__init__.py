@@ -36,7 +36,7 @@ EXPORTED = ["eb_status_string", "eb_config_check", "eb_workspace_size", "eb_crea
             "eb_sync_status", "eb_route", "eb_loads", "eb_schedule", "eb_profile",
             "eb_profile_read", "eb_launch_count", "eb_route_loads_static",
             "eb_selftest_timeout", "eb_set_expert_map", "eb_loads_mapped", "eb_set_router",
-            "eb_router", "eb_engines", "eb_inject_status"]
+            "eb_router", "eb_engines", "eb_inject_status", "eb_expert_ffn"]
 
 PROF_KERNELS = ("route", "schedule", "permute", "gemm_gateup", "gemm_down", "combine",
                 "positions", "router")
@@ -94,6 +94,7 @@ def load() -> ctypes.CDLL:
         "eb_route_loads_static": (I, [P, I, I, I, I, I, I, P, P, P, P, P]),
         "eb_selftest_timeout": (I, [ctypes.c_int64, P, P]),
         "eb_inject_status": (I, [P, I, P]),
+        "eb_expert_ffn": (I, [P, P, I, P, P, P, I, P, P, P, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -261,6 +262,23 @@ class Context:
                                  _ptr(w_down), _ptr(self.workspace), self.ws_bytes,
                                  _stream(stream), ctypes.byref(n)), "eb_episode")
         return n.value
+
+    def eb_expert_ffn(self, rows, seg_off, seg_layer, seg_expert, out, w_gateup, w_down,
+                      stream=None) -> None:
+        """Expert FFN of grouped rows: rows [R, H] (device, cfg dtype), segment
+        i = rows [seg_off[i], seg_off[i+1]) for expert seg_expert[i] of layer
+        seg_layer[i] (host int sequences); out [R, H] receives every row's
+        expert output in the same order.  Synchronous."""
+        nseg = len(seg_layer)
+        off = (ctypes.c_int32 * (nseg + 1))(*[int(v) for v in seg_off])
+        lay = (ctypes.c_int32 * max(nseg, 1))(*[int(v) for v in seg_layer])
+        exp = (ctypes.c_int32 * max(nseg, 1))(*[int(v) for v in seg_expert])
+        R = int(rows.shape[0])
+        _check(load().eb_expert_ffn(self.handle, _ptr(rows), R, ctypes.cast(off, ctypes.c_void_p),
+                                    ctypes.cast(lay, ctypes.c_void_p),
+                                    ctypes.cast(exp, ctypes.c_void_p), nseg, _ptr(out),
+                                    _ptr(w_gateup), _ptr(w_down), _ptr(self.workspace),
+                                    self.ws_bytes, _stream(stream)), "eb_expert_ffn")
 
     def eb_utilization(self):
         a, b, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()

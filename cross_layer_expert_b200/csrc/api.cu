@@ -40,6 +40,8 @@ struct eb_ctx {
   void* deferred_hidden = nullptr;
   // steps enqueued since create; its parity picks the step's StepView slot
   long long seq = 0;
+  // the GEMMs' state for eb_expert_ffn (the step state stays untouched)
+  State* ffn_st = nullptr;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
   // cached TMA maps (rebuilt when a pointer changes)
@@ -194,6 +196,17 @@ cudaError_t timed(eb_ctx* x, int kernel, int n_launch, cudaStream_t s, F&& launc
   return e;
 }
 
+// p[i] = i for i < n (the identity row map of eb_expert_ffn).
+__global__ void k_iota(int32_t* p, int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) p[i] = i;
+}
+
+cudaError_t launch_iota(int32_t* p, int n, cudaStream_t s) {
+  k_iota<<<(n + 255) / 256, 256, 0, s>>>(p, n);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 extern "C" {
@@ -276,7 +289,8 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   // MaxUtil search grid results, when one CTA would search too many subsets
   const bool grid_search = c->policy == EB_SCHED_MAXUTIL && maxutil_uses_grid(c->M, c->m);
   const size_t n_slots = grid_search ? align_up(kSearchCtas * kSearchSlotBytes) : 0;
-  const size_t n_all = n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots;
+  const size_t n_all =
+      n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots + n_state;
   char* p = nullptr;
   if (e == cudaSuccess) e = cudaMalloc(&p, n_all);
   if (e == cudaSuccess) e = cudaMemset(p, 0, n_all);
@@ -293,6 +307,7 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->dev.arrive_bytes = n_arrive;
     x->dev.search_slots =
         n_slots ? (void*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive) : nullptr;
+    x->ffn_st = (State*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots);
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
   for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
@@ -723,6 +738,106 @@ eb_status eb_loads_mapped(const int32_t* hist, int M, int E, int D, const int32_
   if (cuda_error_pending()) return EB_ERR_CUDA;
   return cuda_status(
       launch_loads(hist, M, E, D, expert_rank, w, status_dev, (cudaStream_t)stream));
+}
+
+eb_status eb_expert_ffn(eb_ctx* x, const void* rows, int R, const int32_t* seg_off,
+                        const int32_t* seg_layer, const int32_t* seg_expert, int nseg, void* out,
+                        const void* wgu, const void* wdn, void* workspace, size_t ws_bytes,
+                        void* stream) {
+  if (!x) return EB_ERR_INVALID_ARG;
+  const eb_config& c = x->cfg;
+  if (!c.compute) return EB_ERR_UNSUPPORTED;
+  if (R < 0 || nseg < 0 || !wgu || !wdn || !workspace) return EB_ERR_INVALID_ARG;
+  if (R > 0 && (!rows || !out)) return EB_ERR_INVALID_ARG;
+  if (nseg > 0 && (!seg_off || !seg_layer || !seg_expert)) return EB_ERR_INVALID_ARG;
+  if (((uintptr_t)workspace & (kAlign - 1)) != 0) return EB_ERR_INVALID_ARG;
+  if (!aligned16(wgu) || !aligned16(wdn) || (R > 0 && (!aligned16(rows) || !aligned16(out))))
+    return EB_ERR_INVALID_ARG;
+  Work w;
+  const size_t need = layout(c, (char*)workspace, &w);
+  if (ws_bytes < need) return EB_ERR_WORKSPACE;
+  const int Et = c.E + c.n_shared;
+  if ((long long)R > w.Rcap || nseg > c.M * Et) return EB_ERR_UNSUPPORTED;
+  // the segment table: offsets ascending from 0 to R, (layer, expert) in range
+  if (nseg == 0 ? R != 0 : (seg_off[0] != 0 || seg_off[nseg] != R)) return EB_ERR_INVALID_ARG;
+  for (int i = 0; i < nseg; ++i)
+    if (seg_off[i + 1] < seg_off[i] || seg_layer[i] < 0 || seg_layer[i] >= c.L ||
+        seg_expert[i] < 0 || seg_expert[i] >= Et)
+      return EB_ERR_INVALID_ARG;
+  if (cuda_error_pending()) return EB_ERR_CUDA;
+  if (R == 0) return EB_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  x->last_stream = s;
+  // the engines of the step, without the gather (GEMM 1 reads the rows as
+  // given) and without the fused combine (there is no combine here)
+  const int g1 = !x->use_tc ? EB_GEMM_SIMT : x->eng1 == EB_GEMM_TMG ? EB_GEMM_TM : x->eng1;
+  const int g2 = !x->use_tc ? EB_GEMM_SIMT : x->eng2 == EB_GEMM_TMC ? EB_GEMM_TM : x->eng2;
+  int rn1, fm1, rn2, fm2;
+  engine_tiles(g1, 1, &rn1, &fm1);
+  engine_tiles(g2, 2, &rn2, &fm2);
+  // the plan, built here: rows, (layer, expert) and work items per segment
+  std::vector<int32_t> plan(4 * (size_t)(nseg + 1), 0);
+  int32_t* p_rows = plan.data();
+  int32_t* p_wid = p_rows + (nseg + 1);
+  int32_t* p_it1 = p_wid + (nseg + 1);
+  int32_t* p_it2 = p_it1 + (nseg + 1);
+  const int mb1 = c.F / fm1, mb2 = c.H / fm2;
+  for (int i = 0; i <= nseg; ++i) {
+    p_rows[i] = seg_off[i];
+    if (i == nseg) break;
+    const int n = seg_off[i + 1] - seg_off[i];
+    p_wid[i] = seg_layer[i] * Et + seg_expert[i];
+    p_it1[i + 1] = p_it1[i] + (n + rn1 - 1) / rn1 * mb1;
+    p_it2[i + 1] = p_it2[i] + (n + rn2 - 1) / rn2 * mb2;
+  }
+  State fs{};
+  fs.nseg = nseg;
+  fs.runset = 1u;
+  fs.rows = R;
+  fs.items1 = p_it1[nseg];
+  fs.items2 = p_it2[nseg];
+  // the GEMMs read the rows as given and write each output row in place:
+  // row r's (token, slot) is r
+  Work wf = w;
+  wf.A = const_cast<void*>(rows);
+  wf.y = out;
+  wf.Rcap = R;
+  CtxDev cf = x->dev;
+  cf.st = x->ffn_st;
+  cf.arrive = nullptr;
+  cudaError_t e = cudaMemcpyAsync(w.seg_rows, p_rows, sizeof(int32_t) * (nseg + 1),
+                                  cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w.seg_wid, p_wid, sizeof(int32_t) * nseg, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w.seg_items1, p_it1, sizeof(int32_t) * (nseg + 1), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(w.seg_items2, p_it2, sizeof(int32_t) * (nseg + 1), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(x->ffn_st, &fs, sizeof(State), cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(w.gemm_next, 0, sizeof(int32_t) * 2, s);
+  if (e == cudaSuccess) e = launch_iota(w.rowslot, R, s);
+  // (the host buffers above are pageable: each copy has read its source
+  // before it returns)
+  TcMaps maps;
+  if (e == cudaSuccess && x->use_tc && make_tc_maps(x->d, wf, wgu, wdn, &maps) != cudaSuccess)
+    return EB_ERR_UNSUPPORTED;
+  auto run = [&](int eng, int which) -> cudaError_t {
+    switch (eng) {
+      case EB_GEMM_TC: return launch_gemm_tc(x->d, cf, wf, maps, x->num_sms, s, which);
+      case EB_GEMM_TM:
+        return launch_gemm_tm(x->d, cf, wf, maps, x->num_sms, s, which, nullptr, nullptr);
+      default: return launch_gemm_simt(x->d, cf, wf, wgu, wdn, s, which);
+    }
+  };
+  if (e == cudaSuccess) e = timed(x, 3, 1, s, [&] { return run(g1, 1); });
+  if (e == cudaSuccess) e = timed(x, 4, 1, s, [&] { return run(g2, 2); });
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return EB_ERR_CUDA;
+  int status = EB_OK;
+  if (cudaMemcpy(&status, &x->ffn_st->status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return EB_ERR_CUDA;
+  return status == EB_OK ? EB_OK : (eb_status)status;
 }
 
 eb_status eb_schedule(const int32_t* w, uint32_t pending_mask, int M, int D, int m, int policy,

@@ -28,10 +28,11 @@ One step:
      token's rank sums them in slot order.
 
 Everything here is plumbing over ``torch.distributed``: the all-reduce of
-counts, the all-to-alls of counts and rows, and the agreement check.  The
-routing, scheduling and expert arithmetic are the callers' (the library's
-kernels on a GPU).  Step 5 on a GPU needs a grouped-FFN entry point over
-received rows, which the library does not export yet.
+counts, the all-to-alls of counts and rows, the agreement check, and the
+grouping of received rows into (layer, expert) segments.  The routing,
+scheduling and expert arithmetic are the callers' -- on a GPU the library's
+kernels: ``eb_route`` / the step's routing, ``eb_loads``, ``eb_schedule``,
+and for step 5 ``eb_expert_ffn`` over the segments ``segment_rows`` builds.
 """
 from __future__ import annotations
 
@@ -136,3 +137,24 @@ def exchange_back(results, recv_counts, order, send_counts, group=None):
     out = torch.empty_like(back)
     out[torch.from_numpy(np.asarray(order))] = back
     return out
+
+
+def segment_rows(layer, expert):
+    """Groups received rows by (layer, expert) for the expert FFN of step 5.
+
+    layer, expert: int arrays [n] of each received row.  Returns (order,
+    seg_off, seg_layer, seg_expert): rows[order] lists the rows segment by
+    segment (segments ascending by (layer, expert), rows of a segment in
+    received order), segment i being rows seg_off[i] .. seg_off[i+1] of that
+    list.  The FFN's output row q belongs to received row order[q]."""
+    layer = np.asarray(layer, dtype=np.int64)
+    expert = np.asarray(expert, dtype=np.int64)
+    if len(layer) == 0:
+        empty = np.zeros(0, dtype=np.int64)
+        return empty, np.zeros(1, dtype=np.int64), empty, empty
+    order = np.lexsort((np.arange(len(layer)), expert, layer))
+    key = np.stack([layer[order], expert[order]], 1)
+    starts = [0] + [q for q in range(1, len(order)) if (key[q] != key[q - 1]).any()]
+    seg_off = np.array(starts + [len(order)], dtype=np.int64)
+    return order, seg_off, key[starts, 0], key[starts, 1]
+

@@ -207,6 +207,28 @@ eb_status eb_moe_step(eb_ctx* ctx, const float* logits, void* hidden, const void
                       const void* w_down, void* workspace, size_t workspace_bytes, void* stream,
                       uint32_t* runset_host);
 
+/* The expert computation of expert parallelism ([EB] §2.2: between the
+ * dispatch and combine all-to-alls, a rank runs its experts' FFNs on the
+ * token rows it received): rows [R, H] (cfg.dtype, DEVICE, 16-byte aligned,
+ * caller-owned) are grouped into nseg segments, segment i being rows
+ * [seg_off[i], seg_off[i+1]) for expert seg_expert[i] (0..E+n_shared-1) of
+ * layer seg_layer[i] (HOST int32 arrays; seg_off has nseg + 1 entries,
+ * ascending from 0 to R; segments may come in any order and repeat an
+ * expert).  out [R, H] (cfg.dtype, DEVICE, 16-byte aligned) receives
+ * W_down (silu(W_gate x) * (W_up x)) of every row x, in the same order, with
+ * the step's arithmetic (bf16 activation, fp32 accumulation, one rounding of
+ * each output).  The step's GEMM engines run it (the gathering and
+ * fused-combine engines as their plain token-major form); it uses the
+ * context's workspace, so no step of the context may be in flight, and it
+ * leaves the step state untouched.  Synchronous.  Needs cfg.compute;
+ * R <= M * T * (k + n_shared) and nseg <= M * (E + n_shared)
+ * (EB_ERR_UNSUPPORTED otherwise); EB_ERR_INVALID_ARG for a malformed segment
+ * table; EB_ERR_TIMEOUT if a bounded device wait expired. */
+eb_status eb_expert_ffn(eb_ctx* ctx, const void* rows, int R, const int32_t* seg_off,
+                        const int32_t* seg_layer, const int32_t* seg_expert, int nseg, void* out,
+                        const void* w_gateup, const void* w_down, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
 /* A whole episode: eb_reset, then eb_moe_step until S is empty.  Steps are
  * enqueued a few ahead of the host's completion check, so the GPU never waits
  * for the host; steps enqueued after S became empty do nothing.  Returns the

@@ -76,6 +76,14 @@ def _rank_main(rank, world, port, out_dir, policy):
         payload = torch.from_numpy(np.stack([tok, slot, expert, np.full_like(tok, rank)], 1))
         recv, recv_counts, order, send_counts = ep.exchange(payload, owner[expert], world)
         got = sorted(map(tuple, recv[:, :3].tolist()))
+        # step 5's grouping of the received rows (all at layer 0 here) into
+        # (layer, expert) segments for the expert FFN
+        seg_order, seg_off, seg_layer, seg_expert = ep.segment_rows(
+            np.zeros(recv.shape[0], dtype=np.int64), recv[:, 2].numpy())
+        grouped = recv[:, 2].numpy()[seg_order]
+        seg_ok = (bool(np.all(seg_layer == 0)) and bool(np.all(np.diff(seg_expert) > 0)) and
+                  all(bool(np.all(grouped[seg_off[i]:seg_off[i + 1]] == seg_expert[i]))
+                      for i in range(len(seg_expert))) and int(seg_off[-1]) == recv.shape[0])
         # the rows returned carry a mark of the rank that served them
         served = recv.clone()
         served[:, 3] = rank
@@ -85,7 +93,8 @@ def _rank_main(rank, world, port, out_dir, policy):
                                  for s in steps],
                        "received": got, "recv_owner_ok": bool(np.all(owner[recv[:, 2].numpy()] == rank)),
                        "back_rows_ok": bool(torch.equal(back[:, :3], payload[:, :3])),
-                       "back_served_by_owner": bool(np.all(back[:, 3].numpy() == owner[expert]))}, f)
+                       "back_served_by_owner": bool(np.all(back[:, 3].numpy() == owner[expert])),
+                       "segments_ok": seg_ok}, f)
     finally:
         dist.destroy_process_group()
 
@@ -108,6 +117,7 @@ def test_ep_two_ranks_agree_with_single_process_oracle(tmp_path, policy):
             assert got["runset"] == want["runset"]
             assert {int(k): v for k, v in got["layers"].items()} == want["layers"]
         assert r["recv_owner_ok"] and r["back_rows_ok"] and r["back_served_by_owner"]
+        assert r["segments_ok"]
     # every (token, slot) of micro-batch 0 at layer 0 lands on its expert's owner exactly once
     idx, _ = oracle.route(logits[0, 0], wl.k)
     owner = ep.expert_owner(wl.E, world)
@@ -117,6 +127,15 @@ def test_ep_two_ranks_agree_with_single_process_oracle(tmp_path, policy):
             want[int(owner[idx[t, s]])].append((t, s, int(idx[t, s])))
     for r in range(world):
         assert [tuple(x) for x in res[r]["received"]] == sorted(want[r])
+
+
+def test_segment_rows():
+    from cross_layer_expert_b200 import ep
+    order, off, lay, ex = ep.segment_rows([1, 0, 1, 0, 0], [3, 2, 3, 5, 2])
+    assert order.tolist() == [1, 4, 3, 0, 2]
+    assert off.tolist() == [0, 2, 3, 5] and lay.tolist() == [0, 0, 1] and ex.tolist() == [2, 5, 3]
+    order, off, lay, ex = ep.segment_rows([], [])
+    assert len(order) == 0 and off.tolist() == [0] and len(lay) == 0 and len(ex) == 0
 
 
 def test_token_shards_and_owner_map():

@@ -266,6 +266,38 @@ def test_routing_ahead_equals_step_by_step(small_inputs, name, gemm):
         assert torch.equal(hidden.cpu().view(torch.int16), h_ep.cpu().view(torch.int16)), policy
 
 
+def test_overlapped_episodes_repeat_and_mix_with_single_steps(small_inputs):
+    """One context: an episode, a second episode, a reset and a few single
+    steps, then a third episode.  The overlapped episodes leave nothing
+    pending (the last step's deferred combine is flushed, the routing done
+    ahead of a step that never comes changes nothing), so every episode
+    equals the first bit for bit."""
+    import torch
+    import cross_layer_expert_b200 as eb
+    from _common import lib_config
+    inp = small_inputs["small_bf16"]
+    ctx = eb.Context(lib_config(inp.wl, osch.MAXUTIL, gemm=4))
+    try:
+        outs = []
+        for rep in range(2):
+            hidden = inp.h0.clone()
+            ctx.eb_episode(inp.logits, hidden, inp.w_gateup, inp.w_down)
+            assert ctx.eb_sync_status() == eb.EB_OK
+            outs.append(hidden.cpu())
+        ctx.eb_reset()
+        hidden = inp.h0.clone()
+        for _ in range(3):
+            ctx.eb_moe_step(inp.logits, hidden, inp.w_gateup, inp.w_down)
+        hidden = inp.h0.clone()
+        ctx.eb_episode(inp.logits, hidden, inp.w_gateup, inp.w_down)
+        assert ctx.eb_sync_status() == eb.EB_OK
+        outs.append(hidden.cpu())
+    finally:
+        ctx.close()
+    for o in outs[1:]:
+        assert torch.equal(o.view(torch.int16), outs[0].view(torch.int16))
+
+
 @pytest.mark.parametrize("m", [1, 2, 4])
 def test_small_episode_m_sweep(small_inputs, small_expected, m):
     inp = small_inputs["small_bf16"]

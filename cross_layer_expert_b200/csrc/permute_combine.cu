@@ -198,15 +198,17 @@ __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const Sta
 
 // ---- the copy by the TMA engine ----
 // Rows of up to kBulkMaxRowBytes are copied with bulk copies: a warp's lane 0
-// loads a token's row into one of its two shared-memory slots
+// loads a token's row into one of its kBulkSlots shared-memory slots
 // (cp.async.bulk, completion on an mbarrier), then lanes s < k + n_shared
 // each store it to the row of slot s (cp.async.bulk to global, one bulk
 // group per lane per token).  Before a slot is loaded again, every lane's
-// stores that read it (two tokens back) must have read it.  The copy engine
+// stores that read it (kBulkSlots tokens back) must have read it.  The copy engine
 // moves the bytes; the warps only issue.
 constexpr int kBulkWarps = 8;
-constexpr int kBulkSlots = 2;
+constexpr int kBulkSlots = 3;
 constexpr int kBulkMaxRowBytes = 8192;
+static_assert(kBulkWarps * kBulkSlots * kBulkMaxRowBytes <= 227 * 1024,
+              "the row slots of a CTA fit its shared memory");
 constexpr unsigned long long kBulkWaitNs = 4000000000ull;  // 4 s per wait
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -264,11 +266,11 @@ __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State*
   uint32_t phases = 0;  // bit sl: parity of slot sl's next completion
   int it = 0;
   for (int u = wid; u < units; u += W, ++it) {
-    const int sl = it & 1;
+    const int sl = it % kBulkSlots;
     uint8_t* buf = bulk_rows + (size_t)(warp * kBulkSlots + sl) * bytes;
     const uint32_t bar = smem_u32(&bars[warp][sl]);
     // the stores issued from this slot two tokens ago have read it
-    if (lane < kk) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+    if (lane < kk) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kBulkSlots - 1) : "memory");
     __syncwarp();
     const size_t tok = (size_t)st->run_list[u / d.T] * d.T + (u % d.T);
     if (lane == 0) {

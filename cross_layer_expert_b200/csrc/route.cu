@@ -5,18 +5,24 @@
 // from ([SysLB] §1: L_r = sum_{e in E_r} T_e).
 //
 // A warp routes token rows: the E logits are read coalesced (lane i holds
-// experts i, i+32, ...), each lane sorts its experts once, and the k winners
-// come out of k rounds over the lanes' heads under the order (logit
-// descending, expert index ascending) -- a hardware max-reduction over
-// order-preserving integer keys, then a min-reduction over the expert ids
-// holding the maximum; the winning lane drops its head.  Two rows are routed
-// together, their rounds interleaved.  The gates exp(l_s - l_max) /
-// sum_{s'} exp(l_s' - l_max) are formed from the winners alone when
-// renormalised (the full softmax denominator cancels).  Counts go to
-// shared-memory atomics (integers, so the result is exact and order-free),
-// are written once per (micro-batch, chunk) and are added to the
-// micro-batch's histogram and rank loads with one global atomic per (chunk,
-// expert) and (chunk, rank).
+// experts i, i+32, ...) and mapped to order-preserving integer keys, and each
+// lane sorts its experts by key, descending (a stable sort, so equal keys
+// keep their ascending expert order).  The k winners then come out of k
+// rounds over the lanes' heads: a hardware max-reduction of the head keys,
+// after which the lane holding the maximum pops its head and marks the
+// round.  A lane's winners are thus a prefix of its sorted list, and the
+// rounds it marked are their slots.  When two lanes hold equal maxima in a
+// round, both pop and the warp counts more than k pops; such a row is
+// selected again with the exact order (logit descending, expert index
+// ascending): among the lanes holding the maximum, a min-reduction of their
+// head indices names the one that pops.  Two rows are routed together, their
+// rounds interleaved.  Each lane then writes its own winners: the gates
+// exp(l_s - l_max) / sum_{s'} exp(l_s' - l_max) are formed from the winners
+// alone when renormalised (the full softmax denominator cancels), l_max being
+// the first round's maximum.  Counts go to shared-memory atomics (integers,
+// so the result is exact and order-free), are written once per
+// (micro-batch, chunk) and are added to the micro-batch's histogram and rank
+// loads with one global atomic per (chunk, expert) and (chunk, rank).
 #include <math.h>
 
 #include "eb_internal.cuh"
@@ -32,158 +38,204 @@ __device__ __forceinline__ float warp_sum(float x) {
   return x;
 }
 
-// Order-preserving map of a finite float to uint32 (-0 is folded into +0
-// first, so equal floats map to equal keys).
+// Order-preserving map of a finite float (or -inf) to uint32 (-0 is folded
+// into +0 first, so equal floats map to equal keys).  Every such key is at
+// least order_key(-inf) = 0x007fffff, so 0 is free to mark padding.
 __device__ __forceinline__ uint32_t order_key(float x) {
   const uint32_t u = __float_as_uint(x + 0.0f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Routes R token rows with the calling warp, their k argmax rounds
-// interleaved so the rows' dependency chains overlap.  Lane s < k returns
-// slot s of each row.  Each lane first sorts its VPL experts by (logit
-// descending, expert index ascending); a round then compares only the
-// lanes' heads: the warp maximum of the head keys, then the smallest expert
-// index among the lanes holding it, and the winning lane drops its head.
-// A row with valid[r] false is skipped (its outputs are unspecified).
+// The float order_key maps to this key.
+__device__ __forceinline__ float key_value(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
+}
+
+// One round over the lanes' heads h[0]: returns the warp maximum; every lane
+// holding it pops its head and sets `bit` in `won`.
+template <int VPL>
+__device__ __forceinline__ uint32_t pop_max(uint32_t (&h)[VPL], uint32_t& won, uint32_t bit) {
+  const uint32_t m = __reduce_max_sync(kFull, h[0]);
+  if (h[0] == m) {
+    won |= bit;
+#pragma unroll
+    for (int i = 0; i + 1 < VPL; ++i) h[i] = h[i + 1];
+    h[VPL - 1] = 0u;
+  }
+  return m;
+}
+
+// The k rounds under the exact order: among the lanes whose head holds the
+// maximum key, the one with the smallest expert index pops.
+template <int VPL>
+__device__ __forceinline__ uint32_t exact_rounds(const uint32_t (&key)[VPL], const int (&id)[VPL],
+                                                 int k) {
+  uint32_t h[VPL];
+  int hid[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    h[i] = key[i];
+    hid[i] = id[i];
+  }
+  uint32_t won = 0u;
+  for (int s = 0; s < k; ++s) {
+    const uint32_t m = __reduce_max_sync(kFull, h[0]);
+    const uint32_t me = __reduce_min_sync(kFull, h[0] == m ? (uint32_t)hid[0] : 0xffffffffu);
+    if (h[0] == m && (uint32_t)hid[0] == me) {
+      won |= 1u << s;
+#pragma unroll
+      for (int i = 0; i + 1 < VPL; ++i) {
+        h[i] = h[i + 1];
+        hid[i] = hid[i + 1];
+      }
+      h[VPL - 1] = 0u;
+    }
+  }
+  return won;
+}
+
+// Routes R token rows with the calling warp, their rounds interleaved so the
+// rows' dependency chains overlap, and writes slot s of row r to
+// idx_out[r][s], gate_out[r][s], counting its expert in hist_s.  x[r][i] is
+// the logit of expert i * 32 + lane of row r; a row with valid[r] false is
+// skipped.
 template <int VPL, int R>
-__device__ __forceinline__ void route_rows(const float* const (&row)[R], const bool (&valid)[R],
-                                           int E, int k, int renorm, int lane, int (&out_e)[R],
-                                           float (&out_g)[R], bool& nonfinite) {
-  float v[R][VPL];
+__device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool (&valid)[R], int E,
+                                           int k, int renorm, int lane,
+                                           int32_t* const (&idx_out)[R],
+                                           float* const (&gate_out)[R], int* hist_s,
+                                           bool& nonfinite) {
   uint32_t key[R][VPL];
   int id[R][VPL];
-  float part[R];  // this lane's share of the full softmax denominator (renorm off)
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = i * 32 + lane;
-      float x = -INFINITY;
+      uint32_t kk = 0u;  // padding ranks below every real expert, even one at -inf
       if (valid[r] && e < E) {
-        x = __ldg(row[r] + e);
-        if (!isfinite(x)) {
+        float v = x[r][i];
+        if (!isfinite(v)) {
           nonfinite = true;
-          x = -INFINITY;  // selection stays among real experts; the call reports the error
+          v = -INFINITY;  // selection stays among real experts; the call reports the error
         }
+        kk = order_key(v);
       }
-      v[r][i] = x;
-      key[r][i] = e < E ? order_key(x) : 0u;  // real experts (even -inf) rank above padding
-      if (e < E && key[r][i] == 0u) key[r][i] = 1u;
+      key[r][i] = kk;
       id[r][i] = e;
     }
-  // the first round's maximum is every lane's unsorted maximum
-  float vmax[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    uint32_t bk = 0;
-    int be = 0x7fffffff;
-    float bv = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < VPL; ++i)
-      if (key[r][i] > bk) {
-        bk = key[r][i];
-        be = id[r][i];
-        bv = v[r][i];
-      }
-    const uint32_t wk = __reduce_max_sync(kFull, bk);
-    const int we = (int)__reduce_min_sync(kFull, bk == wk ? (uint32_t)be : 0xffffffffu);
-    vmax[r] = __shfl_sync(kFull, bv, we & 31);
-    part[r] = 0.f;
-    if (!renorm) {
-#pragma unroll
-      for (int i = 0; i < VPL; ++i)
-        if (i * 32 + lane < E) part[r] += expf(v[r][i] - vmax[r]);
-    }
-  }
-  // sort each lane's experts: key descending, index ascending among equal keys
+  // stable sort, key descending: equal keys stay in ascending expert order
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
-    for (int a = 0; a < VPL; ++a)
+    for (int a = 0; a + 1 < VPL; ++a)
 #pragma unroll
-      for (int b = VPL - 1; b > a; --b) {
-        const bool sw = key[r][b] > key[r][b - 1] ||
-                        (key[r][b] == key[r][b - 1] && id[r][b] < id[r][b - 1]);
-        if (sw) {
+      for (int b = VPL - 1; b > a; --b)
+        if (key[r][b] > key[r][b - 1]) {
           const uint32_t tk = key[r][b];
           key[r][b] = key[r][b - 1];
           key[r][b - 1] = tk;
           const int ti = id[r][b];
           id[r][b] = id[r][b - 1];
           id[r][b - 1] = ti;
-          const float tv = v[r][b];
-          v[r][b] = v[r][b - 1];
-          v[r][b - 1] = tv;
         }
-      }
-  float top_v[R];
-  int top_e[R];
+  uint32_t h[R][VPL], won[R], top[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    top_v[r] = -INFINITY;
-    top_e[r] = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) h[r][i] = key[r][i];
+    won[r] = 0u;
+    top[r] = pop_max<VPL>(h[r], won[r], 1u);
   }
-  for (int s = 0; s < k; ++s) {
+#pragma unroll 2
+  for (int s = 1; s < k; ++s) {
+    const uint32_t bit = 1u << s;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const uint32_t wk = __reduce_max_sync(kFull, key[r][0]);
-      const int we = (int)__reduce_min_sync(kFull, key[r][0] == wk ? (uint32_t)id[r][0] : 0xffffffffu);
-      const float wv = __shfl_sync(kFull, v[r][0], we & 31);
-      if (lane == (we & 31)) {  // the winner drops its head
+    for (int r = 0; r < R; ++r) pop_max<VPL>(h[r], won[r], bit);
+  }
 #pragma unroll
-        for (int i = 0; i + 1 < VPL; ++i) {
-          key[r][i] = key[r][i + 1];
-          id[r][i] = id[r][i + 1];
-          v[r][i] = v[r][i + 1];
-        }
-        key[r][VPL - 1] = 0u;
+  for (int r = 0; r < R; ++r) {
+    if (!valid[r]) continue;
+    // equal maxima in two lanes made both pop: select the row again exactly
+    if (__reduce_add_sync(kFull, (unsigned)__popc(won[r])) != (unsigned)k)
+      won[r] = exact_rounds<VPL>(key[r], id[r], k);
+    const float vmax = key_value(top[r]);
+    const int c = __popc(won[r]);
+    // the most winners any lane holds: the loops below stop there
+    const int cmax = (int)__reduce_max_sync(kFull, (unsigned)c);
+    float ex[VPL];
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      ex[i] = 0.f;
+      if (renorm ? (i < cmax && i < c) : (key[r][i] != 0u)) {
+        ex[i] = expf(key_value(key[r][i]) - vmax);
+        sum += ex[i];
       }
-      if (lane == s) {
-        top_v[r] = wv;
-        top_e[r] = we;
+    }
+    const float inv = __frcp_rn(warp_sum(sum));
+    uint32_t rest = won[r];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      if (i >= cmax) break;
+      if (i < c) {
+        const int s = __ffs(rest) - 1;
+        rest &= rest - 1u;
+        idx_out[r][s] = id[r][i];
+        gate_out[r][s] = ex[i] * inv;
+        atomicAdd(&hist_s[id[r][i]], 1);
       }
     }
   }
+}
+
+// Logits of rows t + r * W (r < R) that lie below t1; lane i holds experts
+// i, i + 32, ...
+template <int VPL, int R>
+__device__ __forceinline__ void load_rows(const float* __restrict__ logits, int t, int t1, int E,
+                                          int W, int lane, float (&x)[R][VPL]) {
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    const float ex = (lane < k) ? expf(top_v[r] - vmax[r]) : 0.f;
-    const float denom = warp_sum(renorm ? ex : part[r]);
-    out_e[r] = top_e[r];
-    out_g[r] = ex / denom;
+    const int tr = t + r * W;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = i * 32 + lane;
+      x[r][i] = (tr < t1 && e < E) ? __ldg(logits + (size_t)tr * E + e) : 0.f;
+    }
   }
 }
 
 // Tokens [t0, t1) of a block of rows: warp w routes tokens w, w + W, ...
 // (W warps) R at a time, R = 2 while two rows' registers fit (VPL <= 4).
+// The next R rows' logits are loaded while the current ones are routed.
 template <int VPL>
 __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
                             int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
                             int* hist_s, bool& nonfinite) {
   constexpr int R = VPL <= 4 ? 2 : 1;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  for (int t = t0 + warp; t < t1; t += R * nwarps) {
-    const float* rows[R];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
+  float next[R][VPL];
+  int t = t0 + warp;
+  if (t < t1) load_rows<VPL, R>(logits, t, t1, E, W, lane, next);
+  for (; t < t1; t += R * W) {
+    float x[R][VPL];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) x[r][i] = next[r][i];
+    if (t + R * W < t1) load_rows<VPL, R>(logits, t + R * W, t1, E, W, lane, next);
     bool valid[R];
-    int tr[R];
+    int32_t* io[R];
+    float* go[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      tr[r] = t + r * nwarps;
-      valid[r] = tr[r] < t1;
-      rows[r] = logits + (size_t)(valid[r] ? tr[r] : t) * E;
+      const int tr = t + r * W;
+      valid[r] = tr < t1;
+      const size_t q = (size_t)(valid[r] ? tr : t);
+      io[r] = idx + q * k;
+      go[r] = gate + q * k;
     }
-    int e[R];
-    float g[R];
-    route_rows<VPL, R>(rows, valid, E, k, renorm, lane, e, g, nonfinite);
-    if (lane < k) {
-#pragma unroll
-      for (int r = 0; r < R; ++r)
-        if (valid[r]) {
-          idx[(size_t)tr[r] * k + lane] = e[r];
-          gate[(size_t)tr[r] * k + lane] = g[r];
-          atomicAdd(&hist_s[e[r]], 1);
-        }
-    }
+    route_rows<VPL, R>(x, valid, E, k, renorm, lane, io, go, hist_s, nonfinite);
   }
 }
 
@@ -202,7 +254,7 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
 // after it still start after GEMM 2.  The state it reads was written by the
 // previous scheduler step, which completed before GEMM 2 started.
 template <int VPL>
-__global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__ st,
+__global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict__ st,
                                                      const float* __restrict__ logits,
                                                      int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
@@ -265,7 +317,7 @@ __global__ void __launch_bounds__(1024) k_route_step(Dims d, State* __restrict__
 // Stand-alone path: rows [c*kChunk, ...) of an [n, E] block; counts summed
 // into hist[E] with one global atomic per (CTA, expert) with a non-zero count.
 template <int VPL>
-__global__ void __launch_bounds__(256) k_route_rows(const float* __restrict__ logits, int n, int E,
+__global__ void __launch_bounds__(256, 4) k_route_rows(const float* __restrict__ logits, int n, int E,
                                                      int k, int renorm, int32_t* __restrict__ idx,
                                                      float* __restrict__ gate,
                                                      int32_t* __restrict__ hist,
@@ -293,9 +345,10 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
                               long long mb_stride, long long layer_stride, bool early,
                               cudaStream_t s) {
   dim3 grid(d.NC, d.M);
-  // beside GEMM 2's CTAs (one per SM, most of its registers and shared
-  // memory) an early launch uses 256-thread CTAs
-  const dim3 block(early ? 256 : 1024);
+  // 256-thread CTAs, four per SM: a warp routes a chunk's rows R at a time
+  // while the next ones load, and beside GEMM 2's CTAs (one per SM, most of
+  // its registers and shared memory) an early launch still finds room
+  const dim3 block(256);
   const int32_t* emap = c.use_emap ? c.emap : nullptr;
   const int ea = early ? 1 : 0;
   cudaError_t e;
@@ -405,7 +458,7 @@ cudaError_t static_counts_ptr(int32_t** out) {
 // CTA (c, j): chunk c of micro-batch j of logits [n_mb, T, E]; writes every
 // count of its (j, c) row, so nothing in the scratch needs to start at zero.
 template <int VPL>
-__global__ void __launch_bounds__(1024) k_route_counts_static(const float* __restrict__ logits,
+__global__ void __launch_bounds__(256, 4) k_route_counts_static(const float* __restrict__ logits,
                                                               int T, int E, int k, int renorm, int NC,
                                                               int32_t* __restrict__ idx,
                                                               float* __restrict__ gate,
@@ -461,10 +514,10 @@ extern "C" eb_status eb_route_loads_static(const float* logits, int n_mb, int T,
   cudaStream_t s = (cudaStream_t)stream;
   dim3 grid(NC, n_mb);
   switch (vpl_for(E)) {
-    case 1: k_route_counts_static<1><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
-    case 2: k_route_counts_static<2><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
-    case 4: k_route_counts_static<4><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
-    default: k_route_counts_static<8><<<grid, 1024, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    case 1: k_route_counts_static<1><<<grid, 256, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    case 2: k_route_counts_static<2><<<grid, 256, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    case 4: k_route_counts_static<4><<<grid, 256, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
+    default: k_route_counts_static<8><<<grid, 256, 0, s>>>(logits, T, E, k, renorm, NC, idx, gate, counts, status_dev); break;
   }
   if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   const int n = n_mb * D;

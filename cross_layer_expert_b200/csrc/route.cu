@@ -65,30 +65,60 @@ __device__ __forceinline__ uint32_t pop_max(uint32_t (&h)[VPL], uint32_t& won, u
   return m;
 }
 
+// Sorted position -> expert of a lane: byte i of the packed words is the
+// slot q (expert q * 32 + lane) at sorted position i.
+template <int VPL>
+struct Perm {
+  static constexpr int kW = (VPL + 3) / 4;
+  uint32_t w[kW];
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int q = 0; q < kW; ++q) w[q] = 0x03020100u + 0x04040404u * (uint32_t)q;
+  }
+  // exchanges positions b - 1 and b (b a constant once unrolled)
+  __device__ __forceinline__ void swap(int b) {
+    if ((b & 3) != 0) {
+      const int q = b >> 2, j = b & 3;
+      const uint32_t sel = (0x3210u & ~(0xffu << (4 * (j - 1)))) |
+                           ((uint32_t)j << (4 * (j - 1))) | ((uint32_t)(j - 1) << (4 * j));
+      w[q] = __byte_perm(w[q], 0u, sel);
+    } else if (kW > 1) {  // byte 3 of one word and byte 0 of the next
+      const int q = (b >> 2) - 1, q1 = min(q + 1, kW - 1);
+      const uint32_t lo = __byte_perm(w[q], w[q1], 0x4210u);
+      const uint32_t hi = __byte_perm(w[q], w[q1], 0x7653u);
+      w[q] = lo;
+      w[q1] = hi;
+    }
+  }
+  // drops position 0 (the others move down by one)
+  __device__ __forceinline__ void pop() {
+#pragma unroll
+    for (int q = 0; q + 1 < kW; ++q) w[q] = __funnelshift_r(w[q], w[q + 1], 8);
+    w[kW - 1] >>= 8;
+  }
+  __device__ __forceinline__ int slot(int i) const { return (w[i >> 2] >> (8 * (i & 3))) & 0xff; }
+};
+
 // The k rounds under the exact order: among the lanes whose head holds the
 // maximum key, the one with the smallest expert index pops.
 template <int VPL>
-__device__ __forceinline__ uint32_t exact_rounds(const uint32_t (&key)[VPL], const int (&id)[VPL],
-                                                 int k) {
+__device__ __forceinline__ uint32_t exact_rounds(const uint32_t (&key)[VPL], const Perm<VPL>& perm,
+                                                 int lane, int k) {
   uint32_t h[VPL];
-  int hid[VPL];
 #pragma unroll
-  for (int i = 0; i < VPL; ++i) {
-    h[i] = key[i];
-    hid[i] = id[i];
-  }
+  for (int i = 0; i < VPL; ++i) h[i] = key[i];
+  Perm<VPL> p = perm;
   uint32_t won = 0u;
   for (int s = 0; s < k; ++s) {
     const uint32_t m = __reduce_max_sync(kFull, h[0]);
-    const uint32_t me = __reduce_min_sync(kFull, h[0] == m ? (uint32_t)hid[0] : 0xffffffffu);
-    if (h[0] == m && (uint32_t)hid[0] == me) {
+    const uint32_t hid = h[0] == m ? (uint32_t)(p.slot(0) * 32 + lane) : 0xffffffffu;
+    const uint32_t me = __reduce_min_sync(kFull, hid);
+    if (hid == me) {
       won |= 1u << s;
 #pragma unroll
-      for (int i = 0; i + 1 < VPL; ++i) {
-        h[i] = h[i + 1];
-        hid[i] = hid[i + 1];
-      }
+      for (int i = 0; i + 1 < VPL; ++i) h[i] = h[i + 1];
       h[VPL - 1] = 0u;
+      p.pop();
     }
   }
   return won;
@@ -97,48 +127,53 @@ __device__ __forceinline__ uint32_t exact_rounds(const uint32_t (&key)[VPL], con
 // Routes R token rows with the calling warp, their rounds interleaved so the
 // rows' dependency chains overlap, and writes slot s of row r to
 // idx_out[r][s], gate_out[r][s], counting its expert in hist_s.  x[r][i] is
-// the logit of expert i * 32 + lane of row r; a row with valid[r] false is
-// skipped.
-template <int VPL, int R>
+// the logit of expert i * 32 + lane of row r (0 where that is not below E);
+// FULL: E == 32 * VPL.  A row with valid[r] false is skipped.
+template <int VPL, int R, bool FULL>
 __device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool (&valid)[R], int E,
                                            int k, int renorm, int lane,
                                            int32_t* const (&idx_out)[R],
                                            float* const (&gate_out)[R], int* hist_s,
                                            bool& nonfinite) {
   uint32_t key[R][VPL];
-  int id[R][VPL];
+  Perm<VPL> perm[R];
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int r = 0; r < R; ++r) {
+    float z = 0.f;  // becomes NaN once a logit is infinite or NaN
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      const int e = i * 32 + lane;
-      uint32_t kk = 0u;  // padding ranks below every real expert, even one at -inf
-      if (valid[r] && e < E) {
-        float v = x[r][i];
-        if (!isfinite(v)) {
-          nonfinite = true;
-          v = -INFINITY;  // selection stays among real experts; the call reports the error
-        }
-        kk = order_key(v);
-      }
-      key[r][i] = kk;
-      id[r][i] = e;
+      z = fmaf(x[r][i], 0.f, z);
+      key[r][i] = order_key(x[r][i]);
     }
+    if (__any_sync(kFull, z != 0.f)) {
+      // selection stays among real experts, a non-finite logit ranking as
+      // -inf; the call reports the error
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (!isfinite(x[r][i])) {
+          nonfinite = true;
+          key[r][i] = order_key(-INFINITY);
+        }
+    }
+    if (!FULL) {
+#pragma unroll
+      for (int i = 0; i < VPL; ++i)
+        if (i * 32 + lane >= E) key[r][i] = 0u;  // padding ranks below every real expert
+    }
+    perm[r].init();
+  }
   // stable sort, key descending: equal keys stay in ascending expert order
 #pragma unroll
   for (int r = 0; r < R; ++r)
 #pragma unroll
     for (int a = 0; a + 1 < VPL; ++a)
 #pragma unroll
-      for (int b = VPL - 1; b > a; --b)
-        if (key[r][b] > key[r][b - 1]) {
-          const uint32_t tk = key[r][b];
-          key[r][b] = key[r][b - 1];
-          key[r][b - 1] = tk;
-          const int ti = id[r][b];
-          id[r][b] = id[r][b - 1];
-          id[r][b - 1] = ti;
-        }
+      for (int b = VPL - 1; b > a; --b) {
+        const uint32_t hi = key[r][b - 1], lo = key[r][b];
+        key[r][b - 1] = max(hi, lo);
+        key[r][b] = min(hi, lo);
+        if (lo > hi) perm[r].swap(b);
+      }
   uint32_t h[R][VPL], won[R], top[R];
 #pragma unroll
   for (int r = 0; r < R; ++r) {
@@ -158,7 +193,7 @@ __device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool 
     if (!valid[r]) continue;
     // equal maxima in two lanes made both pop: select the row again exactly
     if (__reduce_add_sync(kFull, (unsigned)__popc(won[r])) != (unsigned)k)
-      won[r] = exact_rounds<VPL>(key[r], id[r], k);
+      won[r] = exact_rounds<VPL>(key[r], perm[r], lane, k);
     const float vmax = key_value(top[r]);
     const int c = __popc(won[r]);
     // the most winners any lane holds: the loops below stop there
@@ -181,9 +216,10 @@ __device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool 
       if (i < c) {
         const int s = __ffs(rest) - 1;
         rest &= rest - 1u;
-        idx_out[r][s] = id[r][i];
+        const int e = perm[r].slot(i) * 32 + lane;
+        idx_out[r][s] = e;
         gate_out[r][s] = ex[i] * inv;
-        atomicAdd(&hist_s[id[r][i]], 1);
+        atomicAdd(&hist_s[e], 1);
       }
     }
   }
@@ -208,8 +244,8 @@ __device__ __forceinline__ void load_rows(const float* __restrict__ logits, int 
 // Tokens [t0, t1) of a block of rows: warp w routes tokens w, w + W, ...
 // (W warps) R at a time, R = 2 while two rows' registers fit (VPL <= 4).
 // The next R rows' logits are loaded while the current ones are routed.
-template <int VPL>
-__device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
+template <int VPL, bool FULL>
+__device__ __forceinline__ void route_chunk_t(const float* __restrict__ logits, int t0, int t1, int E, int k,
                             int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
                             int* hist_s, bool& nonfinite) {
   constexpr int R = VPL <= 4 ? 2 : 1;
@@ -235,8 +271,18 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
       io[r] = idx + q * k;
       go[r] = gate + q * k;
     }
-    route_rows<VPL, R>(x, valid, E, k, renorm, lane, io, go, hist_s, nonfinite);
+    route_rows<VPL, R, FULL>(x, valid, E, k, renorm, lane, io, go, hist_s, nonfinite);
   }
+}
+
+template <int VPL>
+__device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
+                            int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
+                            int* hist_s, bool& nonfinite) {
+  if (E == 32 * VPL)
+    route_chunk_t<VPL, true>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
+  else
+    route_chunk_t<VPL, false>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
 }
 
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j

@@ -7,6 +7,8 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <atomic>
+#include <thread>
 #include <vector>
 
 #include "eb_internal.cuh"
@@ -44,6 +46,10 @@ struct eb_ctx {
   State* ffn_st = nullptr;
   uint32_t* host_pending = nullptr;  // pinned ring for eb_episode's completion checks
   cudaEvent_t events[8] = {};
+  // mapped pinned words the scheduler writes, {S, scheduler launches}; the
+  // host polls them instead (null: the copies and events above are used)
+  volatile uint32_t* host_flag = nullptr;
+  uint32_t sched_launched = 0;  // scheduler launches enqueued since create
   // cached TMA maps (rebuilt when a pointer changes)
   TcMaps maps;
   const void* map_keys[3] = {nullptr, nullptr, nullptr};
@@ -310,6 +316,20 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->ffn_st = (State*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots);
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
+  if (e == cudaSuccess) {
+    void* hf = nullptr;
+    void* hd = nullptr;
+    if (cudaHostAlloc(&hf, 64, cudaHostAllocMapped) == cudaSuccess) {
+      memset(hf, 0, 64);
+      if (cudaHostGetDevicePointer(&hd, hf, 0) == cudaSuccess) {
+        x->host_flag = static_cast<volatile uint32_t*>(hf);
+        x->dev.host_flag = static_cast<volatile uint32_t*>(hd);
+      } else {
+        cudaFreeHost(hf);
+      }
+    }
+    (void)cudaGetLastError();  // without mapped memory eb_episode copies instead
+  }
   for (int i = 0; e == cudaSuccess && i < kLookahead; ++i)
     e = cudaEventCreateWithFlags(&x->events[i], cudaEventDisableTiming);
   if (e == cudaSuccess && x->use_tc) e = gemm_tc_prepare();
@@ -334,6 +354,7 @@ eb_status eb_destroy(eb_ctx* x) {
   }
   for (auto e : x->pool) cudaEventDestroy(e);
   if (x->host_pending) cudaFreeHost(x->host_pending);
+  if (x->host_flag) cudaFreeHost(const_cast<uint32_t*>(x->host_flag));
   if (x->dev_alloc) cudaFree(x->dev_alloc);
   delete x;
   return EB_OK;
@@ -471,9 +492,11 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   x->routed_ahead = false;
   const int slot = (int)(x->seq & 1);
   x->seq += 1;
-  if (e == cudaSuccess)
+  if (e == cudaSuccess) {
     e = timed(x, 1, x->dev.search_slots ? 2 : 1, s,
               [&] { return launch_schedule_step(x->d, x->dev, w, rn1, rn2, fm1, fm2, slot, s); });
+    if (e == cudaSuccess) x->sched_launched += 1u;
+  }
   // the previous step's combine runs beside this step's scheduler: it reads
   // the previous step's view, outputs and gates, none of which the scheduler
   // writes, and the positions pass after it waits for both
@@ -550,6 +573,34 @@ eb_status eb_moe_step(eb_ctx* x, const float* logits, void* hidden, const void* 
   return EB_OK;
 }
 
+// Waits until the scheduler launch numbered `target` (counting from the
+// context's creation) has written the host's mapped words, and returns S as
+// of that step or later (S only shrinks, and an empty S is all the caller
+// tests).  If the stream runs dry first (a launch that never ran, e.g. after
+// an error), S is read from the device state instead.
+static eb_status wait_scheduler(eb_ctx* x, cudaStream_t s, uint32_t target, uint32_t* pending) {
+  for (unsigned it = 1;; ++it) {
+    if ((int32_t)(x->host_flag[1] - target) >= 0) {
+      std::atomic_thread_fence(std::memory_order_acquire);
+      *pending = x->host_flag[0];
+      return EB_OK;
+    }
+    if ((it & 15u) == 0u) {
+      const cudaError_t q = cudaStreamQuery(s);
+      if (q == cudaSuccess) {
+        if ((int32_t)(x->host_flag[1] - target) >= 0) continue;
+        uint32_t p = 0;
+        if (cudaMemcpy(&p, &x->dev.st->pending, sizeof(p), cudaMemcpyDeviceToHost) != cudaSuccess)
+          return EB_ERR_CUDA;
+        *pending = p;
+        return EB_OK;
+      }
+      if (q != cudaErrorNotReady) return EB_ERR_CUDA;
+    }
+    std::this_thread::yield();
+  }
+}
+
 eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* wgu,
                      const void* wdn, void* workspace, size_t ws_bytes, void* stream,
                      int* n_steps) {
@@ -558,9 +609,22 @@ eb_status eb_episode(eb_ctx* x, const float* logits, void* hidden, const void* w
   eb_status st = eb_reset(x, stream);
   if (st != EB_OK) return st;
   const int max_steps = x->d.max_steps;
+  const uint32_t base = x->sched_launched;
   for (int i = 0; i < max_steps; ++i) {
     st = enqueue_step(x, logits, hidden, wgu, wdn, workspace, ws_bytes, s, true);
     if (st != EB_OK) return st;
+    if (x->host_flag) {
+      // the scheduler of the step enqueued kLookahead - 1 steps ago has told
+      // the host S; nothing but kernels sits in the stream
+      const int chk = i - (kLookahead - 1);
+      if (chk >= 0) {
+        uint32_t pending = 0;
+        st = wait_scheduler(x, s, base + (uint32_t)chk + 1u, &pending);
+        if (st != EB_OK) return st;
+        if (pending == 0) break;
+      }
+      continue;
+    }
     const int slot = i % kLookahead;
     cudaError_t e = cudaMemcpyAsync(&x->host_pending[slot], &x->dev.st->pending, sizeof(uint32_t),
                                     cudaMemcpyDeviceToHost, s);

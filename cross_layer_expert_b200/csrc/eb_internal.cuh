@@ -57,6 +57,7 @@ struct State {
   int32_t items2;    // work items of the down GEMM
   int32_t rows;      // permuted rows of this step
   uint32_t gate_buf; // bit j: which of the two gate buffers holds j's current routing
+  uint32_t sched_calls;  // scheduler launches since the context was created (eb_reset keeps it)
   long long num, den, den_sep;  // utilisation accumulators (Eq. (3))
 };
 
@@ -113,6 +114,10 @@ struct CtxDev {
   size_t arrive_bytes;
   void* search_slots;   // [kSearchCtas] MaxUtil search results (MaxUtil with a large
                         // candidate count), else null
+  // mapped pinned host words {S after the step, scheduler launches so far}
+  // that each scheduler launch writes, so that the host learns of the
+  // episode's end without a copy in the stream between the kernels; or null
+  volatile uint32_t* host_flag;
 };
 
 // ---- programmatic dependent launch ----

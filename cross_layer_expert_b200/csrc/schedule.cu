@@ -621,11 +621,21 @@ __global__ void __launch_bounds__(kThreads) k_schedule_step(Dims d, CtxDev c, Wo
   __syncthreads();
   // the micro-batches routed for this step wrote their gates into the
   // buffers their gate_buf bits did not name: from now on those hold them
-  if (tid == 0) ss.gate_buf ^= ss.need_route;
+  if (tid == 0) {
+    ss.gate_buf ^= ss.need_route;
+    ss.sched_calls += 1u;
+  }
+  // the state goes back to global memory; then S and the launch count go to
+  // the host's mapped words, S first (the host reads the count, then S)
   auto write_back = [&]() {
     __syncthreads();
     for (int i = tid; i < kStateWords; i += kThreads)
       reinterpret_cast<int*>(c.st)[i] = reinterpret_cast<const int*>(&ss)[i];
+    if (tid == 0 && c.host_flag) {
+      c.host_flag[0] = ss.pending;
+      __threadfence_system();
+      c.host_flag[1] = ss.sched_calls;
+    }
   };
   auto finish_empty = [&]() {
     if (tid == 0) {

@@ -255,13 +255,17 @@ def run_ours(args, world, rank, local):
     alg = {
         "gemm_gateup": int((P_touch * 2 * wl.F * wl.H * b + R * (wl.H + wl.F) * b).sum()),
         "gemm_down": int((P_touch * wl.H * wl.F * b + R * (wl.F + wl.H) * b).sum()),
+        # the RunSet's rows in, every permuted row out; per row the copy also
+        # reads its pair's expert and rank and writes its position and the
+        # row's (token, slot)
         "permute": int(sum(bin(int(m)).count("1") for m in rows[:, 0]) * wl.T * wl.H * b
-                       + (R * (wl.H * b + 4)).sum()),
+                       + (R * (wl.H * b + 16)).sum()),
         "combine": int((R * (wl.H * b + 8)).sum()
                        + 2 * sum(bin(int(m)).count("1") for m in rows[:, 0]) * wl.T * wl.H * b),
-        # every (micro-batch, layer) is routed once: fp32 logits in, indices
-        # and gates out, one count row per 64-token chunk
-        "route": int(wl.M * wl.L * (wl.T * (4 * wl.E + 8 * wl.k) + -(-wl.T // 64) * 4 * wl.E)),
+        # every (micro-batch, layer) is routed once: fp32 logits in, indices,
+        # gates and in-chunk ranks out, one count row per 64-token chunk
+        # (written, then read back with the chunk offsets written)
+        "route": int(wl.M * wl.L * (wl.T * (4 * wl.E + 12 * wl.k) + -(-wl.T // 64) * 12 * wl.E)),
         # indices in, the row of every (token, slot) and the token of every row out
         "positions": int((R * (4 + 4 + 4)).sum()),
     }

@@ -148,6 +148,10 @@ size_t layout(const eb_config& c, char* base, Work* w) {
   x.idx = (int32_t*)take(sizeof(int32_t) * M * T * c.k);
   x.gate = (float*)take(sizeof(float) * 2 * M * T * c.k);
   x.chunk_hist = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
+  if (c.compute) {
+    x.rank = (int32_t*)take(sizeof(int32_t) * M * T * c.k);
+    x.cbase = (int32_t*)take(sizeof(int32_t) * M * d.NC * c.E);
+  }
   x.views = (StepView*)take(sizeof(StepView) * 2);
   const size_t nseg = M * (size_t)d.Etot;
   if (c.compute) {
@@ -289,6 +293,7 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   const size_t n_trace = align_up(sizeof(long long) * kTraceCols * x->d.max_steps);
   const size_t n_tl = align_up(sizeof(int32_t) * c->M * (size_t)x->d.max_steps);
   const size_t n_map = align_up(sizeof(int32_t) * c->E);
+  const size_t n_tickets = align_up(sizeof(int32_t) * c->M);
   // arrival counters of the fused combine, one per (token, 256-feature block)
   const size_t n_arrive =
       x->eng2 == EB_GEMM_TMC ? align_up(sizeof(int32_t) * (size_t)c->M * c->T * (c->H / kTmFeat2)) : 0;
@@ -296,7 +301,7 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
   const bool grid_search = c->policy == EB_SCHED_MAXUTIL && maxutil_uses_grid(c->M, c->m);
   const size_t n_slots = grid_search ? align_up(kSearchCtas * kSearchSlotBytes) : 0;
   const size_t n_all =
-      n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots + n_state;
+      n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots + n_state + n_tickets;
   char* p = nullptr;
   if (e == cudaSuccess) e = cudaMalloc(&p, n_all);
   if (e == cudaSuccess) e = cudaMemset(p, 0, n_all);
@@ -314,6 +319,8 @@ eb_status eb_create(const eb_config* c, eb_ctx** out) {
     x->dev.search_slots =
         n_slots ? (void*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive) : nullptr;
     x->ffn_st = (State*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots);
+    x->dev.tickets =
+        (int32_t*)(p + n_state + n_hist + n_w + n_trace + n_tl + n_map + n_arrive + n_slots + n_state);
     e = cudaHostAlloc(&x->host_pending, sizeof(uint32_t) * kLookahead, cudaHostAllocDefault);
   }
   if (e == cudaSuccess) {
@@ -507,7 +514,9 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
     });
   }
   if (c.compute) {
-    if (e == cudaSuccess)
+    // the gathering engine reads the rows' positions in GEMM 1; otherwise
+    // the row copy places the rows itself, from the ranks routing wrote
+    if (e == cudaSuccess && gather)
       e = timed(x, 6, 1, s, [&] { return launch_positions(x->d, x->dev, w, s); });
     if (e == cudaSuccess && !gather)
       e = timed(x, 2, 1, s, [&] { return launch_permute_copy(x->d, x->dev, w, hidden, s); });

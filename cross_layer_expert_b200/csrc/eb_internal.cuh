@@ -85,6 +85,9 @@ struct Work {
   int32_t* idx;        // [M][T][k]
   float* gate;         // [2][M][T][k]: two buffers, State::gate_buf picks one per micro-batch
   int32_t* chunk_hist; // [M][NC][E]: counts of each 64-token chunk
+  int32_t* rank;       // [M][T][k]: place of (j, t, s) among its chunk's pairs of its expert
+                       // (expert arithmetic on; else null)
+  int32_t* cbase;      // [M][NC][E]: pairs of expert e in micro-batch j's chunks before c
   int32_t* prior;      // [M][Etot]: rows of (j's segment, expert) taken by earlier RunSet members
   int32_t* pos;        // [M][T][kk]: row of (j, t, slot)
   int32_t* rowslot;    // [Rcap]: slot (j * T + t) * kk + s of each permuted row
@@ -110,6 +113,8 @@ struct CtxDev {
   int32_t* trace_layers;  // [max_steps][M]
   int32_t* emap;        // [E]: rank of each expert (a custom placement)
   int use_emap;         // 0: contiguous map, experts [d E/D, (d+1) E/D) on rank d
+  int32_t* tickets;     // [M]: routing CTAs of micro-batch j done with their chunk (the last
+                        // one writes the chunk offsets and resets it)
   int32_t* arrive;      // [M*T][H/256]: fused-combine arrival counts (engine TMC), else null
   size_t arrive_bytes;
   void* search_slots;   // [kSearchCtas] MaxUtil search results (MaxUtil with a large

@@ -11,10 +11,13 @@
 // [EB-read] §2.1: scheduling may change neither the expert set, the gates nor
 // the aggregation order -- the slot order here is fixed.
 //
-// The permutation is two launches: k_positions computes every (token, slot)
-// row of the RunSet and its inverse, the (token, slot) of every row (a light
-// pass over the routing indices); k_permute_copy then moves the rows --
-// unless GEMM 1 gathers them from the hidden states itself.  GEMM 2 writes
+// The permutation: routing already ranked every (token, slot) pair among its
+// micro-batch's pairs of the same expert (none of which depends on the
+// schedule); the row copy adds the step's segment bases, writes each row's
+// position and its inverse, the (token, slot) of every row, and moves the
+// rows.  When GEMM 1 gathers the rows from the hidden states itself, there is
+// no copy, and k_positions computes the positions from the routing counts
+// in a pass of its own.  GEMM 2 writes
 // each row's output at its (token, slot) position, so the combine reads a
 // token's k + n_shared outputs from one contiguous run.  The copy and the combine are HBM-bound and
 // persistent: a grid of resident CTAs sized to the SM count works through
@@ -140,12 +143,52 @@ __device__ __forceinline__ size_t runset_token(const State* st, int T, int u) {
   return (size_t)st->run_list[u / T] * T + (u % T);
 }
 
+// What the row copy needs to place the rows itself (engines other than the
+// gathering one, which keep k_positions): routing's per-pair ranks and chunk
+// offsets, the step's segment bases and prior rows; the positions it writes.
+struct Place {
+  const int32_t* idx;       // [M][T][k]
+  const int32_t* rank;      // [M][T][k]: place among the chunk's pairs of the expert
+  const int32_t* cbase;     // [M][NC][E]: pairs of the expert in the earlier chunks
+  const int32_t* seg_rows;  // first row of each (group, expert) segment
+  const int32_t* prior;     // [M][Etot]: rows of the segment taken by earlier RunSet members
+  int32_t* pos;             // [M][T][kk]: row of each (token, slot), written here
+  int32_t* rowslot;         // [Rcap]: (token, slot) of each row, written here
+  long long Rcap;
+};
+
+// Row of slot s (< k + n_shared) of token t of RunSet member j, recorded in
+// pos and rowslot: the segment's first row, the rows of earlier RunSet
+// members in it, and the pair's place among j's pairs of that expert in
+// (token, slot) order -- the rows k_positions computes, in the same order.
+// A row outside [0, Rcap) (inconsistent inputs) is returned as -1 and
+// nothing is stored for it.
+__device__ __forceinline__ int place_row(const Dims& d, const State* st, const Place& pl, int j,
+                                         int t, int s) {
+  const size_t tok = (size_t)j * d.T + t;
+  int e, r;
+  if (s < d.k) {
+    e = __ldg(pl.idx + tok * d.k + s);
+    r = __ldg(pl.rank + tok * d.k + s) +
+        __ldg(pl.cbase + ((size_t)j * d.NC + t / kChunk) * d.E + e);
+  } else {  // shared expert: every token of j has one pair
+    e = d.E + (s - d.k);
+    r = t;
+  }
+  const int row = __ldg(pl.seg_rows + st->group_of[j] * d.Etot + e) +
+                  __ldg(pl.prior + j * d.Etot + e) + r;
+  if (row < 0 || (long long)row >= pl.Rcap) return -1;
+  pl.pos[tok * d.kk + s] = row;
+  pl.rowslot[row] = (int)(tok * d.kk + s);
+  return row;
+}
+
 // Persistent copy: warp w moves tokens w, w + W, ... (W = warps in the grid),
 // two at a time: both rows' 16-byte vectors are loaded into registers (8 per
 // lane per token) before the k + n_shared stores of each.
 template <typename T>
 __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const State* __restrict__ st,
-                                                               const int32_t* __restrict__ pos,
+                                                               Place pl,
                                                                const T* __restrict__ hidden,
                                                                T* __restrict__ A) {
   pdl_enter();
@@ -161,8 +204,9 @@ __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const Sta
     const bool two = u2 < units;
     const size_t tok0 = runset_token(st, d.T, u), tok1 = runset_token(st, d.T, two ? u2 : u);
     // slot rows of both tokens, one per lane
-    const int row0 = lane < kk ? __ldg(pos + tok0 * kk + lane) : 0;
-    const int row1 = lane < kk ? __ldg(pos + tok1 * kk + lane) : 0;
+    const int row0 = lane < kk ? place_row(d, st, pl, st->run_list[u / d.T], u % d.T, lane) : 0;
+    const int row1 =
+        two && lane < kk ? place_row(d, st, pl, st->run_list[u2 / d.T], u2 % d.T, lane) : 0;
     const uint4* src0 = reinterpret_cast<const uint4*>(hidden + tok0 * d.H);
     const uint4* src1 = reinterpret_cast<const uint4*>(hidden + tok1 * d.H);
     for (int base = 0; base < nvec; base += 32 * kU) {
@@ -176,14 +220,17 @@ __global__ void __launch_bounds__(kPermThreads) k_permute_copy(Dims d, const Sta
         }
       }
       for (int s = 0; s < kk; ++s) {
-        uint4* dst0 = reinterpret_cast<uint4*>(A + (size_t)__shfl_sync(kFull, row0, s) * d.H);
+        const int r0 = __shfl_sync(kFull, row0, s);
         const int r1 = __shfl_sync(kFull, row1, s);
+        if (r0 >= 0) {
+          uint4* dst0 = reinterpret_cast<uint4*>(A + (size_t)r0 * d.H);
 #pragma unroll
-        for (int q = 0; q < kU; ++q) {
-          const int v = base + q * 32 + lane;
-          if (v < nvec) dst0[v] = v0[q];
+          for (int q = 0; q < kU; ++q) {
+            const int v = base + q * 32 + lane;
+            if (v < nvec) dst0[v] = v0[q];
+          }
         }
-        if (two) {
+        if (two && r1 >= 0) {
           uint4* dst1 = reinterpret_cast<uint4*>(A + (size_t)r1 * d.H);
 #pragma unroll
           for (int q = 0; q < kU; ++q) {
@@ -245,7 +292,7 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
 
 template <typename T>
 __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State* __restrict__ st,
-                                                                  const int32_t* __restrict__ pos,
+                                                                  Place pl,
                                                                   const T* __restrict__ hidden,
                                                                   T* __restrict__ A) {
   pdl_enter();
@@ -265,6 +312,7 @@ __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State*
   __syncwarp();
   uint32_t phases = 0;  // bit sl: parity of slot sl's next completion
   int it = 0;
+  int row = 0;  // this lane's row of the current token (placed one token ahead)
   for (int u = wid; u < units; u += W, ++it) {
     const int sl = it % kBulkSlots;
     uint8_t* buf = bulk_rows + (size_t)(warp * kBulkSlots + sl) * bytes;
@@ -272,7 +320,8 @@ __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State*
     // the stores issued from this slot two tokens ago have read it
     if (lane < kk) asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(kBulkSlots - 1) : "memory");
     __syncwarp();
-    const size_t tok = (size_t)st->run_list[u / d.T] * d.T + (u % d.T);
+    const int j = st->run_list[u / d.T], t = u % d.T;
+    const size_t tok = (size_t)j * d.T + t;
     if (lane == 0) {
       asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                    : "memory");
@@ -281,7 +330,11 @@ __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State*
           ::"r"(smem_u32(buf)), "l"(hidden + tok * d.H), "r"(bytes), "r"(bar)
           : "memory");
     }
-    const int row = lane < kk ? __ldg(pos + tok * kk + lane) : 0;
+    if (it == 0 && lane < kk) row = place_row(d, st, pl, j, t, lane);
+    // the next token's rows are placed while this token's row loads
+    int row_next = 0;
+    const int un = u + W;
+    if (un < units && lane < kk) row_next = place_row(d, st, pl, st->run_list[un / d.T], un % d.T, lane);
     const bool ok = bar_wait(bar, (phases >> sl) & 1u);
     phases ^= 1u << sl;
     if (!__all_sync(0xffffffffu, ok)) {
@@ -292,12 +345,13 @@ __global__ void __launch_bounds__(32 * kBulkWarps) k_permute_bulk(Dims d, State*
       break;
     }
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    if (lane < kk) {
+    if (lane < kk && row >= 0) {
       asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                    ::"l"(A + (size_t)row * d.H), "r"(smem_u32(buf)), "r"(bytes)
                    : "memory");
       asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     }
+    row = row_next;
   }
   // every store has completed (its writes are performed) before the CTA exits
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
@@ -488,6 +542,10 @@ cudaError_t launch_positions(const Dims& d, const CtxDev& c, const Work& w, cuda
 
 int g_grid_bulk_bf16 = 0, g_grid_bulk_f32 = 0;
 
+Place place_of(const Work& w) {
+  return Place{w.idx, w.rank, w.cbase, w.seg_rows, w.prior, w.pos, w.rowslot, w.Rcap};
+}
+
 template <typename T>
 cudaError_t launch_permute_bulk(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
                                 int& grid_cache, cudaStream_t s) {
@@ -508,8 +566,7 @@ cudaError_t launch_permute_bulk(const Dims& d, const CtxDev& c, const Work& w, c
       grid_cache = 148;
   }
   return launch_pdl(k_permute_bulk<T>, dim3(grid_cache), dim3(32 * kBulkWarps), smem, s, 1, d,
-                    c.st, (const int32_t*)w.pos, static_cast<const T*>(hidden),
-                    static_cast<T*>(w.A));
+                    c.st, place_of(w), static_cast<const T*>(hidden), static_cast<T*>(w.A));
 }
 
 cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, const void* hidden,
@@ -523,12 +580,12 @@ cudaError_t launch_permute_copy(const Dims& d, const CtxDev& c, const Work& w, c
     return launch_pdl(k_permute_copy<__nv_bfloat16>,
                       dim3(persistent_grid((const void*)k_permute_copy<__nv_bfloat16>, kPermThreads,
                                            g_grid_copy_bf16)),
-                      dim3(kPermThreads), 0, s, 1, d, c.st, w.pos,
+                      dim3(kPermThreads), 0, s, 1, d, c.st, place_of(w),
                       static_cast<const __nv_bfloat16*>(hidden), static_cast<__nv_bfloat16*>(w.A));
   return launch_pdl(k_permute_copy<float>,
                     dim3(persistent_grid((const void*)k_permute_copy<float>, kPermThreads,
                                          g_grid_copy_f32)),
-                    dim3(kPermThreads), 0, s, 1, d, c.st, w.pos, static_cast<const float*>(hidden),
+                    dim3(kPermThreads), 0, s, 1, d, c.st, place_of(w), static_cast<const float*>(hidden),
                     static_cast<float*>(w.A));
 }
 

@@ -285,12 +285,66 @@ __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, in
     route_chunk_t<VPL, false>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
 }
 
+// Ranks the n (token, slot) pairs of a chunk, ex[p] for p = t * k + s, among
+// the chunk's pairs with the same expert, in p order: out[p] = #{p' < p :
+// ex[p'] == ex[p]}.  A warp's 32 pairs are grouped by expert with a match,
+// the groups' sizes go to cnt[warp][e], and a scan over the warps per expert
+// (carried over rounds of blockDim.x pairs) gives each warp's offset.  All
+// threads of the CTA call it; ex was written by this CTA before a barrier.
+__device__ __forceinline__ unsigned lanemask_lt() {
+  unsigned m;
+  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+  return m;
+}
+
+__device__ void chunk_ranks(const int32_t* ex, int n, int E, int32_t* out) {
+  constexpr int kW = 8;  // warps of a 256-thread CTA
+  __shared__ int cnt[kW][EB_MAX_ETOT];
+  __shared__ int running[EB_MAX_ETOT];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < kW * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+  for (int e = tid; e < E; e += blockDim.x) running[e] = 0;
+  __syncthreads();
+  for (int r0 = 0; r0 < n; r0 += blockDim.x) {
+    const int p = r0 + tid;
+    const int e = p < n ? ex[p] : -1;
+    const unsigned peers = __match_any_sync(kFull, e);
+    const int in_warp = __popc(peers & lanemask_lt());
+    if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] = __popc(peers);
+    __syncthreads();
+    for (int ee = tid; ee < E; ee += blockDim.x) {
+      int run = running[ee];
+      for (int w = 0; w < kW; ++w) {
+        const int c = cnt[w][ee];
+        cnt[w][ee] = run;
+        run += c;
+      }
+      running[ee] = run;
+    }
+    __syncthreads();
+    if (e >= 0) out[p] = cnt[warp][e] + in_warp;
+    __syncthreads();
+    for (int i = tid; i < kW * E; i += blockDim.x) cnt[i / E][i % E] = 0;
+    __syncthreads();
+  }
+}
+
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
 // is in need_route; its counts land in chunk_hist[j][c][:] and are added
 // (integer atomics: exact, order-free) to the micro-batch's histogram
 // hist[j][:] and rank loads w[j][:], which the previous step zeroed.  The
 // loads fold the counts by the context's expert placement: contiguous
 // blocks of E/D experts, or emap[e] if one was set.
+//
+// With `rank` set (expert arithmetic on), the CTA also ranks its chunk's
+// (token, slot) pairs among those with the same expert, in (token, slot)
+// order, into rank[j][t][s]; and the last of micro-batch j's NC CTAs to
+// finish (a ticket taken after every CTA's counts are visible) writes the
+// chunk offsets cbase[j][c][e] = sum over c' < c of chunk_hist[j][c'][e].
+// rank + cbase is the pair's place among micro-batch j's pairs of its
+// expert; none of it depends on the schedule, so the row copy of the step
+// that runs j only adds the segment's base and the rows of earlier RunSet
+// members (see k_permute_bulk).
 //
 // early: launched right after the previous step's GEMM 2 (whose persistent
 // CTAs are all resident), which reads nothing routing writes -- the gates go
@@ -309,7 +363,9 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
                                                      int32_t* __restrict__ wload,
                                                      const int32_t* __restrict__ emap,
                                                      long long mb_stride, long long layer_stride,
-                                                     int early) {
+                                                     int32_t* __restrict__ rank,
+                                                     int32_t* __restrict__ cbase,
+                                                     int32_t* __restrict__ tickets, int early) {
   if (early) pdl_trigger();
   else pdl_enter();
   const int c = blockIdx.x, j = blockIdx.y;
@@ -357,6 +413,30 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
     }
   }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
+  if (rank) {
+    const size_t base = (size_t)j * d.T + t0;
+    chunk_ranks(idx + base * d.k, (t1 - t0) * d.k, d.E, rank + base * d.k);
+    // every thread's counts of this chunk are visible before the ticket
+    __threadfence();
+    __shared__ int last;
+    __syncthreads();
+    if (threadIdx.x == 0) last = atomicAdd(&tickets[j], 1) == d.NC - 1;
+    __syncthreads();
+    if (last) {
+      __threadfence();
+      const int32_t* ch = chunk_hist + (size_t)j * d.NC * d.E;
+      int32_t* cb = cbase + (size_t)j * d.NC * d.E;
+      for (int e = threadIdx.x; e < d.E; e += blockDim.x) {
+        int run = 0;
+#pragma unroll 8
+        for (int cc = 0; cc < d.NC; ++cc) {
+          cb[(size_t)cc * d.E + e] = run;
+          run += __ldcg(ch + (size_t)cc * d.E + e);
+        }
+      }
+      if (threadIdx.x == 0) tickets[j] = 0;
+    }
+  }
   if (early) pdl_wait();
 }
 
@@ -399,10 +479,10 @@ cudaError_t launch_route_step(const Dims& d, const CtxDev& c, const Work& w, con
   const int ea = early ? 1 : 0;
   cudaError_t e;
   switch (vpl_for(d.E)) {
-    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
-    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
-    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
-    default: e = launch_pdl(k_route_step<8>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, ea); break;
+    case 1: e = launch_pdl(k_route_step<1>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, w.rank, w.cbase, c.tickets, ea); break;
+    case 2: e = launch_pdl(k_route_step<2>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, w.rank, w.cbase, c.tickets, ea); break;
+    case 4: e = launch_pdl(k_route_step<4>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, w.rank, w.cbase, c.tickets, ea); break;
+    default: e = launch_pdl(k_route_step<8>, dim3(grid), block, 0, s, 1, d, c.st, logits, w.idx, w.gate, w.chunk_hist, c.hist, c.w, emap, mb_stride, layer_stride, w.rank, w.cbase, c.tickets, ea); break;
   }
   return e;
 }

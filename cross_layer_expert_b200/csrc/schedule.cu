@@ -919,6 +919,8 @@ __global__ void k_reset(Dims d, CtxDev c) {
   State* st = c.st;
   for (int i = threadIdx.x; i < d.M * d.E; i += blockDim.x) c.hist[i] = 0;
   for (int i = threadIdx.x; i < d.M * d.D; i += blockDim.x) c.w[i] = 0;
+  // a routing launch cut short may have left tickets behind
+  for (int i = threadIdx.x; i < d.M; i += blockDim.x) c.tickets[i] = 0;
   if (threadIdx.x != 0) return;
   const uint32_t all = d.M >= 32 ? 0xffffffffu : ((1u << d.M) - 1u);
   for (int j = 0; j < EB_MAX_M; ++j) {

@@ -297,9 +297,11 @@ __device__ __forceinline__ unsigned lanemask_lt() {
   return m;
 }
 
-__device__ void chunk_ranks(const int32_t* ex, int n, int E, int32_t* out) {
-  constexpr int kW = 8;  // warps of a 256-thread CTA
-  __shared__ int cnt[kW][EB_MAX_ETOT];
+constexpr int kRankWarps = 8;  // warps of a 256-thread routing CTA
+
+__device__ void chunk_ranks(const int32_t* ex, int n, int E, int32_t* out,
+                            int (&cnt)[kRankWarps][EB_MAX_ETOT]) {
+  constexpr int kW = kRankWarps;
   __shared__ int running[EB_MAX_ETOT];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kW * E; i += blockDim.x) cnt[i / E][i % E] = 0;
@@ -414,8 +416,9 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
   }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
   if (rank) {
+    __shared__ int scratch[kRankWarps][EB_MAX_ETOT];
     const size_t base = (size_t)j * d.T + t0;
-    chunk_ranks(idx + base * d.k, (t1 - t0) * d.k, d.E, rank + base * d.k);
+    chunk_ranks(idx + base * d.k, (t1 - t0) * d.k, d.E, rank + base * d.k, scratch);
     // every thread's counts of this chunk are visible before the ticket
     __threadfence();
     __shared__ int last;
@@ -423,13 +426,27 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
     if (threadIdx.x == 0) last = atomicAdd(&tickets[j], 1) == d.NC - 1;
     __syncthreads();
     if (last) {
+      // warp w sums its range of chunks per expert (lanes over experts,
+      // loads coalesced), the ranges' totals are scanned in shared memory,
+      // and each warp writes its range's offsets
       __threadfence();
       const int32_t* ch = chunk_hist + (size_t)j * d.NC * d.E;
       int32_t* cb = cbase + (size_t)j * d.NC * d.E;
-      for (int e = threadIdx.x; e < d.E; e += blockDim.x) {
-        int run = 0;
+      const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+      const int per = (d.NC + kRankWarps - 1) / kRankWarps;
+      const int c0 = min(d.NC, warp * per), c1 = min(d.NC, c0 + per);
+      for (int e = lane; e < d.E; e += 32) {
+        int sum = 0;
 #pragma unroll 8
-        for (int cc = 0; cc < d.NC; ++cc) {
+        for (int cc = c0; cc < c1; ++cc) sum += __ldcg(ch + (size_t)cc * d.E + e);
+        scratch[warp][e] = sum;
+      }
+      __syncthreads();
+      for (int e = lane; e < d.E; e += 32) {
+        int run = 0;
+        for (int w = 0; w < warp; ++w) run += scratch[w][e];
+#pragma unroll 8
+        for (int cc = c0; cc < c1; ++cc) {
           cb[(size_t)cc * d.E + e] = run;
           run += __ldcg(ch + (size_t)cc * d.E + e);
         }

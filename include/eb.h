@@ -268,9 +268,12 @@ eb_status eb_trace(eb_ctx* ctx, int64_t* rows, int32_t* layers, int max_steps, i
  * enqueues with CUDA events on the launching stream (eb_profile(ctx, 0) stops;
  * both drop earlier marks).  eb_profile_read waits for them and returns, per
  * kernel, the summed milliseconds and the number of launches since, then
- * clears the marks.  Kernel order: route, schedule+plan, permute (the row
- * copy), GEMM 1 (gate/up + SwiGLU), GEMM 2 (down), combine, positions (the
- * rows of every token slot), router projection (router mode).
+ * clears the marks.  Kernel order: route (with the rows' ranks within their
+ * chunk and the chunk offsets), schedule+plan, permute (the row copy, which
+ * also places the rows), GEMM 1 (gate/up + SwiGLU), GEMM 2 (down), combine,
+ * positions (the rows of every token slot, computed in a pass of its own
+ * only for the gathering GEMM 1, which has no row copy), router projection
+ * (router mode).
  * eb_launch_count returns the kernels the context has enqueued since
  * eb_create.  eb_engines returns the EB_GEMM_* engine that runs GEMM 1 and
  * GEMM 2 (after AUTO and the shape fallbacks above are resolved; SIMT for

@@ -128,12 +128,15 @@ __device__ __forceinline__ uint32_t exact_rounds(const uint32_t (&key)[VPL], con
 // rows' dependency chains overlap, and writes slot s of row r to
 // idx_out[r][s], gate_out[r][s], counting its expert in hist_s.  x[r][i] is
 // the logit of expert i * 32 + lane of row r (0 where that is not below E);
-// FULL: E == 32 * VPL.  A row with valid[r] false is skipped.
+// FULL: E == 32 * VPL.  A row with valid[r] false is skipped.  With emask
+// set, each winner also sets bit tl[r] (the row's token within its 64-token
+// chunk) of its expert's 64-bit mask emask[2e], emask[2e + 1].
 template <int VPL, int R, bool FULL>
 __device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool (&valid)[R], int E,
                                            int k, int renorm, int lane,
                                            int32_t* const (&idx_out)[R],
                                            float* const (&gate_out)[R], int* hist_s,
+                                           uint32_t* emask, const int (&tl)[R],
                                            bool& nonfinite) {
   uint32_t key[R][VPL];
   Perm<VPL> perm[R];
@@ -220,6 +223,7 @@ __device__ __forceinline__ void route_rows(const float (&x)[R][VPL], const bool 
         idx_out[r][s] = e;
         gate_out[r][s] = ex[i] * inv;
         atomicAdd(&hist_s[e], 1);
+        if (emask) atomicOr(&emask[2 * e + (tl[r] >> 5)], 1u << (tl[r] & 31));
       }
     }
   }
@@ -245,9 +249,11 @@ __device__ __forceinline__ void load_rows(const float* __restrict__ logits, int 
 // (W warps) R at a time, R = 2 while two rows' registers fit (VPL <= 4).
 // The next R rows' logits are loaded while the current ones are routed.
 template <int VPL, bool FULL>
-__device__ __forceinline__ void route_chunk_t(const float* __restrict__ logits, int t0, int t1, int E, int k,
-                            int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
-                            int* hist_s, bool& nonfinite) {
+__device__ __forceinline__ void route_chunk_t(const float* __restrict__ logits, int t0, int t1,
+                                              int E, int k, int renorm,
+                                              int32_t* __restrict__ idx,
+                                              float* __restrict__ gate, int* hist_s,
+                                              uint32_t* emask, bool& nonfinite) {
   constexpr int R = VPL <= 4 ? 2 : 1;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, W = blockDim.x >> 5;
   float next[R][VPL];
@@ -263,6 +269,7 @@ __device__ __forceinline__ void route_chunk_t(const float* __restrict__ logits, 
     bool valid[R];
     int32_t* io[R];
     float* go[R];
+    int tl[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
       const int tr = t + r * W;
@@ -270,66 +277,24 @@ __device__ __forceinline__ void route_chunk_t(const float* __restrict__ logits, 
       const size_t q = (size_t)(valid[r] ? tr : t);
       io[r] = idx + q * k;
       go[r] = gate + q * k;
+      tl[r] = (valid[r] ? tr : t) - t0;
     }
-    route_rows<VPL, R, FULL>(x, valid, E, k, renorm, lane, io, go, hist_s, nonfinite);
+    route_rows<VPL, R, FULL>(x, valid, E, k, renorm, lane, io, go, hist_s, emask, tl, nonfinite);
   }
 }
 
 template <int VPL>
 __device__ void route_chunk(const float* __restrict__ logits, int t0, int t1, int E, int k,
                             int renorm, int32_t* __restrict__ idx, float* __restrict__ gate,
-                            int* hist_s, bool& nonfinite) {
+                            int* hist_s, uint32_t* emask, bool& nonfinite) {
   if (E == 32 * VPL)
-    route_chunk_t<VPL, true>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
+    route_chunk_t<VPL, true>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, emask, nonfinite);
   else
-    route_chunk_t<VPL, false>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
-}
-
-// Ranks the n (token, slot) pairs of a chunk, ex[p] for p = t * k + s, among
-// the chunk's pairs with the same expert, in p order: out[p] = #{p' < p :
-// ex[p'] == ex[p]}.  A warp's 32 pairs are grouped by expert with a match,
-// the groups' sizes go to cnt[warp][e], and a scan over the warps per expert
-// (carried over rounds of blockDim.x pairs) gives each warp's offset.  All
-// threads of the CTA call it; ex was written by this CTA before a barrier.
-__device__ __forceinline__ unsigned lanemask_lt() {
-  unsigned m;
-  asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
-  return m;
+    route_chunk_t<VPL, false>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, emask, nonfinite);
 }
 
 constexpr int kRankWarps = 8;  // warps of a 256-thread routing CTA
-
-__device__ void chunk_ranks(const int32_t* ex, int n, int E, int32_t* out,
-                            int (&cnt)[kRankWarps][EB_MAX_ETOT]) {
-  constexpr int kW = kRankWarps;
-  __shared__ int running[EB_MAX_ETOT];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < kW * E; i += blockDim.x) cnt[i / E][i % E] = 0;
-  for (int e = tid; e < E; e += blockDim.x) running[e] = 0;
-  __syncthreads();
-  for (int r0 = 0; r0 < n; r0 += blockDim.x) {
-    const int p = r0 + tid;
-    const int e = p < n ? ex[p] : -1;
-    const unsigned peers = __match_any_sync(kFull, e);
-    const int in_warp = __popc(peers & lanemask_lt());
-    if (e >= 0 && lane == __ffs(peers) - 1) cnt[warp][e] = __popc(peers);
-    __syncthreads();
-    for (int ee = tid; ee < E; ee += blockDim.x) {
-      int run = running[ee];
-      for (int w = 0; w < kW; ++w) {
-        const int c = cnt[w][ee];
-        cnt[w][ee] = run;
-        run += c;
-      }
-      running[ee] = run;
-    }
-    __syncthreads();
-    if (e >= 0) out[p] = cnt[warp][e] + in_warp;
-    __syncthreads();
-    for (int i = tid; i < kW * E; i += blockDim.x) cnt[i / E][i % E] = 0;
-    __syncthreads();
-  }
-}
+static_assert(kChunk <= 64, "a chunk's tokens fit one 64-bit mask per expert");
 
 // Step path: CTA (c, j) routes chunk c of micro-batch j at its layer l_j if j
 // is in need_route; its counts land in chunk_hist[j][c][:] and are added
@@ -382,8 +347,11 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
   __shared__ int hist_s[EB_MAX_ETOT];
   __shared__ int w_s[EB_MAX_D];
   __shared__ int bad;
+  __shared__ uint32_t emask[2 * EB_MAX_ETOT];  // tokens of the chunk that chose each expert
   for (int e = threadIdx.x; e < d.E; e += blockDim.x) hist_s[e] = 0;
   for (int r = threadIdx.x; r < d.D; r += blockDim.x) w_s[r] = 0;
+  if (rank)
+    for (int i = threadIdx.x; i < 2 * d.E; i += blockDim.x) emask[i] = 0u;
   if (threadIdx.x == 0) bad = 0;
   __syncthreads();
   // rows of micro-batch j at layer l: the caller's logits [M, L, T, E], or
@@ -392,7 +360,7 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
   const int t0 = c * kChunk, t1 = min(d.T, t0 + kChunk);
   bool nonfinite = false;
   route_chunk<VPL>(blk, t0, t1, d.E, d.k, d.renorm, idx + (size_t)j * d.T * d.k,
-                   gate_j + (size_t)j * d.T * d.k, hist_s, nonfinite);
+                   gate_j + (size_t)j * d.T * d.k, hist_s, rank ? emask : nullptr, nonfinite);
   if (nonfinite) bad = 1;
   __syncthreads();
   int32_t* out = chunk_hist + ((size_t)j * d.NC + c) * d.E;
@@ -416,9 +384,18 @@ __global__ void __launch_bounds__(256, 4) k_route_step(Dims d, State* __restrict
   }
   if (threadIdx.x == 0 && bad) atomicCAS(&st->status, EB_OK, EB_ERR_NONFINITE);
   if (rank) {
-    __shared__ int scratch[kRankWarps][EB_MAX_ETOT];
+    // a token's k experts are distinct, so the place of (t, s) among the
+    // chunk's pairs of its expert is the number of earlier tokens of the
+    // chunk whose mask bit that expert has
     const size_t base = (size_t)j * d.T + t0;
-    chunk_ranks(idx + base * d.k, (t1 - t0) * d.k, d.E, rank + base * d.k, scratch);
+    const int32_t* ex = idx + base * d.k;
+    int32_t* rk = rank + base * d.k;
+    for (int p = threadIdx.x; p < (t1 - t0) * d.k; p += blockDim.x) {
+      const int t = p / d.k, e = ex[p];
+      const uint32_t lo = emask[2 * e], below = (1u << (t & 31)) - 1u;
+      rk[p] = t < 32 ? __popc(lo & below) : __popc(lo) + __popc(emask[2 * e + 1] & below);
+    }
+    __shared__ int scratch[kRankWarps][EB_MAX_ETOT];
     // every thread's counts of this chunk are visible before the ticket
     __threadfence();
     __shared__ int last;
@@ -472,7 +449,7 @@ __global__ void __launch_bounds__(256, 4) k_route_rows(const float* __restrict__
   __syncthreads();
   const int t0 = blockIdx.x * kChunk, t1 = min(n, t0 + kChunk);
   bool nonfinite = false;
-  route_chunk<VPL>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nonfinite);
+  route_chunk<VPL>(logits, t0, t1, E, k, renorm, idx, gate, hist_s, nullptr, nonfinite);
   if (nonfinite) bad = 1;
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x)
@@ -616,7 +593,7 @@ __global__ void __launch_bounds__(256, 4) k_route_counts_static(const float* __r
   const int t0 = c * kChunk, t1 = min(T, t0 + kChunk);
   bool nonfinite = false;
   route_chunk<VPL>(logits + (size_t)j * T * E, t0, t1, E, k, renorm, idx + (size_t)j * T * k,
-                   gate + (size_t)j * T * k, hist_s, nonfinite);
+                   gate + (size_t)j * T * k, hist_s, nullptr, nonfinite);
   if (nonfinite) bad = 1;
   __syncthreads();
   int32_t* out = counts + ((size_t)j * NC + c) * E;

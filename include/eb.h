@@ -231,7 +231,11 @@ eb_status eb_expert_ffn(eb_ctx* ctx, const void* rows, int R, const int32_t* seg
 
 /* A whole episode: eb_reset, then eb_moe_step until S is empty.  Steps are
  * enqueued a few ahead of the host's completion check, so the GPU never waits
- * for the host; steps enqueued after S became empty do nothing.  Returns the
+ * for the host; steps enqueued after S became empty do nothing.  The check
+ * reads S from pinned host memory that each scheduler launch writes (the
+ * calling thread polls it, yielding), so nothing but kernels is enqueued
+ * between the steps; without mapped host memory it falls back to a copy and
+ * an event per step.  Returns the
  * number of steps that ran in *n_steps (host).  Waits for completion; returns
  * EB_ERR_TIMEOUT if a bounded device wait expired during the episode.
  * Because every step reads the same logits, consecutive steps overlap (same

@@ -234,6 +234,21 @@ def test_fused_combine_bitwise_equals_unfused(small_inputs, name, policy):
 
 
 @pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16"])
+@pytest.mark.parametrize("policy", [0, 1])
+def test_row_placement_in_copy_equals_positions_pass(small_inputs, name, policy):
+    """The token-major engine (4) places the rows in its row copy, from the
+    ranks and chunk offsets routing computed; the gathering engine (6) takes
+    them from the separate positions pass.  Each row's arithmetic is the
+    same on both, so whole episodes agree bit for bit only if every (token,
+    slot) pair lands on a row of its own segment in both."""
+    import torch
+    inp = small_inputs[name]
+    placed = run_episode(inp, policy, gemm=4)[0].cpu()
+    passed = run_episode(inp, policy, gemm=6)[0].cpu()
+    assert torch.equal(placed.view(torch.int16), passed.view(torch.int16))
+
+
+@pytest.mark.parametrize("name", ["small_bf16", "small_shared_bf16"])
 @pytest.mark.parametrize("gemm", [4, 7, 1])
 def test_routing_ahead_equals_step_by_step(small_inputs, name, gemm):
     """eb_episode routes step i+1 beside step i's GEMM 2, into the gate buffer

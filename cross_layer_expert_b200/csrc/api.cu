@@ -506,7 +506,7 @@ static eb_status enqueue_step(eb_ctx* x, const float* logits, void* hidden, cons
   }
   // the previous step's combine runs beside this step's scheduler: it reads
   // the previous step's view, outputs and gates, none of which the scheduler
-  // writes, and the positions pass after it waits for both
+  // writes, and the row copy (or the positions pass) after it waits for both
   if (e == cudaSuccess && x->combine_deferred) {
     x->combine_deferred = false;
     e = timed(x, 5, 1, s, [&] {

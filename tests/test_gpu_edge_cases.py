@@ -1,8 +1,9 @@
 """Degenerate and boundary cases of the step against the oracle: one token,
 one micro-batch, one rank (u = 1), every expert per token (k = E), one
-expert per rank (D = E), m = M (MaxUtil reduces to lock-step), and a ragged
-token count -- on the default tensor-core engine, on SIMT and with the
-combine fused into GEMM 2."""
+expert per rank (D = E), m = M (MaxUtil reduces to lock-step), a ragged
+token count, the largest expert count and one that leaves routing lanes
+padded -- on the default tensor-core engine, on SIMT and with the combine
+fused into GEMM 2."""
 import numpy as np
 import pytest
 
@@ -31,6 +32,11 @@ CASES = {
     "rank_per_expert": dict(D=16),
     "m_equals_M": dict(m=4),
     "ragged_tokens": dict(T=129, M=3, m=2),
+    # 8 experts per lane in routing (one row per warp) and 256 experts in the
+    # rows' per-expert token masks and ranks
+    "many_experts": dict(E=256, k=8, D=8, T=150),
+    # experts that do not fill the last lane column (padded lanes), ragged T
+    "odd_experts": dict(E=40, k=5, D=8, T=77),
 }
 
 
